@@ -1,0 +1,90 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the bench.
+
+This module holds only random-number recipes: it contains none of the
+sparsity method's arithmetic, so both the CPU oracle and the CUDA library
+can be fed from it without sharing any of the method.  Everything is drawn
+on the CPU with torch's Philox-free default CPU generator (``torch.Generator``
+seeded per tensor) and returned as CPU tensors; callers copy to the device.
+
+The workloads stand in for the pages' models (vision and transformer
+linear/conv weights; the pages' datasets and trained weights are not used):
+
+* ``small_fp32``      W 256x256 ~N(0,1) (seed 0), X 256x128 ~N(0,1) (seed 100)
+* ``linear_4096``     W bf16 4096x4096 = bf16(0.02 * N(0,1)) (seed 1),
+                      X bf16 4096x4096 ~N(0,1) (seed 101)
+* ``mlp_pair``        W_up bf16 14336x4096 (seed 2), W_down bf16 4096x14336
+                      (seed 3), both bf16(0.02 * N(0,1)); X bf16 4096x8192 (seed 102)
+* ``ties_fp32``       W fp32 8192x8192 = fp32(k/100), k ~ U{-8..7} (seed 4)
+* ``decode_skinny``   W bf16 28672x8192 = bf16(0.02 * N(0,1)) (seed 5),
+                      X bf16 8192xT ~N(0,1) (seed 105+T), T in {16,64,256,1024}
+"""
+from __future__ import annotations
+
+import torch
+
+SEEDS = {
+    "small_fp32.W": 0, "small_fp32.X": 100,
+    "linear_4096.W": 1, "linear_4096.X": 101,
+    "mlp_pair.W_up": 2, "mlp_pair.W_down": 3, "mlp_pair.X": 102,
+    "ties_fp32.W": 4,
+    "decode_skinny.W": 5,
+}
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return g
+
+
+def normal(shape, seed: int, std: float = 1.0, dtype=torch.float32) -> torch.Tensor:
+    """N(0, std^2) drawn in fp32 then rounded (RNE) to `dtype`."""
+    x = torch.randn(*shape, generator=_gen(seed), dtype=torch.float32)
+    if std != 1.0:
+        x = x * std
+    return x.to(dtype)
+
+
+def ties(shape, seed: int) -> torch.Tensor:
+    """fp32(k/100), k uniform on the integers -8..7 (computed in fp64, rounded once)."""
+    k = torch.randint(-8, 8, shape, generator=_gen(seed), dtype=torch.int64)
+    return (k.to(torch.float64) / 100.0).to(torch.float32)
+
+
+def small_int(shape, seed: int, lo: int = -8, hi: int = 8, dtype=torch.bfloat16) -> torch.Tensor:
+    """Integer values in [lo, hi], exactly representable in bf16/f16/f32."""
+    k = torch.randint(lo, hi + 1, shape, generator=_gen(seed), dtype=torch.int64)
+    return k.to(torch.float32).to(dtype)
+
+
+# ---- the named workloads ---------------------------------------------------
+def small_fp32():
+    return normal((256, 256), SEEDS["small_fp32.W"]), normal((256, 128), SEEDS["small_fp32.X"])
+
+
+def linear_4096():
+    return (normal((4096, 4096), SEEDS["linear_4096.W"], 0.02, torch.bfloat16),
+            normal((4096, 4096), SEEDS["linear_4096.X"], 1.0, torch.bfloat16))
+
+
+def mlp_pair():
+    return (normal((14336, 4096), SEEDS["mlp_pair.W_up"], 0.02, torch.bfloat16),
+            normal((4096, 14336), SEEDS["mlp_pair.W_down"], 0.02, torch.bfloat16),
+            normal((4096, 8192), SEEDS["mlp_pair.X"], 1.0, torch.bfloat16))
+
+
+def ties_fp32(R: int = 8192, C: int = 8192):
+    return ties((R, C), SEEDS["ties_fp32.W"])
+
+
+def decode_skinny_W():
+    return normal((28672, 8192), SEEDS["decode_skinny.W"], 0.02, torch.bfloat16)
+
+
+def decode_skinny_X(T: int):
+    return normal((8192, T), 105 + T, 1.0, torch.bfloat16)
+
+
+def bits_u16(t: torch.Tensor):
+    """numpy uint16 view of a bf16/f16 CPU tensor (bit patterns)."""
+    return t.contiguous().view(torch.int16).numpy().view("uint16")

@@ -1,0 +1,515 @@
+/*
+ * nm_oracle.c -- plain, slow, obviously-correct CPU oracle for N:M
+ * fine-grained structured sparsity (mask selection, 2:4 compression,
+ * decompression, the tensor-core metadata permutation, and the fp64
+ * sparse x dense product).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load
+ * or call this file; only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark do.  It shares no code, header, table or
+ * constant with the CUDA library: every definition here is written out
+ * again from the sources cited next to it.
+ *
+ * Sources (web pages on N:M sparsity; section names as printed there):
+ *  [SRSTE]  "SR-STE sparse training (quantisation-friendly)",
+ *           blog.bakeneko-kuro.com: section "N:M sparsity / concept",
+ *           Apex static mask listing (mn_1d_best / m4n2_1d) and its
+ *           explanation, SR-STE forward (argsort top-N of |w| per group).
+ *  [ASDNN]  Medium review of "Accelerating Sparse Deep Neural Networks":
+ *           "Benefits of 2:4 sparsity" (compressed matrix R*C/2 values,
+ *           2-bit metadata per kept value, groups with more zeros still
+ *           store 2 values, 36 vs 64 bits per 4 16-bit values),
+ *           "Structured sparse GEMM on tensor cores" (sparse x dense =
+ *           dense), "Network pruning workflow, Step-2" (drop the two
+ *           smallest of every 4).
+ *  [PTX]    NVIDIA PTX ISA, tcgen05 "Sparse matrices" (metadata of
+ *           .kind::f16 sparse MMA in tensor memory) -- the pages give no
+ *           hardware layout; this is the public ISA description.
+ *
+ * Readings of points the pages leave open (each is also listed in the
+ * design notes):
+ *  - N is the number of KEPT entries per group of M.
+ *  - Magnitude order: the IEEE bit pattern with the sign cleared, read as
+ *    an unsigned integer (+0 == -0, subnormals below normals, Inf above
+ *    every finite value, NaN above Inf).
+ *  - Ties: equal magnitude -> the lower in-group index is kept.
+ *  - decompress writes +0.0 at pruned positions.
+ *
+ * Floating point: the only arithmetic is in oracle_spmm, done in double
+ * from exactly-decoded inputs.  Mask selection uses exact integers.
+ */
+#include <stdint.h>
+#include <stddef.h>
+#include <string.h>
+#include <stdlib.h>
+#include <math.h>
+#include <pthread.h>
+
+/* element type codes used by this file's callers (tests pass these) */
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F16 = 2 };
+
+/* status codes */
+enum { OR_OK = 0, OR_BAD_ARG = 1, OR_NONFINITE = 2, OR_BAD_MASK = 3 };
+
+static size_t elem_size(int dtype) { return dtype == OR_F32 ? 4 : 2; }
+
+static uint32_t load_bits(const void *base, int dtype, size_t i)
+{
+    if (dtype == OR_F32) return ((const uint32_t *)base)[i];
+    return ((const uint16_t *)base)[i];
+}
+
+static void store_bits(void *base, int dtype, size_t i, uint32_t v)
+{
+    if (dtype == OR_F32) ((uint32_t *)base)[i] = v;
+    else ((uint16_t *)base)[i] = (uint16_t)v;
+}
+
+/* --------------------------------------------------------------------- */
+/* IEEE-754 decoding, written from the format definitions.                */
+/*   binary32: 1 sign, 8 exponent (bias 127), 23 fraction                 */
+/*   bfloat16: the upper 16 bits of a binary32                            */
+/*   binary16: 1 sign, 5 exponent (bias 15), 10 fraction                  */
+/* --------------------------------------------------------------------- */
+static double decode_generic(uint32_t sign, uint32_t e, uint32_t f,
+                             int ebits, int fbits, int bias)
+{
+    double v;
+    uint32_t emax = (1u << ebits) - 1u;
+    if (e == emax) {
+        if (f != 0) return NAN;
+        v = INFINITY;
+    } else if (e == 0) {
+        v = ldexp((double)f, 1 - bias - fbits);          /* subnormal */
+    } else {
+        v = ldexp((double)(f | (1u << fbits)), (int)e - bias - fbits);
+    }
+    return sign ? -v : v;
+}
+
+double oracle_decode(uint32_t bits, int dtype)
+{
+    if (dtype == OR_F16)
+        return decode_generic(bits >> 15, (bits >> 10) & 0x1Fu, bits & 0x3FFu, 5, 10, 15);
+    if (dtype == OR_BF16) bits <<= 16;
+    return decode_generic(bits >> 31, (bits >> 23) & 0xFFu, bits & 0x7FFFFFu, 8, 23, 127);
+}
+
+/* Round a double to the nearest representable value of a binary format
+ * with `fbits` fraction bits, exponent bias `bias` and `ebits` exponent
+ * bits, ties to even; overflow to Inf (round-to-nearest semantics).
+ * Returns the encoded bit pattern. */
+static uint32_t encode_rne(double x, int ebits, int fbits, int bias)
+{
+    uint32_t sign = signbit(x) ? 1u : 0u;
+    uint32_t emax = (1u << ebits) - 1u;
+    uint32_t sbit = 1u << (ebits + fbits);
+    if (isnan(x)) return (sign ? sbit : 0u) | (emax << fbits) | (1u << (fbits - 1));
+    double a = fabs(x);
+    if (isinf(a)) return (sign ? sbit : 0u) | (emax << fbits);
+    if (a == 0.0) return sign ? sbit : 0u;
+    int e2;
+    frexp(a, &e2);                 /* a = m * 2^e2, m in [0.5, 1) */
+    int exp_unb = e2 - 1;          /* a in [2^exp_unb, 2^(exp_unb+1)) */
+    int emin = 1 - bias;
+    int q = (exp_unb < emin ? emin : exp_unb) - fbits;  /* quantum exponent */
+    double scaled = ldexp(a, -q);  /* exact: power-of-two scaling */
+    double fl = floor(scaled);
+    double rem = scaled - fl;
+    uint64_t n = (uint64_t)fl;
+    if (rem > 0.5 || (rem == 0.5 && (n & 1u))) n += 1;
+    /* n * 2^q is the rounded magnitude */
+    uint32_t E, F;
+    if (q == emin - fbits && n < (1ull << fbits)) {
+        E = 0; F = (uint32_t)n;                          /* subnormal */
+    } else {
+        int ee = q + fbits;
+        if (n >= (2ull << fbits)) { n >>= 1; ee += 1; }  /* carried into next binade */
+        if (ee + bias >= (int)emax) return (sign ? sbit : 0u) | (emax << fbits);
+        E = (uint32_t)(ee + bias);
+        F = (uint32_t)(n - (1ull << fbits));
+    }
+    return (sign ? sbit : 0u) | (E << fbits) | F;
+}
+
+uint32_t oracle_encode(double x, int dtype)
+{
+    if (dtype == OR_F16) return encode_rne(x, 5, 10, 15);
+    if (dtype == OR_BF16) return encode_rne(x, 8, 7, 127);
+    return encode_rne(x, 8, 23, 127);
+}
+
+/* Magnitude key: sign bit cleared, read as unsigned. */
+uint32_t oracle_mag(uint32_t bits, int dtype)
+{
+    return dtype == OR_F32 ? (bits & 0x7FFFFFFFu) : (bits & 0x7FFFu);
+}
+
+/* --------------------------------------------------------------------- */
+/* Mask, variant S: rank rule.                                           */
+/* [SRSTE] SR-STE forward: argsort |w| inside each group of M and zero   */
+/* the M-N smallest; [ASDNN] Step-2: drop the smallest of every group.   */
+/* Element i is kept iff fewer than N elements of its group beat it,     */
+/* where j beats i when mag_j > mag_i, or mag_j == mag_i and j < i.       */
+/* Groups are M consecutive entries of a row (the reduction dimension).  */
+/* --------------------------------------------------------------------- */
+int oracle_mask_rank(const void *W, int dtype, int64_t R, int64_t C, int64_t ldw,
+                     int N, int M, uint8_t *mask, int64_t ldm)
+{
+    if (M < 2 || M > 8 || N < 1 || N >= M || C % M != 0 || R < 0 || C < 0)
+        return OR_BAD_ARG;
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t g = 0; g < C / M; ++g) {
+            uint32_t mag[8];
+            for (int i = 0; i < M; ++i)
+                mag[i] = oracle_mag(load_bits(W, dtype, (size_t)(r * ldw + g * M + i)), dtype);
+            for (int i = 0; i < M; ++i) {
+                int beaten_by = 0;
+                for (int j = 0; j < M; ++j) {
+                    if (j == i) continue;
+                    if (mag[j] > mag[i] || (mag[j] == mag[i] && j < i)) beaten_by++;
+                }
+                mask[r * ldm + g * M + i] = (uint8_t)(beaten_by < N ? 1 : 0);
+            }
+        }
+    }
+    return OR_OK;
+}
+
+/* --------------------------------------------------------------------- */
+/* Mask, variant E: exhaustive pattern search.                           */
+/* [SRSTE] Apex listing (mn_1d_best): enumerate every pattern with N     */
+/* ones among M places, score each by the L1 sum of the |w| it keeps,    */
+/* take the argmax.  Here the sums are EXACT (multi-limb integers in     */
+/* units of 2^-149, the smallest binary32 subnormal) so no rounding can  */
+/* create a false tie, patterns are visited in lexicographic order of    */
+/* their ascending index tuples, and the first strictly greater score    */
+/* wins.  Only finite inputs are accepted.                                */
+/* --------------------------------------------------------------------- */
+#define LIMBS 5  /* 320 bits >= 277-bit magnitude + 3 bits of carry */
+typedef struct { uint64_t w[LIMBS]; } big_t;
+
+static void big_zero(big_t *a) { memset(a, 0, sizeof *a); }
+
+static void big_add_shifted(big_t *a, uint64_t m, int shift)
+{
+    /* a += m << shift, m < 2^24 */
+    int limb = shift / 64, off = shift % 64;
+    uint64_t lo = m << off;
+    uint64_t hi = off ? (m >> (64 - off)) : 0;
+    uint64_t carry = 0;
+    for (int i = limb; i < LIMBS; ++i) {
+        uint64_t add = (i == limb) ? lo : (i == limb + 1 ? hi : 0);
+        uint64_t s = a->w[i] + add;
+        uint64_t c1 = s < add;
+        uint64_t s2 = s + carry;
+        uint64_t c2 = s2 < carry;
+        a->w[i] = s2;
+        carry = c1 + c2;
+        if (i > limb + 1 && carry == 0) break;
+    }
+}
+
+static int big_cmp(const big_t *a, const big_t *b)
+{
+    for (int i = LIMBS - 1; i >= 0; --i) {
+        if (a->w[i] != b->w[i]) return a->w[i] > b->w[i] ? 1 : -1;
+    }
+    return 0;
+}
+
+/* |w| = m * 2^(shift-149): returns 0 on success, -1 if non-finite */
+static int exact_magnitude(uint32_t bits, int dtype, uint64_t *m, int *shift)
+{
+    if (dtype == OR_BF16) { bits <<= 16; dtype = OR_F32; }
+    if (dtype == OR_F32) {
+        uint32_t e = (bits >> 23) & 0xFFu, f = bits & 0x7FFFFFu;
+        if (e == 0xFFu) return -1;
+        if (e == 0) { *m = f; *shift = 0; }
+        else { *m = f | (1u << 23); *shift = (int)e - 1; }
+        return 0;
+    }
+    /* binary16: subnormal f * 2^-24 ; normal (1.f) * 2^(e-15) */
+    uint32_t e = (bits >> 10) & 0x1Fu, f = bits & 0x3FFu;
+    if (e == 0x1Fu) return -1;
+    if (e == 0) { *m = f; *shift = 125; }                 /* 2^-24 = 2^(125-149) */
+    else { *m = f | (1u << 10); *shift = (int)e + 124; }   /* 2^(e-25) */
+    return 0;
+}
+
+int oracle_mask_exhaustive(const void *W, int dtype, int64_t R, int64_t C, int64_t ldw,
+                           int N, int M, uint8_t *mask, int64_t ldm)
+{
+    if (M < 2 || M > 8 || N < 1 || N >= M || C % M != 0 || R < 0 || C < 0)
+        return OR_BAD_ARG;
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t g = 0; g < C / M; ++g) {
+            uint64_t m[8]; int sh[8];
+            for (int i = 0; i < M; ++i) {
+                uint32_t b = load_bits(W, dtype, (size_t)(r * ldw + g * M + i));
+                if (exact_magnitude(b, dtype, &m[i], &sh[i]) != 0) return OR_NONFINITE;
+            }
+            int idx[8], best[8];
+            for (int i = 0; i < N; ++i) idx[i] = i;   /* first combination */
+            big_t best_score; int have_best = 0;
+            for (;;) {
+                big_t s; big_zero(&s);
+                for (int i = 0; i < N; ++i) big_add_shifted(&s, m[idx[i]], sh[idx[i]]);
+                if (!have_best || big_cmp(&s, &best_score) > 0) {
+                    best_score = s; have_best = 1;
+                    memcpy(best, idx, sizeof(int) * (size_t)N);
+                }
+                /* next combination in lexicographic order */
+                int p = N - 1;
+                while (p >= 0 && idx[p] == M - N + p) --p;
+                if (p < 0) break;
+                idx[p]++;
+                for (int q = p + 1; q < N; ++q) idx[q] = idx[q - 1] + 1;
+            }
+            for (int i = 0; i < M; ++i) mask[r * ldm + g * M + i] = 0;
+            for (int i = 0; i < N; ++i) mask[r * ldm + g * M + best[i]] = 1;
+        }
+    }
+    return OR_OK;
+}
+
+/* --------------------------------------------------------------------- */
+/* 2:4 compression. [ASDNN] "Benefits of 2:4 sparsity": the compressed   */
+/* matrix holds R*C/2 values, and 2-bit metadata gives the in-group      */
+/* position of each kept value; every group stores exactly 2 values even */
+/* when it holds more zeros.                                              */
+/* Canonical layout (this library's documented choice):                   */
+/*   values[r][2g+j] = W[r][4g+idx_j], idx_0 < idx_1, bits copied as-is   */
+/*   meta: kept entry k = 2g+j of row r -> its 2-bit idx_j in bits        */
+/*   2*(k%4) .. 2*(k%4)+1 of byte r*(C/8) + k/4 (LSB first).              */
+/* The mask must hold exactly 2 ones per group; otherwise OR_BAD_MASK.    */
+/* --------------------------------------------------------------------- */
+int oracle_compress24(const void *W, const uint8_t *mask, int dtype, int64_t R, int64_t C,
+                      void *values, uint8_t *meta)
+{
+    if (C % 8 != 0 || R < 0) return OR_BAD_ARG;
+    memset(meta, 0, (size_t)(R * C / 8));
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t g = 0; g < C / 4; ++g) {
+            int kept[4], nk = 0;
+            for (int i = 0; i < 4; ++i) {
+                uint8_t mv = mask[r * C + g * 4 + i];
+                if (mv > 1) return OR_BAD_MASK;
+                if (mv) { if (nk == 2) return OR_BAD_MASK; kept[nk++] = i; }
+            }
+            if (nk != 2) return OR_BAD_MASK;
+            for (int j = 0; j < 2; ++j) {
+                int64_t k = 2 * g + j;
+                uint32_t b = load_bits(W, dtype, (size_t)(r * C + g * 4 + kept[j]));
+                store_bits(values, dtype, (size_t)(r * (C / 2) + k), b);
+                meta[r * (C / 8) + k / 4] |= (uint8_t)(kept[j] << (2 * (k % 4)));
+            }
+        }
+    }
+    return OR_OK;
+}
+
+/* Inverse of the above: kept positions get their value, others +0.0. */
+int oracle_decompress24(const void *values, const uint8_t *meta, int dtype, int64_t R, int64_t C,
+                        void *W_out)
+{
+    if (C % 8 != 0 || R < 0) return OR_BAD_ARG;
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t c = 0; c < C; ++c) store_bits(W_out, dtype, (size_t)(r * C + c), 0u);
+        for (int64_t k = 0; k < C / 2; ++k) {
+            int idx = (meta[r * (C / 8) + k / 4] >> (2 * (k % 4))) & 3;
+            int64_t g = k / 2;
+            uint32_t b = load_bits(values, dtype, (size_t)(r * (C / 2) + k));
+            store_bits(W_out, dtype, (size_t)(r * C + g * 4 + idx), b);
+        }
+    }
+    return OR_OK;
+}
+
+/* --------------------------------------------------------------------- */
+/* Tensor-core metadata layout for the sm_100 sparse MMA (.kind::f16).    */
+/* [PTX] tcgen05 sparse matrices: for an MMA of 128 rows x 32 (logical)  */
+/* K, each row's metadata is 32 bits: 8 groups of 4, a 4-bit field per   */
+/* group holding idx_0 | idx_1 << 2.  In tensor memory, lane L of the     */
+/* 32-bit column holds, for m2 = L/16, h = (L%16)/8, m0 = L%8:            */
+/*     bits  0..15: row 16*m2 + m0,     groups 4h..4h+3 of the 32-K slice */
+/*     bits 16..31: row 16*m2 + 8 + m0, groups 4h..4h+3 of the 32-K slice */
+/* This library stores, per block of 128 rows x 128 logical K, the exact  */
+/* 2048-byte image that one 128-lane x 128-bit copy puts in tensor memory:*/
+/*   block (rt, kt) at byte ((rt * ceil(C/128)) + kt) * 2048              */
+/*   16 bytes per lane L, 4 bytes per 32-K slice s = (c%128)/32.          */
+/* Rows are padded to a multiple of 128 and C to a multiple of 128; the   */
+/* padding carries the valid pattern (0,1), nibble 0x4.                   */
+/* --------------------------------------------------------------------- */
+int64_t oracle_meta_sm100_bytes(int64_t R, int64_t C)
+{
+    int64_t Rp = (R + 127) / 128 * 128, Cp = (C + 127) / 128 * 128;
+    return Rp * Cp / 8;
+}
+
+int oracle_meta_sm100(const uint8_t *meta, int64_t R, int64_t C, uint8_t *out)
+{
+    if (C % 8 != 0 || R < 0) return OR_BAD_ARG;
+    int64_t Rp = (R + 127) / 128 * 128, Cp = (C + 127) / 128 * 128;
+    int64_t kblocks = Cp / 128;
+    memset(out, 0, (size_t)(Rp * Cp / 8));
+    for (int64_t r = 0; r < Rp; ++r) {
+        for (int64_t g = 0; g < Cp / 4; ++g) {
+            uint32_t nib;
+            if (r < R && g < C / 4) {
+                /* group g holds kept entries 2g and 2g+1 */
+                int i0 = (meta[r * (C / 8) + (2 * g) / 4] >> (2 * ((2 * g) % 4))) & 3;
+                int i1 = (meta[r * (C / 8) + (2 * g + 1) / 4] >> (2 * ((2 * g + 1) % 4))) & 3;
+                nib = (uint32_t)(i0 | (i1 << 2));
+            } else {
+                nib = 0x4u;
+            }
+            int64_t c = 4 * g;                       /* first logical column of the group */
+            int64_t rt = r / 128, kt = c / 128;
+            int64_t rr = r % 128, cc = c % 128;
+            int64_t lane = (rr % 8) + 8 * ((cc % 32) / 16) + 16 * (rr / 16);
+            int64_t slice = cc / 32;
+            int64_t bit = 16 * ((rr % 16) / 8) + 4 * ((cc % 16) / 4);
+            int64_t byte = (rt * kblocks + kt) * 2048 + lane * 16 + slice * 4 + bit / 8;
+            out[byte] |= (uint8_t)(nib << (bit % 8));
+        }
+    }
+    return OR_OK;
+}
+
+/* --------------------------------------------------------------------- */
+/* Sparse x dense product in double.  [ASDNN] "Structured sparse GEMM on  */
+/* tensor cores": sparse matrix x dense matrix = dense matrix; only the  */
+/* kept values are multiplied.                                            */
+/*   Y[r][t] = alpha * sum_k values[r][k] * X[4*(k/2) + idx_k][t]         */
+/*             + beta * Y_in[r][t]        (Y_in not read when beta == 0)  */
+/* values/meta in the canonical layout, X is K x T row-major, Y_in R x T  */
+/* row-major (y_dtype).  Only the listed rows are computed (rows == NULL  */
+/* means all R rows); Y_out is nrows x T doubles.                          */
+/* --------------------------------------------------------------------- */
+typedef struct {
+    const void *values; const uint8_t *meta; int ab_dtype;
+    const void *X; int64_t T; const void *Y_in; int y_dtype;
+    int64_t R, K; double alpha, beta;
+    const int64_t *rows; int64_t nrows; double *Y_out;
+    int64_t lo, hi;
+} spmm_job;
+
+/* exact decode of one element to double: a 65536-entry table for the
+ * 16-bit formats (filled by oracle_decode), a plain float->double
+ * conversion (exact in C) for binary32 */
+static double *g_tab[3];
+static pthread_once_t g_tab_once = PTHREAD_ONCE_INIT;
+static void build_tables(void)
+{
+    for (int d = OR_BF16; d <= OR_F16; ++d) {
+        g_tab[d] = (double *)malloc(sizeof(double) * 65536);
+        for (uint32_t b = 0; b < 65536; ++b) g_tab[d][b] = oracle_decode(b, d);
+    }
+}
+
+static double decode_fast(const void *base, int dtype, size_t i)
+{
+    if (dtype == OR_F32) {
+        float f;
+        memcpy(&f, (const char *)base + 4 * i, 4);
+        return (double)f;
+    }
+    return g_tab[dtype][((const uint16_t *)base)[i]];
+}
+
+static void *spmm_worker(void *arg)
+{
+    spmm_job *j = (spmm_job *)arg;
+    double *acc = (double *)malloc(sizeof(double) * (size_t)(j->T > 0 ? j->T : 1));
+    for (int64_t i = j->lo; i < j->hi; ++i) {
+        int64_t r = j->rows ? j->rows[i] : i;
+        for (int64_t t = 0; t < j->T; ++t) acc[t] = 0.0;
+        for (int64_t k = 0; k < j->K / 2; ++k) {
+            int idx = (j->meta[r * (j->K / 8) + k / 4] >> (2 * (k % 4))) & 3;
+            int64_t kk = 4 * (k / 2) + idx;            /* logical column of this value */
+            double v = decode_fast(j->values, j->ab_dtype, (size_t)(r * (j->K / 2) + k));
+            for (int64_t t = 0; t < j->T; ++t)
+                acc[t] += v * decode_fast(j->X, j->ab_dtype, (size_t)(kk * j->T + t));
+        }
+        for (int64_t t = 0; t < j->T; ++t) {
+            double y = j->alpha * acc[t];
+            if (j->beta != 0.0)
+                y += j->beta * decode_fast(j->Y_in, j->y_dtype, (size_t)(r * j->T + t));
+            j->Y_out[i * j->T + t] = y;
+        }
+    }
+    free(acc);
+    return NULL;
+}
+
+int oracle_spmm(const void *values, const uint8_t *meta, int ab_dtype,
+                const void *X, int64_t T, const void *Y_in, int y_dtype,
+                int64_t R, int64_t K, double alpha, double beta,
+                const int64_t *rows, int64_t nrows, int nthreads, double *Y_out)
+{
+    if (K % 8 != 0 || R < 0 || T < 0) return OR_BAD_ARG;
+    if (rows == NULL) nrows = R;
+    for (int64_t i = 0; rows && i < nrows; ++i) if (rows[i] < 0 || rows[i] >= R) return OR_BAD_ARG;
+    pthread_once(&g_tab_once, build_tables);
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (nrows < nthreads) nthreads = (int)(nrows > 0 ? nrows : 1);
+    spmm_job jobs[256];
+    pthread_t th[256];
+    for (int i = 0; i < nthreads; ++i) {
+        spmm_job j = { values, meta, ab_dtype, X, T, Y_in, y_dtype, R, K, alpha, beta,
+                       rows, nrows, Y_out, nrows * i / nthreads, nrows * (i + 1) / nthreads };
+        jobs[i] = j;
+    }
+    if (nthreads == 1) { spmm_worker(&jobs[0]); return OR_OK; }
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, spmm_worker, &jobs[i]);
+    for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
+    return OR_OK;
+}
+
+/* --------------------------------------------------------------------- */
+/* Row-parallel drivers for timing the oracle on many cores (the mask and */
+/* compress steps are independent per row).                               */
+/* --------------------------------------------------------------------- */
+typedef struct {
+    const void *W; int dtype; int64_t C; int N, M; uint8_t *mask;
+    void *values; uint8_t *meta; int64_t lo, hi; int what; int status;
+} rows_job;
+
+static void *rows_worker(void *arg)
+{
+    rows_job *j = (rows_job *)arg;
+    int64_t n = j->hi - j->lo;
+    const char *Wr = (const char *)j->W + (size_t)(j->lo * j->C) * elem_size(j->dtype);
+    uint8_t *mr = j->mask + j->lo * j->C;
+    if (j->what == 0) {
+        j->status = oracle_mask_rank(Wr, j->dtype, n, j->C, j->C, j->N, j->M, mr, j->C);
+    } else {
+        j->status = oracle_mask_rank(Wr, j->dtype, n, j->C, j->C, 2, 4, mr, j->C);
+        if (j->status == OR_OK)
+            j->status = oracle_compress24(Wr, mr, j->dtype, n, j->C,
+                                          (char *)j->values + (size_t)(j->lo * j->C / 2) * elem_size(j->dtype),
+                                          j->meta + j->lo * j->C / 8);
+    }
+    return NULL;
+}
+
+/* what = 0: mask only (N:M); what = 1: 2:4 mask then compress. */
+int oracle_rows_parallel(int what, const void *W, int dtype, int64_t R, int64_t C, int N, int M,
+                         uint8_t *mask, void *values, uint8_t *meta, int nthreads)
+{
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > 256) nthreads = 256;
+    if (R < nthreads) nthreads = (int)(R > 0 ? R : 1);
+    rows_job jobs[256];
+    pthread_t th[256];
+    for (int i = 0; i < nthreads; ++i) {
+        rows_job j = { W, dtype, C, N, M, mask, values, meta, R * i / nthreads, R * (i + 1) / nthreads, what, 0 };
+        jobs[i] = j;
+    }
+    for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, rows_worker, &jobs[i]);
+    int st = OR_OK;
+    for (int i = 0; i < nthreads; ++i) { pthread_join(th[i], NULL); if (jobs[i].status) st = jobs[i].status; }
+    return st;
+}
