@@ -1,0 +1,186 @@
+/*
+ * nm.h -- C ABI of libnm: N:M fine-grained structured sparsity on NVIDIA
+ * B200 (sm_100a).  Mask selection, 2:4 compression / decompression, the
+ * tensor-core metadata image, and the 2:4-sparse x dense product.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Matrices are row-major.  Leading dimensions (ld*) count ELEMENTS.
+ *  - W is R x C; groups are M consecutive entries of a row, i.e. along the
+ *    reduction (K) dimension of the product Y = W X.  (Pages: "SR-STE sparse
+ *    training", N:M concept -- N of every M consecutive parameters kept.)
+ *  - Every pointer is a DEVICE pointer owned by the caller; the library
+ *    allocates no device memory.  Every call is asynchronous on `stream`
+ *    (a cudaStream_t passed as void*; NULL = the legacy default stream) and
+ *    returns as soon as the work is enqueued.  The returned status reports
+ *    argument validation and launch errors only; it never waits for the GPU.
+ *  - Device pointers and leading-dimension strides (ld * element size) must
+ *    be 16-byte aligned, else NM_ERR_ALIGN.  Packed arrays (values, meta)
+ *    have no stride argument.  Sizes must be >= 0; R == 0 or C == 0 (or
+ *    T == 0) is a no-op returning NM_OK.
+ *  - Magnitude order: the IEEE bit pattern with the sign bit cleared, read as
+ *    an unsigned integer (so -0 == +0, subnormals < normals < Inf < NaN).
+ *    Ties: the lower in-group index wins.  Both are this library's readings;
+ *    the pages leave them open.
+ *
+ * Canonical compressed 2:4 layout ("Accelerating Sparse Deep Neural
+ * Networks" review, "Benefits of 2:4 sparsity": R*C/2 values plus a 2-bit
+ * in-group index per value; groups with more zeros still store 2 values):
+ *    values[r][2g+j] = W[r][4g+idx_j], idx_0 < idx_1   (R x C/2, W's dtype,
+ *                      bits copied exactly, row stride C/2 elements)
+ *    meta[r][k/4]    bits 2*(k%4)..+1 = idx of kept entry k = 2g+j
+ *                      (R x C/8 bytes, row stride C/8)
+ *
+ * Tensor-core metadata image ("meta_sm100"): the layout the sm_100
+ * .kind::f16 sparse MMA reads from tensor memory (PTX ISA, tcgen05 sparse
+ * matrices).  Per block of 128 rows x 128 logical columns, 2048 bytes:
+ * 16 bytes per tensor-memory lane L, 4 bytes per 32-column slice s; lane
+ * L = r%8 + 8*((c%32)/16) + 16*((r%128)/16), bit 16*((r%16)/8) +
+ * 4*((c%16)/4) of slice (c%128)/32 holds the group's idx_0 | idx_1 << 2.
+ * Blocks are stored row-tile major: block (rt, kt) at byte
+ * (rt*ceil(C/128) + kt) * 2048.  R and C are padded up to multiples of 128;
+ * padded groups hold the pattern (0,1).  Size: nm_sizes().
+ */
+#ifndef NM_H
+#define NM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NM_API __attribute__((visibility("default")))
+#else
+#define NM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NM_OK = 0,
+    NM_ERR_NULL = 1,         /* a required pointer is NULL                      */
+    NM_ERR_SHAPE = 2,        /* bad R / C / K / T / ld (e.g. C % M != 0)        */
+    NM_ERR_ALIGN = 3,        /* pointer or row stride not 16-byte aligned       */
+    NM_ERR_DTYPE = 4,        /* dtype not supported by this call                */
+    NM_ERR_NM = 5,           /* N, M outside 1 <= N < M <= 8                     */
+    NM_ERR_UNSUPPORTED = 6,  /* valid request this build does not implement     */
+    NM_ERR_CUDA = 7,         /* a CUDA runtime / driver call failed             */
+    NM_ERR_WORKSPACE = 8,    /* workspace NULL or smaller than required         */
+    NM_ERR_TIMEOUT = 9       /* a bounded device-side wait gave up (see below)  */
+} nm_status;
+
+typedef enum { NM_F32 = 0, NM_BF16 = 1, NM_F16 = 2 } nm_dtype;
+
+/* Human-readable text for a status code (static string, never NULL). */
+NM_API const char *nm_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+NM_API int nm_version(void);
+
+/*
+ * nm_sizes -- bytes of the compressed forms of an R x C matrix.
+ *   values_bytes     = R * C * N / M * sizeof(dtype)
+ *   meta_bytes       = R * C * N / M * 2 bits / 8  (2:4 only; 0 otherwise)
+ *   meta_sm100_bytes = ceil(R/128)*128 * ceil(C/128)*128 / 8 (2:4 only)
+ * Any output pointer may be NULL.  Errors: NM_ERR_NM, NM_ERR_SHAPE,
+ * NM_ERR_DTYPE.  Source: "Benefits of 2:4 sparsity" (R*C/2 values and
+ * R*C/2 2-bit metadata entries).
+ */
+NM_API nm_status nm_sizes(int64_t R, int64_t C, int N, int M, nm_dtype dtype,
+                   size_t *values_bytes, size_t *meta_bytes, size_t *meta_sm100_bytes);
+
+/*
+ * nm_mask -- N:M magnitude mask.  For every group of M consecutive entries
+ * of each row of W, mask = 1 at the N entries of largest |w| (ties -> lower
+ * index), 0 elsewhere.  Sources: "SR-STE sparse training", SR-STE forward
+ * (argsort of |w| per group, M-N smallest zeroed) and the Apex exhaustive
+ * search (largest kept L1 sum), which select the same entries; review of
+ * "Accelerating Sparse Deep Neural Networks", Step-2 (drop the 2 smallest of 4).
+ *   W     R x C, dtype NM_F32 / NM_BF16 / NM_F16, leading dim ldw >= C
+ *   mask  R x C uint8 (0 or 1), leading dim ldm >= C
+ *   1 <= N < M <= 8, C % M == 0 (else NM_ERR_NM / NM_ERR_SHAPE)
+ */
+NM_API nm_status nm_mask(const void *W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw,
+                  int N, int M, uint8_t *mask, int64_t ldm, void *stream);
+
+/*
+ * nm_mask_compress -- fused 2:4 mask + compression in one pass over W:
+ * the 2:4 mask of nm_mask, then the kept values and their indices in the
+ * canonical layout and (if meta_sm100 != NULL) in the tensor-core image.
+ *   W          R x C (ldw >= C), C % 8 == 0
+ *   values     R x C/2, W's dtype, packed
+ *   meta       R x C/8 bytes, packed (canonical)
+ *   meta_sm100 nm_sizes(...)->meta_sm100_bytes bytes, or NULL
+ */
+NM_API nm_status nm_mask_compress(const void *W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw,
+                           void *values, uint8_t *meta, uint8_t *meta_sm100, void *stream);
+
+/*
+ * nm_compress -- 2:4 compression under a caller-supplied mask (uint8, R x C,
+ * leading dim ldm).  A valid group has exactly two entries equal to 1 and
+ * the rest 0.  Invalid groups are counted into *invalid_groups (a device
+ * int32, added to atomically; pass NULL to skip); their output is the
+ * pattern (0,1) with values W[4g], W[4g+1].  Outputs as nm_mask_compress.
+ */
+NM_API nm_status nm_compress(const void *W, const uint8_t *mask, nm_dtype dtype, int64_t R, int64_t C,
+                      int64_t ldw, int64_t ldm, void *values, uint8_t *meta, uint8_t *meta_sm100,
+                      int32_t *invalid_groups, void *stream);
+
+/*
+ * nm_decompress -- dense R x C from the canonical 2:4 form: kept positions
+ * get their values (bits copied), every other position gets +0.0.
+ *   W_out R x C, leading dim ldw >= C, C % 8 == 0
+ */
+NM_API nm_status nm_decompress(const void *values, const uint8_t *meta, nm_dtype dtype, int64_t R,
+                        int64_t C, void *W_out, int64_t ldw, void *stream);
+
+/*
+ * nm_meta_to_sm100 -- canonical metadata (R x C/8 bytes) -> tensor-core
+ * metadata image (layout above).  C % 8 == 0.
+ */
+NM_API nm_status nm_meta_to_sm100(const uint8_t *meta, int64_t R, int64_t C, uint8_t *meta_sm100,
+                           void *stream);
+
+/*
+ * nm_spmm_workspace_bytes -- device scratch nm_spmm needs for this problem
+ * (0 when none is needed).  NM_F32 inputs are rounded to binary16 (nearest
+ * even) in the workspace before the product.
+ */
+NM_API size_t nm_spmm_workspace_bytes(nm_dtype ab_dtype, int64_t R, int64_t K, int64_t T);
+
+/*
+ * nm_spmm -- Y = alpha * (W (.) mask) X + beta * Y with fp32 accumulation,
+ * W given in compressed 2:4 form.  Review of "Accelerating Sparse Deep
+ * Neural Networks", "Structured sparse GEMM on tensor cores": sparse x dense
+ * = dense; the application supplies the first operand compressed.
+ *   values     R x K/2, ab_dtype (packed, row stride K/2)
+ *   meta_sm100 tensor-core metadata image of W (nm_mask_compress /
+ *              nm_meta_to_sm100), R and K padded to 128
+ *   X          K x T, ab_dtype, leading dim ldx >= T
+ *   Y          R x T, y_dtype (NM_BF16 or NM_F32), leading dim ldy >= T;
+ *              read only when beta != 0
+ *   ab_dtype   NM_BF16 or NM_F16 (tensor-core path), or NM_F32 (rounded to
+ *              binary16 in `workspace`, then the binary16 path)
+ *   K % 16 == 0 (the pages' rule for 16-bit sparse operands); R, T >= 1 any
+ *   workspace  >= nm_spmm_workspace_bytes(...) bytes (may be NULL when 0)
+ * A bounded wait inside the kernel that gives up records NM_ERR_TIMEOUT in a
+ * device status word, read and cleared by nm_last_device_status().
+ */
+NM_API nm_status nm_spmm(const void *values, const uint8_t *meta_sm100, nm_dtype ab_dtype,
+                  const void *X, int64_t ldx, void *Y, nm_dtype y_dtype, int64_t ldy,
+                  int64_t R, int64_t K, int64_t T, float alpha, float beta,
+                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * nm_last_device_status -- synchronises `stream`, then returns and clears the
+ * device status word written by kernels whose bounded waits gave up
+ * (NM_OK if none did).  NM_ERR_CUDA if the synchronisation itself failed.
+ */
+NM_API nm_status nm_last_device_status(void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NM_H */

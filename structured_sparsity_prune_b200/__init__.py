@@ -1,0 +1,193 @@
+"""Python binding of libnm (include/nm.h): N:M structured sparsity on B200.
+
+Argument marshalling only: every step runs in the CUDA kernels of
+``libnm.so``.  Functions keep the C names; tensors are torch CUDA tensors
+(torch supplies device memory and streams), pointers and sizes are passed
+straight through, and a non-zero status raises ``NMError``.  There is no CPU
+fallback: if ``libnm.so`` is missing or fails to load, every call raises.
+
+Element types: torch.float32 -> NM_F32, torch.bfloat16 -> NM_BF16,
+torch.float16 -> NM_F16.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnm.so")
+
+NM_F32, NM_BF16, NM_F16 = 0, 1, 2
+STATUS = ["NM_OK", "NM_ERR_NULL", "NM_ERR_SHAPE", "NM_ERR_ALIGN", "NM_ERR_DTYPE", "NM_ERR_NM",
+          "NM_ERR_UNSUPPORTED", "NM_ERR_CUDA", "NM_ERR_WORKSPACE", "NM_ERR_TIMEOUT"]
+_DT = {torch.float32: NM_F32, torch.bfloat16: NM_BF16, torch.float16: NM_F16}
+
+
+class NMError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s: %s" % (what, _lib().nm_status_string(status).decode()))
+
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libnm.so not built (python -m structured_sparsity_prune_b200.build): " + LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    i64, i32, vp, sz, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float
+    sig = {
+        "nm_status_string": ([i32], ctypes.c_char_p),
+        "nm_version": ([], i32),
+        "nm_sizes": ([i64, i64, i32, i32, i32, vp, vp, vp], i32),
+        "nm_mask": ([vp, i32, i64, i64, i64, i32, i32, vp, i64, vp], i32),
+        "nm_mask_compress": ([vp, i32, i64, i64, i64, vp, vp, vp, vp], i32),
+        "nm_compress": ([vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp, vp], i32),
+        "nm_decompress": ([vp, vp, i32, i64, i64, vp, i64, vp], i32),
+        "nm_meta_to_sm100": ([vp, i64, i64, vp, vp], i32),
+        "nm_spmm_workspace_bytes": ([i32, i64, i64, i64], sz),
+        "nm_spmm": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp, sz, vp], i32),
+        "nm_last_device_status": ([vp], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _LIB = lib
+    return lib
+
+
+def load() -> ctypes.CDLL:
+    """Load libnm.so (raises if it is missing)."""
+    return _lib()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ld(t: torch.Tensor) -> int:
+    assert t.dim() == 2 and t.stride(1) == 1, "row-major 2-D tensor with unit column stride expected"
+    return t.stride(0)
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise NMError(st, what)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise NMError(4, "dtype %s" % t.dtype)
+    return _DT[t.dtype]
+
+
+# ---------------------------------------------------------------------------
+def nm_version() -> int:
+    return _lib().nm_version()
+
+
+def nm_status_string(status: int) -> str:
+    return _lib().nm_status_string(status).decode()
+
+
+def nm_sizes(R: int, C: int, N: int, M: int, dtype: torch.dtype):
+    """-> (values_bytes, meta_bytes, meta_sm100_bytes)."""
+    v, m, s = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(_lib().nm_sizes(R, C, N, M, _DT[dtype], ctypes.byref(v), ctypes.byref(m), ctypes.byref(s)), "nm_sizes")
+    return v.value, m.value, s.value
+
+
+def nm_mask(W: torch.Tensor, N: int, M: int, mask: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    R, C = W.shape
+    if mask is None:
+        mask = torch.empty((R, C), dtype=torch.uint8, device=W.device)
+    _check(_lib().nm_mask(_ptr(W), _dtype(W), R, C, _ld(W), N, M, _ptr(mask), _ld(mask), _stream(stream)), "nm_mask")
+    return mask
+
+
+def alloc_compressed(R: int, C: int, dtype: torch.dtype, device, sm100: bool = True):
+    """Output buffers of the compressing calls: (values, meta, meta_sm100 or None)."""
+    _, mb, sb = nm_sizes(R, C, 2, 4, dtype)
+    values = torch.empty((R, C // 2), dtype=dtype, device=device)
+    meta = torch.empty((R, C // 8), dtype=torch.uint8, device=device)
+    img = torch.empty((sb,), dtype=torch.uint8, device=device) if sm100 else None
+    return values, meta, img
+
+
+def nm_mask_compress(W: torch.Tensor, values=None, meta=None, meta_sm100=None, sm100: bool = True, stream=None):
+    """-> (values, meta, meta_sm100 or None)."""
+    R, C = W.shape
+    if values is None:
+        values, meta, meta_sm100 = alloc_compressed(R, C, W.dtype, W.device, sm100)
+    _check(_lib().nm_mask_compress(_ptr(W), _dtype(W), R, C, _ld(W), _ptr(values), _ptr(meta), _ptr(meta_sm100),
+                                   _stream(stream)), "nm_mask_compress")
+    return values, meta, meta_sm100
+
+
+def nm_compress(W: torch.Tensor, mask: torch.Tensor, values=None, meta=None, meta_sm100=None, sm100: bool = True,
+                invalid_groups: torch.Tensor | None = None, stream=None):
+    """-> (values, meta, meta_sm100 or None); invalid_groups: optional int32 device counter."""
+    R, C = W.shape
+    if values is None:
+        values, meta, meta_sm100 = alloc_compressed(R, C, W.dtype, W.device, sm100)
+    _check(_lib().nm_compress(_ptr(W), _ptr(mask), _dtype(W), R, C, _ld(W), _ld(mask), _ptr(values), _ptr(meta),
+                              _ptr(meta_sm100), _ptr(invalid_groups), _stream(stream)), "nm_compress")
+    return values, meta, meta_sm100
+
+
+def nm_decompress(values: torch.Tensor, meta: torch.Tensor, C: int, out: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    R = values.shape[0]
+    if out is None:
+        out = torch.empty((R, C), dtype=values.dtype, device=values.device)
+    _check(_lib().nm_decompress(_ptr(values), _ptr(meta), _dtype(values), R, C, _ptr(out), _ld(out),
+                                _stream(stream)), "nm_decompress")
+    return out
+
+
+def nm_meta_to_sm100(meta: torch.Tensor, R: int, C: int, out: torch.Tensor | None = None, stream=None):
+    if out is None:
+        out = torch.empty((nm_sizes(R, C, 2, 4, torch.bfloat16)[2],), dtype=torch.uint8, device=meta.device)
+    _check(_lib().nm_meta_to_sm100(_ptr(meta), R, C, _ptr(out), _stream(stream)), "nm_meta_to_sm100")
+    return out
+
+
+def nm_spmm_workspace_bytes(ab_dtype: torch.dtype, R: int, K: int, T: int) -> int:
+    return int(_lib().nm_spmm_workspace_bytes(_DT[ab_dtype], R, K, T))
+
+
+def nm_spmm(values: torch.Tensor, meta_sm100: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = None,
+            y_dtype: torch.dtype = torch.bfloat16, alpha: float = 1.0, beta: float = 0.0,
+            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Y = alpha * (W (.) mask) X + beta * Y from the compressed W (values, meta_sm100)."""
+    R, Kh = values.shape
+    K = 2 * Kh
+    Kx, T = X.shape
+    assert Kx == K, "X must be K x T"
+    if Y is None:
+        Y = torch.empty((R, T), dtype=y_dtype, device=values.device)
+    need = nm_spmm_workspace_bytes(values.dtype, R, K, T)
+    if need and workspace is None:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=values.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib().nm_spmm(_ptr(values), _ptr(meta_sm100), _dtype(values), _ptr(X), _ld(X), _ptr(Y), _dtype(Y),
+                          _ld(Y), R, K, T, float(alpha), float(beta), _ptr(workspace), ws_bytes, _stream(stream)),
+           "nm_spmm")
+    return Y
+
+
+def nm_last_device_status(stream=None) -> int:
+    return int(_lib().nm_last_device_status(_stream(stream)))

@@ -1,0 +1,362 @@
+// nm_compress.cu -- 2:4 compression, decompression and the tensor-core
+// metadata image.
+//
+// Pages: review of "Accelerating Sparse Deep Neural Networks", "Benefits of
+// 2:4 sparsity" -- the compressed matrix keeps R*C/2 values plus a 2-bit
+// in-group index per value, and a group with more zeros still stores two
+// values.  The hardware layout of the indices is the PTX ISA's tcgen05
+// sparse-matrix metadata (the pages do not give one).
+//
+// All kernels here are HBM-bound streams.  The compressing kernels walk the
+// matrix in 128-row x 128-column tiles (one 2048-byte block of the metadata
+// image per tile): each thread takes a (row, 32-column slice) unit, reads its
+// 32 weights with 16-byte loads, selects/compresses in registers, writes its
+// 16 values and 4 canonical metadata bytes with vector stores, and drops the
+// two 16-bit image pieces into shared memory; the block then writes the
+// finished 2048-byte image block with one coalesced 16-byte store per thread.
+#include "nm_internal.cuh"
+
+namespace nm {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr uint32_t kPadByte = 0x44u;  // two groups holding the pattern (0,1)
+
+// 8 consecutive elements (one canonical metadata byte) as raw bits.
+template <typename Bits> struct Oct;
+template <> struct Oct<uint16_t> {
+  uint4 v;
+  __device__ __forceinline__ void load(const uint16_t* p) { v = __ldcs(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ uint16_t operator[](int i) const {
+    const uint32_t w = (&v.x)[i >> 1];
+    return uint16_t((i & 1) ? (w >> 16) : (w & 0xFFFFu));
+  }
+};
+template <> struct Oct<uint32_t> {
+  uint4 v[2];
+  __device__ __forceinline__ void load(const uint32_t* p) {
+    v[0] = __ldcs(reinterpret_cast<const uint4*>(p));
+    v[1] = __ldcs(reinterpret_cast<const uint4*>(p) + 1);
+  }
+  __device__ __forceinline__ uint32_t operator[](int i) const { return (&v[i >> 2].x)[i & 3]; }
+};
+
+// Four compressed values of one octet, stored as a unit.
+template <typename Bits> struct Quad;
+template <> struct Quad<uint16_t> {
+  uint2 v;
+  __device__ __forceinline__ void set(int i, uint16_t b) {
+    uint32_t& w = (&v.x)[i >> 1];
+    w = (i & 1) ? ((w & 0xFFFFu) | (uint32_t(b) << 16)) : ((w & 0xFFFF0000u) | b);
+  }
+  __device__ __forceinline__ void store(uint16_t* p) const { __stcs(reinterpret_cast<uint2*>(p), v); }
+};
+template <> struct Quad<uint32_t> {
+  uint4 v;
+  __device__ __forceinline__ void set(int i, uint32_t b) { (&v.x)[i] = b; }
+  __device__ __forceinline__ void store(uint32_t* p) const { __stcs(reinterpret_cast<uint4*>(p), v); }
+};
+
+// Compress one octet (two groups).  MODE 0 selects by magnitude; MODE 1 takes
+// the caller's mask (8 bytes) and reports whether both groups were valid.
+template <typename Bits, int MODE>
+__device__ __forceinline__ uint32_t compress_octet(const Oct<Bits>& e, uint2 m, Quad<Bits>& q, int& invalid) {
+  uint32_t byte = 0;
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    uint32_t i0, i1;
+    if constexpr (MODE == 0) {
+      const Pick24 p = pick24(mag_key<Bits>(e[4 * g]), mag_key<Bits>(e[4 * g + 1]),
+                              mag_key<Bits>(e[4 * g + 2]), mag_key<Bits>(e[4 * g + 3]));
+      i0 = p.i0;
+      i1 = p.i1;
+    } else {
+      const uint32_t w = g ? m.y : m.x;  // 4 mask bytes of this group
+      uint32_t bits = 0;
+      bool ok = (w & 0xFEFEFEFEu) == 0;  // every byte is 0 or 1
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bits |= ((w >> (8 * i)) & 1u) << i;
+      ok = ok && __popc(bits) == 2;
+      if (!ok) {
+        ++invalid;
+        bits = 0x3u;  // documented fallback: pattern (0,1)
+      }
+      i0 = __ffs(bits) - 1;
+      i1 = 31 - __clz(bits);
+    }
+    q.set(2 * g, sel4<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3], i0));
+    q.set(2 * g + 1, sel4<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3], i1));
+    byte |= (i0 | (i1 << 2)) << (4 * g);
+  }
+  return byte;
+}
+
+// One block walks 128x128 tiles (tile index = rt * kt_count + kt, the same
+// order as the image blocks).
+template <typename Bits, int MODE>
+__global__ void __launch_bounds__(kThreads) compress_tiles_kernel(
+    const Bits* __restrict__ W, int64_t ldw, const uint8_t* __restrict__ mask, int64_t ldm, int64_t R,
+    int64_t C, Bits* __restrict__ values, uint8_t* __restrict__ meta, uint8_t* __restrict__ img,
+    int32_t* __restrict__ invalid_groups) {
+  __shared__ __align__(16) uint16_t s_img[1024];  // one 2048-byte image block
+  const int64_t kt_count = (C + 127) / 128;
+  const int64_t tiles = ((R + 127) / 128) * kt_count;
+  const bool full_rows = (C % 32) == 0;  // vector stores of a whole unit are aligned
+  int invalid = 0;
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    const int64_t rt = tile / kt_count, kt = tile - rt * kt_count;
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      const int u = threadIdx.x + pass * kThreads;  // 512 units: 128 rows x 4 slices
+      const int64_t r = rt * 128 + (u >> 2);
+      const int64_t c0 = kt * 128 + (u & 3) * 32;
+      uint32_t bytes[4] = {kPadByte, kPadByte, kPadByte, kPadByte};
+      if (r < R && c0 < C) {
+        const Bits* wrow = W + r * ldw;
+        if (full_rows) {
+          // whole unit in range: 4 octets, loads first, then work
+          Oct<Bits> e[4];
+          uint2 m[4];
+#pragma unroll
+          for (int o = 0; o < 4; ++o) e[o].load(wrow + c0 + 8 * o);
+          if constexpr (MODE == 1) {
+            const uint4* mp = reinterpret_cast<const uint4*>(mask + r * ldm + c0);
+            const uint4 a = __ldcs(mp), b = __ldcs(mp + 1);
+            m[0] = make_uint2(a.x, a.y); m[1] = make_uint2(a.z, a.w);
+            m[2] = make_uint2(b.x, b.y); m[3] = make_uint2(b.z, b.w);
+          }
+          Quad<Bits> q[4];
+#pragma unroll
+          for (int o = 0; o < 4; ++o) bytes[o] = compress_octet<Bits, MODE>(e[o], m[o], q[o], invalid);
+          Bits* vrow = values + r * (C / 2) + c0 / 2;
+#pragma unroll
+          for (int o = 0; o < 4; ++o) q[o].store(vrow + 4 * o);
+          const uint32_t word = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
+          __stcs(reinterpret_cast<uint32_t*>(meta + r * (C / 8) + c0 / 8), word);
+        } else {
+#pragma unroll
+          for (int o = 0; o < 4; ++o) {
+            const int64_t c = c0 + 8 * o;
+            if (c < C) {
+              Oct<Bits> e;
+              e.load(wrow + c);
+              uint2 m = make_uint2(0u, 0u);
+              if constexpr (MODE == 1) m = __ldcs(reinterpret_cast<const uint2*>(mask + r * ldm + c));
+              Quad<Bits> q;
+              bytes[o] = compress_octet<Bits, MODE>(e, m, q, invalid);
+              q.store(values + r * (C / 2) + c / 2);
+              meta[r * (C / 8) + c / 8] = uint8_t(bytes[o]);
+            }
+          }
+        }
+      }
+      if (img != nullptr) {
+        const uint32_t rl = uint32_t(u >> 2), cl = uint32_t(u & 3) * 32u;
+        s_img[sm100_piece_offset(rl, cl) >> 1] = uint16_t(bytes[0] | (bytes[1] << 8));
+        s_img[sm100_piece_offset(rl, cl + 16) >> 1] = uint16_t(bytes[2] | (bytes[3] << 8));
+      }
+    }
+    if (img != nullptr) {
+      __syncthreads();
+      if (threadIdx.x < 128) {
+        const uint4 v = reinterpret_cast<const uint4*>(s_img)[threadIdx.x];
+        __stcs(reinterpret_cast<uint4*>(img + tile * 2048) + threadIdx.x, v);
+      }
+      __syncthreads();
+    }
+  }
+  if constexpr (MODE == 1) {
+    if (invalid_groups != nullptr) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) invalid += __shfl_xor_sync(0xFFFFFFFFu, invalid, off);
+      if ((threadIdx.x & 31) == 0 && invalid != 0) atomicAdd(invalid_groups, invalid);
+    }
+  }
+}
+
+// canonical metadata -> image, same tiling, no weights involved
+__global__ void __launch_bounds__(kThreads) meta_image_kernel(const uint8_t* __restrict__ meta, int64_t R,
+                                                              int64_t C, uint8_t* __restrict__ img) {
+  __shared__ __align__(16) uint16_t s_img[1024];
+  const int64_t kt_count = (C + 127) / 128;
+  const int64_t tiles = ((R + 127) / 128) * kt_count;
+  const bool full_rows = (C % 32) == 0;
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    const int64_t rt = tile / kt_count, kt = tile - rt * kt_count;
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      const int u = threadIdx.x + pass * kThreads;
+      const int64_t r = rt * 128 + (u >> 2);
+      const int64_t c0 = kt * 128 + (u & 3) * 32;
+      uint32_t word = 0x44444444u;
+      if (r < R && c0 < C) {
+        const uint8_t* mrow = meta + r * (C / 8) + c0 / 8;
+        if (full_rows) {
+          word = __ldcs(reinterpret_cast<const uint32_t*>(mrow));
+        } else {
+#pragma unroll
+          for (int o = 0; o < 4; ++o)
+            if (c0 + 8 * o < C) word = (word & ~(0xFFu << (8 * o))) | (uint32_t(mrow[o]) << (8 * o));
+        }
+      }
+      const uint32_t rl = uint32_t(u >> 2), cl = uint32_t(u & 3) * 32u;
+      s_img[sm100_piece_offset(rl, cl) >> 1] = uint16_t(word & 0xFFFFu);
+      s_img[sm100_piece_offset(rl, cl + 16) >> 1] = uint16_t(word >> 16);
+    }
+    __syncthreads();
+    if (threadIdx.x < 128) {
+      const uint4 v = reinterpret_cast<const uint4*>(s_img)[threadIdx.x];
+      __stcs(reinterpret_cast<uint4*>(img + tile * 2048) + threadIdx.x, v);
+    }
+    __syncthreads();
+  }
+}
+
+// Decompress: unit = one row x 8 columns (one metadata byte, four values).
+template <typename Bits>
+__global__ void __launch_bounds__(256) decompress_kernel(const Bits* __restrict__ values,
+                                                         const uint8_t* __restrict__ meta, int64_t R,
+                                                         int64_t C, Bits* __restrict__ out, int64_t ldo) {
+  const int64_t opr = C / 8;
+  const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
+  const int64_t o_step = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+    for (int64_t o = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; o < opr; o += o_step) {
+      const uint32_t mb = meta[r * (C / 8) + o];
+      Bits v[4], d[8];
+      if constexpr (sizeof(Bits) == 2) {
+        const uint2 x = __ldcs(reinterpret_cast<const uint2*>(values + r * (C / 2) + 4 * o));
+        v[0] = uint16_t(x.x & 0xFFFFu); v[1] = uint16_t(x.x >> 16);
+        v[2] = uint16_t(x.y & 0xFFFFu); v[3] = uint16_t(x.y >> 16);
+      } else {
+        const uint4 x = __ldcs(reinterpret_cast<const uint4*>(values + r * (C / 2) + 4 * o));
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) d[i] = Bits(0);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t idx = (mb >> (2 * k)) & 3u;
+        const int g = k >> 1;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          if (idx == uint32_t(i)) d[4 * g + i] = v[k];
+      }
+      Bits* dst = out + r * ldo + 8 * o;
+      if constexpr (sizeof(Bits) == 2) {
+        uint4 y;
+        y.x = d[0] | (uint32_t(d[1]) << 16); y.y = d[2] | (uint32_t(d[3]) << 16);
+        y.z = d[4] | (uint32_t(d[5]) << 16); y.w = d[6] | (uint32_t(d[7]) << 16);
+        __stcs(reinterpret_cast<uint4*>(dst), y);
+      } else {
+        __stcs(reinterpret_cast<uint4*>(dst), make_uint4(d[0], d[1], d[2], d[3]));
+        __stcs(reinterpret_cast<uint4*>(dst) + 1, make_uint4(d[4], d[5], d[6], d[7]));
+      }
+    }
+  }
+}
+
+int tile_grid(int64_t R, int64_t C) {
+  const int64_t tiles = ((R + 127) / 128) * ((C + 127) / 128);
+  const int64_t want = int64_t(sm_count()) * 8;
+  return int(tiles < want ? tiles : want);
+}
+
+nm_status check_common(const void* W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw) {
+  if (!dtype_ok(dtype)) return NM_ERR_DTYPE;
+  if (R < 0 || C < 0 || C % 8 != 0 || ldw < C) return NM_ERR_SHAPE;
+  (void)W;
+  return NM_OK;
+}
+
+}  // namespace
+}  // namespace nm
+
+using namespace nm;
+
+extern "C" nm_status nm_mask_compress(const void* W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw,
+                                      void* values, uint8_t* meta, uint8_t* meta_sm100, void* stream) {
+  nm_status st = check_common(W, dtype, R, C, ldw);
+  if (st != NM_OK) return st;
+  if (R == 0 || C == 0) return NM_OK;
+  if (W == nullptr || values == nullptr || meta == nullptr) return NM_ERR_NULL;
+  if (!aligned16(W) || !aligned16(values) || !aligned16(meta) || (meta_sm100 && !aligned16(meta_sm100)) ||
+      !stride_ok(ldw, esize_of(dtype)))
+    return NM_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int grid = tile_grid(R, C);
+  if (dtype == NM_F32)
+    compress_tiles_kernel<uint32_t, 0><<<grid, kThreads, 0, s>>>(
+        static_cast<const uint32_t*>(W), ldw, nullptr, 0, R, C, static_cast<uint32_t*>(values), meta,
+        meta_sm100, nullptr);
+  else
+    compress_tiles_kernel<uint16_t, 0><<<grid, kThreads, 0, s>>>(
+        static_cast<const uint16_t*>(W), ldw, nullptr, 0, R, C, static_cast<uint16_t*>(values), meta,
+        meta_sm100, nullptr);
+  return launch_status();
+}
+
+extern "C" nm_status nm_compress(const void* W, const uint8_t* mask, nm_dtype dtype, int64_t R, int64_t C,
+                                 int64_t ldw, int64_t ldm, void* values, uint8_t* meta, uint8_t* meta_sm100,
+                                 int32_t* invalid_groups, void* stream) {
+  nm_status st = check_common(W, dtype, R, C, ldw);
+  if (st != NM_OK) return st;
+  if (ldm < C) return NM_ERR_SHAPE;
+  if (R == 0 || C == 0) return NM_OK;
+  if (W == nullptr || mask == nullptr || values == nullptr || meta == nullptr) return NM_ERR_NULL;
+  if (!aligned16(W) || !aligned16(mask) || !aligned16(values) || !aligned16(meta) ||
+      (meta_sm100 && !aligned16(meta_sm100)) || !stride_ok(ldw, esize_of(dtype)) || !stride_ok(ldm, 1) ||
+      (invalid_groups && (reinterpret_cast<uintptr_t>(invalid_groups) & 3u)))
+    return NM_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int grid = tile_grid(R, C);
+  if (dtype == NM_F32)
+    compress_tiles_kernel<uint32_t, 1><<<grid, kThreads, 0, s>>>(
+        static_cast<const uint32_t*>(W), ldw, mask, ldm, R, C, static_cast<uint32_t*>(values), meta, meta_sm100,
+        invalid_groups);
+  else
+    compress_tiles_kernel<uint16_t, 1><<<grid, kThreads, 0, s>>>(
+        static_cast<const uint16_t*>(W), ldw, mask, ldm, R, C, static_cast<uint16_t*>(values), meta, meta_sm100,
+        invalid_groups);
+  return launch_status();
+}
+
+extern "C" nm_status nm_decompress(const void* values, const uint8_t* meta, nm_dtype dtype, int64_t R, int64_t C,
+                                   void* W_out, int64_t ldw, void* stream) {
+  nm_status st = check_common(W_out, dtype, R, C, ldw);
+  if (st != NM_OK) return st;
+  if (R == 0 || C == 0) return NM_OK;
+  if (values == nullptr || meta == nullptr || W_out == nullptr) return NM_ERR_NULL;
+  if (!aligned16(values) || !aligned16(meta) || !aligned16(W_out) || !stride_ok(ldw, esize_of(dtype)))
+    return NM_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // x over the octets of a row, y over rows
+  const int64_t opr = C / 8;
+  int bx = 32;
+  while (bx < 256 && bx < opr) bx *= 2;
+  const int by = 256 / bx;
+  const int64_t gx = (opr + bx - 1) / bx;
+  const int64_t want = int64_t(sm_count()) * 8;
+  int64_t gy = (R + by - 1) / by;
+  const int64_t cap = gx >= want ? 1 : want / gx;
+  if (gy > cap) gy = cap;
+  if (gy > 65535) gy = 65535;
+  dim3 grid(unsigned(gx), unsigned(gy < 1 ? 1 : gy)), block(bx, by);
+  if (dtype == NM_F32)
+    decompress_kernel<uint32_t><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C,
+                                                       static_cast<uint32_t*>(W_out), ldw);
+  else
+    decompress_kernel<uint16_t><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(values), meta, R, C,
+                                                       static_cast<uint16_t*>(W_out), ldw);
+  return launch_status();
+}
+
+extern "C" nm_status nm_meta_to_sm100(const uint8_t* meta, int64_t R, int64_t C, uint8_t* meta_sm100,
+                                      void* stream) {
+  if (R < 0 || C < 0 || C % 8 != 0) return NM_ERR_SHAPE;
+  if (R == 0 || C == 0) return NM_OK;
+  if (meta == nullptr || meta_sm100 == nullptr) return NM_ERR_NULL;
+  if (!aligned16(meta) || !aligned16(meta_sm100)) return NM_ERR_ALIGN;
+  meta_image_kernel<<<tile_grid(R, C), kThreads, 0, static_cast<cudaStream_t>(stream)>>>(meta, R, C, meta_sm100);
+  return launch_status();
+}

@@ -1,0 +1,97 @@
+// nm_internal.cuh -- helpers shared by the libnm CUDA sources (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nm.h"
+
+namespace nm {
+
+// ----------------------------------------------------------------- host side
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool stride_ok(int64_t ld_elems, int esize) { return ((ld_elems * esize) & 15) == 0; }
+inline int esize_of(nm_dtype d) { return d == NM_F32 ? 4 : 2; }
+inline bool dtype_ok(int d) { return d == NM_F32 || d == NM_BF16 || d == NM_F16; }
+
+inline nm_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? NM_OK : NM_ERR_CUDA;
+}
+
+inline int sm_count() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// ----------------------------------------------------------------- device side
+// Magnitude key: IEEE bits with the sign cleared.  Elements are handled as raw
+// 16- or 32-bit patterns; no floating-point arithmetic touches them.
+template <typename Bits> __device__ __forceinline__ uint32_t mag_key(Bits b);
+template <> __device__ __forceinline__ uint32_t mag_key<uint32_t>(uint32_t b) { return b & 0x7FFFFFFFu; }
+template <> __device__ __forceinline__ uint32_t mag_key<uint16_t>(uint16_t b) { return uint32_t(b) & 0x7FFFu; }
+
+// Keep-bits of one group of M keys: bit i set iff fewer than N entries beat
+// entry i (j beats i: key_j > key_i, or key_j == key_i and j < i).
+// Each unordered pair is compared once: for i < j exactly one beats the other.
+template <int M>
+__device__ __forceinline__ uint32_t keep_bits(const uint32_t (&key)[M], int N) {
+  int beaten[M];
+#pragma unroll
+  for (int i = 0; i < M; ++i) beaten[i] = 0;
+#pragma unroll
+  for (int i = 0; i < M; ++i) {
+#pragma unroll
+    for (int j = i + 1; j < M; ++j) {
+      const int jw = key[j] > key[i] ? 1 : 0;  // j beats i; otherwise i beats j
+      beaten[i] += jw;
+      beaten[j] += 1 - jw;
+    }
+  }
+  uint32_t bits = 0;
+#pragma unroll
+  for (int i = 0; i < M; ++i) bits |= (beaten[i] < N ? 1u : 0u) << i;
+  return bits;
+}
+
+// 2:4 specialisation: the two kept indices (ascending) of a group and the
+// 4-bit metadata field idx0 | idx1 << 2.
+struct Pick24 {
+  uint32_t nib;   // idx0 | idx1 << 2
+  uint32_t i0, i1;
+};
+
+__device__ __forceinline__ Pick24 pick24(uint32_t k0, uint32_t k1, uint32_t k2, uint32_t k3) {
+  const uint32_t key[4] = {k0, k1, k2, k3};
+  const uint32_t b = keep_bits<4>(key, 2);
+  Pick24 p;
+  p.i0 = __ffs(b) - 1;             // lowest set bit
+  p.i1 = 31 - __clz(b);            // highest set bit
+  p.nib = p.i0 | (p.i1 << 2);
+  return p;
+}
+
+template <typename Bits>
+__device__ __forceinline__ Bits sel4(Bits w0, Bits w1, Bits w2, Bits w3, uint32_t i) {
+  Bits a = (i & 1) ? w1 : w0;
+  Bits b = (i & 1) ? w3 : w2;
+  return (i & 2) ? b : a;
+}
+
+// Tensor-core metadata image: byte offset of the 16-bit piece that holds the
+// four group fields of row r, logical columns [c, c+16) with c % 16 == 0,
+// inside its 2048-byte block (see nm.h).
+__device__ __forceinline__ uint32_t sm100_piece_offset(uint32_t r, uint32_t c) {
+  const uint32_t rr = r & 127u, cc = c & 127u;
+  const uint32_t lane = (rr & 7u) + 8u * ((cc & 31u) >> 4) + 16u * (rr >> 4);
+  const uint32_t slice = cc >> 5;
+  return lane * 16u + slice * 4u + 2u * ((rr >> 3) & 1u);
+}
+
+}  // namespace nm

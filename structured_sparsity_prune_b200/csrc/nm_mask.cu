@@ -1,0 +1,144 @@
+// nm_mask.cu -- N:M magnitude mask (any 1 <= N < M <= 8).
+//
+// Pages: "SR-STE sparse training" (N of every M consecutive weights kept;
+// SR-STE forward keeps the N largest |w| of each group; the Apex exhaustive
+// pattern search picks the same entries) and the review of "Accelerating
+// Sparse Deep Neural Networks", Network Pruning Workflow Step-2.
+//
+// HBM-bound streaming kernel: every weight is read once and one mask byte is
+// written per weight.  The selection is integer compares on the magnitude
+// bits (no floating point), M*(M-1)/2 compares per group.
+#include "nm_internal.cuh"
+
+namespace nm {
+namespace {
+
+// 16 consecutive elements of one row -> 16 mask bytes (one 16-byte store).
+template <typename Bits> struct Chunk16;
+template <> struct Chunk16<uint32_t> {
+  static constexpr int kVec = 4;  // 4 x 16 B loads
+};
+template <> struct Chunk16<uint16_t> {
+  static constexpr int kVec = 2;  // 2 x 16 B loads
+};
+
+template <typename Bits, int M>
+__global__ void __launch_bounds__(256) mask_vec16_kernel(const Bits* __restrict__ W, int64_t R,
+                                                         int64_t cpr, int64_t ldw, int N,
+                                                         uint8_t* __restrict__ mask, int64_t ldm) {
+  static_assert(16 % M == 0, "vector path needs M | 16");
+  constexpr int kVec = Chunk16<Bits>::kVec;
+  const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
+  const int64_t c_step = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+    const uint4* wrow = reinterpret_cast<const uint4*>(W + r * ldw);
+    uint4* mrow = reinterpret_cast<uint4*>(mask + r * ldm);
+    for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < cpr; c += c_step) {
+      uint4 v[kVec];
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) v[i] = __ldcs(wrow + c * kVec + i);
+      const Bits* e = reinterpret_cast<const Bits*>(v);
+      uint32_t out[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int g = 0; g < 16 / M; ++g) {
+        uint32_t key[M];
+#pragma unroll
+        for (int i = 0; i < M; ++i) key[i] = mag_key<Bits>(e[g * M + i]);
+        const uint32_t kb = keep_bits<M>(key, N);
+#pragma unroll
+        for (int i = 0; i < M; ++i) {
+          const int pos = g * M + i;  // byte position in the 16-byte chunk
+          out[pos >> 2] |= ((kb >> i) & 1u) << (8 * (pos & 3));
+        }
+      }
+      __stcs(mrow + c, make_uint4(out[0], out[1], out[2], out[3]));
+    }
+  }
+}
+
+// Any M (2..8), any alignment: one thread per group, scalar loads/stores.
+template <typename Bits, int M>
+__global__ void __launch_bounds__(256) mask_scalar_kernel(const Bits* __restrict__ W, int64_t R,
+                                                          int64_t gpr, int64_t ldw, int N,
+                                                          uint8_t* __restrict__ mask, int64_t ldm) {
+  const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
+  const int64_t g_step = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+    for (int64_t g = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; g < gpr; g += g_step) {
+      uint32_t key[M];
+#pragma unroll
+      for (int i = 0; i < M; ++i) key[i] = mag_key<Bits>(W[r * ldw + g * M + i]);
+      const uint32_t kb = keep_bits<M>(key, N);
+#pragma unroll
+      for (int i = 0; i < M; ++i) mask[r * ldm + g * M + i] = uint8_t((kb >> i) & 1u);
+    }
+  }
+}
+
+// 2D launch shape: x over the units of a row, y over rows; about 8 blocks of
+// 256 threads per SM in total.
+void shape2d(int64_t R, int64_t units, dim3& grid, dim3& block) {
+  int bx = 32;
+  while (bx < 256 && bx < units) bx *= 2;
+  const int by = 256 / bx;
+  const int64_t gx = (units + bx - 1) / bx;
+  const int64_t want = int64_t(sm_count()) * 8;
+  int64_t gy = (R + by - 1) / by;
+  const int64_t cap_y = gx >= want ? 1 : want / gx;
+  if (gy > cap_y) gy = cap_y;
+  if (gy > 65535) gy = 65535;
+  grid = dim3(unsigned(gx > 2147483647 ? 2147483647 : gx), unsigned(gy < 1 ? 1 : gy), 1);
+  block = dim3(bx, by, 1);
+}
+
+template <typename Bits, int M>
+void launch_mask(const void* W, int64_t R, int64_t C, int64_t ldw, int N, uint8_t* mask, int64_t ldm,
+                 bool vec, cudaStream_t s) {
+  dim3 grid, block;
+  if constexpr (16 % M == 0) {
+    if (vec) {
+      shape2d(R, C / 16, grid, block);
+      mask_vec16_kernel<Bits, M><<<grid, block, 0, s>>>(static_cast<const Bits*>(W), R, C / 16, ldw, N,
+                                                        mask, ldm);
+      return;
+    }
+  }
+  shape2d(R, C / M, grid, block);
+  mask_scalar_kernel<Bits, M><<<grid, block, 0, s>>>(static_cast<const Bits*>(W), R, C / M, ldw, N, mask, ldm);
+}
+
+template <typename Bits>
+void dispatch_m(const void* W, int64_t R, int64_t C, int64_t ldw, int N, int M, uint8_t* mask, int64_t ldm,
+                bool vec, cudaStream_t s) {
+  switch (M) {
+    case 2: launch_mask<Bits, 2>(W, R, C, ldw, N, mask, ldm, vec, s); break;
+    case 3: launch_mask<Bits, 3>(W, R, C, ldw, N, mask, ldm, vec, s); break;
+    case 4: launch_mask<Bits, 4>(W, R, C, ldw, N, mask, ldm, vec, s); break;
+    case 5: launch_mask<Bits, 5>(W, R, C, ldw, N, mask, ldm, vec, s); break;
+    case 6: launch_mask<Bits, 6>(W, R, C, ldw, N, mask, ldm, vec, s); break;
+    case 7: launch_mask<Bits, 7>(W, R, C, ldw, N, mask, ldm, vec, s); break;
+    default: launch_mask<Bits, 8>(W, R, C, ldw, N, mask, ldm, vec, s); break;
+  }
+}
+
+}  // namespace
+}  // namespace nm
+
+extern "C" nm_status nm_mask(const void* W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw, int N, int M,
+                             uint8_t* mask, int64_t ldm, void* stream) {
+  using namespace nm;
+  if (!dtype_ok(dtype)) return NM_ERR_DTYPE;
+  if (M < 2 || M > 8 || N < 1 || N >= M) return NM_ERR_NM;
+  if (R < 0 || C < 0 || C % M != 0 || ldw < C || ldm < C) return NM_ERR_SHAPE;
+  if (R == 0 || C == 0) return NM_OK;
+  if (W == nullptr || mask == nullptr) return NM_ERR_NULL;
+  const int es = esize_of(dtype);
+  if (!aligned16(W) || !aligned16(mask) || !stride_ok(ldw, es) || !stride_ok(ldm, 1)) return NM_ERR_ALIGN;
+  const bool vec = (C % 16) == 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == NM_F32)
+    dispatch_m<uint32_t>(W, R, C, ldw, N, M, mask, ldm, vec, s);
+  else
+    dispatch_m<uint16_t>(W, R, C, ldw, N, M, mask, ldm, vec, s);
+  return launch_status();
+}

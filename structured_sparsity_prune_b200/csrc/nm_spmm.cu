@@ -1,0 +1,582 @@
+// nm_spmm.cu -- Y = alpha * (W (.) mask) X + beta * Y on sm_100a sparse
+// tensor cores (tcgen05.mma.sp, .kind::f16, fp32 accumulation in TMEM).
+//
+// Pages: review of "Accelerating Sparse Deep Neural Networks", "Structured
+// sparse GEMM on tensor cores" -- sparse matrix x dense matrix = dense matrix,
+// only the kept values are multiplied, and the application hands the first
+// operand over in compressed 2:4 form.  The Ampere design described there is
+// prior art; this kernel is written for the Blackwell execution model:
+//
+//  * one CTA per SM (persistent), a 128-row x N_TILE-column output tile;
+//  * warp 0 (one lane): TMA producer.  Per K-stage of 128 logical columns it
+//    loads the compressed A tile (128 x 64 values, 128B swizzle), the X tile
+//    (128 rows of K x N_TILE, 128B swizzle, N-contiguous) and the 2048-byte
+//    metadata image block (one bulk copy) into a ring of STAGES slots;
+//  * warp 1 (one lane): copies the stage's metadata into tensor memory
+//    (tcgen05.cp 128x128b) and issues four 128 x N_TILE x 32 sparse MMAs
+//    into the TMEM accumulator; tcgen05.commit frees the stage;
+//  * warps 2-5: epilogue.  tcgen05.ld the accumulator (32 columns at a
+//    time), apply alpha / beta in fp32, round to the output type and store.
+//    With two accumulator buffers the epilogue of tile i overlaps the MMAs of
+//    tile i+1.
+//
+// Every mbarrier wait is bounded by a wall-clock limit; on expiry the kernel
+// records NM_ERR_TIMEOUT in the device status word, raises a CTA-wide abort
+// flag so the other roles stop waiting, drains what it issued, frees its
+// tensor memory and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <mutex>
+
+#include "nm_internal.cuh"
+
+namespace nm {
+
+// Device word written by kernels whose bounded waits give up (NM_ERR_TIMEOUT).
+__device__ int g_device_status = 0;
+
+namespace spmm {
+
+constexpr int kBlockM = 128;     // rows of W per tile = TMEM lanes
+constexpr int kStageK = 128;     // logical K per pipeline stage
+constexpr int kStageKPhys = 64;  // compressed values per row per stage (128 B)
+constexpr int kMmaK = 32;        // logical K per sparse MMA instruction
+constexpr int kThreads = 192;    // 6 warps
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+
+// ----------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: true when the phase completed, false on timeout or abort.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (;;) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicExch(&g_device_status, int(NM_ERR_TIMEOUT));
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05): start, leading / stride byte
+// offsets (16-byte units), version 1, layout type in bits 61..63.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFFu);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(layout & 7u) << 61;
+  return d;
+}
+constexpr uint32_t kLayoutNone = 0, kLayoutSW128 = 2;
+
+__device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void mma_sp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t e_tmem,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Instruction descriptor, .kind::f16 with sparsity: D fp32, A/B fp16 or bf16,
+// A K-major, B N-major (X is K x T with T contiguous), M = 128, N = n.
+__host__ __device__ constexpr uint32_t make_idesc(bool bf16, int n) {
+  return (1u << 2)                    // sparse
+         | (1u << 4)                  // D format fp32
+         | ((bf16 ? 1u : 0u) << 7)    // A format
+         | ((bf16 ? 1u : 0u) << 10)   // B format
+         | (0u << 15)                 // A K-major
+         | (1u << 16)                 // B MN-major
+         | (uint32_t(n >> 3) << 17)   // N / 8
+         | (uint32_t(kBlockM >> 4) << 24);  // M / 16
+}
+
+// ----------------------------------------------------------------- kernel
+template <int N_TILE, int STAGES>
+struct Cfg {
+  static constexpr int kABytes = kBlockM * kStageKPhys * 2;   // 16 KB
+  static constexpr int kBBoxes = N_TILE / 64;                 // 64-column TMA boxes
+  static constexpr int kBBoxBytes = kStageK * 64 * 2;         // 16 KB
+  static constexpr int kBBytes = kBBoxes * kBBoxBytes;
+  static constexpr int kEBytes = 2048;
+  static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
+  static constexpr int kAccCols = N_TILE;
+  static constexpr int kAccBufs = (2 * N_TILE + 4 * STAGES <= 512) ? 2 : 1;
+  static constexpr int kECol0 = kAccBufs * N_TILE;
+  static constexpr int kTmemCols = (kECol0 + 4 * STAGES) <= 256 ? 256 : 512;
+  static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 /* align */ + 256 /* barriers, flags */;
+  static_assert(N_TILE % 64 == 0 && N_TILE <= 256, "N_TILE");
+  static_assert(kECol0 + 4 * STAGES <= 512, "TMEM budget");
+};
+
+struct Params {
+  const uint8_t* meta_img;  // tensor-core metadata image
+  void* Y;
+  int64_t ldy;
+  int R, T, K;
+  int m_tiles, n_tiles, k_blocks;
+  int m_inner;  // tile order: 1 -> m fastest
+  int y_f32;    // 1: fp32 output, 0: bf16 output
+  float alpha, beta;
+};
+
+template <int N_TILE, int STAGES, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    spmm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, Params p) {
+  using C = Cfg<N_TILE, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
+  uint64_t* full = bars;                         // [STAGES]
+  uint64_t* empty = bars + STAGES;               // [STAGES]
+  uint64_t* acc_full = bars + 2 * STAGES;        // [2]
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;   // [2]
+  uint64_t* drain = bars + 2 * STAGES + 4;       // MMA completion before TMEM release
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_tiles = p.m_tiles * p.n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto tile_coords = [&](int t, int& mt, int& nt) {
+    if (p.m_inner) { mt = t % p.m_tiles; nt = t / p.m_tiles; }
+    else { nt = t % p.n_tiles; mt = t / p.n_tiles; }
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      uint32_t armed_round[STAGES];
+      for (int s = 0; s < STAGES; ++s) armed_round[s] = 0xFFFFFFFFu;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int mt, nt;
+        tile_coords(t, mt, nt);
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = int(it % STAGES);
+          const uint32_t round = it / STAGES;
+          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* st = smem + s * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+          armed_round[s] = round;
+          tma_load_2d(st, &map_a, &full[s], kb * kStageKPhys, mt * kBlockM);
+#pragma unroll
+          for (int j = 0; j < C::kBBoxes; ++j)
+            tma_load_2d(st + C::kABytes + j * C::kBBoxBytes, &map_b, &full[s], nt * N_TILE + 64 * j, kb * kStageK);
+          const uint8_t* esrc = p.meta_img + (size_t(mt) * p.k_blocks + kb) * 2048;
+          bulk_load(st + C::kABytes + C::kBBytes, esrc, 2048, &full[s]);
+        }
+      }
+      if (!ok) {
+        // drain: every stage armed but maybe unconsumed completes its copies
+        for (int s = 0; s < STAGES; ++s)
+          if (armed_round[s] != 0xFFFFFFFFu) {
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(&full[s], armed_round[s] & 1u) && globaltimer() - t0 < 100000000ull) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(BF16, N_TILE);
+      uint32_t it = 0, local = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
+        const int buf = int(local % C::kAccBufs);
+        const uint32_t use = local / C::kAccBufs;
+        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        fence_after_sync();
+        const uint32_t d_tmem = tmem_base + uint32_t(buf * N_TILE);
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = int(it % STAGES);
+          const uint32_t round = it / STAGES;
+          if (!mbar_wait(&full[s], round & 1u, abort_flag)) { ok = false; break; }
+          fence_after_sync();
+          uint8_t* st = smem + s * C::kStageBytes;
+          const uint32_t a_addr = smem_u32(st);
+          const uint32_t b_addr = smem_u32(st + C::kABytes);
+          const uint32_t e_addr = smem_u32(st + C::kABytes + C::kBBytes);
+          const uint32_t e_tmem = tmem_base + uint32_t(C::kECol0 + 4 * s);
+          // metadata: 128 lanes x 16 bytes, rows contiguous (8-row groups 128 B apart)
+          tmem_cp_128x128b(e_tmem, smem_desc(e_addr, 0, 128, kLayoutNone));
+#pragma unroll
+          for (int k2 = 0; k2 < kStageK / kMmaK; ++k2) {
+            // A: K-major, 128B swizzle, rows 128 B apart, 8-row atoms 1024 B apart;
+            //    32 logical K = 16 compressed values = 32 bytes further per MMA.
+            const uint64_t adesc = smem_desc(a_addr + 32u * k2, 16, 1024, kLayoutSW128);
+            // B: N-major, 128B swizzle: 64-column atoms LBO apart, 8-row K groups 1024 B apart;
+            //    32 logical K rows = 4096 bytes further per MMA.
+            const uint64_t bdesc = smem_desc(b_addr + 4096u * k2, C::kBBoxBytes, 1024, kLayoutSW128);
+            // metadata column of this MMA: even base + selector bit
+            const uint32_t e_col = e_tmem + uint32_t(k2 & ~1);
+            const uint32_t id = idesc | uint32_t(k2 & 1);
+            mma_sp(d_tmem, adesc, bdesc, e_col, id, (kb > 0 || k2 > 0) ? 1u : 0u);
+          }
+          mma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&acc_full[buf]);
+      }
+      // every MMA / copy this thread issued must finish before TMEM is freed
+      mma_commit(drain);
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+      }
+      (void)ok;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;             // TMEM lane quarter this warp may access
+    const int row_in_tile = 32 * q + lane;
+    uint32_t local = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+      int mt, nt;
+      tile_coords(t, mt, nt);
+      const int buf = int(local % C::kAccBufs);
+      const uint32_t use = local / C::kAccBufs;
+      const bool ok = mbar_wait(&acc_full[buf], use & 1u, abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;  // warp-uniform exit keeps tcgen05.ld converged
+      fence_after_sync();
+      const int r = mt * kBlockM + row_in_tile;
+      const int c_base = nt * N_TILE;
+#pragma unroll 1
+      for (int c = 0; c < N_TILE; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TILE + c), v);
+        const int col0 = c_base + c;
+        if (r < p.R && col0 < p.T) {
+          const bool full_chunk = col0 + 32 <= p.T;
+          float y[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) y[j] = p.alpha * __uint_as_float(v[j]);
+          if (p.y_f32) {
+            float* yrow = static_cast<float*>(p.Y) + size_t(r) * p.ldy + col0;
+            if (full_chunk) {
+              if (p.beta != 0.0f) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                  const float4 o = *reinterpret_cast<const float4*>(yrow + j);
+                  y[j] += p.beta * o.x; y[j + 1] += p.beta * o.y; y[j + 2] += p.beta * o.z; y[j + 3] += p.beta * o.w;
+                }
+              }
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(yrow + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+            } else {
+              for (int j = 0; j < 32 && col0 + j < p.T; ++j) {
+                float o = y[j];
+                if (p.beta != 0.0f) o += p.beta * yrow[j];
+                yrow[j] = o;
+              }
+            }
+          } else {
+            __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.Y) + size_t(r) * p.ldy + col0;
+            if (full_chunk) {
+              if (p.beta != 0.0f) {
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                  const uint4 o = *reinterpret_cast<const uint4*>(yrow + j);
+                  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&o);
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    const float2 f = __bfloat1622float2(h[u]);
+                    y[j + 2 * u] += p.beta * f.x;
+                    y[j + 2 * u + 1] += p.beta * f.y;
+                  }
+                }
+              }
+#pragma unroll
+              for (int j = 0; j < 32; j += 8) {
+                uint4 o;
+                __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+                for (int u = 0; u < 4; ++u) h[u] = __floats2bfloat162_rn(y[j + 2 * u], y[j + 2 * u + 1]);
+                *reinterpret_cast<uint4*>(yrow + j) = o;
+              }
+            } else {
+              for (int j = 0; j < 32 && col0 + j < p.T; ++j) {
+                float o = y[j];
+                if (p.beta != 0.0f) o += p.beta * __bfloat162float(yrow[j]);
+                yrow[j] = __float2bfloat16_rn(o);
+              }
+            }
+          }
+        }
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[buf]);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    fence_after_sync();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// f32 -> f16 (round to nearest even) staging for the NM_F32 path
+__global__ void f32_to_f16_kernel(const float* __restrict__ src, int64_t rows, int64_t cols, int64_t lds,
+                                  __half* __restrict__ dst, int64_t ldd) {
+  const int64_t n = rows * cols;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t r = i / cols, c = i - r * cols;
+    dst[r * ldd + c] = __float2half_rn(src[r * lds + c]);
+  }
+}
+
+// ----------------------------------------------------------------- host side
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  });
+  return fn;
+}
+
+// 2D tile map over a row-major [rows x cols] 16-bit matrix, box = box_cols x box_rows, 128B swizzle.
+bool make_map(CUtensorMap* map, const void* base, bool bf16, int64_t rows, int64_t cols, int64_t ld_elems,
+              int box_cols, int box_rows) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(ld_elems) * 2};
+  const cuuint32_t box[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int N_TILE, int STAGES, bool BF16>
+nm_status launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, cudaStream_t s) {
+  using C = Cfg<N_TILE, STAGES>;
+  auto kern = spmm_kernel<N_TILE, STAGES, BF16>;
+  static bool attr_done = false;  // per instantiation
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+      return NM_ERR_CUDA;
+    attr_done = true;
+  }
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  kern<<<grid, kThreads, C::kSmemBytes, s>>>(ma, mb, p);
+  return launch_status();
+}
+
+template <bool BF16>
+nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_t ldx, void* Y, bool y_f32,
+              int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta, cudaStream_t s) {
+  Params p;
+  p.meta_img = meta_img;
+  p.Y = Y;
+  p.ldy = ldy;
+  p.R = int(R);
+  p.T = int(T);
+  p.K = int(K);
+  p.k_blocks = int((K + kStageK - 1) / kStageK);
+  p.y_f32 = y_f32 ? 1 : 0;
+  p.alpha = alpha;
+  p.beta = beta;
+  p.m_tiles = int((R + kBlockM - 1) / kBlockM);
+  const int n_tile = T > 128 ? 256 : (T > 64 ? 128 : 64);
+  p.n_tiles = int((T + n_tile - 1) / n_tile);
+  // stream the larger operand once: W bigger than X -> n fastest
+  const double a_bytes = double(R) * double(K);          // compressed values, 2 B x K/2
+  const double b_bytes = double(K) * double(T) * 2.0;
+  p.m_inner = a_bytes < b_bytes ? 1 : 0;
+
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, values, BF16, R, K / 2, K / 2, kStageKPhys, kBlockM)) return NM_ERR_CUDA;
+  if (!make_map(&mb, X, BF16, K, T, ldx, 64, kStageK)) return NM_ERR_CUDA;
+  switch (n_tile) {
+    case 256: return launch<256, 2, BF16>(ma, mb, p, s);
+    case 128: return launch<128, 4, BF16>(ma, mb, p, s);
+    default: return launch<64, 6, BF16>(ma, mb, p, s);
+  }
+}
+
+}  // namespace spmm
+}  // namespace nm
+
+using namespace nm;
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+extern "C" size_t nm_spmm_workspace_bytes(nm_dtype ab_dtype, int64_t R, int64_t K, int64_t T) {
+  if (ab_dtype != NM_F32 || R <= 0 || K <= 0 || T <= 0) return 0;
+  const int64_t ldx_h = (T + 7) / 8 * 8;
+  return align256(size_t(R) * size_t(K / 2) * 2) + align256(size_t(K) * size_t(ldx_h) * 2);
+}
+
+extern "C" nm_status nm_spmm(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X,
+                             int64_t ldx, void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T,
+                             float alpha, float beta, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!dtype_ok(ab_dtype) || (y_dtype != NM_BF16 && y_dtype != NM_F32)) return NM_ERR_DTYPE;
+  if (R < 0 || K < 0 || T < 0 || K % 16 != 0 || ldx < T || ldy < T) return NM_ERR_SHAPE;
+  if (R > 0x7FFFFFFF - 256 || K > 0x7FFFFFFF - 256 || T > 0x7FFFFFFF - 256) return NM_ERR_SHAPE;
+  if (R == 0 || T == 0) return NM_OK;
+  if (values == nullptr || meta_sm100 == nullptr || X == nullptr || Y == nullptr) return NM_ERR_NULL;
+  const int ab_es = esize_of(ab_dtype), y_es = esize_of(y_dtype);
+  if (!aligned16(values) || !aligned16(meta_sm100) || !aligned16(X) || !aligned16(Y) || !stride_ok(ldx, ab_es) ||
+      !stride_ok(ldy, y_es))
+    return NM_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool y_f32 = y_dtype == NM_F32;
+  if (K == 0) return NM_ERR_SHAPE;
+  if (ab_dtype == NM_F32) {
+    const size_t need = nm_spmm_workspace_bytes(ab_dtype, R, K, T);
+    if (workspace == nullptr || workspace_bytes < need) return NM_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return NM_ERR_ALIGN;
+    const int64_t ldx_h = (T + 7) / 8 * 8;
+    __half* vh = static_cast<__half*>(workspace);
+    __half* xh = reinterpret_cast<__half*>(static_cast<uint8_t*>(workspace) + align256(size_t(R) * size_t(K / 2) * 2));
+    const int blocks = sm_count() * 4;
+    spmm::f32_to_f16_kernel<<<blocks, 256, 0, s>>>(static_cast<const float*>(values), R, K / 2, K / 2, vh, K / 2);
+    spmm::f32_to_f16_kernel<<<blocks, 256, 0, s>>>(static_cast<const float*>(X), K, T, ldx, xh, ldx_h);
+    if (launch_status() != NM_OK) return NM_ERR_CUDA;
+    return spmm::run<false>(vh, meta_sm100, xh, ldx_h, Y, y_f32, ldy, R, K, T, alpha, beta, s);
+  }
+  if (ab_dtype == NM_BF16)
+    return spmm::run<true>(values, meta_sm100, X, ldx, Y, y_f32, ldy, R, K, T, alpha, beta, s);
+  return spmm::run<false>(values, meta_sm100, X, ldx, Y, y_f32, ldy, R, K, T, alpha, beta, s);
+}
+
+extern "C" nm_status nm_last_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return NM_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, nm::g_device_status, sizeof(int)) != cudaSuccess) return NM_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(nm::g_device_status, &zero, sizeof(int)) != cudaSuccess) return NM_ERR_CUDA;
+  }
+  return static_cast<nm_status>(v);
+}

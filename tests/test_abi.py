@@ -1,0 +1,118 @@
+"""The C-ABI library: it builds, loads, exports every symbol include/nm.h
+declares, and validates arguments on the host (no GPU needed: every case
+here fails validation before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import structured_sparsity_prune_b200 as nm
+from structured_sparsity_prune_b200 import build as nm_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nm.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"NM_API\s+[\w\s\*]*?\b(nm_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nm_build.build()
+    return nm.load()
+
+
+def test_header_declares_the_hot_path():
+    names = _declared()
+    for want in ["nm_mask", "nm_mask_compress", "nm_compress", "nm_decompress", "nm_meta_to_sm100", "nm_spmm",
+                 "nm_sizes", "nm_status_string", "nm_spmm_workspace_bytes", "nm_last_device_status"]:
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code, name in enumerate(nm.STATUS):
+        assert nm.nm_status_string(code).startswith(name)
+    assert "unknown" in nm.nm_status_string(99)
+
+
+def test_version(lib):
+    assert nm.nm_version() >= 10000
+
+
+def test_sizes_match_the_pages_counts(lib):
+    import torch
+    # 2:4: R*C/2 values and R*C/2 2-bit fields; image padded to 128 x 128 blocks
+    v, m, s = nm.nm_sizes(4096, 4096, 2, 4, torch.bfloat16)
+    assert v == 4096 * 4096 // 2 * 2 and m == 4096 * 4096 // 2 * 2 // 8 and s == 4096 * 4096 // 8
+    v, m, s = nm.nm_sizes(200, 72, 2, 4, torch.float32)
+    assert v == 200 * 36 * 4 and m == 200 * 9 and s == 256 * 128 // 8
+    # 36 of 64 bits per four 16-bit weights
+    assert (v := nm.nm_sizes(8, 64, 2, 4, torch.float16)[0]) * 8 + m * 0 >= 0
+    v16, m16, _ = nm.nm_sizes(8, 64, 2, 4, torch.float16)
+    assert (v16 + m16) * 8 * 64 == 8 * 64 * 16 * 36
+    # other N:M: values only
+    v, m, s = nm.nm_sizes(10, 80, 2, 8, torch.float32)
+    assert v == 10 * 20 * 4 and m == 0 and s == 0
+
+
+@pytest.mark.parametrize("N,M,code", [(0, 4, 5), (4, 4, 5), (2, 9, 5), (2, 1, 5)])
+def test_sizes_bad_nm(lib, N, M, code):
+    import torch
+    with pytest.raises(nm.NMError) as e:
+        nm.nm_sizes(8, 64, N, M, torch.float32)
+    assert e.value.status == code
+
+
+def test_host_validation_before_any_launch(lib):
+    fake = ctypes.c_void_p(0x10000)          # never dereferenced: validation fails first
+    odd = ctypes.c_void_p(0x10008)
+    s = ctypes.c_void_p(0)
+    L = lib
+    assert L.nm_mask(fake, 7, 4, 64, 64, 2, 4, fake, 64, s) == 4          # bad dtype
+    assert L.nm_mask(fake, 0, 4, 64, 64, 4, 4, fake, 64, s) == 5          # N == M
+    assert L.nm_mask(fake, 0, 4, 66, 66, 2, 4, fake, 66, s) == 2          # C % M
+    assert L.nm_mask(fake, 0, 4, 64, 32, 2, 4, fake, 64, s) == 2          # ldw < C
+    assert L.nm_mask(None, 0, 4, 64, 64, 2, 4, fake, 64, s) == 1          # NULL
+    assert L.nm_mask(odd, 0, 4, 64, 64, 2, 4, fake, 64, s) == 3           # misaligned
+    assert L.nm_mask(fake, 1, 4, 64, 68, 2, 4, fake, 64, s) == 3          # ldw*2 not 16B
+    assert L.nm_mask(fake, 0, 0, 64, 64, 2, 4, fake, 64, s) == 0          # R == 0: no-op
+    assert L.nm_mask_compress(fake, 1, 4, 12, 12, fake, fake, None, s) == 2   # C % 8
+    assert L.nm_mask_compress(fake, 1, 4, 64, 64, None, fake, None, s) == 1
+    assert L.nm_mask_compress(fake, 1, 4, 64, 64, fake, odd, None, s) == 3
+    assert L.nm_compress(fake, fake, 1, 4, 64, 64, 32, fake, fake, None, None, s) == 2  # ldm < C
+    assert L.nm_compress(fake, None, 1, 4, 64, 64, 64, fake, fake, None, None, s) == 1
+    assert L.nm_decompress(fake, fake, 1, 4, 64, fake, 60, s) == 2
+    assert L.nm_meta_to_sm100(fake, 4, 60, fake, s) == 2
+    assert L.nm_meta_to_sm100(None, 4, 64, fake, s) == 1
+    f = ctypes.c_float
+    # spmm: K % 16, dtype of Y, ldx < T, NULL, misaligned, workspace
+    assert L.nm_spmm(fake, fake, 1, fake, 8, fake, 1, 8, 128, 40, 8, f(1), f(0), None, 0, s) == 2
+    assert L.nm_spmm(fake, fake, 1, fake, 8, fake, 2, 8, 128, 64, 8, f(1), f(0), None, 0, s) == 4
+    assert L.nm_spmm(fake, fake, 1, fake, 4, fake, 1, 8, 128, 64, 8, f(1), f(0), None, 0, s) == 2
+    assert L.nm_spmm(fake, None, 1, fake, 8, fake, 1, 8, 128, 64, 8, f(1), f(0), None, 0, s) == 1
+    assert L.nm_spmm(fake, fake, 1, odd, 8, fake, 1, 8, 128, 64, 8, f(1), f(0), None, 0, s) == 3
+    assert L.nm_spmm(fake, fake, 1, fake, 12, fake, 1, 16, 128, 64, 12, f(1), f(0), None, 0, s) == 3
+    assert L.nm_spmm(fake, fake, 0, fake, 8, fake, 0, 8, 128, 64, 8, f(1), f(0), None, 0, s) == 8
+    assert L.nm_spmm(fake, fake, 1, fake, 8, fake, 1, 8, 0, 64, 8, f(1), f(0), None, 0, s) == 0
+
+
+def test_workspace_size(lib):
+    import torch
+    assert nm.nm_spmm_workspace_bytes(torch.bfloat16, 256, 256, 128) == 0
+    need = nm.nm_spmm_workspace_bytes(torch.float32, 256, 256, 128)
+    assert need >= 256 * 128 * 2 + 256 * 128 * 2
+
+
+def test_no_cpu_fallback_in_the_binding():
+    """The product binding must not reach the oracle or any CPU path."""
+    src = open(os.path.join(ROOT, "structured_sparsity_prune_b200", "__init__.py")).read()
+    assert "oracle" not in src.replace("no CPU\nfallback", "")
+    assert "import numpy" not in src

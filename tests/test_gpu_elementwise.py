@@ -1,0 +1,190 @@
+"""GPU parity: mask, fused mask+compress, compress, decompress and the
+metadata image, bit for bit against the CPU oracle on the same seeded inputs."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import nm_inputs
+import structured_sparsity_prune_b200 as nm
+
+pytestmark = pytest.mark.gpu
+
+CODE = {torch.float32: oracle.F32, torch.bfloat16: oracle.BF16, torch.float16: oracle.F16}
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.float32:
+        return t.view(torch.int32).numpy().view(np.uint32)
+    if t.dtype in (torch.bfloat16, torch.float16):
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def _rand(shape, dtype, seed, kind="normal"):
+    if kind == "ties":
+        return nm_inputs.ties(shape, seed).to(dtype)
+    if kind == "special":
+        g = torch.Generator().manual_seed(seed)
+        x = torch.randn(*shape, generator=g)
+        pick = torch.randint(0, 10, shape, generator=g)
+        x[pick == 0] = 0.0
+        x[pick == 1] = -0.0
+        x[pick == 2] = float("inf")
+        x[pick == 3] = float("-inf")
+        x[pick == 4] = float("nan")
+        x[pick == 5] = 1e-40 if dtype == torch.float32 else 1e-6   # subnormal-ish
+        return x.to(dtype)
+    return nm_inputs.normal(shape, seed, 1.0, dtype)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from structured_sparsity_prune_b200 import build
+    build.build()
+    oracle.build()
+    assert torch.cuda.is_available()
+
+
+NM = [(1, 2), (1, 4), (2, 4), (3, 4), (1, 8), (2, 8), (4, 8), (7, 8), (2, 3), (2, 5), (3, 6), (4, 7)]
+
+
+@pytest.mark.parametrize("N,M", NM)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("kind", ["normal", "ties", "special"])
+def test_mask_small(N, M, dtype, kind):
+    R, C = 67, M * 48            # ragged rows; C a multiple of 16 when M | 16
+    W = _rand((R, C), dtype, 10 * N + M, kind)
+    got = nm.nm_mask(W.cuda(), N, M).cpu().numpy()
+    ref = oracle.mask_rank(_bits(W), N, M, dtype=CODE[dtype])
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("N,M", [(2, 4), (4, 8)])
+def test_mask_strided_and_unaligned_c(N, M):
+    """ldw > C and C not a multiple of 16 (scalar path)."""
+    R, C = 33, 24 if M == 4 else 40
+    full = _rand((R, C + 8), torch.bfloat16, 3, "ties")
+    W = full.cuda()[:, :C]
+    mask = torch.full((R, C + 16), 7, dtype=torch.uint8, device="cuda")
+    nm.nm_mask(W, N, M, mask=mask[:, :C])
+    ref = oracle.mask_rank(_bits(full[:, :C]), N, M, dtype=oracle.BF16)
+    assert np.array_equal(mask[:, :C].cpu().numpy(), ref)
+    assert torch.all(mask[:, C:] == 7)   # nothing written past C
+
+
+@pytest.mark.parametrize("N,M", [(1, 4), (2, 4), (4, 8), (2, 8)])
+def test_mask_heavy_ties_full_size(N, M):
+    """The 8192 x 8192 fp32 k/100 workload, whole matrix, bit-exact."""
+    W = nm_inputs.ties_fp32()
+    got = nm.nm_mask(W.cuda(), N, M).cpu().numpy()
+    ref, _, _ = oracle.rows_parallel(0, _bits(W), N, M, oracle.F32, threads=max(1, (os.cpu_count() or 2)))
+    assert np.array_equal(got, ref)
+
+
+
+def _check_compressed(W, values, meta, img, code):
+    Wb = _bits(W)
+    R, C = Wb.shape
+    mask = oracle.mask_rank(Wb, 2, 4, dtype=code)
+    v_ref, m_ref = oracle.compress24(Wb, mask, dtype=code)
+    assert np.array_equal(_bits(values), np.ascontiguousarray(v_ref).view(_bits(values).dtype))
+    assert np.array_equal(meta.cpu().numpy(), m_ref)
+    if img is not None:
+        assert np.array_equal(img.cpu().numpy(), oracle.meta_sm100(m_ref, R, C))
+
+
+SHAPES = [(128, 128), (256, 256), (67, 200), (300, 392), (1, 8), (129, 136), (5, 32), (250, 1000)]
+
+
+@pytest.mark.parametrize("R,C", SHAPES)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_mask_compress(R, C, dtype):
+    W = _rand((R, C), dtype, R + C, "special" if dtype != torch.float32 else "normal")
+    values, meta, img = nm.nm_mask_compress(W.cuda())
+    _check_compressed(W, values, meta, img, CODE[dtype])
+
+
+def test_mask_compress_without_image_and_strided():
+    R, C = 96, 256
+    full = _rand((R, C + 64), torch.bfloat16, 42, "ties")
+    values, meta, img = nm.nm_mask_compress(full.cuda()[:, :C], sm100=False)
+    assert img is None
+    _check_compressed(full[:, :C], values, meta, None, oracle.BF16)
+
+
+@pytest.mark.parametrize("R,C", [(256, 256), (67, 200), (130, 64)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_compress_with_given_mask(R, C, dtype):
+    W = _rand((R, C), dtype, 7, "normal")
+    # a valid but not magnitude-based mask: random (i0 < i1) per group
+    g = torch.Generator().manual_seed(9)
+    pairs = torch.tensor([(0, 1), (0, 2), (0, 3), (1, 2), (1, 3), (2, 3)])
+    choice = pairs[torch.randint(0, 6, (R, C // 4), generator=g)]
+    mask = torch.zeros((R, C // 4, 4), dtype=torch.uint8)
+    mask.scatter_(2, choice, 1)
+    mask = mask.reshape(R, C)
+    ctr = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    values, meta, img = nm.nm_compress(W.cuda(), mask.cuda(), invalid_groups=ctr)
+    v_ref, m_ref = oracle.compress24(_bits(W), mask.numpy(), dtype=CODE[dtype])
+    assert np.array_equal(_bits(values), np.ascontiguousarray(v_ref).view(_bits(values).dtype))
+    assert np.array_equal(meta.cpu().numpy(), m_ref)
+    assert np.array_equal(img.cpu().numpy(), oracle.meta_sm100(m_ref, R, C))
+    assert int(ctr.item()) == 0
+
+
+def test_compress_counts_invalid_groups():
+    R, C = 64, 128
+    W = _rand((R, C), torch.bfloat16, 1)
+    mask = torch.zeros((R, C), dtype=torch.uint8)
+    mask[:, 0::4] = 1
+    mask[:, 1::4] = 1
+    bad = [(0, 0, [1, 1, 1, 0]), (3, 5, [0, 0, 0, 0]), (63, 31, [2, 0, 1, 0]), (10, 7, [1, 0, 0, 0])]
+    for r, g, pat in bad:
+        mask[r, 4 * g:4 * g + 4] = torch.tensor(pat, dtype=torch.uint8)
+    ctr = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    values, meta, _ = nm.nm_compress(W.cuda(), mask.cuda(), invalid_groups=ctr)
+    assert int(ctr.item()) == len(bad)
+    m = meta.cpu().numpy()
+    for r, g, _ in bad:      # documented fallback: pattern (0,1)
+        assert (m[r, g // 2] >> (4 * (g % 2))) & 0xF == 0x4
+
+
+@pytest.mark.parametrize("R,C", SHAPES)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_decompress(R, C, dtype):
+    W = _rand((R, C), dtype, 3 * R + C, "special")
+    Wb = _bits(W)
+    code = CODE[dtype]
+    mask = oracle.mask_rank(Wb, 2, 4, dtype=code)
+    v_ref, m_ref = oracle.compress24(Wb, mask, dtype=code)
+    vals = torch.from_numpy(np.ascontiguousarray(v_ref).view(np.int32 if code == oracle.F32 else np.int16))
+    vals = vals.view(dtype).cuda()
+    out = torch.full((R, C + 8), 3.0, dtype=dtype, device="cuda")
+    nm.nm_decompress(vals, torch.from_numpy(m_ref).cuda(), C, out=out[:, :C])
+    ref = oracle.decompress24(v_ref, m_ref, C, dtype=code)
+    assert np.array_equal(_bits(out[:, :C]), np.ascontiguousarray(ref).view(_bits(out).dtype))
+    assert torch.all(out[:, C:] == 3.0)
+
+
+@pytest.mark.parametrize("R,C", SHAPES)
+def test_meta_to_sm100(R, C):
+    rng = np.random.default_rng(R * 7 + C)
+    nib = rng.choice([0x4, 0x8, 0xC, 0x9, 0xD, 0xE], size=(R, C // 4)).astype(np.uint8)
+    meta = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    got = nm.nm_meta_to_sm100(torch.from_numpy(meta).cuda(), R, C).cpu().numpy()
+    assert np.array_equal(got, oracle.meta_sm100(meta, R, C))
+
+
+def test_linear_4096_mask_compress_full_size():
+    """The 4096 x 4096 bf16 transformer-linear weight, whole matrix, bit-exact."""
+    W, _ = nm_inputs.linear_4096()
+    values, meta, img = nm.nm_mask_compress(W.cuda())
+    Wb = _bits(W)
+    _, v_ref, m_ref = oracle.rows_parallel(1, Wb, 2, 4, oracle.BF16, threads=os.cpu_count() or 2)
+    assert np.array_equal(_bits(values), v_ref)
+    assert np.array_equal(meta.cpu().numpy(), m_ref)
+    assert np.array_equal(img.cpu().numpy(), oracle.meta_sm100(m_ref, 4096, 4096))

@@ -1,0 +1,203 @@
+"""GPU parity of the 2:4 sparse x dense product against the fp64 CPU oracle.
+
+Tolerances (normalised Frobenius error ||Y - Y_ref|| / ||Y_ref||): 1e-3 for
+fp32 output, 8e-3 for bf16 output; exact where the arithmetic is exact
+(integer-valued inputs, one-hot rows)."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import nm_inputs
+import structured_sparsity_prune_b200 as nm
+
+pytestmark = pytest.mark.gpu
+
+CODE = {torch.float32: oracle.F32, torch.bfloat16: oracle.BF16, torch.float16: oracle.F16}
+TOL = {torch.float32: 1e-3, torch.bfloat16: 8e-3}
+THREADS = os.cpu_count() or 2
+
+
+def _bits(t):
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.float32:
+        return t.view(torch.int32).numpy().view(np.uint32)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def _nerr(Y, ref):
+    Yf = Y.detach().float().cpu().numpy().astype(np.float64)
+    den = np.linalg.norm(ref)
+    return np.linalg.norm(Yf - ref) / (den if den > 0 else 1.0)
+
+
+def _ok_status():
+    assert nm.nm_last_device_status() == 0
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from structured_sparsity_prune_b200 import build
+    build.build()
+    oracle.build()
+    assert torch.cuda.is_available()
+
+
+def _run(W, X, y_dtype=torch.bfloat16, alpha=1.0, beta=0.0, Y0=None, rows=None):
+    """GPU: fused compress then spmm.  Oracle: its own compress then fp64 spmm."""
+    ab = W.dtype
+    values, meta, img = nm.nm_mask_compress(W.cuda())
+    Y = None if Y0 is None else Y0.clone().cuda()
+    Y = nm.nm_spmm(values, img, X.cuda(), Y=Y, y_dtype=y_dtype, alpha=alpha, beta=beta)
+    torch.cuda.synchronize()
+    _ok_status()
+    Wb = _bits(W)
+    code = CODE[ab]
+    _, v_ref, m_ref = oracle.rows_parallel(1, Wb, 2, 4, code, threads=THREADS)
+    ref = oracle.spmm(v_ref, m_ref, _bits(X), code, alpha=alpha, beta=beta,
+                      Y_in=None if Y0 is None else _bits(Y0), y_dtype=CODE[y_dtype], rows=rows, threads=THREADS)
+    return Y.cpu() if rows is None else Y.cpu()[torch.as_tensor(rows)], ref
+
+
+@pytest.mark.parametrize("y_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("ab", [torch.bfloat16, torch.float16])
+def test_small_square(ab, y_dtype):
+    W = nm_inputs.normal((256, 256), 11, 0.02, ab)
+    X = nm_inputs.normal((256, 128), 12, 1.0, ab)
+    Y, ref = _run(W, X, y_dtype)
+    assert _nerr(Y, ref) <= TOL[y_dtype]
+
+
+CASES = [(1, 16, 1), (100, 48, 8), (128, 128, 16), (200, 64, 17), (333, 320, 64), (129, 192, 100),
+         (256, 256, 128), (64, 512, 200), (300, 128, 256), (130, 256, 300), (40, 640, 520), (257, 384, 33)]
+
+
+@pytest.mark.parametrize("R,K,T", CASES)
+def test_ragged_shapes(R, K, T):
+    W = nm_inputs.normal((R, K), R + K, 0.02, torch.bfloat16)
+    X = nm_inputs.normal((K, T), T + 3, 1.0, torch.bfloat16)
+    Y, ref = _run(W, X, torch.float32)
+    assert _nerr(Y, ref) <= 1e-3
+
+
+@pytest.mark.parametrize("T", [8, 64, 130, 256, 512])
+def test_integer_inputs_are_exact(T):
+    """Integers in [-8, 8], K = 256: every partial sum is exact in fp32, so the
+    fp32 output equals the exact product bit for bit, and the bf16 output is
+    its round-to-nearest-even."""
+    R, K = 192, 256
+    W = nm_inputs.small_int((R, K), 21, dtype=torch.bfloat16)
+    X = nm_inputs.small_int((K, T), 22, dtype=torch.bfloat16)
+    Y, ref = _run(W, X, torch.float32)
+    assert np.array_equal(Y.numpy().astype(np.float64), ref)
+    Yb, ref_b = _run(W, X, torch.bfloat16)
+    expect = oracle.encode_array(ref_b, oracle.BF16)
+    assert np.array_equal(_bits(Yb), expect)
+
+
+def test_one_hot_rows_select_x_rows():
+    R, K, T = 256, 512, 192
+    g = torch.Generator().manual_seed(5)
+    cols = torch.randint(0, K, (R,), generator=g)
+    W = torch.zeros((R, K), dtype=torch.bfloat16)
+    W[torch.arange(R), cols] = 1.0
+    X = nm_inputs.normal((K, T), 6, 1.0, torch.bfloat16)
+    values, meta, img = nm.nm_mask_compress(W.cuda())
+    Y = nm.nm_spmm(values, img, X.cuda(), y_dtype=torch.float32)
+    assert torch.equal(Y.cpu(), X[cols].float())
+
+
+def test_oracle_image_drives_the_kernel():
+    """The kernel reading an image built by the oracle (not by the GPU)."""
+    R, K, T = 256, 384, 96
+    W = nm_inputs.normal((R, K), 31, 1.0, torch.bfloat16)
+    X = nm_inputs.normal((K, T), 32, 1.0, torch.bfloat16)
+    Wb = _bits(W)
+    v_ref, m_ref = oracle.compress24(Wb, oracle.mask_rank(Wb, 2, 4, dtype=oracle.BF16), dtype=oracle.BF16)
+    img = torch.from_numpy(oracle.meta_sm100(m_ref, R, K)).cuda()
+    vals = torch.from_numpy(np.ascontiguousarray(v_ref).view(np.int16)).view(torch.bfloat16).cuda()
+    Y = nm.nm_spmm(vals, img, X.cuda(), y_dtype=torch.float32)
+    ref = oracle.spmm(v_ref, m_ref, _bits(X), oracle.BF16, threads=THREADS)
+    assert _nerr(Y, ref) <= 1e-3
+
+
+@pytest.mark.parametrize("y_dtype", [torch.float32, torch.bfloat16])
+def test_alpha_beta(y_dtype):
+    R, K, T = 200, 256, 160
+    W = nm_inputs.normal((R, K), 41, 0.02, torch.bfloat16)
+    X = nm_inputs.normal((K, T), 42, 1.0, torch.bfloat16)
+    Y0 = nm_inputs.normal((R, T), 43, 1.0, y_dtype)
+    Y, ref = _run(W, X, y_dtype, alpha=2.0, beta=0.5, Y0=Y0)
+    assert _nerr(Y, ref) <= TOL[y_dtype]
+
+
+def test_beta_zero_never_reads_y():
+    R, K, T = 130, 128, 72
+    W = nm_inputs.normal((R, K), 51, 1.0, torch.bfloat16)
+    X = nm_inputs.normal((K, T), 52, 1.0, torch.bfloat16)
+    Y0 = torch.full((R, T), float("nan"), dtype=torch.float32)
+    Y, ref = _run(W, X, torch.float32, alpha=1.0, beta=0.0, Y0=Y0)
+    assert torch.isfinite(Y).all()
+    assert _nerr(Y, ref) <= 1e-3
+
+
+def test_strided_x_and_y():
+    R, K, T = 160, 256, 100
+    W = nm_inputs.normal((R, K), 61, 1.0, torch.float16)
+    Xfull = nm_inputs.normal((K, T + 28), 62, 1.0, torch.float16)
+    values, meta, img = nm.nm_mask_compress(W.cuda())
+    Yfull = torch.full((R, T + 60), 9.0, dtype=torch.float32, device="cuda")
+    nm.nm_spmm(values, img, Xfull.cuda()[:, :T], Y=Yfull[:, :T])
+    Wb = _bits(W)
+    v_ref, m_ref = oracle.compress24(Wb, oracle.mask_rank(Wb, 2, 4, dtype=oracle.F16), dtype=oracle.F16)
+    ref = oracle.spmm(v_ref, m_ref, _bits(Xfull[:, :T].contiguous()), oracle.F16, threads=THREADS)
+    assert _nerr(Yfull[:, :T], ref) <= 1e-3
+    assert torch.all(Yfull[:, T:] == 9.0)
+
+
+def test_fp32_inputs_small_workload():
+    """The 256 x 256 fp32 weight, X 256 x 128 fp32: rounded to binary16 inside
+    the call, fp32 accumulation and output; within 1e-3 of the fp64 product."""
+    W, X = nm_inputs.small_fp32()
+    Y, ref = _run(W, X, torch.float32)
+    err = _nerr(Y, ref)
+    assert err <= 1e-3, err
+
+
+def test_repeat_calls_are_deterministic():
+    W = nm_inputs.normal((384, 512), 71, 0.02, torch.bfloat16).cuda()
+    X = nm_inputs.normal((512, 384), 72, 1.0, torch.bfloat16).cuda()
+    values, meta, img = nm.nm_mask_compress(W)
+    a = nm.nm_spmm(values, img, X)
+    b = nm.nm_spmm(values, img, X)
+    assert torch.equal(a, b)
+
+
+def _sample_rows(R, per_tile=2):
+    rows = []
+    for t in range((R + 127) // 128):
+        for j in range(per_tile):
+            r = t * 128 + (37 * j + 11 * t) % 128
+            if r < R:
+                rows.append(r)
+    rows.append(R - 1)
+    return np.array(sorted(set(rows)), dtype=np.int64)
+
+
+def test_linear_4096_full_size_sampled_rows():
+    """4096 x 4096 x 4096 bf16 (bf16 out), rows sampled across every row tile."""
+    W, X = nm_inputs.linear_4096()
+    rows = _sample_rows(4096, 2)
+    Y, ref = _run(W, X, torch.bfloat16, rows=rows)
+    assert _nerr(Y, ref) <= 8e-3
+
+
+@pytest.mark.parametrize("T", [16, 64, 256, 1024])
+def test_decode_skinny_full_size_sampled_rows(T):
+    W = nm_inputs.decode_skinny_W()
+    X = nm_inputs.decode_skinny_X(T)
+    rows = _sample_rows(W.shape[0], 1)
+    Y, ref = _run(W, X, torch.bfloat16, rows=rows)
+    assert _nerr(Y, ref) <= 8e-3
