@@ -1,0 +1,474 @@
+"""Benchmark of the N:M sparsity hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload linear_4096|mlp_pair|decode_T16|decode_T64|decode_T256|decode_T1024|ties_mask]
+
+One step is one pass of every step of the path over one batch of synthetic
+input (default: the transformer-linear workload, bf16 W 4096x4096 pruned 2:4
+along K, X 4096x4096 tokens):
+    nm_mask (2:4) -> nm_compress (that mask) -> nm_mask_compress (fused)
+    -> nm_meta_to_sm100 -> nm_decompress -> nm_spmm (Y = W' X, bf16 out).
+`value` is the dense-equivalent TFLOP/s of the whole step (2*R*K*T flops per
+step over the device time of the full step); the per-kernel breakdown, the
+roofline of the dominant kernel (nm_spmm, sparse tensor peak) and the
+bandwidth kernels' GB/s against HBM are reported beside it.
+
+Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
+events on the launching stream, with L2 flushed (a 256 MiB write) between
+steps outside the events; barrier + synchronize around the loop; the max over
+ranks.  N > 1 runs one independent copy of the workload per GPU (the path
+has no exchange step; weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import nm_inputs  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+SPARSE_RATIO = 2.0   # 2:4 sparse tensor peak = 2x dense (dense-equivalent flops)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------- workloads
+def make_workload(name: str):
+    """-> dict(W, X, R, K, T, desc) with CPU tensors."""
+    if name == "linear_4096":
+        W, X = nm_inputs.linear_4096()
+        desc = "transformer linear: bf16 W 4096x4096 ~N(0,0.02) 2:4 along K; X bf16 4096x4096 ~N(0,1)"
+    elif name.startswith("decode_T"):
+        T = int(name[len("decode_T"):])
+        W, X = nm_inputs.decode_skinny_W(), nm_inputs.decode_skinny_X(T)
+        desc = "decode-like skinny: bf16 W 28672x8192 ~N(0,0.02) 2:4; X bf16 8192x%d ~N(0,1)" % T
+    elif name == "mlp_pair":
+        W_up, W_down, X = nm_inputs.mlp_pair()
+        return {"W": W_up, "W2": W_down, "X": X, "R": W_up.shape[0], "K": W_up.shape[1], "T": X.shape[1],
+                "desc": "MLP pair: bf16 W_up 14336x4096, W_down 4096x14336 ~N(0,0.02) 2:4; X bf16 4096x8192 ~N(0,1);"
+                        " up then down"}
+    elif name == "ties_mask":
+        W = nm_inputs.ties_fp32()
+        return {"W": W, "X": None, "R": 8192, "K": 8192, "T": 0,
+                "desc": "mask-only: fp32 W 8192x8192 = k/100, k ~ U{-8..7}; 1:4, 2:4, 4:8, 2:8"}
+    else:
+        raise SystemExit("unknown workload " + name)
+    return {"W": W, "X": X, "R": W.shape[0], "K": W.shape[1], "T": X.shape[1], "desc": desc}
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", "nm_clocks_%d_%d.csv" % (os.getpid(), index))
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons, n = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                n += 1
+                for name, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": n}
+
+
+# ----------------------------------------------------------------- GPU arm
+def _dev_x(X: torch.Tensor, dev) -> torch.Tensor:
+    """X on the device in a buffer whose rows are 16-byte aligned."""
+    K, T = X.shape
+    buf = torch.zeros((K, (T + 7) // 8 * 8), dtype=X.dtype, device=dev)
+    buf[:, :T].copy_(X)
+    return buf[:, :T]
+
+
+class Step:
+    """Device buffers and the launch sequence of one step of the path."""
+
+    def __init__(self, nm, wl, dev):
+        self.nm, self.wl, self.dev = nm, wl, dev
+        R, K, T = wl["R"], wl["K"], wl["T"]
+        self.kind = "ties" if wl["X"] is None else ("mlp" if "W2" in wl else "linear")
+        self.W = wl["W"].to(dev)
+        if self.kind == "ties":
+            self.masks = [torch.empty((R, K), dtype=torch.uint8, device=dev) for _ in range(4)]
+            self.names = ["nm_mask_1:4", "nm_mask_2:4", "nm_mask_4:8", "nm_mask_2:8"]
+            G = R * K
+            self.bytes = {n: G * (4 + 1) for n in self.names}
+            self.flops = 0
+            return
+        self.X = _dev_x(wl["X"], dev)
+        v, m, img = nm.alloc_compressed(R, K, self.W.dtype, dev)
+        self.values, self.meta, self.img = v, m, img
+        if self.kind == "mlp":
+            self.W2 = wl["W2"].to(dev)
+            R2, K2 = self.W2.shape
+            self.v2, self.m2, self.img2 = nm.alloc_compressed(R2, K2, self.W2.dtype, dev)
+            self.H = torch.empty((R, (T + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)[:, :T]
+            self.Y = torch.empty((R2, T), dtype=torch.bfloat16, device=dev)
+            self.names = ["nm_mask_compress_up", "nm_mask_compress_down", "nm_spmm_up", "nm_spmm_down"]
+            G1, G2 = R * K, R2 * K2
+            self.bytes = {"nm_mask_compress_up": G1 * 3.25, "nm_mask_compress_down": G2 * 3.25,
+                          "nm_spmm_up": G1 * 1.125 + K * T * 2 + R * T * 2,
+                          "nm_spmm_down": G2 * 1.125 + K2 * T * 2 + R2 * T * 2}
+            self.flop_k = {"nm_spmm_up": 2.0 * R * K * T, "nm_spmm_down": 2.0 * R2 * K2 * T}
+            self.flops = sum(self.flop_k.values())
+            return
+        self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
+        self.v_c, self.m_c, self.img_c = nm.alloc_compressed(R, K, self.W.dtype, dev)
+        self.img_r = torch.empty_like(self.img)
+        self.Wd = torch.empty_like(self.W)
+        self.Y = torch.empty((R, T), dtype=torch.bfloat16, device=dev)
+        self.names = ["nm_mask", "nm_compress", "nm_mask_compress", "nm_meta_to_sm100", "nm_decompress", "nm_spmm"]
+        G = R * K
+        es = self.W.element_size()
+        self.bytes = {"nm_mask": G * (es + 1), "nm_compress": G * (es + 1 + es / 2 + 0.25),
+                      "nm_mask_compress": G * (es + es / 2 + 0.25), "nm_meta_to_sm100": G * 0.25,
+                      "nm_decompress": G * (es / 2 + 0.125 + es),
+                      "nm_spmm": G * (es / 2 + 0.125) + K * T * es + R * T * 2}
+        self.flop_k = {"nm_spmm": 2.0 * R * K * T}
+        self.flops = self.flop_k["nm_spmm"]
+
+    def launches(self):
+        return len(self.names)
+
+    def run(self, events=None):
+        nm, s = self.nm, torch.cuda.current_stream()
+        rec = (lambda i: events[i].record(s)) if events is not None else (lambda i: None)
+        rec(0)
+        if self.kind == "ties":
+            for i, (N, M) in enumerate([(1, 4), (2, 4), (4, 8), (2, 8)]):
+                nm.nm_mask(self.W, N, M, mask=self.masks[i])
+                rec(i + 1)
+        elif self.kind == "mlp":
+            nm.nm_mask_compress(self.W, self.values, self.meta, self.img)
+            rec(1)
+            nm.nm_mask_compress(self.W2, self.v2, self.m2, self.img2)
+            rec(2)
+            nm.nm_spmm(self.values, self.img, self.X, Y=self.H)
+            rec(3)
+            nm.nm_spmm(self.v2, self.img2, self.H, Y=self.Y)
+            rec(4)
+        else:
+            K = self.wl["K"]
+            nm.nm_mask(self.W, 2, 4, mask=self.mask)
+            rec(1)
+            nm.nm_compress(self.W, self.mask, self.v_c, self.m_c, self.img_c)
+            rec(2)
+            nm.nm_mask_compress(self.W, self.values, self.meta, self.img)
+            rec(3)
+            nm.nm_meta_to_sm100(self.meta, self.wl["R"], K, out=self.img_r)
+            rec(4)
+            nm.nm_decompress(self.values, self.meta, K, out=self.Wd)
+            rec(5)
+            nm.nm_spmm(self.values, self.img, self.X, Y=self.Y)
+            rec(6)
+
+    def result(self):
+        return self.masks[1] if self.kind == "ties" else self.Y
+
+
+def timed_steps(step: Step, steps: int, flush: torch.Tensor):
+    """-> (per-step ms list, per-kernel ms lists) over exactly `steps` steps."""
+    n = step.launches()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()                      # evict L2 between steps (outside the events)
+        step.run(ev[i])
+    torch.cuda.synchronize()
+    tot = [ev[i][0].elapsed_time(ev[i][n]) for i in range(steps)]
+    per = {name: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps)] for j, name in enumerate(step.names)}
+    return tot, per
+
+
+def e2e_steps(step: Step, steps: int, flush: torch.Tensor):
+    """Same step through the public API with host buffers: pinned H2D of the
+    step's inputs, the step, D2H of its result, all inside the events."""
+    W_h = step.wl["W"].pin_memory()
+    X_h = None if step.wl["X"] is None else step.wl["X"].pin_memory()
+    res = step.result()
+    out_h = torch.empty(res.shape, dtype=res.dtype).pin_memory()
+    h2d = W_h.numel() * W_h.element_size() + (0 if X_h is None else X_h.numel() * X_h.element_size())
+    if "W2" in step.wl:
+        W2_h = step.wl["W2"].pin_memory()
+        h2d += W2_h.numel() * W2_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+    s = torch.cuda.current_stream()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        step.W.copy_(W_h, non_blocking=True)
+        if X_h is not None:
+            step.X.copy_(X_h, non_blocking=True)
+        if "W2" in step.wl:
+            step.W2.copy_(W2_h, non_blocking=True)
+        step.run()
+        out_h.copy_(res, non_blocking=True)
+        b.record(s)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return times, h2d, d2h
+
+
+# ----------------------------------------------------------------- CPU oracle (baseline / reference arm)
+def _u16(t):
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def oracle_step(wl, rows: int, threads: int):
+    """The oracle doing the step's work on the first `rows` rows of W.
+    -> (seconds, units) with units in the metric's unit (dense-eq flops or bytes)."""
+    import oracle
+    if wl["X"] is None:           # mask-only workload
+        W = wl["W"][:rows].contiguous().numpy()
+        t0 = time.perf_counter()
+        for N, M in [(1, 4), (2, 4), (4, 8), (2, 8)]:
+            oracle.rows_parallel(0, W, N, M, oracle.F32, threads)
+        return time.perf_counter() - t0, 4.0 * rows * W.shape[1] * 5
+    W = wl["W"][:rows].contiguous()
+    Wb = _u16(W)
+    code = oracle.BF16
+    X = _u16(wl["X"])
+    K, T = wl["K"], wl["T"]
+    t0 = time.perf_counter()
+    mask, _, _ = oracle.rows_parallel(0, Wb, 2, 4, code, threads)          # mask
+    v1, m1 = oracle.compress24(Wb, mask, dtype=code)                        # compress (given mask)
+    _, values, meta = oracle.rows_parallel(1, Wb, 2, 4, code, threads)     # fused mask + compress
+    oracle.meta_sm100(meta, rows, K)                                        # metadata image
+    oracle.decompress24(values, meta, K, dtype=code)                        # decompress
+    oracle.spmm(values, meta, X, code, threads=threads)                     # product
+    if "W2" in wl:
+        # down projection on the same number of rows of W_down, fed by X's first rows
+        W2 = _u16(wl["W2"][:rows].contiguous())
+        _, v2, m2 = oracle.rows_parallel(1, W2, 2, 4, code, threads)
+        H = np.zeros((wl["W2"].shape[1], T), dtype=np.uint16)
+        oracle.spmm(v2, m2, H, code, threads=threads)
+        units = 2.0 * rows * K * T + 2.0 * rows * wl["W2"].shape[1] * T
+    else:
+        units = 2.0 * rows * K * T
+    return time.perf_counter() - t0, units
+
+
+def size_oracle_sample(wl, threads: int, target_s: float):
+    """Rows of W whose oracle step takes about target_s seconds (probe on 8 rows)."""
+    probe = 8
+    t, _ = oracle_step(wl, probe, threads)
+    per_row = max(t / probe, 1e-6)
+    rows = int(max(probe, min(wl["R"], target_s / per_row)))
+    return rows
+
+
+def cpu_baseline(wl, target_s: float = 15.0):
+    threads = os.cpu_count() or 1
+    rows = size_oracle_sample(wl, threads, target_s)
+    secs, units = oracle_step(wl, rows, threads)
+    scale, unit = (1e12, "TFLOP/s") if wl["X"] is not None else (1e9, "GB/s")
+    return {"value": units / secs / scale, "unit": unit, "cores": threads, "kind": "oracle",
+            "sample": "first %d of %d rows of W, whole step (mask, compress, fused mask+compress, image, "
+                      "decompress, fp64 product), %.1f s" % (rows, wl["R"], secs)}
+
+
+def run_reference(args, wl, metric):
+    """The oracle as it stands on the host cores, `steps` bounded samples."""
+    threads = os.cpu_count() or 1
+    per_step_s = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    rows = size_oracle_sample(wl, threads, per_step_s)
+    for _ in range(args.warmup):
+        oracle_step(wl, rows, threads)
+    tot_s, tot_u = 0.0, 0.0
+    for _ in range(args.steps):
+        s, u = oracle_step(wl, rows, threads)
+        tot_s += s
+        tot_u += u
+    scale, unit = (1e12, "TFLOP/s") if wl["X"] is not None else (1e9, "GB/s")
+    value = tot_u / tot_s / scale
+    sample = "first %d of %d rows of W per step, whole step on the CPU oracle" % (rows, wl["R"])
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "desc": wl["desc"], "R": wl["R"], "K": wl["K"], "T": wl["T"]},
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------- main
+METRIC = "nm_spmm dense-equiv TFLOP/s + mask/compress GB/s, % of B200 roofline"
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="nm", choices=["nm", "reference"])
+    ap.add_argument("--workload", default="linear_4096")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, make_workload(args.workload), METRIC)
+        return
+
+    warmup = max(3, args.warmup)
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+        pg = dist
+
+    import structured_sparsity_prune_b200 as nm
+    nm.load()                                    # fails loudly without the CUDA library
+    wl = make_workload(args.workload)
+    step = Step(nm, wl, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    for _ in range(warmup):
+        step.run()
+    torch.cuda.synchronize()
+    if nm.nm_last_device_status() != 0:
+        raise SystemExit("device status reports a timed-out wait")
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    tot, per = timed_steps(step, args.steps, flush)
+    torch.cuda.synchronize()
+    if pg:
+        pg.barrier()
+    clk = clocks.stop()
+
+    total_ms = float(np.sum(tot))
+    e2e_t, h2d, d2h = e2e_steps(step, args.steps, flush)
+    e2e_ms = float(np.sum(e2e_t))
+    if pg:
+        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+    if nm.nm_last_device_status() != 0:
+        raise SystemExit("device status reports a timed-out wait")
+
+    peaks, peak_src = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    sparse_peak = float(peaks["bf16_tflops"]) * SPARSE_RATIO
+    kernels = {}
+    for name in step.names:
+        ms = float(np.mean(per[name]))
+        k = {"us": 1e3 * ms, "GB/s": step.bytes[name] / (ms * 1e-3) / 1e9,
+             "hbm_frac": step.bytes[name] / (ms * 1e-3) / 1e9 / hbm}
+        if hasattr(step, "flop_k") and name in step.flop_k:
+            tf = step.flop_k[name] / (ms * 1e-3) / 1e12
+            k.update({"TFLOP/s": tf, "tensor_frac": tf / sparse_peak})
+        kernels[name] = k
+
+    if step.kind == "ties":
+        units_per_step = sum(step.bytes.values())
+        value = world * units_per_step * args.steps / (total_ms * 1e-3) / 1e9
+        unit = "GB/s"
+        dom = "nm_mask_2:4"
+        roof = {"bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": hbm, "unit": "GB/s",
+                "frac": kernels[dom]["GB/s"] / hbm, "kernel": dom,
+                "algorithmic_bytes_per_launch": step.bytes[dom]}
+        e2e_value = world * units_per_step * args.steps / (e2e_ms * 1e-3) / 1e9
+    else:
+        value = world * step.flops * args.steps / (total_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        dom = max(step.flop_k, key=lambda n: np.mean(per[n]))
+        roof = {"bound": "tensor", "achieved": kernels[dom]["TFLOP/s"], "peak": sparse_peak, "unit": "TFLOP/s",
+                "frac": kernels[dom]["TFLOP/s"] / sparse_peak, "kernel": dom,
+                "algorithmic_flops_per_launch": step.flop_k[dom]}
+        e2e_value = world * step.flops * args.steps / (e2e_ms * 1e-3) / 1e12
+    roof["peak_source"] = "%s: 2 x dense bf16 burst" % peak_src if roof["bound"] == "tensor" else \
+        "%s: HBM copy" % peak_src
+    roof["traffic"] = None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
+                "warmup": warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": str(wl["W"].dtype).replace("torch.", ""),
+                "data": "synthetic",
+                "config": {"workload": args.workload, "desc": wl["desc"], "R": wl["R"], "K": wl["K"], "T": wl["T"],
+                           "sparsity": "2:4 along K" if step.kind != "ties" else "N:M along K",
+                           "l2": "flushed: 256 MiB write between timed steps, outside the events",
+                           "parallelism": "independent replica per GPU" if world > 1 else "single GPU"},
+                "roofline": roof, "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "gpu_launches": step.launches() * args.steps,
+                "clocks": clk, "kernels": kernels}
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

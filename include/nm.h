@@ -159,7 +159,9 @@ NM_API size_t nm_spmm_workspace_bytes(nm_dtype ab_dtype, int64_t R, int64_t K, i
  *              nm_meta_to_sm100), R and K padded to 128
  *   X          K x T, ab_dtype, leading dim ldx >= T
  *   Y          R x T, y_dtype (NM_BF16 or NM_F32), leading dim ldy >= T;
- *              read only when beta != 0
+ *              read only when beta != 0.  Y needs only element alignment;
+ *              16-byte aligned Y and ldy get vector stores
+ *   X, values, meta_sm100: 16-byte aligned; ldx * element size % 16 == 0
  *   ab_dtype   NM_BF16 or NM_F16 (tensor-core path), or NM_F32 (rounded to
  *              binary16 in `workspace`, then the binary16 path)
  *   K % 16 == 0 (the pages' rule for 16-bit sparse operands); R, T >= 1 any

@@ -28,7 +28,9 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <cstdlib>
 #include <mutex>
+#include <string>
 
 #include "nm_internal.cuh"
 
@@ -170,9 +172,77 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// ---- CTA-pair (cluster of 2) helpers for the cta_group::2 kernel
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// shared::cluster address of the same shared-memory object in CTA `rank`
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA tile load into this CTA's shared memory whose completion is counted on
+// an mbarrier of either CTA of the pair (here: the MMA-issuing CTA's).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
+                                                 int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tmem_cp_pair_128x128b(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void mma_sp_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t e_tmem,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// completion of this thread's earlier tcgen05 ops arrives on the mbarrier at
+// the same offset in both CTAs of the pair
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .b16 m;\n\tmov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
 // Instruction descriptor, .kind::f16 with sparsity: D fp32, A/B fp16 or bf16,
 // A K-major, B N-major (X is K x T with T contiguous), M = 128, N = n.
-__host__ __device__ constexpr uint32_t make_idesc(bool bf16, int n) {
+__host__ __device__ constexpr uint32_t make_idesc(bool bf16, int n, int m = kBlockM) {
   return (1u << 2)                    // sparse
          | (1u << 4)                  // D format fp32
          | ((bf16 ? 1u : 0u) << 7)    // A format
@@ -180,7 +250,7 @@ __host__ __device__ constexpr uint32_t make_idesc(bool bf16, int n) {
          | (0u << 15)                 // A K-major
          | (1u << 16)                 // B MN-major
          | (uint32_t(n >> 3) << 17)   // N / 8
-         | (uint32_t(kBlockM >> 4) << 24);  // M / 16
+         | (uint32_t(m >> 4) << 24);  // M / 16
 }
 
 // ----------------------------------------------------------------- kernel
@@ -209,8 +279,72 @@ struct Params {
   int m_tiles, n_tiles, k_blocks;
   int m_inner;  // tile order: 1 -> m fastest
   int y_f32;    // 1: fp32 output, 0: bf16 output
+  int y_vec;    // 1: Y and ldy allow 16-byte vector stores
   float alpha, beta;
 };
+
+// Epilogue of one 32-column chunk of one output row: y = alpha * acc (+ beta * y_old),
+// rounded to the output type; vector stores when Y allows them, scalar at the T edge.
+__device__ __forceinline__ void store_chunk(const Params& p, int r, int col0, const uint32_t (&v)[32]) {
+  if (r < p.R && col0 < p.T) {
+    const bool full_chunk = p.y_vec && col0 + 32 <= p.T;
+    float y[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) y[j] = p.alpha * __uint_as_float(v[j]);
+    if (p.y_f32) {
+      float* yrow = static_cast<float*>(p.Y) + size_t(r) * p.ldy + col0;
+      if (full_chunk) {
+        if (p.beta != 0.0f) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 4) {
+            const float4 o = *reinterpret_cast<const float4*>(yrow + j);
+            y[j] += p.beta * o.x; y[j + 1] += p.beta * o.y; y[j + 2] += p.beta * o.z; y[j + 3] += p.beta * o.w;
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<float4*>(yrow + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+      } else {
+        for (int j = 0; j < 32 && col0 + j < p.T; ++j) {
+          float o = y[j];
+          if (p.beta != 0.0f) o += p.beta * yrow[j];
+          yrow[j] = o;
+        }
+      }
+    } else {
+      __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.Y) + size_t(r) * p.ldy + col0;
+      if (full_chunk) {
+        if (p.beta != 0.0f) {
+#pragma unroll
+          for (int j = 0; j < 32; j += 8) {
+            const uint4 o = *reinterpret_cast<const uint4*>(yrow + j);
+            const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&o);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 f = __bfloat1622float2(h[u]);
+              y[j + 2 * u] += p.beta * f.x;
+              y[j + 2 * u + 1] += p.beta * f.y;
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; j += 8) {
+          uint4 o;
+          __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) h[u] = __floats2bfloat162_rn(y[j + 2 * u], y[j + 2 * u + 1]);
+          *reinterpret_cast<uint4*>(yrow + j) = o;
+        }
+      } else {
+        for (int j = 0; j < 32 && col0 + j < p.T; ++j) {
+          float o = y[j];
+          if (p.beta != 0.0f) o += p.beta * __bfloat162float(yrow[j]);
+          yrow[j] = __float2bfloat16_rn(o);
+        }
+      }
+    }
+  }
+}
 
 template <int N_TILE, int STAGES, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -358,65 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < N_TILE; c += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TILE + c), v);
-        const int col0 = c_base + c;
-        if (r < p.R && col0 < p.T) {
-          const bool full_chunk = col0 + 32 <= p.T;
-          float y[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] = p.alpha * __uint_as_float(v[j]);
-          if (p.y_f32) {
-            float* yrow = static_cast<float*>(p.Y) + size_t(r) * p.ldy + col0;
-            if (full_chunk) {
-              if (p.beta != 0.0f) {
-#pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                  const float4 o = *reinterpret_cast<const float4*>(yrow + j);
-                  y[j] += p.beta * o.x; y[j + 1] += p.beta * o.y; y[j + 2] += p.beta * o.z; y[j + 3] += p.beta * o.w;
-                }
-              }
-#pragma unroll
-              for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(yrow + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
-            } else {
-              for (int j = 0; j < 32 && col0 + j < p.T; ++j) {
-                float o = y[j];
-                if (p.beta != 0.0f) o += p.beta * yrow[j];
-                yrow[j] = o;
-              }
-            }
-          } else {
-            __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.Y) + size_t(r) * p.ldy + col0;
-            if (full_chunk) {
-              if (p.beta != 0.0f) {
-#pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                  const uint4 o = *reinterpret_cast<const uint4*>(yrow + j);
-                  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&o);
-#pragma unroll
-                  for (int u = 0; u < 4; ++u) {
-                    const float2 f = __bfloat1622float2(h[u]);
-                    y[j + 2 * u] += p.beta * f.x;
-                    y[j + 2 * u + 1] += p.beta * f.y;
-                  }
-                }
-              }
-#pragma unroll
-              for (int j = 0; j < 32; j += 8) {
-                uint4 o;
-                __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
-#pragma unroll
-                for (int u = 0; u < 4; ++u) h[u] = __floats2bfloat162_rn(y[j + 2 * u], y[j + 2 * u + 1]);
-                *reinterpret_cast<uint4*>(yrow + j) = o;
-              }
-            } else {
-              for (int j = 0; j < 32 && col0 + j < p.T; ++j) {
-                float o = y[j];
-                if (p.beta != 0.0f) o += p.beta * __bfloat162float(yrow[j]);
-                yrow[j] = __float2bfloat16_rn(o);
-              }
-            }
-          }
-        }
+        store_chunk(p, r, c_base + c, v);
       }
       fence_before_sync();
       __syncwarp();
@@ -430,6 +506,202 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     fence_after_sync();
     tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------- CTA-pair kernel
+// A cluster of two CTAs on two SMs computes a 256-row x N_TOTAL output tile with
+// tcgen05.mma.sp.cta_group::2 (M = 256): each CTA stages its own 128 rows of A,
+// its own metadata block and HALF of the X tile (N_TOTAL / 2 columns); the MMA
+// issued by the even CTA reads both halves, so each SM's shared memory feeds
+// only half of B.  Both CTAs' TMA loads complete on the even CTA's full
+// barrier; the even CTA's commits arrive on both CTAs' barriers.
+template <int N_TOTAL, int STAGES>
+struct PairCfg {
+  static constexpr int kNHalf = N_TOTAL / 2;
+  static constexpr int kABytes = kBlockM * kStageKPhys * 2;   // 16 KB
+  static constexpr int kBBoxes = kNHalf / 64;
+  static constexpr int kBBoxBytes = kStageK * 64 * 2;         // 16 KB
+  static constexpr int kBBytes = kBBoxes * kBBoxBytes;
+  static constexpr int kEBytes = 2048;
+  static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
+  static constexpr int kAccBufs = (2 * N_TOTAL + 4 * STAGES <= 512) ? 2 : 1;
+  static constexpr int kECol0 = kAccBufs * N_TOTAL;
+  static constexpr int kTmemCols = (kECol0 + 4 * STAGES) <= 256 ? 256 : 512;
+  static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 + 256;
+  static_assert(kNHalf % 64 == 0 && N_TOTAL <= 256, "N_TOTAL");
+  static_assert(kECol0 + 4 * STAGES <= 512, "TMEM budget");
+};
+
+template <int N_TOTAL, int STAGES, bool BF16>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    spmm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                     const __grid_constant__ CUtensorMap map_e, Params p) {
+  using C = PairCfg<N_TOTAL, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
+  uint64_t* full = bars;                        // [STAGES], used in the even CTA
+  uint64_t* empty = bars + STAGES;              // [STAGES], both CTAs
+  uint64_t* acc_full = bars + 2 * STAGES;       // [2], both CTAs
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;  // [2], used in the even CTA
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = int(blockIdx.x >> 1), num_pairs = int(gridDim.x >> 1);
+  const int num_tiles = p.m_tiles * p.n_tiles;  // m_tiles counts 256-row tiles here
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);  // 4 epilogue warps in each CTA
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, C::kTmemCols);
+  fence_before_sync();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive / copy
+  fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  auto tile_coords = [&](int t, int& mt, int& nt) {
+    if (p.m_inner) { mt = t % p.m_tiles; nt = t / p.m_tiles; }
+    else { nt = t % p.n_tiles; mt = t / p.n_tiles; }
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      uint32_t it = 0;
+      uint32_t armed_round[STAGES];
+      for (int s = 0; s < STAGES; ++s) armed_round[s] = 0xFFFFFFFFu;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += num_pairs) {
+        int mt, nt;
+        tile_coords(t, mt, nt);
+        const int row_tile = 2 * mt + int(rank);  // this CTA's 128-row tile
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = int(it % STAGES);
+          const uint32_t round = it / STAGES;
+          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* st = smem + s * C::kStageBytes;
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
+          armed_round[s] = round;
+          const uint32_t bar = mapa(smem_u32(&full[s]), 0);
+          tma_load_2d_pair(st, &map_a, bar, kb * kStageKPhys, row_tile * kBlockM);
+#pragma unroll
+          for (int j = 0; j < C::kBBoxes; ++j)
+            tma_load_2d_pair(st + C::kABytes + j * C::kBBoxBytes, &map_b, bar,
+                             nt * N_TOTAL + int(rank) * C::kNHalf + 64 * j, kb * kStageK);
+          tma_load_2d_pair(st + C::kABytes + C::kBBytes, &map_e, bar, 0,
+                           (row_tile * p.k_blocks + kb) * kBlockM);
+        }
+      }
+      if (!ok) {
+        // let copies already issued land before the CTA can leave
+        if (leader) {
+          for (int s = 0; s < STAGES; ++s)
+            if (armed_round[s] != 0xFFFFFFFFu) {
+              const uint64_t t0 = globaltimer();
+              while (!mbar_try_wait(&full[s], armed_round[s] & 1u) && globaltimer() - t0 < 100000000ull) {
+              }
+            }
+        } else {
+          const uint64_t t0 = globaltimer();
+          while (globaltimer() - t0 < 2000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
+      const uint32_t idesc = make_idesc(BF16, N_TOTAL, 2 * kBlockM);
+      uint32_t it = 0, local = 0;
+      bool ok = true;
+      for (int t = pair; t < num_tiles && ok; t += num_pairs, ++local) {
+        const int buf = int(local % C::kAccBufs);
+        const uint32_t use = local / C::kAccBufs;
+        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        fence_after_sync();
+        const uint32_t d_tmem = tmem_base + uint32_t(buf * N_TOTAL);
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = int(it % STAGES);
+          const uint32_t round = it / STAGES;
+          if (!mbar_wait(&full[s], round & 1u, abort_flag)) { ok = false; break; }
+          fence_after_sync();
+          uint8_t* st = smem + s * C::kStageBytes;
+          const uint32_t a_addr = smem_u32(st);
+          const uint32_t b_addr = smem_u32(st + C::kABytes);
+          const uint32_t e_addr = smem_u32(st + C::kABytes + C::kBBytes);
+          const uint32_t e_tmem = tmem_base + uint32_t(C::kECol0 + 4 * s);
+          tmem_cp_pair_128x128b(e_tmem, smem_desc(e_addr, 0, 128, kLayoutNone));
+#pragma unroll
+          for (int k2 = 0; k2 < kStageK / kMmaK; ++k2) {
+            const uint64_t adesc = smem_desc(a_addr + 32u * k2, 16, 1024, kLayoutSW128);
+            const uint64_t bdesc = smem_desc(b_addr + 4096u * k2, C::kBBoxBytes, 1024, kLayoutSW128);
+            mma_sp_pair(d_tmem, adesc, bdesc, e_tmem + uint32_t(k2 & ~1), idesc | uint32_t(k2 & 1),
+                        (kb > 0 || k2 > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(&empty[s]);
+        }
+        if (!ok) break;
+        mma_commit_pair(&acc_full[buf]);
+      }
+      asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                       smem_u32(drain))
+                   : "memory");
+      const uint64_t t0 = globaltimer();
+      while (!mbar_try_wait(drain, 0) && globaltimer() - t0 < kWaitLimitNs) {
+      }
+      (void)ok;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;
+    const int row_in_tile = 32 * q + lane;
+    const uint32_t acc_empty_leader[2] = {mapa(smem_u32(&acc_empty[0]), 0), mapa(smem_u32(&acc_empty[1]), 0)};
+    uint32_t local = 0;
+    for (int t = pair; t < num_tiles; t += num_pairs, ++local) {
+      int mt, nt;
+      tile_coords(t, mt, nt);
+      const int buf = int(local % C::kAccBufs);
+      const uint32_t use = local / C::kAccBufs;
+      const bool ok = mbar_wait(&acc_full[buf], use & 1u, abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      fence_after_sync();
+      const int r = (2 * mt + int(rank)) * kBlockM + row_in_tile;
+      const int c_base = nt * N_TOTAL;
+#pragma unroll 1
+      for (int c = 0; c < N_TOTAL; c += 32) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TOTAL + c), v);
+        store_chunk(p, r, c_base + c, v);
+      }
+      fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc_empty_leader[buf]);
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  fence_before_sync();
+  __syncthreads();
+  cluster_sync();  // the even CTA's MMAs are done and no remote arrive is pending
+  if (warp == 1) {
+    fence_after_sync();
+    tmem_dealloc_pair(tmem_base, C::kTmemCols);
   }
 }
 
@@ -492,6 +764,61 @@ nm_status launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, 
   return launch_status();
 }
 
+// 2D byte map over the metadata image seen as rows of 16 bytes (one row per
+// tensor-memory lane), box = 128 rows = one 2048-byte block.
+bool make_map_image(CUtensorMap* map, const uint8_t* img, int64_t rows16) {
+  EncodeFn enc = get_encode();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {16, cuuint64_t(rows16)};
+  const cuuint64_t strides[1] = {16};
+  const cuuint32_t box[2] = {16, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(img), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int N_TOTAL, int STAGES, bool BF16>
+nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me, const Params& p,
+                      cudaStream_t s) {
+  using C = PairCfg<N_TOTAL, STAGES>;
+  auto kern = spmm_pair_kernel<N_TOTAL, STAGES, BF16>;
+  static bool attr_done = false;  // per instantiation
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
+      return NM_ERR_CUDA;
+    attr_done = true;
+  }
+  const int pairs = p.m_tiles * p.n_tiles;
+  const int max_pairs = sm_count() / 2;
+  const int grid = 2 * (pairs < max_pairs ? pairs : max_pairs);
+  kern<<<grid, kThreads, C::kSmemBytes, s>>>(ma, mb, me, p);
+  return launch_status();
+}
+
+// Kernel choice: the CTA-pair kernel when the row tiles pair up and the
+// output is wide enough to fill 128+ columns; the single-CTA kernel
+// otherwise.  NM_SPMM_KERNEL = pair256 | pair128 | single256 | single128 |
+// single64 overrides the choice (for tuning; an inapplicable override falls
+// back to the default).
+enum class Kern { Pair256, Pair128, Single256, Single128, Single64 };
+
+Kern choose_kernel(int64_t R, int64_t T) {
+  const bool pairable = ((R + kBlockM - 1) / kBlockM) % 2 == 0;
+  Kern k;
+  if (pairable && T > 64) k = T > 128 ? Kern::Pair256 : Kern::Pair128;
+  else k = T > 128 ? Kern::Single256 : (T > 64 ? Kern::Single128 : Kern::Single64);
+  if (const char* env = getenv("NM_SPMM_KERNEL")) {
+    const std::string e(env);
+    if (e == "pair256" && pairable) k = Kern::Pair256;
+    else if (e == "pair128" && pairable) k = Kern::Pair128;
+    else if (e == "single256") k = Kern::Single256;
+    else if (e == "single128") k = Kern::Single128;
+    else if (e == "single64") k = Kern::Single64;
+  }
+  return k;
+}
+
 template <bool BF16>
 nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_t ldx, void* Y, bool y_f32,
               int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta, cudaStream_t s) {
@@ -504,10 +831,15 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
   p.K = int(K);
   p.k_blocks = int((K + kStageK - 1) / kStageK);
   p.y_f32 = y_f32 ? 1 : 0;
+  p.y_vec = (aligned16(Y) && stride_ok(ldy, y_f32 ? 4 : 2)) ? 1 : 0;
   p.alpha = alpha;
   p.beta = beta;
-  p.m_tiles = int((R + kBlockM - 1) / kBlockM);
-  const int n_tile = T > 128 ? 256 : (T > 64 ? 128 : 64);
+  const Kern kern = choose_kernel(R, T);
+  const bool pair = kern == Kern::Pair256 || kern == Kern::Pair128;
+  const int block_m = pair ? 2 * kBlockM : kBlockM;
+  const int n_tile = (kern == Kern::Pair256 || kern == Kern::Single256) ? 256
+                     : (kern == Kern::Pair128 || kern == Kern::Single128) ? 128 : 64;
+  p.m_tiles = int((R + block_m - 1) / block_m);
   p.n_tiles = int((T + n_tile - 1) / n_tile);
   // stream the larger operand once: W bigger than X -> n fastest
   const double a_bytes = double(R) * double(K);          // compressed values, 2 B x K/2
@@ -517,9 +849,16 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
   CUtensorMap ma, mb;
   if (!make_map(&ma, values, BF16, R, K / 2, K / 2, kStageKPhys, kBlockM)) return NM_ERR_CUDA;
   if (!make_map(&mb, X, BF16, K, T, ldx, 64, kStageK)) return NM_ERR_CUDA;
-  switch (n_tile) {
-    case 256: return launch<256, 2, BF16>(ma, mb, p, s);
-    case 128: return launch<128, 4, BF16>(ma, mb, p, s);
+  if (pair) {
+    CUtensorMap me;
+    const int64_t rows16 = ((R + 127) / 128) * int64_t(p.k_blocks) * 128;
+    if (!make_map_image(&me, meta_img, rows16)) return NM_ERR_CUDA;
+    if (kern == Kern::Pair256) return launch_pair<256, 4, BF16>(ma, mb, me, p, s);
+    return launch_pair<128, 6, BF16>(ma, mb, me, p, s);
+  }
+  switch (kern) {
+    case Kern::Single256: return launch<256, 2, BF16>(ma, mb, p, s);
+    case Kern::Single128: return launch<128, 4, BF16>(ma, mb, p, s);
     default: return launch<64, 6, BF16>(ma, mb, p, s);
   }
 }
@@ -546,8 +885,8 @@ extern "C" nm_status nm_spmm(const void* values, const uint8_t* meta_sm100, nm_d
   if (R == 0 || T == 0) return NM_OK;
   if (values == nullptr || meta_sm100 == nullptr || X == nullptr || Y == nullptr) return NM_ERR_NULL;
   const int ab_es = esize_of(ab_dtype), y_es = esize_of(y_dtype);
-  if (!aligned16(values) || !aligned16(meta_sm100) || !aligned16(X) || !aligned16(Y) || !stride_ok(ldx, ab_es) ||
-      !stride_ok(ldy, y_es))
+  if (!aligned16(values) || !aligned16(meta_sm100) || !aligned16(X) || !stride_ok(ldx, ab_es) ||
+      (reinterpret_cast<uintptr_t>(Y) % uintptr_t(y_es)) != 0)
     return NM_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool y_f32 = y_dtype == NM_F32;

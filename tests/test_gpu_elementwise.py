@@ -69,7 +69,7 @@ def test_mask_strided_and_unaligned_c(N, M):
     R, C = 33, 24 if M == 4 else 40
     full = _rand((R, C + 8), torch.bfloat16, 3, "ties")
     W = full.cuda()[:, :C]
-    mask = torch.full((R, C + 16), 7, dtype=torch.uint8, device="cuda")
+    mask = torch.full((R, 64), 7, dtype=torch.uint8, device="cuda")
     nm.nm_mask(W, N, M, mask=mask[:, :C])
     ref = oracle.mask_rank(_bits(full[:, :C]), N, M, dtype=oracle.BF16)
     assert np.array_equal(mask[:, :C].cpu().numpy(), ref)
@@ -128,7 +128,9 @@ def test_compress_with_given_mask(R, C, dtype):
     mask.scatter_(2, choice, 1)
     mask = mask.reshape(R, C)
     ctr = torch.zeros((1,), dtype=torch.int32, device="cuda")
-    values, meta, img = nm.nm_compress(W.cuda(), mask.cuda(), invalid_groups=ctr)
+    mbuf = torch.zeros((R, (C + 15) // 16 * 16), dtype=torch.uint8, device="cuda")   # 16-byte rows
+    mbuf[:, :C] = mask.cuda()
+    values, meta, img = nm.nm_compress(W.cuda(), mbuf[:, :C], invalid_groups=ctr)
     v_ref, m_ref = oracle.compress24(_bits(W), mask.numpy(), dtype=CODE[dtype])
     assert np.array_equal(_bits(values), np.ascontiguousarray(v_ref).view(_bits(values).dtype))
     assert np.array_equal(meta.cpu().numpy(), m_ref)

@@ -33,6 +33,14 @@ def _nerr(Y, ref):
     return np.linalg.norm(Yf - ref) / (den if den > 0 else 1.0)
 
 
+def _dev(X):
+    """Device copy of X in a buffer whose rows are 16-byte aligned (ldx % 8 == 0)."""
+    K, T = X.shape
+    buf = torch.zeros((K, (T + 7) // 8 * 8), dtype=X.dtype, device="cuda")
+    buf[:, :T] = X.cuda()
+    return buf[:, :T]
+
+
 def _ok_status():
     assert nm.nm_last_device_status() == 0
 
@@ -50,7 +58,7 @@ def _run(W, X, y_dtype=torch.bfloat16, alpha=1.0, beta=0.0, Y0=None, rows=None):
     ab = W.dtype
     values, meta, img = nm.nm_mask_compress(W.cuda())
     Y = None if Y0 is None else Y0.clone().cuda()
-    Y = nm.nm_spmm(values, img, X.cuda(), Y=Y, y_dtype=y_dtype, alpha=alpha, beta=beta)
+    Y = nm.nm_spmm(values, img, _dev(X), Y=Y, y_dtype=y_dtype, alpha=alpha, beta=beta)
     torch.cuda.synchronize()
     _ok_status()
     Wb = _bits(W)
