@@ -76,7 +76,7 @@ def make_workload(name: str):
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled during the timed region."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -95,6 +95,9 @@ class ClockSampler:
             self.proc = None
         self.t0 = time.time()
 
+    def mark(self, what: str):
+        setattr(self, what, time.time())
+
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
@@ -104,22 +107,33 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
+        import datetime
         sm, smax, reasons, n = [], None, set(), 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        t_lo = getattr(self, "t_begin", 0.0) - 0.05
+        t_hi = getattr(self, "t_end", 1e30) + 0.05
+        samples = []
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) < 9:
                     continue
                 try:
-                    sm.append(float(parts[1]))
-                    smax = float(parts[2])
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    samples.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
                 except ValueError:
                     continue
-                n += 1
-                for name, v in zip(names, parts[5:9]):
-                    if v.lower().startswith("active"):
-                        reasons.add(name)
+        inside = [x for x in samples if t_lo <= x[0] <= t_hi]
+        if not inside and samples:   # region shorter than the sampling period: nearest sample
+            mid = 0.5 * (t_lo + t_hi)
+            inside = [min(samples, key=lambda x: abs(x[0] - mid))]
+        for ts, mhz, mx, flags in inside:
+            sm.append(mhz)
+            smax = mx
+            n += 1
+            for name, v in zip(names, flags):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
         os.unlink(self.path)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
                 "reasons": sorted(reasons), "samples": n}
@@ -354,7 +368,7 @@ METRIC = "nm_spmm dense-equiv TFLOP/s + mask/compress GB/s, % of B200 roofline"
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nm", choices=["nm", "reference"])
     ap.add_argument("--workload", default="linear_4096")
@@ -394,11 +408,14 @@ def main():
 
     clocks = ClockSampler(local_rank)
     clocks.start()
+    time.sleep(0.5)                              # let the sampler start emitting
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
+    clocks.mark("t_begin")
     tot, per = timed_steps(step, args.steps, flush)
     torch.cuda.synchronize()
+    clocks.mark("t_end")
     if pg:
         pg.barrier()
     clk = clocks.stop()

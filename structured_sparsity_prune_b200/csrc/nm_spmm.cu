@@ -45,7 +45,8 @@ constexpr int kBlockM = 128;     // rows of W per tile = TMEM lanes
 constexpr int kStageK = 128;     // logical K per pipeline stage
 constexpr int kStageKPhys = 64;  // compressed values per row per stage (128 B)
 constexpr int kMmaK = 32;        // logical K per sparse MMA instruction
-constexpr int kThreads = 192;    // 6 warps
+constexpr int kThreads = 192;    // 6 warps (single-CTA kernel)
+constexpr int kPairThreads = 320;  // 10 warps: producer, MMA, 8 epilogue warps (CTA-pair kernel)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 
 // ----------------------------------------------------------------- PTX helpers
@@ -238,6 +239,23 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], m;\n\t}" ::"r"(
           smem_u32(bar))
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld_32x32b_x32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 // Instruction descriptor, .kind::f16 with sparsity: D fp32, A/B fp16 or bf16,
@@ -534,7 +552,7 @@ struct PairCfg {
 };
 
 template <int N_TOTAL, int STAGES, bool BF16>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     spmm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                      const __grid_constant__ CUtensorMap map_e, Params p) {
   using C = PairCfg<N_TOTAL, STAGES>;
@@ -562,7 +580,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 8);  // 4 epilogue warps in each CTA
+      mbar_init(&acc_empty[b], 16);  // 8 epilogue warps in each CTA
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -669,9 +687,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    // Warps 2..9: warp w reads TMEM lanes 32*(w%4).. (its rows) and columns
+    // [half * N/2, (half+1) * N/2) with half = (w-2)/4.  For bf16 output with
+    // beta == 0 a thread converts its whole row segment into registers first
+    // and releases the accumulator before storing, so the next tile's MMAs
+    // overlap the global stores.
+    constexpr int kCols = N_TOTAL / 2;
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row_in_tile = 32 * q + lane;
     const uint32_t acc_empty_leader[2] = {mapa(smem_u32(&acc_empty[0]), 0), mapa(smem_u32(&acc_empty[1]), 0)};
+    const bool early = !p.y_f32 && p.beta == 0.0f && p.y_vec;
     uint32_t local = 0;
     for (int t = pair; t < num_tiles; t += num_pairs, ++local) {
       int mt, nt;
@@ -682,16 +708,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       fence_after_sync();
       const int r = (2 * mt + int(rank)) * kBlockM + row_in_tile;
-      const int c_base = nt * N_TOTAL;
+      const int c_base = nt * N_TOTAL + half * kCols;
+      const uint32_t taddr = tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TOTAL + half * kCols);
+      if (early) {
+        uint32_t packed[kCols / 2];
+#pragma unroll
+        for (int c = 0; c < kCols; c += 64) {
+          uint32_t v0[32], v1[32];
+          tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c), v0);
+          tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c + 32), v1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            packed[c / 2 + j] = pack_bf16x2(p.alpha * __uint_as_float(v0[2 * j]), p.alpha * __uint_as_float(v0[2 * j + 1]));
+            packed[c / 2 + 16 + j] =
+                pack_bf16x2(p.alpha * __uint_as_float(v1[2 * j]), p.alpha * __uint_as_float(v1[2 * j + 1]));
+          }
+        }
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader[buf]);
+        if (r < p.R) {
+          __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.Y) + size_t(r) * p.ldy;
+#pragma unroll
+          for (int c = 0; c < kCols; c += 8) {
+            const int col = c_base + c;
+            if (col + 8 <= p.T) {
+              *reinterpret_cast<uint4*>(yrow + col) =
+                  make_uint4(packed[c / 2], packed[c / 2 + 1], packed[c / 2 + 2], packed[c / 2 + 3]);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                if (col + j < p.T) {
+                  const uint32_t w = packed[c / 2 + j / 2];
+                  const uint16_t h = uint16_t((j & 1) ? (w >> 16) : (w & 0xFFFFu));
+                  reinterpret_cast<uint16_t*>(yrow)[col + j] = h;
+                }
+              }
+            }
+          }
+        }
+      } else {
 #pragma unroll 1
-      for (int c = 0; c < N_TOTAL; c += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TOTAL + c), v);
-        store_chunk(p, r, c_base + c, v);
+        for (int c = 0; c < kCols; c += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + uint32_t(c), v);
+          store_chunk(p, r, c_base + c, v);
+        }
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader[buf]);
       }
-      fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(acc_empty_leader[buf]);
     }
   }
 
@@ -792,7 +859,7 @@ nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   const int pairs = p.m_tiles * p.n_tiles;
   const int max_pairs = sm_count() / 2;
   const int grid = 2 * (pairs < max_pairs ? pairs : max_pairs);
-  kern<<<grid, kThreads, C::kSmemBytes, s>>>(ma, mb, me, p);
+  kern<<<grid, kPairThreads, C::kSmemBytes, s>>>(ma, mb, me, p);
   return launch_status();
 }
 
