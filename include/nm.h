@@ -175,6 +175,31 @@ NM_API nm_status nm_spmm(const void *values, const uint8_t *meta_sm100, nm_dtype
                   void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * nm_spmm_noalloc -- nm_spmm that allocates nothing and takes no workspace.
+ * (No counterpart on the pages: this is an interface for callers.)  For
+ * callers that are not allowed to allocate device memory: code running inside
+ * a host framework that owns every device allocation (a serving engine or a
+ * plugin host with a pre-reserved memory budget), or a latency-critical path
+ * that cannot afford cudaMalloc's implicit device-wide synchronisation.
+ *   Arguments as nm_spmm, without workspace / workspace_bytes.
+ *   For NM_F32 inputs the binary16 staging buffers live in a fixed 16 MiB
+ *   device array inside the library (held by every GPU that loads it, until
+ *   exit); problems needing more (nm_spmm_workspace_bytes(...) > 16 MiB)
+ *   return NM_ERR_WORKSPACE.  NM_BF16 / NM_F16 inputs need no scratch.
+ *   The first NM_F32 call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   All calls on a device share its one array, and it keeps the previous
+ *   call's contents (every call overwrites what it reads, so nothing needs
+ *   clearing).  Calls that may overlap on the same GPU -- issued to
+ *   different streams, or from concurrent host threads -- race on it and
+ *   must be serialised by the caller.
+ */
+NM_API nm_status nm_spmm_noalloc(const void *values, const uint8_t *meta_sm100, nm_dtype ab_dtype,
+                                 const void *X, int64_t ldx, void *Y, nm_dtype y_dtype, int64_t ldy,
+                                 int64_t R, int64_t K, int64_t T, float alpha, float beta, void *stream);
+
+/*
  * nm_last_device_status -- synchronises `stream`, then returns and clears the
  * device status word written by kernels whose bounded waits gave up
  * (NM_OK if none did).  NM_ERR_CUDA if the synchronisation itself failed.

@@ -53,6 +53,7 @@ def _lib():
         "nm_meta_to_sm100": ([vp, i64, i64, vp, vp], i32),
         "nm_spmm_workspace_bytes": ([i32, i64, i64, i64], sz),
         "nm_spmm": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp, sz, vp], i32),
+        "nm_spmm_noalloc": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp], i32),
         "nm_last_device_status": ([vp], i32),
     }
     for name, (args, res) in sig.items():

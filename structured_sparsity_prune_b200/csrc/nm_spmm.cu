@@ -986,3 +986,51 @@ extern "C" nm_status nm_last_device_status(void* stream) {
   }
   return static_cast<nm_status>(v);
 }
+
+// ---------------------------------------------------------------------------
+// nm_spmm_noalloc: nm_spmm for callers that cannot allocate device memory.
+// The fp32 path of nm_spmm needs scratch (inputs rounded to binary16).  This
+// variant takes it from a fixed, file-scope device array instead of a
+// caller-supplied workspace, so the call itself never allocates.  The array
+// is part of the module: every GPU that loads the library holds it until the
+// process exits.
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  Looked up once
+// per device, on the first call made with that device current.  In host code
+// the array's name is only a host-side stand-in, never a device address.
+nm_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return NM_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return NM_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return NM_OK;
+}
+}  // namespace
+
+extern "C" nm_status nm_spmm_noalloc(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype,
+                                     const void* X, int64_t ldx, void* Y, nm_dtype y_dtype, int64_t ldy,
+                                     int64_t R, int64_t K, int64_t T, float alpha, float beta, void* stream) {
+  if (ab_dtype != NM_F32)  // the 16-bit paths use no scratch at all
+    return nm_spmm(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, nullptr, 0, stream);
+  const size_t need = nm_spmm_workspace_bytes(ab_dtype, R, K, T);
+  if (need > kNoAllocScratchBytes) return NM_ERR_WORKSPACE;  // problem larger than the fixed scratch
+  void* scratch = nullptr;
+  if (need > 0) {
+    const nm_status st = noalloc_scratch(&scratch);
+    if (st != NM_OK) return st;
+  }
+  return nm_spmm(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, scratch,
+                 need > 0 ? kNoAllocScratchBytes : 0, stream);
+}
