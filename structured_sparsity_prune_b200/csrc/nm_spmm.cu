@@ -295,11 +295,34 @@ struct Params {
   int64_t ldy;
   int R, T, K;
   int m_tiles, n_tiles, k_blocks;
-  int m_inner;  // tile order: 1 -> m fastest
+  int m_inner;  // tile order: 1 -> m fastest inside a group of `group` m-tiles, 0 -> n fastest
+  int group;    // tiles of the slow operand kept together (sized so the group stays in L2)
   int y_f32;    // 1: fp32 output, 0: bf16 output
   int y_vec;    // 1: Y and ldy allow 16-byte vector stores
   float alpha, beta;
 };
+
+// Tile order.  Tiles run in groups: with m_inner, `group` consecutive m-tiles
+// (rows of W) are swept across every n-tile with m fastest, so the group's
+// slices of W stay in L2 while X streams through once per group; without
+// m_inner the roles of W and X swap.
+__device__ __forceinline__ void grouped_tile(const Params& p, int t, int& mt, int& nt) {
+  if (p.m_inner) {
+    const int span = p.group * p.n_tiles;
+    const int g = t / span, first = g * p.group;
+    const int gm = min(p.group, p.m_tiles - first);
+    const int local = t - g * span;
+    mt = first + local % gm;
+    nt = local / gm;
+  } else {
+    const int span = p.group * p.m_tiles;
+    const int g = t / span, first = g * p.group;
+    const int gn = min(p.group, p.n_tiles - first);
+    const int local = t - g * span;
+    nt = first + local % gn;
+    mt = local / gn;
+  }
+}
 
 // Epilogue of one 32-column chunk of one output row: y = alpha * acc (+ beta * y_old),
 // rounded to the output type; vector stores when Y allows them, scalar at the T edge.
@@ -402,10 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
-  auto tile_coords = [&](int t, int& mt, int& nt) {
-    if (p.m_inner) { mt = t % p.m_tiles; nt = t / p.m_tiles; }
-    else { nt = t % p.n_tiles; mt = t / p.n_tiles; }
-  };
+  auto tile_coords = [&](int t, int& mt, int& nt) { grouped_tile(p, t, mt, nt); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -538,7 +558,7 @@ template <int N_TOTAL, int STAGES>
 struct PairCfg {
   static constexpr int kNHalf = N_TOTAL / 2;
   static constexpr int kABytes = kBlockM * kStageKPhys * 2;   // 16 KB
-  static constexpr int kBBoxes = kNHalf / 64;
+  static constexpr int kBBoxes = (kNHalf + 63) / 64;           // the last box may be partly unused
   static constexpr int kBBoxBytes = kStageK * 64 * 2;         // 16 KB
   static constexpr int kBBytes = kBBoxes * kBBoxBytes;
   static constexpr int kEBytes = 2048;
@@ -547,7 +567,7 @@ struct PairCfg {
   static constexpr int kECol0 = kAccBufs * N_TOTAL;
   static constexpr int kTmemCols = (kECol0 + 4 * STAGES) <= 256 ? 256 : 512;
   static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 + 256;
-  static_assert(kNHalf % 64 == 0 && N_TOTAL <= 256, "N_TOTAL");
+  static_assert(kNHalf % 32 == 0 && N_TOTAL <= 256, "N_TOTAL");
   static_assert(kECol0 + 4 * STAGES <= 512, "TMEM budget");
 };
 
@@ -593,10 +613,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
-  auto tile_coords = [&](int t, int& mt, int& nt) {
-    if (p.m_inner) { mt = t % p.m_tiles; nt = t / p.m_tiles; }
-    else { nt = t % p.n_tiles; mt = t / p.n_tiles; }
-  };
+  auto tile_coords = [&](int t, int& mt, int& nt) { grouped_tile(p, t, mt, nt); };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -716,13 +733,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         for (int c = 0; c < kCols; c += 64) {
           uint32_t v0[32], v1[32];
           tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c), v0);
-          tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c + 32), v1);
+          if (c + 64 <= kCols) tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c + 32), v1);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 16; ++j)
             packed[c / 2 + j] = pack_bf16x2(p.alpha * __uint_as_float(v0[2 * j]), p.alpha * __uint_as_float(v0[2 * j + 1]));
-            packed[c / 2 + 16 + j] =
-                pack_bf16x2(p.alpha * __uint_as_float(v1[2 * j]), p.alpha * __uint_as_float(v1[2 * j + 1]));
+          if (c + 64 <= kCols) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              packed[c / 2 + 16 + j] =
+                  pack_bf16x2(p.alpha * __uint_as_float(v1[2 * j]), p.alpha * __uint_as_float(v1[2 * j + 1]));
           }
         }
         fence_before_sync();
@@ -868,7 +888,7 @@ nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
 // otherwise.  NM_SPMM_KERNEL = pair256 | pair128 | single256 | single128 |
 // single64 overrides the choice (for tuning; an inapplicable override falls
 // back to the default).
-enum class Kern { Pair256, Pair128, Single256, Single128, Single64 };
+enum class Kern { Pair256, Pair192, Pair128, Single256, Single128, Single64 };
 
 Kern choose_kernel(int64_t R, int64_t T) {
   const bool pairable = ((R + kBlockM - 1) / kBlockM) % 2 == 0;
@@ -878,6 +898,7 @@ Kern choose_kernel(int64_t R, int64_t T) {
   if (const char* env = getenv("NM_SPMM_KERNEL")) {
     const std::string e(env);
     if (e == "pair256" && pairable) k = Kern::Pair256;
+    else if (e == "pair192" && pairable) k = Kern::Pair192;
     else if (e == "pair128" && pairable) k = Kern::Pair128;
     else if (e == "single256") k = Kern::Single256;
     else if (e == "single128") k = Kern::Single128;
@@ -902,16 +923,21 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
   p.alpha = alpha;
   p.beta = beta;
   const Kern kern = choose_kernel(R, T);
-  const bool pair = kern == Kern::Pair256 || kern == Kern::Pair128;
+  const bool pair = kern == Kern::Pair256 || kern == Kern::Pair192 || kern == Kern::Pair128;
   const int block_m = pair ? 2 * kBlockM : kBlockM;
   const int n_tile = (kern == Kern::Pair256 || kern == Kern::Single256) ? 256
+                     : kern == Kern::Pair192                                 ? 192
                      : (kern == Kern::Pair128 || kern == Kern::Single128) ? 128 : 64;
   p.m_tiles = int((R + block_m - 1) / block_m);
   p.n_tiles = int((T + n_tile - 1) / n_tile);
-  // stream the larger operand once: W bigger than X -> n fastest
-  const double a_bytes = double(R) * double(K);          // compressed values, 2 B x K/2
-  const double b_bytes = double(K) * double(T) * 2.0;
-  p.m_inner = a_bytes < b_bytes ? 1 : 0;
+  // Tile order: the operand with fewer bytes is swept fastest, so consecutive
+  // tiles (running at the same time) share a slice of the larger one.
+  {
+    const double a_bytes = double(R) * double(K);          // compressed values, 2 B x K/2
+    const double b_bytes = double(K) * double(T) * 2.0;
+    p.m_inner = a_bytes < b_bytes ? 1 : 0;
+    p.group = p.m_inner ? p.m_tiles : p.n_tiles;
+  }
 
   CUtensorMap ma, mb;
   if (!make_map(&ma, values, BF16, R, K / 2, K / 2, kStageKPhys, kBlockM)) return NM_ERR_CUDA;
@@ -921,6 +947,7 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
     const int64_t rows16 = ((R + 127) / 128) * int64_t(p.k_blocks) * 128;
     if (!make_map_image(&me, meta_img, rows16)) return NM_ERR_CUDA;
     if (kern == Kern::Pair256) return launch_pair<256, 4, BF16>(ma, mb, me, p, s);
+    if (kern == Kern::Pair192) return launch_pair<192, 4, BF16>(ma, mb, me, p, s);
     return launch_pair<128, 6, BF16>(ma, mb, me, p, s);
   }
   switch (kern) {
