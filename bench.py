@@ -172,6 +172,9 @@ class Step:
             self.v2, self.m2, self.img2 = nm.alloc_compressed(R2, K2, self.W2.dtype, dev)
             self.H = torch.empty((R, (T + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)[:, :T]
             self.Y = torch.empty((R2, T), dtype=torch.bfloat16, device=dev)
+            ws = max(nm.nm_spmm_workspace_bytes(torch.bfloat16, R, K, T),
+                     nm.nm_spmm_workspace_bytes(torch.bfloat16, R2, K2, T))
+            self.ws = torch.empty((ws,), dtype=torch.uint8, device=dev) if ws else None
             self.names = ["nm_mask_compress_up", "nm_mask_compress_down", "nm_spmm_up", "nm_spmm_down"]
             G1, G2 = R * K, R2 * K2
             self.bytes = {"nm_mask_compress_up": G1 * 3.25, "nm_mask_compress_down": G2 * 3.25,
@@ -185,6 +188,8 @@ class Step:
         self.img_r = torch.empty_like(self.img)
         self.Wd = torch.empty_like(self.W)
         self.Y = torch.empty((R, T), dtype=torch.bfloat16, device=dev)
+        ws = nm.nm_spmm_workspace_bytes(self.W.dtype, R, K, T)
+        self.ws = torch.empty((max(ws, 1),), dtype=torch.uint8, device=dev) if ws else None
         self.names = ["nm_mask", "nm_compress", "nm_mask_compress", "nm_meta_to_sm100", "nm_decompress", "nm_spmm"]
         G = R * K
         es = self.W.element_size()
@@ -211,9 +216,9 @@ class Step:
             rec(1)
             nm.nm_mask_compress(self.W2, self.v2, self.m2, self.img2)
             rec(2)
-            nm.nm_spmm(self.values, self.img, self.X, Y=self.H)
+            nm.nm_spmm(self.values, self.img, self.X, Y=self.H, workspace=self.ws)
             rec(3)
-            nm.nm_spmm(self.v2, self.img2, self.H, Y=self.Y)
+            nm.nm_spmm(self.v2, self.img2, self.H, Y=self.Y, workspace=self.ws)
             rec(4)
         else:
             K = self.wl["K"]
@@ -227,7 +232,7 @@ class Step:
             rec(4)
             nm.nm_decompress(self.values, self.meta, K, out=self.Wd)
             rec(5)
-            nm.nm_spmm(self.values, self.img, self.X, Y=self.Y)
+            nm.nm_spmm(self.values, self.img, self.X, Y=self.Y, workspace=self.ws)
             rec(6)
 
     def result(self):

@@ -66,10 +66,18 @@ __device__ __forceinline__ uint32_t compress_octet(const Oct<Bits>& e, uint2 m, 
   for (int g = 0; g < 2; ++g) {
     uint32_t i0, i1;
     if constexpr (MODE == 0) {
-      const Pick24 p = pick24(mag_key<Bits>(e[4 * g]), mag_key<Bits>(e[4 * g + 1]),
-                              mag_key<Bits>(e[4 * g + 2]), mag_key<Bits>(e[4 * g + 3]));
-      i0 = p.i0;
-      i1 = p.i1;
+      // branch-free 2:4 selection; exactly two of the four are kept, so the
+      // first kept index is 0, 1 or 2 and the second 1, 2 or 3
+      uint32_t x0, x1, x2, x3;
+      drop4<2>(mag_key<Bits>(e[4 * g]), mag_key<Bits>(e[4 * g + 1]), mag_key<Bits>(e[4 * g + 2]),
+               mag_key<Bits>(e[4 * g + 3]), x0, x1, x2, x3);
+      const bool k0 = int32_t(x0) >= 0, k1 = int32_t(x1) >= 0, k2 = int32_t(x2) >= 0, k3 = int32_t(x3) >= 0;
+      i0 = k0 ? 0u : (k1 ? 1u : 2u);
+      i1 = k3 ? 3u : (k2 ? 2u : 1u);
+      q.set(2 * g, k0 ? e[4 * g] : (k1 ? e[4 * g + 1] : e[4 * g + 2]));
+      q.set(2 * g + 1, k3 ? e[4 * g + 3] : (k2 ? e[4 * g + 2] : e[4 * g + 1]));
+      byte |= (i0 | (i1 << 2)) << (4 * g);
+      continue;
     } else {
       const uint32_t w = g ? m.y : m.x;  // 4 mask bytes of this group
       uint32_t bits = 0;
@@ -174,39 +182,48 @@ __global__ void __launch_bounds__(kThreads) compress_tiles_kernel(
   }
 }
 
-// canonical metadata -> image, same tiling, no weights involved
+// canonical metadata -> image, same tiling, no weights involved.  Each thread
+// takes one row of the tile (16 canonical bytes, one 16-byte load when the row
+// is whole) and drops its eight 16-bit pieces into the shared image block.
 __global__ void __launch_bounds__(kThreads) meta_image_kernel(const uint8_t* __restrict__ meta, int64_t R,
                                                               int64_t C, uint8_t* __restrict__ img) {
-  __shared__ __align__(16) uint16_t s_img[1024];
+  __shared__ __align__(16) uint16_t s_img[2][1024];
   const int64_t kt_count = (C + 127) / 128;
   const int64_t tiles = ((R + 127) / 128) * kt_count;
-  const bool full_rows = (C % 32) == 0;
-  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-    const int64_t rt = tile / kt_count, kt = tile - rt * kt_count;
-#pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-      const int u = threadIdx.x + pass * kThreads;
-      const int64_t r = rt * 128 + (u >> 2);
-      const int64_t c0 = kt * 128 + (u & 3) * 32;
-      uint32_t word = 0x44444444u;
-      if (r < R && c0 < C) {
-        const uint8_t* mrow = meta + r * (C / 8) + c0 / 8;
-        if (full_rows) {
-          word = __ldcs(reinterpret_cast<const uint32_t*>(mrow));
+  const bool vec = (C % 128) == 0;  // whole 16-byte row pieces, 16-byte aligned
+  const int half = threadIdx.x >> 7;  // two tiles per block iteration
+  const int rl = threadIdx.x & 127;
+  for (int64_t base = int64_t(blockIdx.x) * 2; base < tiles; base += int64_t(gridDim.x) * 2) {
+    const int64_t tile = base + half;
+    if (tile < tiles) {
+      const int64_t rt = tile / kt_count, kt = tile - rt * kt_count;
+      const int64_t r = rt * 128 + rl;
+      uint32_t w[4] = {0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u};
+      if (r < R) {
+        const uint8_t* mrow = meta + r * (C / 8) + kt * 16;
+        if (vec) {
+          const uint4 v = __ldcs(reinterpret_cast<const uint4*>(mrow));
+          w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
         } else {
 #pragma unroll
-          for (int o = 0; o < 4; ++o)
-            if (c0 + 8 * o < C) word = (word & ~(0xFFu << (8 * o))) | (uint32_t(mrow[o]) << (8 * o));
+          for (int b = 0; b < 16; ++b) {
+            if (kt * 128 + 8 * b < C) {
+              const int wi = b >> 2, sh = 8 * (b & 3);
+              w[wi] = (w[wi] & ~(0xFFu << sh)) | (uint32_t(mrow[b]) << sh);
+            }
+          }
         }
       }
-      const uint32_t rl = uint32_t(u >> 2), cl = uint32_t(u & 3) * 32u;
-      s_img[sm100_piece_offset(rl, cl) >> 1] = uint16_t(word & 0xFFFFu);
-      s_img[sm100_piece_offset(rl, cl + 16) >> 1] = uint16_t(word >> 16);
+#pragma unroll
+      for (int sl = 0; sl < 4; ++sl) {
+        s_img[half][sm100_piece_offset(uint32_t(rl), uint32_t(32 * sl)) >> 1] = uint16_t(w[sl] & 0xFFFFu);
+        s_img[half][sm100_piece_offset(uint32_t(rl), uint32_t(32 * sl + 16)) >> 1] = uint16_t(w[sl] >> 16);
+      }
     }
     __syncthreads();
-    if (threadIdx.x < 128) {
-      const uint4 v = reinterpret_cast<const uint4*>(s_img)[threadIdx.x];
-      __stcs(reinterpret_cast<uint4*>(img + tile * 2048) + threadIdx.x, v);
+    if (tile < tiles) {
+      const uint4 v = reinterpret_cast<const uint4*>(s_img[half])[rl];
+      __stcs(reinterpret_cast<uint4*>(img + tile * 2048) + rl, v);
     }
     __syncthreads();
   }
@@ -232,23 +249,31 @@ __global__ void __launch_bounds__(256) decompress_kernel(const Bits* __restrict_
         const uint4 x = __ldcs(reinterpret_cast<const uint4*>(values + r * (C / 2) + 4 * o));
         v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
       }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) d[i] = Bits(0);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t idx = (mb >> (2 * k)) & 3u;
-        const int g = k >> 1;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-          if (idx == uint32_t(i)) d[4 * g + i] = v[k];
-      }
       Bits* dst = out + r * ldo + 8 * o;
       if constexpr (sizeof(Bits) == 2) {
+        // each group's four outputs form one 64-bit word: the two kept values
+        // shifted to 16 * idx, zeros elsewhere
+        uint64_t g01[2];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const uint32_t i0 = (mb >> (4 * g)) & 3u, i1 = (mb >> (4 * g + 2)) & 3u;
+          g01[g] = (uint64_t(v[2 * g]) << (16 * i0)) | (uint64_t(v[2 * g + 1]) << (16 * i1));
+        }
         uint4 y;
-        y.x = d[0] | (uint32_t(d[1]) << 16); y.y = d[2] | (uint32_t(d[3]) << 16);
-        y.z = d[4] | (uint32_t(d[5]) << 16); y.w = d[6] | (uint32_t(d[7]) << 16);
+        y.x = uint32_t(g01[0]); y.y = uint32_t(g01[0] >> 32);
+        y.z = uint32_t(g01[1]); y.w = uint32_t(g01[1] >> 32);
         __stcs(reinterpret_cast<uint4*>(dst), y);
       } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) d[i] = Bits(0);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t idx = (mb >> (2 * k)) & 3u;
+          const int g = k >> 1;
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (idx == uint32_t(i)) d[4 * g + i] = v[k];
+        }
         __stcs(reinterpret_cast<uint4*>(dst), make_uint4(d[0], d[1], d[2], d[3]));
         __stcs(reinterpret_cast<uint4*>(dst) + 1, make_uint4(d[4], d[5], d[6], d[7]));
       }

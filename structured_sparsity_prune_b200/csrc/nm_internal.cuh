@@ -60,6 +60,43 @@ __device__ __forceinline__ uint32_t keep_bits(const uint32_t (&key)[M], int N) {
   return bits;
 }
 
+// Groups of four, any N (1..3), branch-free.  For i < j let d_ij = k_i - k_j
+// (keys are below 2^31, so the difference is an exact int32): its sign bit is
+// set iff k_j > k_i, i.e. iff j beats i; its complement says i beats j (ties go
+// to the lower index).  Entry i is beaten by 0..3 others; it is dropped when
+// beaten by at least N of them, which over three 0/1 terms is an OR (N = 1), a
+// majority (N = 2) or an AND (N = 3) -- one 3-input logic op per entry.
+// Returns x_i whose bit 31 is set iff entry i is dropped.
+template <int N>
+__device__ __forceinline__ void drop4(uint32_t k0, uint32_t k1, uint32_t k2, uint32_t k3, uint32_t& x0,
+                                      uint32_t& x1, uint32_t& x2, uint32_t& x3) {
+  const uint32_t d01 = k0 - k1, d02 = k0 - k2, d03 = k0 - k3;
+  const uint32_t d12 = k1 - k2, d13 = k1 - k3, d23 = k2 - k3;
+  // terms "j beats i" for each entry
+  const uint32_t a0 = d01, b0 = d02, c0 = d03;     // entry 0: beaten by 1, 2, 3
+  const uint32_t a1 = ~d01, b1 = d12, c1 = d13;    // entry 1: by 0, 2, 3
+  const uint32_t a2 = ~d02, b2 = ~d12, c2 = d23;   // entry 2: by 0, 1, 3
+  const uint32_t a3 = ~d03, b3 = ~d13, c3 = ~d23;  // entry 3: by 0, 1, 2
+  if constexpr (N == 1) {
+    x0 = a0 | b0 | c0; x1 = a1 | b1 | c1; x2 = a2 | b2 | c2; x3 = a3 | b3 | c3;
+  } else if constexpr (N == 2) {
+    x0 = (a0 & b0) | (a0 & c0) | (b0 & c0);
+    x1 = (a1 & b1) | (a1 & c1) | (b1 & c1);
+    x2 = (a2 & b2) | (a2 & c2) | (b2 & c2);
+    x3 = (a3 & b3) | (a3 & c3) | (b3 & c3);
+  } else {
+    x0 = a0 & b0 & c0; x1 = a1 & b1 & c1; x2 = a2 & b2 & c2; x3 = a3 & b3 & c3;
+  }
+}
+
+// Four 0/1 mask bytes (entry i in byte i) from the drop words of drop4.
+__device__ __forceinline__ uint32_t keep_bytes4(uint32_t x0, uint32_t x1, uint32_t x2, uint32_t x3) {
+  const uint32_t t01 = __byte_perm(x0, x1, 0x0073);  // byte0 = x0.byte3, byte1 = x1.byte3
+  const uint32_t t23 = __byte_perm(x2, x3, 0x0073);
+  const uint32_t t = __byte_perm(t01, t23, 0x5410);  // the four sign bytes
+  return (~t >> 7) & 0x01010101u;
+}
+
 // 2:4 specialisation: the two kept indices (ascending) of a group and the
 // 4-bit metadata field idx0 | idx1 << 2.
 struct Pick24 {

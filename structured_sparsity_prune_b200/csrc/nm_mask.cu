@@ -56,6 +56,35 @@ __global__ void __launch_bounds__(256) mask_vec16_kernel(const Bits* __restrict_
   }
 }
 
+// M = 4 fast path: 16 elements (four groups) per thread, the branch-free
+// selection of drop4 and the byte packing of keep_bytes4.
+template <typename Bits, int N>
+__global__ void __launch_bounds__(256) mask4_vec16_kernel(const Bits* __restrict__ W, int64_t R, int64_t cpr,
+                                                          int64_t ldw, uint8_t* __restrict__ mask, int64_t ldm) {
+  constexpr int kVec = Chunk16<Bits>::kVec;
+  const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
+  const int64_t c_step = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+    const uint4* wrow = reinterpret_cast<const uint4*>(W + r * ldw);
+    uint4* mrow = reinterpret_cast<uint4*>(mask + r * ldm);
+    for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < cpr; c += c_step) {
+      uint4 v[kVec];
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) v[i] = __ldcs(wrow + c * kVec + i);
+      const Bits* e = reinterpret_cast<const Bits*>(v);
+      uint32_t out[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        uint32_t x0, x1, x2, x3;
+        drop4<N>(mag_key<Bits>(e[4 * g]), mag_key<Bits>(e[4 * g + 1]), mag_key<Bits>(e[4 * g + 2]),
+                 mag_key<Bits>(e[4 * g + 3]), x0, x1, x2, x3);
+        out[g] = keep_bytes4(x0, x1, x2, x3);
+      }
+      __stcs(mrow + c, make_uint4(out[0], out[1], out[2], out[3]));
+    }
+  }
+}
+
 // Any M (2..8), any alignment: one thread per group, scalar loads/stores.
 template <typename Bits, int M>
 __global__ void __launch_bounds__(256) mask_scalar_kernel(const Bits* __restrict__ W, int64_t R,
@@ -95,6 +124,16 @@ template <typename Bits, int M>
 void launch_mask(const void* W, int64_t R, int64_t C, int64_t ldw, int N, uint8_t* mask, int64_t ldm,
                  bool vec, cudaStream_t s) {
   dim3 grid, block;
+  if constexpr (M == 4) {
+    if (vec) {
+      shape2d(R, C / 16, grid, block);
+      const Bits* w = static_cast<const Bits*>(W);
+      if (N == 1) mask4_vec16_kernel<Bits, 1><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);
+      else if (N == 2) mask4_vec16_kernel<Bits, 2><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);
+      else mask4_vec16_kernel<Bits, 3><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);
+      return;
+    }
+  }
   if constexpr (16 % M == 0) {
     if (vec) {
       shape2d(R, C / 16, grid, block);

@@ -209,3 +209,4 @@ def test_decode_skinny_full_size_sampled_rows(T):
     rows = _sample_rows(W.shape[0], 1)
     Y, ref = _run(W, X, torch.bfloat16, rows=rows)
     assert _nerr(Y, ref) <= 8e-3
+
