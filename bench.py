@@ -49,6 +49,32 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+# ncu summaries that carry a per-launch DRAM traffic figure for the dominant
+# kernel of a workload; the figure is reported only while the kernel source is
+# unchanged since the capture (its sha256 is recorded in the summary).
+TRAFFIC_PROFILES = {("linear_4096", "nm_spmm"): "profiles/spmm_pair_linear_4096.md"}
+
+
+def profiled_traffic(workload: str, kernel: str):
+    import hashlib
+    rel = TRAFFIC_PROFILES.get((workload, kernel))
+    if rel is None or not os.path.exists(os.path.join(ROOT, rel)):
+        return None
+    fields = {}
+    with open(os.path.join(ROOT, rel)) as f:
+        for line in f:
+            if ":" in line and line.split(":")[0] in ("traffic_bytes_per_launch", "source_sha256", "source_file"):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+    try:
+        src = open(os.path.join(ROOT, fields["source_file"]), "rb").read()
+        if hashlib.sha256(src).hexdigest() != fields["source_sha256"]:
+            return None
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, OSError, ValueError):
+        return None
+
+
 # ----------------------------------------------------------------- workloads
 def make_workload(name: str):
     """-> dict(W, X, R, K, T, desc) with CPU tensors."""
@@ -467,7 +493,7 @@ def main():
         e2e_value = world * step.flops * args.steps / (e2e_ms * 1e-3) / 1e12
     roof["peak_source"] = "%s: 2 x dense bf16 burst" % peak_src if roof["bound"] == "tensor" else \
         "%s: HBM copy" % peak_src
-    roof["traffic"] = None
+    roof["traffic"] = profiled_traffic(args.workload, "nm_spmm" if dom.startswith("nm_spmm") else dom)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -281,6 +281,54 @@ __global__ void __launch_bounds__(256) decompress_kernel(const Bits* __restrict_
   }
 }
 
+// Decompress, wide unit: one row x 32 columns (four canonical metadata bytes,
+// sixteen values) per thread, 16-byte loads and stores.  Needs C % 32 == 0.
+template <typename Bits>
+__global__ void __launch_bounds__(256) decompress32_kernel(const Bits* __restrict__ values,
+                                                           const uint8_t* __restrict__ meta, int64_t R,
+                                                           int64_t C, Bits* __restrict__ out, int64_t ldo) {
+  constexpr int kVals = 16 * int(sizeof(Bits)) / 16;  // 16-byte loads of values per unit: 2 or 4
+  const int64_t upr = C / 32;
+  const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
+  const int64_t u_step = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+    for (int64_t u = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u < upr; u += u_step) {
+      const uint32_t mw = __ldcs(reinterpret_cast<const uint32_t*>(meta + r * (C / 8) + 4 * u));
+      uint4 vv[kVals];
+#pragma unroll
+      for (int i = 0; i < kVals; ++i) vv[i] = __ldcs(reinterpret_cast<const uint4*>(values + r * (C / 2) + 16 * u) + i);
+      uint4* dst = reinterpret_cast<uint4*>(out + r * ldo + 32 * u);
+      if constexpr (sizeof(Bits) == 2) {
+        const uint32_t* vw = reinterpret_cast<const uint32_t*>(vv);  // value pair of group g in word g
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {  // two groups -> one 16-byte store
+          uint64_t g2[2];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int g = 2 * h + k;
+            const uint32_t nib = (mw >> (4 * g)) & 0xFu;
+            const uint32_t w = vw[g];
+            g2[k] = (uint64_t(w & 0xFFFFu) << (16 * (nib & 3u))) | (uint64_t(w >> 16) << (16 * (nib >> 2)));
+          }
+          __stcs(dst + h, make_uint4(uint32_t(g2[0]), uint32_t(g2[0] >> 32), uint32_t(g2[1]), uint32_t(g2[1] >> 32)));
+        }
+      } else {
+        const uint32_t* vw = reinterpret_cast<const uint32_t*>(vv);
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {  // one group -> one 16-byte store
+          const uint32_t nib = (mw >> (4 * g)) & 0xFu;
+          const uint32_t i0 = nib & 3u, i1 = nib >> 2;
+          const uint32_t v0 = vw[2 * g], v1 = vw[2 * g + 1];
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) o[i] = (uint32_t(i) == i0) ? v0 : ((uint32_t(i) == i1) ? v1 : 0u);
+          __stcs(dst + g, make_uint4(o[0], o[1], o[2], o[3]));
+        }
+      }
+    }
+  }
+}
+
 int tile_grid(int64_t R, int64_t C) {
   const int64_t tiles = ((R + 127) / 128) * ((C + 127) / 128);
   const int64_t want = int64_t(sm_count()) * 8;
@@ -355,8 +403,9 @@ extern "C" nm_status nm_decompress(const void* values, const uint8_t* meta, nm_d
   if (!aligned16(values) || !aligned16(meta) || !aligned16(W_out) || !stride_ok(ldw, esize_of(dtype)))
     return NM_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // x over the octets of a row, y over rows
-  const int64_t opr = C / 8;
+  // x over the units of a row, y over rows
+  const bool wide = (C % 32) == 0;
+  const int64_t opr = wide ? C / 32 : C / 8;
   int bx = 32;
   while (bx < 256 && bx < opr) bx *= 2;
   const int by = 256 / bx;
@@ -367,12 +416,21 @@ extern "C" nm_status nm_decompress(const void* values, const uint8_t* meta, nm_d
   if (gy > cap) gy = cap;
   if (gy > 65535) gy = 65535;
   dim3 grid(unsigned(gx), unsigned(gy < 1 ? 1 : gy)), block(bx, by);
-  if (dtype == NM_F32)
-    decompress_kernel<uint32_t><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C,
-                                                       static_cast<uint32_t*>(W_out), ldw);
-  else
-    decompress_kernel<uint16_t><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(values), meta, R, C,
-                                                       static_cast<uint16_t*>(W_out), ldw);
+  if (dtype == NM_F32) {
+    if (wide)
+      decompress32_kernel<uint32_t><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C,
+                                                           static_cast<uint32_t*>(W_out), ldw);
+    else
+      decompress_kernel<uint32_t><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C,
+                                                         static_cast<uint32_t*>(W_out), ldw);
+  } else {
+    if (wide)
+      decompress32_kernel<uint16_t><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(values), meta, R, C,
+                                                           static_cast<uint16_t*>(W_out), ldw);
+    else
+      decompress_kernel<uint16_t><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(values), meta, R, C,
+                                                         static_cast<uint16_t*>(W_out), ldw);
+  }
   return launch_status();
 }
 
