@@ -21,6 +21,8 @@ What each function follows (page title and section):
   (the pages give none).
 * ``spmm`` -- same review, "Structured sparse GEMM on tensor cores":
   sparse x dense = dense; computed in double.
+* ``srste`` -- "SR-STE sparse training", SR-STE forward / backward:
+  masked weight and grad + decay * (1 - mask) * w.
 """
 from __future__ import annotations
 
@@ -78,6 +80,8 @@ def _load():
     lib.oracle_spmm.restype = i32
     lib.oracle_rows_parallel.argtypes = [i32, vp, i32, i64, i64, i32, i32, vp, vp, vp, i32]
     lib.oracle_rows_parallel.restype = i32
+    lib.oracle_srste.argtypes = [vp, vp, i32, i64, i64, i32, i32, ctypes.c_float, vp, vp, vp]
+    lib.oracle_srste.restype = i32
     _lib = lib
     return lib
 
@@ -235,3 +239,18 @@ def rows_parallel(what: int, W: np.ndarray, N: int, M: int, dtype: int, threads:
                                         values.ctypes.data, meta.ctypes.data, int(threads)),
            "rows_parallel")
     return mask, values, meta
+
+
+def srste(W: np.ndarray, grad: np.ndarray, N: int, M: int, decay: float, dtype: int | None = None):
+    """SR-STE step -> (W_sparse, grad_out, mask); arrays of W's bit type."""
+    code = dtype_code(W, dtype)
+    Wb, Gb = _bits(W, code), _bits(grad, code)
+    R, C = Wb.shape
+    ws = np.zeros_like(Wb)
+    go = np.zeros_like(Wb)
+    mask = np.zeros((R, C), dtype=np.uint8)
+    _check(_load().oracle_srste(Wb.ctypes.data, Gb.ctypes.data, code, R, C, N, M, float(decay),
+                                ws.ctypes.data, go.ctypes.data, mask.ctypes.data), "srste")
+    if W.dtype != np.uint16:
+        return ws.view(W.dtype), go.view(W.dtype), mask
+    return ws, go, mask

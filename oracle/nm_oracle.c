@@ -513,3 +513,41 @@ int oracle_rows_parallel(int what, const void *W, int dtype, int64_t R, int64_t 
     for (int i = 0; i < nthreads; ++i) { pthread_join(th[i], NULL); if (jobs[i].status) st = jobs[i].status; }
     return st;
 }
+
+/* --------------------------------------------------------------------- */
+/* SR-STE step.  [SRSTE] "SR-STE sparse training", SR-STE forward and     */
+/* backward: the forward keeps the N:M mask of |w| (recomputed every     */
+/* step) and returns the masked weight; the backward returns              */
+/*     grad + decay * (1 - mask) * w                                       */
+/* so pruned entries receive an extra decay * w (the page's default       */
+/* decay is 0.0002).  Readings: the masked weight is select(mask, w, +0); */
+/* the decay term is one fused multiply-add in binary32 (fmaf, correctly  */
+/* rounded), rounded once to the element type; kept entries return grad  */
+/* bit for bit.  mask may be NULL.                                         */
+/* --------------------------------------------------------------------- */
+int oracle_srste(const void *W, const void *grad, int dtype, int64_t R, int64_t C, int N, int M, float decay,
+                 void *W_sparse, void *grad_out, uint8_t *mask_out)
+{
+    if (M < 2 || M > 8 || N < 1 || N >= M || C % M != 0 || R < 0) return OR_BAD_ARG;
+    uint8_t *m = (uint8_t *)malloc((size_t)(C > 0 ? C : 1));
+    for (int64_t r = 0; r < R; ++r) {
+        int st = oracle_mask_rank((const char *)W + (size_t)(r * C) * elem_size(dtype), dtype, 1, C, C, N, M, m, C);
+        if (st != OR_OK) { free(m); return st; }
+        for (int64_t c = 0; c < C; ++c) {
+            size_t i = (size_t)(r * C + c);
+            uint32_t wb = load_bits(W, dtype, i), gb = load_bits(grad, dtype, i);
+            if (mask_out) mask_out[i] = m[c];
+            if (m[c]) {
+                store_bits(W_sparse, dtype, i, wb);
+                store_bits(grad_out, dtype, i, gb);
+            } else {
+                store_bits(W_sparse, dtype, i, 0u);
+                float w = (float)oracle_decode(wb, dtype), g = (float)oracle_decode(gb, dtype);
+                float y = fmaf(decay, w, g);                 /* binary32, one rounding */
+                store_bits(grad_out, dtype, i, oracle_encode((double)y, dtype));
+            }
+        }
+    }
+    free(m);
+    return OR_OK;
+}
