@@ -90,6 +90,10 @@ def make_workload(name: str):
         return {"W": W_up, "W2": W_down, "X": X, "R": W_up.shape[0], "K": W_up.shape[1], "T": X.shape[1],
                 "desc": "MLP pair: bf16 W_up 14336x4096, W_down 4096x14336 ~N(0,0.02) 2:4; X bf16 4096x8192 ~N(0,1);"
                         " up then down"}
+    elif name == "srste":
+        W, _ = nm_inputs.linear_4096()
+        return {"W": W, "G": nm_inputs.srste_grad(), "X": None, "R": 4096, "K": 4096, "T": 0,
+                "desc": "SR-STE step: bf16 W 4096x4096 ~N(0,0.02) and bf16 gradient ~N(0,1e-3); 2:4, decay 0.0002"}
     elif name == "ties_mask":
         W = nm_inputs.ties_fp32()
         return {"W": W, "X": None, "R": 8192, "K": 8192, "T": 0,
@@ -180,8 +184,18 @@ class Step:
     def __init__(self, nm, wl, dev):
         self.nm, self.wl, self.dev = nm, wl, dev
         R, K, T = wl["R"], wl["K"], wl["T"]
-        self.kind = "ties" if wl["X"] is None else ("mlp" if "W2" in wl else "linear")
+        self.kind = "srste" if "G" in wl else ("ties" if wl["X"] is None else ("mlp" if "W2" in wl else "linear"))
         self.W = wl["W"].to(dev)
+        if self.kind == "srste":
+            self.G = wl["G"].to(dev)
+            self.WS = torch.empty_like(self.W)
+            self.GO = torch.empty_like(self.W)
+            self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
+            self.names = ["nm_srste_step"]
+            es = self.W.element_size()
+            self.bytes = {"nm_srste_step": R * K * (4 * es + 1)}
+            self.flops = 0
+            return
         if self.kind == "ties":
             self.masks = [torch.empty((R, K), dtype=torch.uint8, device=dev) for _ in range(4)]
             self.names = ["nm_mask_1:4", "nm_mask_2:4", "nm_mask_4:8", "nm_mask_2:8"]
@@ -233,7 +247,10 @@ class Step:
         nm, s = self.nm, torch.cuda.current_stream()
         rec = (lambda i: events[i].record(s)) if events is not None else (lambda i: None)
         rec(0)
-        if self.kind == "ties":
+        if self.kind == "srste":
+            nm.nm_srste_step(self.W, self.G, 2, 4, 0.0002, W_sparse=self.WS, grad_out=self.GO, mask=self.mask)
+            rec(1)
+        elif self.kind == "ties":
             for i, (N, M) in enumerate([(1, 4), (2, 4), (4, 8), (2, 8)]):
                 nm.nm_mask(self.W, N, M, mask=self.masks[i])
                 rec(i + 1)
@@ -262,6 +279,8 @@ class Step:
             rec(6)
 
     def result(self):
+        if self.kind == "srste":
+            return self.GO
         return self.masks[1] if self.kind == "ties" else self.Y
 
 
@@ -289,6 +308,9 @@ def e2e_steps(step: Step, steps: int, flush: torch.Tensor):
     if "W2" in step.wl:
         W2_h = step.wl["W2"].pin_memory()
         h2d += W2_h.numel() * W2_h.element_size()
+    if "G" in step.wl:
+        G_h = step.wl["G"].pin_memory()
+        h2d += G_h.numel() * G_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
     s = torch.cuda.current_stream()
     times = []
@@ -301,6 +323,8 @@ def e2e_steps(step: Step, steps: int, flush: torch.Tensor):
             step.X.copy_(X_h, non_blocking=True)
         if "W2" in step.wl:
             step.W2.copy_(W2_h, non_blocking=True)
+        if "G" in step.wl:
+            step.G.copy_(G_h, non_blocking=True)
         step.run()
         out_h.copy_(res, non_blocking=True)
         b.record(s)
@@ -318,6 +342,12 @@ def oracle_step(wl, rows: int, threads: int):
     """The oracle doing the step's work on the first `rows` rows of W.
     -> (seconds, units) with units in the metric's unit (dense-eq flops or bytes)."""
     import oracle
+    if "G" in wl:                 # SR-STE step
+        Wb = _u16(wl["W"][:rows].contiguous())
+        Gb = _u16(wl["G"][:rows].contiguous())
+        t0 = time.perf_counter()
+        oracle.srste(Wb, Gb, 2, 4, 0.0002, dtype=oracle.BF16)
+        return time.perf_counter() - t0, float(rows * wl["K"] * 9)
     if wl["X"] is None:           # mask-only workload
         W = wl["W"][:rows].contiguous().numpy()
         t0 = time.perf_counter()
@@ -362,9 +392,11 @@ def cpu_baseline(wl, target_s: float = 15.0):
     rows = size_oracle_sample(wl, threads, target_s)
     secs, units = oracle_step(wl, rows, threads)
     scale, unit = (1e12, "TFLOP/s") if wl["X"] is not None else (1e9, "GB/s")
+    what = ("SR-STE step (mask, masked weight, decay gradient)" if "G" in wl else
+            "mask at 1:4, 2:4, 4:8, 2:8" if wl["X"] is None else
+            "whole step (mask, compress, fused mask+compress, image, decompress, fp64 product)")
     return {"value": units / secs / scale, "unit": unit, "cores": threads, "kind": "oracle",
-            "sample": "first %d of %d rows of W, whole step (mask, compress, fused mask+compress, image, "
-                      "decompress, fp64 product), %.1f s" % (rows, wl["R"], secs)}
+            "sample": "first %d of %d rows of W, %s, %.1f s" % (rows, wl["R"], what, secs)}
 
 
 def run_reference(args, wl, metric):
@@ -474,11 +506,11 @@ def main():
             k.update({"TFLOP/s": tf, "tensor_frac": tf / sparse_peak})
         kernels[name] = k
 
-    if step.kind == "ties":
+    if step.kind in ("ties", "srste"):
         units_per_step = sum(step.bytes.values())
         value = world * units_per_step * args.steps / (total_ms * 1e-3) / 1e9
         unit = "GB/s"
-        dom = "nm_mask_2:4"
+        dom = "nm_mask_2:4" if step.kind == "ties" else "nm_srste_step"
         roof = {"bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": hbm, "unit": "GB/s",
                 "frac": kernels[dom]["GB/s"] / hbm, "kernel": dom,
                 "algorithmic_bytes_per_launch": step.bytes[dom]}

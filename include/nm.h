@@ -143,6 +143,24 @@ NM_API nm_status nm_meta_to_sm100(const uint8_t *meta, int64_t R, int64_t C, uin
                            void *stream);
 
 /*
+ * nm_srste_step -- one SR-STE training step, fused ("SR-STE sparse training",
+ * SR-STE forward and backward): the N:M magnitude mask of W is recomputed
+ * (same rule as nm_mask), and
+ *   W_sparse = W where kept, +0 elsewhere                      (forward)
+ *   grad_out = grad where kept, grad + decay * W elsewhere     (backward,
+ *              i.e. grad + decay * (1 - mask) * W)
+ * The decay term is one binary32 fused multiply-add, rounded once (nearest
+ * even) to dtype; kept entries return grad bit for bit.  The page's default
+ * decay is 0.0002.
+ *   W, grad, W_sparse, grad_out: R x C, dtype, common leading dim ld >= C
+ *   mask: R x C uint8 with row stride ld, or NULL
+ *   1 <= N < M <= 8, C % M == 0
+ */
+NM_API nm_status nm_srste_step(const void *W, const void *grad, nm_dtype dtype, int64_t R, int64_t C,
+                               int64_t ld, int N, int M, float decay, void *W_sparse, void *grad_out,
+                               uint8_t *mask, void *stream);
+
+/*
  * nm_spmm_workspace_bytes -- device scratch nm_spmm needs for this problem
  * (0 when none is needed).  NM_F32 inputs are rounded to binary16 (nearest
  * even) in the workspace before the product.

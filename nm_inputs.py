@@ -17,6 +17,8 @@ linear/conv weights; the pages' datasets and trained weights are not used):
 * ``ties_fp32``       W fp32 8192x8192 = fp32(k/100), k ~ U{-8..7} (seed 4)
 * ``decode_skinny``   W bf16 28672x8192 = bf16(0.02 * N(0,1)) (seed 5),
                       X bf16 8192xT ~N(0,1) (seed 105+T), T in {16,64,256,1024}
+* ``srste``           the linear_4096 weight and a gradient bf16(1e-3 * N(0,1))
+                      of the same shape (seed 6)
 """
 from __future__ import annotations
 
@@ -28,6 +30,7 @@ SEEDS = {
     "mlp_pair.W_up": 2, "mlp_pair.W_down": 3, "mlp_pair.X": 102,
     "ties_fp32.W": 4,
     "decode_skinny.W": 5,
+    "srste.grad": 6,
 }
 
 
@@ -88,3 +91,7 @@ def decode_skinny_X(T: int):
 def bits_u16(t: torch.Tensor):
     """numpy uint16 view of a bf16/f16 CPU tensor (bit patterns)."""
     return t.contiguous().view(torch.int16).numpy().view("uint16")
+
+
+def srste_grad(shape=(4096, 4096)):
+    return normal(shape, SEEDS["srste.grad"], 1e-3, torch.bfloat16)

@@ -54,6 +54,7 @@ def _lib():
         "nm_spmm_workspace_bytes": ([i32, i64, i64, i64], sz),
         "nm_spmm": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp, sz, vp], i32),
         "nm_spmm_noalloc": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp], i32),
+        "nm_srste_step": ([vp, vp, i32, i64, i64, i64, i32, i32, f32, vp, vp, vp, vp], i32),
         "nm_last_device_status": ([vp], i32),
     }
     for name, (args, res) in sig.items():
@@ -192,3 +193,22 @@ def nm_spmm(values: torch.Tensor, meta_sm100: torch.Tensor, X: torch.Tensor, Y: 
 
 def nm_last_device_status(stream=None) -> int:
     return int(_lib().nm_last_device_status(_stream(stream)))
+
+
+def nm_srste_step(W: torch.Tensor, grad: torch.Tensor, N: int = 2, M: int = 4, decay: float = 0.0002,
+                  W_sparse: torch.Tensor | None = None, grad_out: torch.Tensor | None = None,
+                  mask: torch.Tensor | None = None, want_mask: bool = False, stream=None):
+    """SR-STE step -> (W_sparse, grad_out, mask or None).  W, grad and the outputs
+    share one leading dimension (that of W)."""
+    R, C = W.shape
+    ld = _ld(W)
+    assert _ld(grad) == ld
+    if W_sparse is None:
+        W_sparse = torch.empty_strided((R, C), (ld, 1), dtype=W.dtype, device=W.device)
+    if grad_out is None:
+        grad_out = torch.empty_strided((R, C), (ld, 1), dtype=W.dtype, device=W.device)
+    if mask is None and want_mask:
+        mask = torch.empty_strided((R, C), (ld, 1), dtype=torch.uint8, device=W.device)
+    _check(_lib().nm_srste_step(_ptr(W), _ptr(grad), _dtype(W), R, C, ld, N, M, float(decay), _ptr(W_sparse),
+                                _ptr(grad_out), _ptr(mask), _stream(stream)), "nm_srste_step")
+    return W_sparse, grad_out, mask
