@@ -140,7 +140,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   d |= uint64_t(layout & 7u) << 61;
   return d;
 }
-constexpr uint32_t kLayoutNone = 0, kLayoutSW128 = 2;
+constexpr uint32_t kLayoutNone = 0, kLayoutSW128 = 2, kLayoutSW64 = 4, kLayoutSW32 = 6;
 
 __device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
@@ -258,6 +258,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // Instruction descriptor, .kind::f16 with sparsity: D fp32, A/B fp16 or bf16,
 // A K-major, B N-major (X is K x T with T contiguous), M = 128, N = n.
 __host__ __device__ constexpr uint32_t make_idesc(bool bf16, int n, int m = kBlockM) {
@@ -275,17 +284,27 @@ __host__ __device__ constexpr uint32_t make_idesc(bool bf16, int n, int m = kBlo
 template <int N_TILE, int STAGES>
 struct Cfg {
   static constexpr int kABytes = kBlockM * kStageKPhys * 2;   // 16 KB
-  static constexpr int kBBoxes = N_TILE / 64;                 // 64-column TMA boxes
-  static constexpr int kBBoxBytes = kStageK * 64 * 2;         // 16 KB
+  // X tile: N_TILE >= 64 -> 64-column boxes with 128-byte rows; narrower tiles
+  // (16 or 32 columns) use one box whose 32- or 64-byte rows carry only the
+  // columns the MMA reads, with the matching swizzle.
+  static constexpr int kBoxCols = N_TILE < 64 ? N_TILE : 64;
+  static constexpr int kBRowBytes = kBoxCols * 2;             // 32, 64 or 128
+  static constexpr int kBBoxes = N_TILE < 64 ? 1 : N_TILE / 64;
+  static constexpr int kBBoxBytes = kStageK * kBRowBytes;
   static constexpr int kBBytes = kBBoxes * kBBoxBytes;
+  static constexpr uint32_t kBLayout = kBRowBytes == 128 ? kLayoutSW128 : (kBRowBytes == 64 ? kLayoutSW64 : kLayoutSW32);
   static constexpr int kEBytes = 2048;
   static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
   static constexpr int kAccCols = N_TILE;
   static constexpr int kAccBufs = (2 * N_TILE + 4 * STAGES <= 512) ? 2 : 1;
   static constexpr int kECol0 = kAccBufs * N_TILE;
-  static constexpr int kTmemCols = (kECol0 + 4 * STAGES) <= 256 ? 256 : 512;
+  static constexpr int kTmemNeed = kECol0 + 4 * STAGES;
+  static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
+                                   : kTmemNeed <= 256 ? 256 : 512;
   static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 /* align */ + 256 /* barriers, flags */;
-  static_assert(N_TILE % 64 == 0 && N_TILE <= 256, "N_TILE");
+  static constexpr int kChunk = N_TILE < 32 ? N_TILE : 32;      // epilogue columns per TMEM load
+  static_assert((N_TILE % 64 == 0 || N_TILE == 16 || N_TILE == 32) && N_TILE <= 256, "N_TILE");
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kECol0 + 4 * STAGES <= 512, "TMEM budget");
 };
 
@@ -326,27 +345,28 @@ __device__ __forceinline__ void grouped_tile(const Params& p, int t, int& mt, in
 
 // Epilogue of one 32-column chunk of one output row: y = alpha * acc (+ beta * y_old),
 // rounded to the output type; vector stores when Y allows them, scalar at the T edge.
-__device__ __forceinline__ void store_chunk(const Params& p, int r, int col0, const uint32_t (&v)[32]) {
+template <int CW>
+__device__ __forceinline__ void store_chunk_n(const Params& p, int r, int col0, const uint32_t (&v)[CW]) {
   if (r < p.R && col0 < p.T) {
-    const bool full_chunk = p.y_vec && col0 + 32 <= p.T;
-    float y[32];
+    const bool full_chunk = p.y_vec && col0 + CW <= p.T;
+    float y[CW];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) y[j] = p.alpha * __uint_as_float(v[j]);
+    for (int j = 0; j < CW; ++j) y[j] = p.alpha * __uint_as_float(v[j]);
     if (p.y_f32) {
       float* yrow = static_cast<float*>(p.Y) + size_t(r) * p.ldy + col0;
       if (full_chunk) {
         if (p.beta != 0.0f) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 4) {
+          for (int j = 0; j < CW; j += 4) {
             const float4 o = *reinterpret_cast<const float4*>(yrow + j);
             y[j] += p.beta * o.x; y[j + 1] += p.beta * o.y; y[j + 2] += p.beta * o.z; y[j + 3] += p.beta * o.w;
           }
         }
 #pragma unroll
-        for (int j = 0; j < 32; j += 4)
+        for (int j = 0; j < CW; j += 4)
           *reinterpret_cast<float4*>(yrow + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
       } else {
-        for (int j = 0; j < 32 && col0 + j < p.T; ++j) {
+        for (int j = 0; j < CW && col0 + j < p.T; ++j) {
           float o = y[j];
           if (p.beta != 0.0f) o += p.beta * yrow[j];
           yrow[j] = o;
@@ -357,7 +377,7 @@ __device__ __forceinline__ void store_chunk(const Params& p, int r, int col0, co
       if (full_chunk) {
         if (p.beta != 0.0f) {
 #pragma unroll
-          for (int j = 0; j < 32; j += 8) {
+          for (int j = 0; j < CW; j += 8) {
             const uint4 o = *reinterpret_cast<const uint4*>(yrow + j);
             const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&o);
 #pragma unroll
@@ -369,7 +389,7 @@ __device__ __forceinline__ void store_chunk(const Params& p, int r, int col0, co
           }
         }
 #pragma unroll
-        for (int j = 0; j < 32; j += 8) {
+        for (int j = 0; j < CW; j += 8) {
           uint4 o;
           __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll
@@ -377,7 +397,7 @@ __device__ __forceinline__ void store_chunk(const Params& p, int r, int col0, co
           *reinterpret_cast<uint4*>(yrow + j) = o;
         }
       } else {
-        for (int j = 0; j < 32 && col0 + j < p.T; ++j) {
+        for (int j = 0; j < CW && col0 + j < p.T; ++j) {
           float o = y[j];
           if (p.beta != 0.0f) o += p.beta * __bfloat162float(yrow[j]);
           yrow[j] = __float2bfloat16_rn(o);
@@ -386,9 +406,12 @@ __device__ __forceinline__ void store_chunk(const Params& p, int r, int col0, co
     }
   }
 }
+__device__ __forceinline__ void store_chunk(const Params& p, int r, int col0, const uint32_t (&v)[32]) {
+  store_chunk_n<32>(p, r, col0, v);
+}
 
 template <int N_TILE, int STAGES, bool BF16>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 113 * 1024 ? 2 : 1)
     spmm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, Params p) {
   using C = Cfg<N_TILE, STAGES>;
   extern __shared__ uint8_t smem_raw[];
@@ -493,7 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t adesc = smem_desc(a_addr + 32u * k2, 16, 1024, kLayoutSW128);
             // B: N-major, 128B swizzle: 64-column atoms LBO apart, 8-row K groups 1024 B apart;
             //    32 logical K rows = 4096 bytes further per MMA.
-            const uint64_t bdesc = smem_desc(b_addr + 4096u * k2, C::kBBoxBytes, 1024, kLayoutSW128);
+            const uint64_t bdesc = smem_desc(b_addr + uint32_t(32 * C::kBRowBytes) * k2, C::kBBoxBytes,
+                                             uint32_t(8 * C::kBRowBytes), C::kBLayout);
             // metadata column of this MMA: even base + selector bit
             const uint32_t e_col = e_tmem + uint32_t(k2 & ~1);
             const uint32_t id = idesc | uint32_t(k2 & 1);
@@ -526,11 +550,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_after_sync();
       const int r = mt * kBlockM + row_in_tile;
       const int c_base = nt * N_TILE;
+      if constexpr (C::kChunk == 16) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TILE), v);
+        store_chunk_n<16>(p, r, c_base, v);
+      } else {
 #pragma unroll 1
-      for (int c = 0; c < N_TILE; c += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TILE + c), v);
-        store_chunk(p, r, c_base + c, v);
+        for (int c = 0; c < N_TILE; c += 32) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TILE + c), v);
+          store_chunk(p, r, c_base + c, v);
+        }
       }
       fence_before_sync();
       __syncwarp();
@@ -822,7 +852,7 @@ EncodeFn get_encode() {
 
 // 2D tile map over a row-major [rows x cols] 16-bit matrix, box = box_cols x box_rows, 128B swizzle.
 bool make_map(CUtensorMap* map, const void* base, bool bf16, int64_t rows, int64_t cols, int64_t ld_elems,
-              int box_cols, int box_rows) {
+              int box_cols, int box_rows, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeFn enc = get_encode();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
@@ -831,13 +861,17 @@ bool make_map(CUtensorMap* map, const void* base, bool bf16, int64_t rows, int64
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int N_TILE, int STAGES, bool BF16>
-nm_status launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, cudaStream_t s) {
+nm_status launch(const CUtensorMap& ma, const void* X, int64_t ldx, int64_t K, int64_t T, const Params& p,
+                 cudaStream_t s) {
   using C = Cfg<N_TILE, STAGES>;
+  CUtensorMap mb;
+  const CUtensorMapSwizzle sw = C::kBRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : C::kBRowBytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  if (!make_map(&mb, X, BF16, K, T, ldx, C::kBoxCols, kStageK, sw)) return NM_ERR_CUDA;
   auto kern = spmm_kernel<N_TILE, STAGES, BF16>;
   static bool attr_done = false;  // per instantiation
   if (!attr_done) {
@@ -846,7 +880,9 @@ nm_status launch(const CUtensorMap& ma, const CUtensorMap& mb, const Params& p, 
     attr_done = true;
   }
   const int tiles = p.m_tiles * p.n_tiles;
-  const int grid = tiles < sm_count() ? tiles : sm_count();
+  const int per_sm = C::kSmemBytes <= 113 * 1024 ? 2 : 1;  // two CTAs per SM when the ring is small
+  const int slots = per_sm * sm_count();
+  const int grid = tiles < slots ? tiles : slots;
   kern<<<grid, kThreads, C::kSmemBytes, s>>>(ma, mb, p);
   return launch_status();
 }
@@ -888,13 +924,17 @@ nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
 // otherwise.  NM_SPMM_KERNEL = pair256 | pair128 | single256 | single128 |
 // single64 overrides the choice (for tuning; an inapplicable override falls
 // back to the default).
-enum class Kern { Pair256, Pair192, Pair128, Single256, Single128, Single64 };
+enum class Kern { Pair256, Pair192, Pair128, Single256, Single128, Single64, Single64x2, Single32x2, Single16x2 };
 
 Kern choose_kernel(int64_t R, int64_t T) {
   const bool pairable = ((R + kBlockM - 1) / kBlockM) % 2 == 0;
   Kern k;
   if (pairable && T > 64) k = T > 128 ? Kern::Pair256 : Kern::Pair128;
-  else k = T > 128 ? Kern::Single256 : (T > 64 ? Kern::Single128 : Kern::Single64);
+  else if (T > 128) k = Kern::Single256;
+  else if (T > 64) k = Kern::Single128;
+  else if (T > 32) k = Kern::Single64x2;
+  else if (T > 16) k = Kern::Single32x2;
+  else k = Kern::Single16x2;
   if (const char* env = getenv("NM_SPMM_KERNEL")) {
     const std::string e(env);
     if (e == "pair256" && pairable) k = Kern::Pair256;
@@ -903,6 +943,9 @@ Kern choose_kernel(int64_t R, int64_t T) {
     else if (e == "single256") k = Kern::Single256;
     else if (e == "single128") k = Kern::Single128;
     else if (e == "single64") k = Kern::Single64;
+    else if (e == "single64x2") k = Kern::Single64x2;
+    else if (e == "single32x2") k = Kern::Single32x2;
+    else if (e == "single16x2") k = Kern::Single16x2;
   }
   return k;
 }
@@ -927,7 +970,9 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
   const int block_m = pair ? 2 * kBlockM : kBlockM;
   const int n_tile = (kern == Kern::Pair256 || kern == Kern::Single256) ? 256
                      : kern == Kern::Pair192                                 ? 192
-                     : (kern == Kern::Pair128 || kern == Kern::Single128) ? 128 : 64;
+                     : (kern == Kern::Pair128 || kern == Kern::Single128) ? 128
+                     : kern == Kern::Single32x2                              ? 32
+                     : kern == Kern::Single16x2                              ? 16 : 64;
   p.m_tiles = int((R + block_m - 1) / block_m);
   p.n_tiles = int((T + n_tile - 1) / n_tile);
   // Tile order: the operand with fewer bytes is swept fastest, so consecutive
@@ -951,9 +996,12 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
     return launch_pair<128, 6, BF16>(ma, mb, me, p, s);
   }
   switch (kern) {
-    case Kern::Single256: return launch<256, 2, BF16>(ma, mb, p, s);
-    case Kern::Single128: return launch<128, 4, BF16>(ma, mb, p, s);
-    default: return launch<64, 6, BF16>(ma, mb, p, s);
+    case Kern::Single256: return launch<256, 2, BF16>(ma, X, ldx, K, T, p, s);
+    case Kern::Single128: return launch<128, 4, BF16>(ma, X, ldx, K, T, p, s);
+    case Kern::Single64x2: return launch<64, 3, BF16>(ma, X, ldx, K, T, p, s);
+    case Kern::Single32x2: return launch<32, 4, BF16>(ma, X, ldx, K, T, p, s);
+    case Kern::Single16x2: return launch<16, 5, BF16>(ma, X, ldx, K, T, p, s);
+    default: return launch<64, 6, BF16>(ma, X, ldx, K, T, p, s);
   }
 }
 
