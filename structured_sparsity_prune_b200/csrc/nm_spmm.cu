@@ -30,6 +30,7 @@
 
 #include <cstdlib>
 #include <mutex>
+#include <cstring>
 #include <string>
 
 #include "nm_internal.cuh"
@@ -197,6 +198,26 @@ __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
 
 // TMA tile load into this CTA's shared memory whose completion is counted on
 // an mbarrier of either CTA of the pair (here: the MMA-issuing CTA's).
+// Output staging: a shared-memory tile written by the generic proxy and
+// stored to global memory by the bulk (async) proxy.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(smem_u32(src)), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// the bulk stores committed by this thread have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// ... and have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int x,
                                                  int y) {
   asm volatile(
@@ -318,6 +339,7 @@ struct Params {
   int group;    // tiles of the slow operand kept together (sized so the group stays in L2)
   int y_f32;    // 1: fp32 output, 0: bf16 output
   int y_vec;    // 1: Y and ldy allow 16-byte vector stores
+  int y_tma;    // 1: bf16 output with beta == 0 leaves through staged bulk tensor stores (pair kernel)
   float alpha, beta;
 };
 
@@ -596,7 +618,13 @@ struct PairCfg {
   static constexpr int kAccBufs = (2 * N_TOTAL + 4 * STAGES <= 512) ? 2 : 1;
   static constexpr int kECol0 = kAccBufs * N_TOTAL;
   static constexpr int kTmemCols = (kECol0 + 4 * STAGES) <= 256 ? 256 : 512;
-  static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 + 256;
+  // One 2 KB output slot (32 rows x 32 bf16 columns, 64-byte swizzle) per
+  // epilogue warp, 1024-byte aligned after the barriers.
+  static constexpr int kOutSlotBytes = 2048;
+  static constexpr int kOutOff = STAGES * kStageBytes + 1024;
+  static constexpr int kSmemBytes = kOutOff + 8 * kOutSlotBytes + 1024 /* base alignment */;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kNHalf % 32 == 0 && N_TOTAL <= 256, "N_TOTAL");
   static_assert(kECol0 + 4 * STAGES <= 512, "TMEM budget");
 };
@@ -604,7 +632,8 @@ struct PairCfg {
 template <int N_TOTAL, int STAGES, bool BF16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     spmm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                     const __grid_constant__ CUtensorMap map_e, Params p) {
+                     const __grid_constant__ CUtensorMap map_e, const __grid_constant__ CUtensorMap map_y,
+                     Params p) {
   using C = PairCfg<N_TOTAL, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -745,6 +774,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int row_in_tile = 32 * q + lane;
     const uint32_t acc_empty_leader[2] = {mapa(smem_u32(&acc_empty[0]), 0), mapa(smem_u32(&acc_empty[1]), 0)};
     const bool early = !p.y_f32 && p.beta == 0.0f && p.y_vec;
+    const uint32_t out_slot = smem_u32(smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes);
     uint32_t local = 0;
     for (int t = pair; t < num_tiles; t += num_pairs, ++local) {
       int mt, nt;
@@ -778,7 +808,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(acc_empty_leader[buf]);
-        if (r < p.R) {
+        if (p.y_tma) {
+          // 32 x 32 chunks through this warp's slot: lane = row, four 16-byte
+          // pieces per row placed with the 64-byte swizzle (piece ^ ((row >> 1) & 3)),
+          // so a warp's shared stores hit all 32 banks; one bulk tensor store per
+          // chunk, which the tensor map clips at R and T.
+          const uint32_t slot = out_slot + uint32_t(lane) * 64u;
+          const uint32_t sw = (uint32_t(lane) >> 1) & 3u;
+          const int row0 = (2 * mt + int(rank)) * kBlockM + 32 * q;
+#pragma unroll
+          for (int c = 0; c < kCols; c += 32) {
+            if (lane == 0) bulk_wait_read_all();  // the slot's previous store has read it
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              st_shared_v4(slot + 16u * (uint32_t(j) ^ sw), packed[c / 2 + 4 * j], packed[c / 2 + 4 * j + 1],
+                           packed[c / 2 + 4 * j + 2], packed[c / 2 + 4 * j + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0 && row0 < p.R && c_base + c < p.T) {  // boxes start inside Y
+              tma_store_2d(&map_y, smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes, c_base + c, row0);
+              bulk_commit();
+            }
+          }
+        } else if (r < p.R) {
           __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.Y) + size_t(r) * p.ldy;
 #pragma unroll
           for (int c = 0; c < kCols; c += 8) {
@@ -810,6 +863,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (lane == 0) mbar_arrive_remote(acc_empty_leader[buf]);
       }
     }
+    if (lane == 0) bulk_wait_all();  // output stores complete before the CTA leaves
   }
 
   // ---------------------------------------------------------------- teardown
@@ -902,8 +956,8 @@ bool make_map_image(CUtensorMap* map, const uint8_t* img, int64_t rows16) {
 }
 
 template <int N_TOTAL, int STAGES, bool BF16>
-nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me, const Params& p,
-                      cudaStream_t s) {
+nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me, const CUtensorMap& my,
+                      const Params& p, cudaStream_t s) {
   using C = PairCfg<N_TOTAL, STAGES>;
   auto kern = spmm_pair_kernel<N_TOTAL, STAGES, BF16>;
   static bool attr_done = false;  // per instantiation
@@ -915,7 +969,7 @@ nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   const int pairs = p.m_tiles * p.n_tiles;
   const int max_pairs = sm_count() / 2;
   const int grid = 2 * (pairs < max_pairs ? pairs : max_pairs);
-  kern<<<grid, kPairThreads, C::kSmemBytes, s>>>(ma, mb, me, p);
+  kern<<<grid, kPairThreads, C::kSmemBytes, s>>>(ma, mb, me, my, p);
   return launch_status();
 }
 
@@ -954,6 +1008,7 @@ template <bool BF16>
 nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_t ldx, void* Y, bool y_f32,
               int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta, cudaStream_t s) {
   Params p;
+  p.y_tma = 0;
   p.meta_img = meta_img;
   p.Y = Y;
   p.ldy = ldy;
@@ -988,12 +1043,16 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
   if (!make_map(&ma, values, BF16, R, K / 2, K / 2, kStageKPhys, kBlockM)) return NM_ERR_CUDA;
   if (!make_map(&mb, X, BF16, K, T, ldx, 64, kStageK)) return NM_ERR_CUDA;
   if (pair) {
-    CUtensorMap me;
+    CUtensorMap me, my;
     const int64_t rows16 = ((R + 127) / 128) * int64_t(p.k_blocks) * 128;
     if (!make_map_image(&me, meta_img, rows16)) return NM_ERR_CUDA;
-    if (kern == Kern::Pair256) return launch_pair<256, 4, BF16>(ma, mb, me, p, s);
-    if (kern == Kern::Pair192) return launch_pair<192, 4, BF16>(ma, mb, me, p, s);
-    return launch_pair<128, 6, BF16>(ma, mb, me, p, s);
+    // bf16 output without beta leaves through bulk tensor stores (32 x 32 boxes)
+    p.y_tma = (!y_f32 && beta == 0.0f && p.y_vec) ? 1 : 0;
+    memset(&my, 0, sizeof(my));
+    if (p.y_tma && !make_map(&my, Y, true, R, T, ldy, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return NM_ERR_CUDA;
+    if (kern == Kern::Pair256) return launch_pair<256, 4, BF16>(ma, mb, me, my, p, s);
+    if (kern == Kern::Pair192) return launch_pair<192, 4, BF16>(ma, mb, me, my, p, s);
+    return launch_pair<128, 6, BF16>(ma, mb, me, my, p, s);
   }
   switch (kern) {
     case Kern::Single256: return launch<256, 2, BF16>(ma, X, ldx, K, T, p, s);

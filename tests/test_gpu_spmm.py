@@ -210,3 +210,34 @@ def test_decode_skinny_full_size_sampled_rows(T):
     Y, ref = _run(W, X, torch.bfloat16, rows=rows)
     assert _nerr(Y, ref) <= 8e-3
 
+
+
+KERNELS = ["pair256", "pair192", "pair128", "single256", "single128", "single64", "single64x2",
+           "single32x2", "single16x2"]
+
+
+@pytest.mark.parametrize("kern", KERNELS)
+def test_every_tile_shape_is_exact_on_integers(kern, monkeypatch):
+    """Each tile configuration, forced through NM_SPMM_KERNEL, on a shape
+    ragged in R (700 = 5.5 row tiles) and T (500 columns, a partial last tile
+    for every width): integer inputs make the fp32 output exact and the bf16
+    output its round-to-nearest-even, on both epilogue paths."""
+    monkeypatch.setenv("NM_SPMM_KERNEL", kern)
+    R, K, T = 700, 384, 500
+    W = nm_inputs.small_int((R, K), 81, dtype=torch.bfloat16)
+    X = nm_inputs.small_int((K, T), 82, dtype=torch.bfloat16)
+    Y, ref = _run(W, X, torch.float32)
+    assert np.array_equal(Y.numpy().astype(np.float64), ref)
+    Yb, ref_b = _run(W, X, torch.bfloat16)
+    assert np.array_equal(_bits(Yb), oracle.encode_array(ref_b, oracle.BF16))
+
+
+@pytest.mark.parametrize("kern", KERNELS)
+def test_every_tile_shape_alpha_beta(kern, monkeypatch):
+    monkeypatch.setenv("NM_SPMM_KERNEL", kern)
+    R, K, T = 700, 256, 500
+    W = nm_inputs.normal((R, K), 83, 0.02, torch.bfloat16)
+    X = nm_inputs.normal((K, T), 84, 1.0, torch.bfloat16)
+    Y0 = nm_inputs.normal((R, T), 85, 1.0, torch.bfloat16)
+    Y, ref = _run(W, X, torch.bfloat16, alpha=1.5, beta=0.5, Y0=Y0)
+    assert _nerr(Y, ref) <= 8e-3
