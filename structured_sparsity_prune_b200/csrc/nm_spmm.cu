@@ -340,6 +340,10 @@ struct Params {
   int y_f32;    // 1: fp32 output, 0: bf16 output
   int y_vec;    // 1: Y and ldy allow 16-byte vector stores
   int y_tma;    // 1: bf16 output with beta == 0 leaves through staged bulk tensor stores (pair kernel)
+  // Pair kernel work list: items [0, split_from) are whole tiles; the tiles
+  // from split_from on are each done as two half-width items (the last,
+  // partly filled wave then takes half as long).
+  int split_from, num_work;
   float alpha, beta;
 };
 
@@ -363,6 +367,21 @@ __device__ __forceinline__ void grouped_tile(const Params& p, int t, int& mt, in
     nt = first + local % gn;
     mt = local / gn;
   }
+}
+
+// Work item w of the pair kernel: its tile (mt, nt), first output column and
+// whether it is a half-width item.
+struct PairWork {
+  int mt, nt, col0, narrow;
+};
+__device__ __forceinline__ PairWork pair_work(const Params& p, int w, int n_total) {
+  PairWork k;
+  const bool narrow = w >= p.split_from;
+  const int t = narrow ? p.split_from + ((w - p.split_from) >> 1) : w;
+  grouped_tile(p, t, k.mt, k.nt);
+  k.narrow = narrow ? 1 : 0;
+  k.col0 = k.nt * n_total + (narrow ? ((w - p.split_from) & 1) * (n_total / 2) : 0);
+  return k;
 }
 
 // Epilogue of one 32-column chunk of one output row: y = alpha * acc (+ beta * y_old),
@@ -650,7 +669,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const uint32_t rank = cluster_rank();
   const bool leader = rank == 0;
   const int pair = int(blockIdx.x >> 1), num_pairs = int(gridDim.x >> 1);
-  const int num_tiles = p.m_tiles * p.n_tiles;  // m_tiles counts 256-row tiles here
+  const int num_work = p.num_work;  // m_tiles counts 256-row tiles here
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -672,8 +691,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
-  auto tile_coords = [&](int t, int& mt, int& nt) { grouped_tile(p, t, mt, nt); };
-
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
@@ -681,23 +698,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       uint32_t armed_round[STAGES];
       for (int s = 0; s < STAGES; ++s) armed_round[s] = 0xFFFFFFFFu;
       bool ok = true;
-      for (int t = pair; t < num_tiles && ok; t += num_pairs) {
-        int mt, nt;
-        tile_coords(t, mt, nt);
-        const int row_tile = 2 * mt + int(rank);  // this CTA's 128-row tile
+      for (int w = pair; w < num_work && ok; w += num_pairs) {
+        const PairWork wk = pair_work(p, w, N_TOTAL);
+        const int row_tile = 2 * wk.mt + int(rank);  // this CTA's 128-row tile
+        // a half-width item stages one 64-column B atom per CTA
+        const int b_boxes = wk.narrow ? 1 : C::kBBoxes;
+        const int b_cols = wk.narrow ? 64 : C::kNHalf;
+        const uint32_t tx = 2u * uint32_t(C::kABytes + b_boxes * C::kBBoxBytes + C::kEBytes);
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = int(it % STAGES);
           const uint32_t round = it / STAGES;
           if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag)) { ok = false; break; }
           uint8_t* st = smem + s * C::kStageBytes;
-          if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
+          if (leader) mbar_arrive_expect_tx(&full[s], tx);
           armed_round[s] = round;
           const uint32_t bar = mapa(smem_u32(&full[s]), 0);
           tma_load_2d_pair(st, &map_a, bar, kb * kStageKPhys, row_tile * kBlockM);
 #pragma unroll
           for (int j = 0; j < C::kBBoxes; ++j)
-            tma_load_2d_pair(st + C::kABytes + j * C::kBBoxBytes, &map_b, bar,
-                             nt * N_TOTAL + int(rank) * C::kNHalf + 64 * j, kb * kStageK);
+            if (j < b_boxes)
+              tma_load_2d_pair(st + C::kABytes + j * C::kBBoxBytes, &map_b, bar,
+                               wk.col0 + int(rank) * b_cols + 64 * j, kb * kStageK);
           tma_load_2d_pair(st + C::kABytes + C::kBBytes, &map_e, bar, 0,
                            (row_tile * p.k_blocks + kb) * kBlockM);
         }
@@ -721,10 +742,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && leader) {
-      const uint32_t idesc = make_idesc(BF16, N_TOTAL, 2 * kBlockM);
+      const uint32_t idesc_full = make_idesc(BF16, N_TOTAL, 2 * kBlockM);
+      const uint32_t idesc_narrow = make_idesc(BF16, N_TOTAL / 2, 2 * kBlockM);
       uint32_t it = 0, local = 0;
       bool ok = true;
-      for (int t = pair; t < num_tiles && ok; t += num_pairs, ++local) {
+      for (int w = pair; w < num_work && ok; w += num_pairs, ++local) {
+        const uint32_t idesc = w >= p.split_from ? idesc_narrow : idesc_full;
         const int buf = int(local % C::kAccBufs);
         const uint32_t use = local / C::kAccBufs;
         if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
@@ -776,21 +799,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const bool early = !p.y_f32 && p.beta == 0.0f && p.y_vec;
     const uint32_t out_slot = smem_u32(smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes);
     uint32_t local = 0;
-    for (int t = pair; t < num_tiles; t += num_pairs, ++local) {
-      int mt, nt;
-      tile_coords(t, mt, nt);
+    for (int w = pair; w < num_work; w += num_pairs, ++local) {
+      const PairWork wk = pair_work(p, w, N_TOTAL);
+      const int mt = wk.mt;
+      // columns of this warp: kc of them (kCols, or half that for a half-width
+      // item); loops below run to kCols with steps past kc skipped, so the
+      // register arrays keep compile-time indexes
+      const int kc = wk.narrow ? kCols / 2 : kCols;
       const int buf = int(local % C::kAccBufs);
       const uint32_t use = local / C::kAccBufs;
       const bool ok = mbar_wait(&acc_full[buf], use & 1u, abort_flag);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       fence_after_sync();
       const int r = (2 * mt + int(rank)) * kBlockM + row_in_tile;
-      const int c_base = nt * N_TOTAL + half * kCols;
-      const uint32_t taddr = tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TOTAL + half * kCols);
+      const int c_base = wk.col0 + half * kc;
+      const uint32_t taddr = tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TOTAL + half * kc);
       if (early) {
         uint32_t packed[kCols / 2];
 #pragma unroll
         for (int c = 0; c < kCols; c += 64) {
+          if (c >= kc) break;
           uint32_t v0[32], v1[32];
           tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c), v0);
           if (c + 64 <= kCols) tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c + 32), v1);
@@ -818,6 +846,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           const int row0 = (2 * mt + int(rank)) * kBlockM + 32 * q;
 #pragma unroll
           for (int c = 0; c < kCols; c += 32) {
+            if (c >= kc) break;
             if (lane == 0) bulk_wait_read_all();  // the slot's previous store has read it
             __syncwarp();
 #pragma unroll
@@ -835,6 +864,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(p.Y) + size_t(r) * p.ldy;
 #pragma unroll
           for (int c = 0; c < kCols; c += 8) {
+            if (c >= kc) break;
             const int col = c_base + c;
             if (col + 8 <= p.T) {
               *reinterpret_cast<uint4*>(yrow + col) =
@@ -853,7 +883,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < kCols; c += 32) {
+        for (int c = 0; c < kc; c += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(taddr + uint32_t(c), v);
           store_chunk(p, r, c_base + c, v);
@@ -955,6 +985,12 @@ bool make_map_image(CUtensorMap* map, const uint8_t* img, int64_t rows16) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// NM_SPMM_TAIL_SPLIT=0 turns the half-width last wave off (for comparison).
+bool split_tail_enabled() {
+  const char* e = getenv("NM_SPMM_TAIL_SPLIT");
+  return !(e && e[0] == '0');
+}
+
 template <int N_TOTAL, int STAGES, bool BF16>
 nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me, const CUtensorMap& my,
                       const Params& p, cudaStream_t s) {
@@ -966,10 +1002,20 @@ nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
       return NM_ERR_CUDA;
     attr_done = true;
   }
-  const int pairs = p.m_tiles * p.n_tiles;
+  const int tiles = p.m_tiles * p.n_tiles;
   const int max_pairs = sm_count() / 2;
-  const int grid = 2 * (pairs < max_pairs ? pairs : max_pairs);
-  kern<<<grid, kPairThreads, C::kSmemBytes, s>>>(ma, mb, me, my, p);
+  const int pairs = tiles < max_pairs ? tiles : max_pairs;
+  Params q = p;
+  q.split_from = tiles;
+  q.num_work = tiles;
+  // A last wave that fills at most half of the pairs is done in half-width
+  // items (whole 64-column B atoms per CTA, so only for 256-column tiles).
+  const int rem = tiles % pairs;
+  if (N_TOTAL == 256 && tiles > pairs && rem > 0 && 2 * rem <= pairs && split_tail_enabled()) {
+    q.split_from = tiles - rem;
+    q.num_work = tiles + rem;
+  }
+  kern<<<2 * pairs, kPairThreads, C::kSmemBytes, s>>>(ma, mb, me, my, q);
   return launch_status();
 }
 

@@ -241,3 +241,31 @@ def test_every_tile_shape_alpha_beta(kern, monkeypatch):
     Y0 = nm_inputs.normal((R, T), 85, 1.0, torch.bfloat16)
     Y, ref = _run(W, X, torch.bfloat16, alpha=1.5, beta=0.5, Y0=Y0)
     assert _nerr(Y, ref) <= 8e-3
+
+
+@pytest.mark.parametrize("R,T", [(2560, 2048), (2500, 2000)])
+def test_half_width_last_wave_is_exact(R, T, monkeypatch):
+    """80 pair tiles on 74 pairs: the last 6 tiles run as 12 half-width items
+    (ragged in R and T in the second case); integer inputs make the fp32
+    output exact and the bf16 output its round-to-nearest-even."""
+    monkeypatch.setenv("NM_SPMM_KERNEL", "pair256")
+    K = 128
+    W = nm_inputs.small_int((R, K), 91, dtype=torch.bfloat16)
+    X = nm_inputs.small_int((K, T), 92, dtype=torch.bfloat16)
+    Y, ref = _run(W, X, torch.float32)
+    assert np.array_equal(Y.numpy().astype(np.float64), ref)
+    Yb, ref_b = _run(W, X, torch.bfloat16)
+    assert np.array_equal(_bits(Yb), oracle.encode_array(ref_b, oracle.BF16))
+
+
+def test_half_width_last_wave_matches_whole_tiles(monkeypatch):
+    """Splitting the last wave does not change the summation order, so the
+    result equals the unsplit run bit for bit."""
+    W = nm_inputs.normal((4096, 1024), 93, 0.02, torch.bfloat16).cuda()
+    X = nm_inputs.normal((1024, 4096), 94, 1.0, torch.bfloat16).cuda()
+    values, meta, img = nm.nm_mask_compress(W)
+    a = nm.nm_spmm(values, img, X)
+    monkeypatch.setenv("NM_SPMM_TAIL_SPLIT", "0")
+    b = nm.nm_spmm(values, img, X)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
