@@ -19,6 +19,12 @@ linear/conv weights; the pages' datasets and trained weights are not used):
                       X bf16 8192xT ~N(0,1) (seed 105+T), T in {16,64,256,1024}
 * ``srste``           the linear_4096 weight and a gradient bf16(1e-3 * N(0,1))
                       of the same shape (seed 6)
+* ``saliency``        the linear_4096 weight and d of length 4096: the diagonal
+                      of the upper Cholesky factor of H^-1, H = (2/n) X^T X +
+                      0.01 * mean(diag) * I from n = 512 synthetic calibration
+                      rows X ~ N(0,1) (seed 7), prepared in float64 the way
+                      "sparsegpt.py" prepares its inverse Hessian, then
+                      rounded to float32.  This stands in for calibration data.
 """
 from __future__ import annotations
 
@@ -31,6 +37,7 @@ SEEDS = {
     "ties_fp32.W": 4,
     "decode_skinny.W": 5,
     "srste.grad": 6,
+    "saliency.X": 7,
 }
 
 
@@ -95,3 +102,15 @@ def bits_u16(t: torch.Tensor):
 
 def srste_grad(shape=(4096, 4096)):
     return normal(shape, SEEDS["srste.grad"], 1e-3, torch.bfloat16)
+
+
+def saliency_d(C: int = 4096, n: int = 512, seed: int | None = None) -> torch.Tensor:
+    """float32 vector of length C: diag of the upper Cholesky factor of the
+    inverse of a damped synthetic Gram matrix (see the module docstring)."""
+    g = _gen(SEEDS["saliency.X"] if seed is None else seed)
+    X = torch.randn(n, C, generator=g, dtype=torch.float64)
+    H = (2.0 / n) * (X.T @ X)
+    H.diagonal().add_(0.01 * H.diagonal().mean())
+    Hinv = torch.cholesky_inverse(torch.linalg.cholesky(H))
+    U = torch.linalg.cholesky(Hinv, upper=True)
+    return U.diagonal().to(torch.float32).contiguous()

@@ -46,7 +46,7 @@ def build(force: bool = False) -> str:
     """Compile nm_oracle.c into liboracle.so next to it (gcc, -O2)."""
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
         tmp = _LIB + ".tmp.%d" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fPIC", "-shared", "-pthread",
                                "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
@@ -80,6 +80,8 @@ def _load():
     lib.oracle_spmm.restype = i32
     lib.oracle_rows_parallel.argtypes = [i32, vp, i32, i64, i64, i32, i32, vp, vp, vp, i32]
     lib.oracle_rows_parallel.restype = i32
+    lib.oracle_mask_scored.argtypes = [vp, i32, vp, i64, i64, i64, i32, i32, vp, i64]
+    lib.oracle_mask_scored.restype = i32
     lib.oracle_srste.argtypes = [vp, vp, i32, i64, i64, i32, i32, ctypes.c_float, vp, vp, vp]
     lib.oracle_srste.restype = i32
     _lib = lib
@@ -149,6 +151,20 @@ def mask_rank(W: np.ndarray, N: int, M: int, dtype: int | None = None) -> np.nda
     mask = np.zeros((R, C), dtype=np.uint8)
     _check(_load().oracle_mask_rank(Wb.ctypes.data, code, R, C, C, N, M, mask.ctypes.data, C),
            "mask_rank")
+    return mask
+
+
+def mask_scored(W: np.ndarray, d: np.ndarray, N: int, M: int, dtype: int | None = None) -> np.ndarray:
+    """Saliency-scored N:M mask: keep the N largest binary32 scores w^2 / d^2
+    of each group ("sparsegpt.py", fasterprune, semi-structured branch)."""
+    code = dtype_code(W, dtype)
+    Wb = _bits(W, code)
+    R, C = Wb.shape
+    dv = np.ascontiguousarray(d, dtype=np.float32).ravel()
+    assert dv.size == C
+    mask = np.zeros((R, C), dtype=np.uint8)
+    _check(_load().oracle_mask_scored(Wb.ctypes.data, code, dv.ctypes.data, R, C, C, N, M, mask.ctypes.data, C),
+           "mask_scored")
     return mask
 
 

@@ -22,6 +22,11 @@
  *           "Structured sparse GEMM on tensor cores" (sparse x dense =
  *           dense), "Network pruning workflow, Step-2" (drop the two
  *           smallest of every 4).
+ *  [SPGPT]  "sparsegpt.py" source page (ken1301225.github.io, code_math
+ *           articles): fasterprune, semi-structured branch (prunen of
+ *           every prunem columns pruned by the score w^2 / d^2, d the
+ *           diagonal of the upper Cholesky factor of the damped inverse
+ *           Hessian; weights and Hessian in float32).
  *  [PTX]    NVIDIA PTX ISA, tcgen05 "Sparse matrices" (metadata of
  *           .kind::f16 sparse MMA in tensor memory) -- the pages give no
  *           hardware layout; this is the public ISA description.
@@ -35,8 +40,10 @@
  *  - Ties: equal magnitude -> the lower in-group index is kept.
  *  - decompress writes +0.0 at pruned positions.
  *
- * Floating point: the only arithmetic is in oracle_spmm, done in double
- * from exactly-decoded inputs.  Mask selection uses exact integers.
+ * Floating point: oracle_spmm works in double from exactly-decoded
+ * inputs; oracle_srste's decay term and oracle_mask_scored's scores are
+ * binary32, as their sources compute them.  Magnitude masks use exact
+ * integers.
  */
 #include <stdint.h>
 #include <stddef.h>
@@ -168,6 +175,54 @@ int oracle_mask_rank(const void *W, int dtype, int64_t R, int64_t C, int64_t ldw
                 for (int j = 0; j < M; ++j) {
                     if (j == i) continue;
                     if (mag[j] > mag[i] || (mag[j] == mag[i] && j < i)) beaten_by++;
+                }
+                mask[r * ldm + g * M + i] = (uint8_t)(beaten_by < N ? 1 : 0);
+            }
+        }
+    }
+    return OR_OK;
+}
+
+/* --------------------------------------------------------------------- */
+/* Saliency-scored mask.  [SPGPT] semi-structured branch: inside every    */
+/* group of M consecutive columns the score of w is w^2 / d^2, with d the */
+/* entry of its column in the caller's vector (the diagonal of the upper  */
+/* Cholesky factor of the inverse Hessian there), and the M-N smallest    */
+/* scores are pruned (topk with largest=False).  In binary32, as there:   */
+/*   s = fl( fl(w*w) / fl(d*d) )                                          */
+/* each product and the quotient rounded once to nearest even.  Scores    */
+/* are ranked by their bit pattern with the sign cleared (the magnitude   */
+/* order above; 0/0 gives NaN, which ranks highest); equal scores keep    */
+/* the lower in-group index.                                              */
+/* --------------------------------------------------------------------- */
+static uint32_t f32_bits(float x)
+{
+    uint32_t u;
+    memcpy(&u, &x, sizeof u);
+    return u;
+}
+
+int oracle_mask_scored(const void *W, int dtype, const float *d, int64_t R, int64_t C, int64_t ldw,
+                       int N, int M, uint8_t *mask, int64_t ldm)
+{
+    if (M < 2 || M > 8 || N < 1 || N >= M || C % M != 0 || R < 0 || C < 0)
+        return OR_BAD_ARG;
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t g = 0; g < C / M; ++g) {
+            uint32_t key[8];
+            for (int i = 0; i < M; ++i) {
+                const int64_t c = g * M + i;
+                const float w = (float)oracle_decode(load_bits(W, dtype, (size_t)(r * ldw + c)), dtype);
+                volatile float ww = w * w;          /* binary32, rounded once */
+                volatile float dd = d[c] * d[c];
+                volatile float sc = ww / dd;
+                key[i] = f32_bits(sc) & 0x7FFFFFFFu;
+            }
+            for (int i = 0; i < M; ++i) {
+                int beaten_by = 0;
+                for (int j = 0; j < M; ++j) {
+                    if (j == i) continue;
+                    if (key[j] > key[i] || (key[j] == key[i] && j < i)) beaten_by++;
                 }
                 mask[r * ldm + g * M + i] = (uint8_t)(beaten_by < N ? 1 : 0);
             }
