@@ -1,7 +1,8 @@
 """Benchmark of the N:M sparsity hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload linear_4096|mlp_pair|decode_T16|decode_T64|decode_T256|decode_T1024|ties_mask]
+                    [--workload linear_4096|mlp_pair|decode_T16|decode_T64|decode_T256|decode_T1024|ties_mask|
+                               srste|saliency_mask]
 
 One step is one pass of every step of the path over one batch of synthetic
 input (default: the transformer-linear workload, bf16 W 4096x4096 pruned 2:4
@@ -94,6 +95,11 @@ def make_workload(name: str):
         W, _ = nm_inputs.linear_4096()
         return {"W": W, "G": nm_inputs.srste_grad(), "X": None, "R": 4096, "K": 4096, "T": 0,
                 "desc": "SR-STE step: bf16 W 4096x4096 ~N(0,0.02) and bf16 gradient ~N(0,1e-3); 2:4, decay 0.0002"}
+    elif name == "saliency_mask":
+        W = nm_inputs.decode_skinny_W()
+        return {"W": W, "D": nm_inputs.saliency_d(W.shape[1]), "X": None, "R": W.shape[0], "K": W.shape[1], "T": 0,
+                "desc": "saliency-scored 2:4 mask: bf16 W 28672x8192 ~N(0,0.02); d = diag of the upper Cholesky factor"
+                        " of the inverse of a damped synthetic Gram matrix (512 calibration rows ~N(0,1))"}
     elif name == "ties_mask":
         W = nm_inputs.ties_fp32()
         return {"W": W, "X": None, "R": 8192, "K": 8192, "T": 0,
@@ -184,8 +190,16 @@ class Step:
     def __init__(self, nm, wl, dev):
         self.nm, self.wl, self.dev = nm, wl, dev
         R, K, T = wl["R"], wl["K"], wl["T"]
-        self.kind = "srste" if "G" in wl else ("ties" if wl["X"] is None else ("mlp" if "W2" in wl else "linear"))
+        self.kind = "srste" if "G" in wl else "scored" if "D" in wl else \
+            ("ties" if wl["X"] is None else ("mlp" if "W2" in wl else "linear"))
         self.W = wl["W"].to(dev)
+        if self.kind == "scored":
+            self.D = wl["D"].to(dev)
+            self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
+            self.names = ["nm_mask_scored"]
+            self.bytes = {"nm_mask_scored": R * K * (self.W.element_size() + 1) + K * 4}
+            self.flops = 0
+            return
         if self.kind == "srste":
             self.G = wl["G"].to(dev)
             self.WS = torch.empty_like(self.W)
@@ -250,6 +264,9 @@ class Step:
         if self.kind == "srste":
             nm.nm_srste_step(self.W, self.G, 2, 4, 0.0002, W_sparse=self.WS, grad_out=self.GO, mask=self.mask)
             rec(1)
+        elif self.kind == "scored":
+            nm.nm_mask_scored(self.W, self.D, 2, 4, mask=self.mask)
+            rec(1)
         elif self.kind == "ties":
             for i, (N, M) in enumerate([(1, 4), (2, 4), (4, 8), (2, 8)]):
                 nm.nm_mask(self.W, N, M, mask=self.masks[i])
@@ -281,6 +298,8 @@ class Step:
     def result(self):
         if self.kind == "srste":
             return self.GO
+        if self.kind == "scored":
+            return self.mask
         return self.masks[1] if self.kind == "ties" else self.Y
 
 
@@ -311,6 +330,9 @@ def e2e_steps(step: Step, steps: int, flush: torch.Tensor):
     if "G" in step.wl:
         G_h = step.wl["G"].pin_memory()
         h2d += G_h.numel() * G_h.element_size()
+    if "D" in step.wl:
+        D_h = step.wl["D"].pin_memory()
+        h2d += D_h.numel() * D_h.element_size()
     d2h = out_h.numel() * out_h.element_size()
     s = torch.cuda.current_stream()
     times = []
@@ -325,6 +347,8 @@ def e2e_steps(step: Step, steps: int, flush: torch.Tensor):
             step.W2.copy_(W2_h, non_blocking=True)
         if "G" in step.wl:
             step.G.copy_(G_h, non_blocking=True)
+        if "D" in step.wl:
+            step.D.copy_(D_h, non_blocking=True)
         step.run()
         out_h.copy_(res, non_blocking=True)
         b.record(s)
@@ -348,6 +372,12 @@ def oracle_step(wl, rows: int, threads: int):
         t0 = time.perf_counter()
         oracle.srste(Wb, Gb, 2, 4, 0.0002, dtype=oracle.BF16)
         return time.perf_counter() - t0, float(rows * wl["K"] * 9)
+    if "D" in wl:                 # saliency-scored mask
+        Wb = _u16(wl["W"][:rows].contiguous())
+        d = wl["D"].numpy()
+        t0 = time.perf_counter()
+        oracle.mask_scored(Wb, d, 2, 4, dtype=oracle.BF16)
+        return time.perf_counter() - t0, float(rows * wl["K"] * 3)
     if wl["X"] is None:           # mask-only workload
         W = wl["W"][:rows].contiguous().numpy()
         t0 = time.perf_counter()
@@ -393,6 +423,7 @@ def cpu_baseline(wl, target_s: float = 15.0):
     secs, units = oracle_step(wl, rows, threads)
     scale, unit = (1e12, "TFLOP/s") if wl["X"] is not None else (1e9, "GB/s")
     what = ("SR-STE step (mask, masked weight, decay gradient)" if "G" in wl else
+            "saliency-scored 2:4 mask" if "D" in wl else
             "mask at 1:4, 2:4, 4:8, 2:8" if wl["X"] is None else
             "whole step (mask, compress, fused mask+compress, image, decompress, fp64 product)")
     return {"value": units / secs / scale, "unit": unit, "cores": threads, "kind": "oracle",
@@ -416,7 +447,9 @@ def run_reference(args, wl, metric):
     sample = "first %d of %d rows of W per step, whole step on the CPU oracle" % (rows, wl["R"])
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / max(1, args.steps), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "data": "synthetic",
+            # the oracle's arithmetic: fp64 product, binary32 decay term / scores, integer magnitude keys
+            "dtype": "f64" if wl["X"] is not None else ("f32" if ("G" in wl or "D" in wl) else "u32"),
             "config": {"workload": args.workload, "desc": wl["desc"], "R": wl["R"], "K": wl["K"], "T": wl["T"]},
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample},
@@ -506,11 +539,11 @@ def main():
             k.update({"TFLOP/s": tf, "tensor_frac": tf / sparse_peak})
         kernels[name] = k
 
-    if step.kind in ("ties", "srste"):
+    if step.kind in ("ties", "srste", "scored"):
         units_per_step = sum(step.bytes.values())
         value = world * units_per_step * args.steps / (total_ms * 1e-3) / 1e9
         unit = "GB/s"
-        dom = "nm_mask_2:4" if step.kind == "ties" else "nm_srste_step"
+        dom = {"ties": "nm_mask_2:4", "srste": "nm_srste_step", "scored": "nm_mask_scored"}[step.kind]
         roof = {"bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": hbm, "unit": "GB/s",
                 "frac": kernels[dom]["GB/s"] / hbm, "kernel": dom,
                 "algorithmic_bytes_per_launch": step.bytes[dom]}

@@ -105,6 +105,27 @@ NM_API nm_status nm_mask(const void *W, nm_dtype dtype, int64_t R, int64_t C, in
                   int N, int M, uint8_t *mask, int64_t ldm, void *stream);
 
 /*
+ * nm_mask_scored -- saliency-scored N:M mask.  Source: "sparsegpt.py"
+ * (fasterprune, semi-structured branch): inside every group of M
+ * consecutive columns the score of w is w^2 / d^2, with d the entry of its
+ * column in the diagonal of the upper Cholesky factor of the damped inverse
+ * Hessian, and the M-N smallest scores are pruned.  Here d is any
+ * caller-supplied vector and the score is evaluated in binary32 as in that
+ * listing, s = fl(fl(w*w) / fl(d[c]*d[c])), each operation rounded once to
+ * nearest even.  mask = 1 at the N largest scores of each group, ranked by
+ * the bit pattern of s with the sign cleared (0/0 gives NaN, which ranks
+ * highest); equal scores keep the lower in-group index.  The weight update
+ * of that listing is not part of this call.
+ *   W     R x C, dtype NM_F32 / NM_BF16 / NM_F16, leading dim ldw >= C
+ *   d     C floats (device), 16-byte aligned
+ *   mask  R x C uint8 (0 or 1), leading dim ldm >= C
+ *   1 <= N < M <= 8, C % M == 0 (else NM_ERR_NM / NM_ERR_SHAPE);
+ *   NM_ERR_NULL for a null W, d or mask, NM_ERR_ALIGN as nm_mask or for d
+ */
+NM_API nm_status nm_mask_scored(const void *W, nm_dtype dtype, const float *d, int64_t R, int64_t C,
+                         int64_t ldw, int N, int M, uint8_t *mask, int64_t ldm, void *stream);
+
+/*
  * nm_mask_compress -- fused 2:4 mask + compression in one pass over W:
  * the 2:4 mask of nm_mask, then the kept values and their indices in the
  * canonical layout and (if meta_sm100 != NULL) in the tensor-core image.

@@ -47,6 +47,7 @@ def _lib():
         "nm_version": ([], i32),
         "nm_sizes": ([i64, i64, i32, i32, i32, vp, vp, vp], i32),
         "nm_mask": ([vp, i32, i64, i64, i64, i32, i32, vp, i64, vp], i32),
+        "nm_mask_scored": ([vp, i32, vp, i64, i64, i64, i32, i32, vp, i64, vp], i32),
         "nm_mask_compress": ([vp, i32, i64, i64, i64, vp, vp, vp, vp], i32),
         "nm_compress": ([vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp, vp], i32),
         "nm_decompress": ([vp, vp, i32, i64, i64, vp, i64, vp], i32),
@@ -117,6 +118,19 @@ def nm_mask(W: torch.Tensor, N: int, M: int, mask: torch.Tensor | None = None, s
     if mask is None:
         mask = torch.empty((R, C), dtype=torch.uint8, device=W.device)
     _check(_lib().nm_mask(_ptr(W), _dtype(W), R, C, _ld(W), N, M, _ptr(mask), _ld(mask), _stream(stream)), "nm_mask")
+    return mask
+
+
+def nm_mask_scored(W: torch.Tensor, d: torch.Tensor, N: int, M: int, mask: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """Saliency-scored N:M mask; d: fp32 device vector of length W.shape[1]."""
+    R, C = W.shape
+    if d.dtype != torch.float32 or d.numel() != C or not d.is_contiguous():
+        raise NMError(2, "nm_mask_scored: d must be a contiguous float32 vector of length C")
+    if mask is None:
+        mask = torch.empty((R, C), dtype=torch.uint8, device=W.device)
+    _check(_lib().nm_mask_scored(_ptr(W), _dtype(W), _ptr(d), R, C, _ld(W), N, M, _ptr(mask), _ld(mask),
+                                 _stream(stream)), "nm_mask_scored")
     return mask
 
 
