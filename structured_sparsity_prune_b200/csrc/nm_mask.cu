@@ -143,10 +143,20 @@ __global__ void __launch_bounds__(256) scored_vec16_kernel(const Bits* __restric
       const float4 t = __ldg(d4 + c * 4 + i);
       dv[4 * i] = t.x; dv[4 * i + 1] = t.y; dv[4 * i + 2] = t.z; dv[4 * i + 3] = t.w;
     }
-    for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+    int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y;
+    uint4 nxt[kVec];
+    if (r < R) {
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) nxt[i] = __ldcs(reinterpret_cast<const uint4*>(W + r * ldw) + c * kVec + i);
+    }
+    for (; r < R; r += r_step) {
       uint4 v[kVec];
 #pragma unroll
-      for (int i = 0; i < kVec; ++i) v[i] = __ldcs(reinterpret_cast<const uint4*>(W + r * ldw) + c * kVec + i);
+      for (int i = 0; i < kVec; ++i) v[i] = nxt[i];
+      if (r + r_step < R) {   // prefetch the next row's chunk before working on this one
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) nxt[i] = __ldcs(reinterpret_cast<const uint4*>(W + (r + r_step) * ldw) + c * kVec + i);
+      }
       const Bits* e = reinterpret_cast<const Bits*>(v);
       uint32_t out[4] = {0u, 0u, 0u, 0u};
       if constexpr (M == 4) {

@@ -67,10 +67,18 @@ def test_zero_d_and_zero_weights():
 
 
 def test_scalar_path_when_c_is_not_a_multiple_of_16():
-    W = nm_inputs.normal((130, 36), 71, 1.0, torch.bfloat16)
-    d = nm_inputs.normal((36,), 72).abs() + 0.1
-    _check(W, d, 2, 4)
-    _check(W, d, 1, 3)
+    """C = 40 (not a multiple of 16) takes the per-group path; rows of W and
+    of the mask sit in buffers padded to 16-byte row strides."""
+    C = 40
+    Wfull = nm_inputs.normal((130, 48), 71, 1.0, torch.bfloat16).cuda()
+    W = Wfull[:, :C]
+    d = (nm_inputs.normal((C,), 72).abs() + 0.1).cuda()
+    for N, M in [(2, 4), (1, 5), (3, 8)]:
+        mfull = torch.full((130, 48), 9, dtype=torch.uint8, device="cuda")
+        nm.nm_mask_scored(W, d, N, M, mask=mfull[:, :C])
+        ref = oracle.mask_scored(_bits(W.contiguous()), d.cpu().numpy(), N, M, dtype=oracle.BF16)
+        assert np.array_equal(mfull[:, :C].cpu().numpy(), ref)
+        assert torch.all(mfull[:, C:] == 9)
 
 
 def test_strided_rows():
@@ -107,3 +115,16 @@ def test_argument_errors():
     assert lib.nm_mask_scored(W.data_ptr(), 1, d.data_ptr() + 4, 8, 16, 16, 2, 4, m.data_ptr(), 16, s) == 3  # ALIGN
     assert lib.nm_mask_scored(W.data_ptr(), 1, d.data_ptr(), 8, 16, 16, 4, 4, m.data_ptr(), 16, s) == 5  # NM_ERR_NM
     assert lib.nm_mask_scored(W.data_ptr(), 1, d.data_ptr(), 8, 15, 16, 2, 4, m.data_ptr(), 16, s) == 2  # SHAPE
+
+
+@pytest.mark.parametrize("N,M", [(2, 4), (1, 4), (4, 8)])
+def test_scores_one_ulp_apart(N, M):
+    """w = c * d in binary32: every score of a group is c^2 up to the rounding
+    of the two squares and the quotient, so scores tie or differ by an ulp or
+    two and the mask depends on every quotient's last bit."""
+    g = torch.Generator().manual_seed(76)
+    R, C = 1024, 512
+    d = (torch.rand(C, generator=g) * 3.5 + 0.5).float()
+    c = (torch.rand(R, 1, generator=g) * 2.0 + 0.01).float()
+    W = (c * d[None, :]).float()
+    _check(W, d, N, M)
