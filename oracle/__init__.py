@@ -80,6 +80,8 @@ def _load():
     lib.oracle_spmm.restype = i32
     lib.oracle_rows_parallel.argtypes = [i32, vp, i32, i64, i64, i32, i32, vp, vp, vp, i32]
     lib.oracle_rows_parallel.restype = i32
+    lib.oracle_mask_transposable.argtypes = [vp, i32, i64, i64, i64, i32, i32, vp, i64]
+    lib.oracle_mask_transposable.restype = i32
     lib.oracle_mask_scored.argtypes = [vp, i32, vp, i64, i64, i64, i32, i32, vp, i64]
     lib.oracle_mask_scored.restype = i32
     lib.oracle_srste.argtypes = [vp, vp, i32, i64, i64, i32, i32, ctypes.c_float, vp, vp, vp]
@@ -165,6 +167,18 @@ def mask_scored(W: np.ndarray, d: np.ndarray, N: int, M: int, dtype: int | None 
     mask = np.zeros((R, C), dtype=np.uint8)
     _check(_load().oracle_mask_scored(Wb.ctypes.data, code, dv.ctypes.data, R, C, C, N, M, mask.ctypes.data, C),
            "mask_scored")
+    return mask
+
+
+def mask_transposable(W: np.ndarray, N: int, M: int, dtype: int | None = None) -> np.ndarray:
+    """Greedy transposable N:M mask over MxM blocks (at most N kept per row
+    and per column of every block), as described in the oracle source."""
+    code = dtype_code(W, dtype)
+    Wb = _bits(W, code)
+    R, C = Wb.shape
+    mask = np.zeros((R, C), dtype=np.uint8)
+    _check(_load().oracle_mask_transposable(Wb.ctypes.data, code, R, C, C, N, M, mask.ctypes.data, C),
+           "mask_transposable")
     return mask
 
 

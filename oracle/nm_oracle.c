@@ -27,6 +27,11 @@
  *           every prunem columns pruned by the score w^2 / d^2, d the
  *           diagonal of the upper Cholesky factor of the damped inverse
  *           Hessian; weights and Hessian in float32).
+ *  [TRANS]  nubint.ai review of "Accelerated Sparse Neural Training: A
+ *           Provable and Efficient Method to Find N:M Transposable Masks":
+ *           in every MxM block keep the largest L1 norm with N non-zeros
+ *           per row and per column (W and W^T both N:M); an exact min-cost
+ *           flow and a fast greedy 2-approximation.
  *  [PTX]    NVIDIA PTX ISA, tcgen05 "Sparse matrices" (metadata of
  *           .kind::f16 sparse MMA in tensor memory) -- the pages give no
  *           hardware layout; this is the public ISA description.
@@ -225,6 +230,60 @@ int oracle_mask_scored(const void *W, int dtype, const float *d, int64_t R, int6
                     if (key[j] > key[i] || (key[j] == key[i] && j < i)) beaten_by++;
                 }
                 mask[r * ldm + g * M + i] = (uint8_t)(beaten_by < N ? 1 : 0);
+            }
+        }
+    }
+    return OR_OK;
+}
+
+/* --------------------------------------------------------------------- */
+/* Transposable N:M mask, greedy.  [TRANS]: inside every MxM block (rows  */
+/* r0..r0+M-1, columns c0..c0+M-1) the mask should keep as much |w| as     */
+/* possible with at most N kept entries in each row and in each column,    */
+/* so that W and its transpose are both N:M.  The page names a fast        */
+/* 2-approximation without printing it; the reading here is the standard   */
+/* greedy for this weighted b-matching:                                    */
+/*   1. order the M*M entries by magnitude (as oracle_mag), largest first, */
+/*      equal magnitudes by row-major position within the block;           */
+/*   2. walk that order and keep an entry when its row and its column each */
+/*      hold fewer than N kept entries.                                    */
+/* The result keeps at least half of the optimum's |w| (each optimal entry */
+/* left out is blocked by a kept entry at least as large in its row or     */
+/* column, and each kept entry blocks at most two such).                   */
+/* --------------------------------------------------------------------- */
+typedef struct { uint32_t key; int pos; } tr_entry;
+
+static int tr_cmp(const void *pa, const void *pb)
+{
+    const tr_entry *a = (const tr_entry *)pa, *b = (const tr_entry *)pb;
+    if (a->key != b->key) return a->key > b->key ? -1 : 1;   /* larger magnitude first */
+    return a->pos - b->pos;                                  /* then lower position    */
+}
+
+int oracle_mask_transposable(const void *W, int dtype, int64_t R, int64_t C, int64_t ldw,
+                             int N, int M, uint8_t *mask, int64_t ldm)
+{
+    if (M < 2 || M > 8 || N < 1 || N >= M || R % M != 0 || C % M != 0 || R < 0 || C < 0)
+        return OR_BAD_ARG;
+    for (int64_t br = 0; br < R / M; ++br) {
+        for (int64_t bc = 0; bc < C / M; ++bc) {
+            tr_entry e[64];
+            int row_kept[8] = {0}, col_kept[8] = {0};
+            for (int i = 0; i < M; ++i)
+                for (int j = 0; j < M; ++j) {
+                    const int64_t r = br * M + i, c = bc * M + j;
+                    e[i * M + j].key = oracle_mag(load_bits(W, dtype, (size_t)(r * ldw + c)), dtype);
+                    e[i * M + j].pos = i * M + j;
+                    mask[r * ldm + c] = 0;
+                }
+            qsort(e, (size_t)(M * M), sizeof e[0], tr_cmp);
+            for (int t = 0; t < M * M; ++t) {
+                const int i = e[t].pos / M, j = e[t].pos % M;
+                if (row_kept[i] < N && col_kept[j] < N) {
+                    row_kept[i]++;
+                    col_kept[j]++;
+                    mask[(br * M + i) * ldm + bc * M + j] = 1;
+                }
             }
         }
     }
