@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload linear_4096|mlp_pair|decode_T16|decode_T64|decode_T256|decode_T1024|ties_mask|
-                               srste|saliency_mask]
+                               srste|saliency_mask|transposable_mask]
 
 One step is one pass of every step of the path over one batch of synthetic
 input (default: the transformer-linear workload, bf16 W 4096x4096 pruned 2:4
@@ -100,6 +100,10 @@ def make_workload(name: str):
         return {"W": W, "D": nm_inputs.saliency_d(W.shape[1]), "X": None, "R": W.shape[0], "K": W.shape[1], "T": 0,
                 "desc": "saliency-scored 2:4 mask: bf16 W 28672x8192 ~N(0,0.02); d = diag of the upper Cholesky factor"
                         " of the inverse of a damped synthetic Gram matrix (512 calibration rows ~N(0,1))"}
+    elif name == "transposable_mask":
+        W, _ = nm_inputs.linear_4096()
+        return {"W": W, "TM": (4, 8), "X": None, "R": 4096, "K": 4096, "T": 0,
+                "desc": "greedy transposable 4:8 mask over 8x8 blocks: bf16 W 4096x4096 ~N(0,0.02)"}
     elif name == "ties_mask":
         W = nm_inputs.ties_fp32()
         return {"W": W, "X": None, "R": 8192, "K": 8192, "T": 0,
@@ -190,9 +194,15 @@ class Step:
     def __init__(self, nm, wl, dev):
         self.nm, self.wl, self.dev = nm, wl, dev
         R, K, T = wl["R"], wl["K"], wl["T"]
-        self.kind = "srste" if "G" in wl else "scored" if "D" in wl else \
+        self.kind = "srste" if "G" in wl else "scored" if "D" in wl else "transposable" if "TM" in wl else \
             ("ties" if wl["X"] is None else ("mlp" if "W2" in wl else "linear"))
         self.W = wl["W"].to(dev)
+        if self.kind == "transposable":
+            self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
+            self.names = ["nm_mask_transposable"]
+            self.bytes = {"nm_mask_transposable": R * K * (self.W.element_size() + 1)}
+            self.flops = 0
+            return
         if self.kind == "scored":
             self.D = wl["D"].to(dev)
             self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
@@ -267,6 +277,9 @@ class Step:
         elif self.kind == "scored":
             nm.nm_mask_scored(self.W, self.D, 2, 4, mask=self.mask)
             rec(1)
+        elif self.kind == "transposable":
+            nm.nm_mask_transposable(self.W, *self.wl["TM"], mask=self.mask)
+            rec(1)
         elif self.kind == "ties":
             for i, (N, M) in enumerate([(1, 4), (2, 4), (4, 8), (2, 8)]):
                 nm.nm_mask(self.W, N, M, mask=self.masks[i])
@@ -298,7 +311,7 @@ class Step:
     def result(self):
         if self.kind == "srste":
             return self.GO
-        if self.kind == "scored":
+        if self.kind in ("scored", "transposable"):
             return self.mask
         return self.masks[1] if self.kind == "ties" else self.Y
 
@@ -372,6 +385,12 @@ def oracle_step(wl, rows: int, threads: int):
         t0 = time.perf_counter()
         oracle.srste(Wb, Gb, 2, 4, 0.0002, dtype=oracle.BF16)
         return time.perf_counter() - t0, float(rows * wl["K"] * 9)
+    if "TM" in wl:                # transposable mask (whole M-row blocks)
+        rows = max(wl["TM"][1], rows - rows % wl["TM"][1])
+        Wb = _u16(wl["W"][:rows].contiguous())
+        t0 = time.perf_counter()
+        oracle.mask_transposable(Wb, *wl["TM"], dtype=oracle.BF16)
+        return time.perf_counter() - t0, float(rows * wl["K"] * 3)
     if "D" in wl:                 # saliency-scored mask
         Wb = _u16(wl["W"][:rows].contiguous())
         d = wl["D"].numpy()
@@ -424,6 +443,7 @@ def cpu_baseline(wl, target_s: float = 15.0):
     scale, unit = (1e12, "TFLOP/s") if wl["X"] is not None else (1e9, "GB/s")
     what = ("SR-STE step (mask, masked weight, decay gradient)" if "G" in wl else
             "saliency-scored 2:4 mask" if "D" in wl else
+            "greedy transposable 4:8 mask" if "TM" in wl else
             "mask at 1:4, 2:4, 4:8, 2:8" if wl["X"] is None else
             "whole step (mask, compress, fused mask+compress, image, decompress, fp64 product)")
     return {"value": units / secs / scale, "unit": unit, "cores": threads, "kind": "oracle",
@@ -544,11 +564,12 @@ def main():
             k.update({"TFLOP/s": tf, "tensor_frac": tf / sparse_peak})
         kernels[name] = k
 
-    if step.kind in ("ties", "srste", "scored"):
+    if step.kind in ("ties", "srste", "scored", "transposable"):
         units_per_step = sum(step.bytes.values())
         value = world * units_per_step * args.steps / (total_ms * 1e-3) / 1e9
         unit = "GB/s"
-        dom = {"ties": "nm_mask_2:4", "srste": "nm_srste_step", "scored": "nm_mask_scored"}[step.kind]
+        dom = {"ties": "nm_mask_2:4", "srste": "nm_srste_step", "scored": "nm_mask_scored",
+               "transposable": "nm_mask_transposable"}[step.kind]
         roof = {"bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": hbm, "unit": "GB/s",
                 "frac": kernels[dom]["GB/s"] / hbm, "kernel": dom,
                 "algorithmic_bytes_per_launch": step.bytes[dom]}

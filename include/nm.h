@@ -126,6 +126,25 @@ NM_API nm_status nm_mask_scored(const void *W, nm_dtype dtype, const float *d, i
                          int64_t ldw, int N, int M, uint8_t *mask, int64_t ldm, void *stream);
 
 /*
+ * nm_mask_transposable -- transposable N:M mask, greedy.  Source: nubint.ai
+ * review of "Accelerated Sparse Neural Training: A Provable and Efficient
+ * Method to Find N:M Transposable Masks": in every M x M block keep as much
+ * |w| as possible with at most N kept entries per row and per column (W and
+ * W^T both N:M), found there by min-cost flow or by a fast greedy
+ * 2-approximation.  This is the greedy: inside each block, entries in order
+ * of decreasing magnitude (the nm_mask order; equal magnitudes by row-major
+ * position within the block); an entry is kept when its row and its column
+ * each hold fewer than N kept entries.  Rows or columns can end with fewer
+ * than N kept entries; the kept |w| is at least half of the optimum.
+ *   W     R x C, dtype NM_F32 / NM_BF16 / NM_F16, leading dim ldw >= C
+ *   mask  R x C uint8 (0 or 1), leading dim ldm >= C
+ *   1 <= N < M <= 8 (else NM_ERR_NM); R % M == 0 and C % M == 0 (else
+ *   NM_ERR_SHAPE); alignment as nm_mask
+ */
+NM_API nm_status nm_mask_transposable(const void *W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw,
+                               int N, int M, uint8_t *mask, int64_t ldm, void *stream);
+
+/*
  * nm_mask_compress -- fused 2:4 mask + compression in one pass over W:
  * the 2:4 mask of nm_mask, then the kept values and their indices in the
  * canonical layout and (if meta_sm100 != NULL) in the tensor-core image.

@@ -48,6 +48,7 @@ def _lib():
         "nm_sizes": ([i64, i64, i32, i32, i32, vp, vp, vp], i32),
         "nm_mask": ([vp, i32, i64, i64, i64, i32, i32, vp, i64, vp], i32),
         "nm_mask_scored": ([vp, i32, vp, i64, i64, i64, i32, i32, vp, i64, vp], i32),
+        "nm_mask_transposable": ([vp, i32, i64, i64, i64, i32, i32, vp, i64, vp], i32),
         "nm_mask_compress": ([vp, i32, i64, i64, i64, vp, vp, vp, vp], i32),
         "nm_compress": ([vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp, vp], i32),
         "nm_decompress": ([vp, vp, i32, i64, i64, vp, i64, vp], i32),
@@ -131,6 +132,18 @@ def nm_mask_scored(W: torch.Tensor, d: torch.Tensor, N: int, M: int, mask: torch
         mask = torch.empty((R, C), dtype=torch.uint8, device=W.device)
     _check(_lib().nm_mask_scored(_ptr(W), _dtype(W), _ptr(d), R, C, _ld(W), N, M, _ptr(mask), _ld(mask),
                                  _stream(stream)), "nm_mask_scored")
+    return mask
+
+
+def nm_mask_transposable(W: torch.Tensor, N: int, M: int, mask: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    """Greedy transposable N:M mask over M x M blocks (at most N kept per row
+    and per column of every block)."""
+    R, C = W.shape
+    if mask is None:
+        mask = torch.empty((R, C), dtype=torch.uint8, device=W.device)
+    _check(_lib().nm_mask_transposable(_ptr(W), _dtype(W), R, C, _ld(W), N, M, _ptr(mask), _ld(mask),
+                                       _stream(stream)), "nm_mask_transposable")
     return mask
 
 
