@@ -38,6 +38,31 @@ sys.path.insert(0, ROOT)
 import nm_inputs  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Integer (ALU) pipe of a B200 SM: 16 lanes per clock in each of its 4 sub-partitions
+# (ncu shows the ALU pipe busy for two issue cycles per warp instruction), 148 SMs at the
+# 1965 MHz maximum clock.
+ALU_PEAK_TOPS = 148 * 64 * 1.965e9 / 1e12
+
+
+def transposable_int_ops(M: int) -> float:
+    """Integer operations the greedy transposable mask needs per M x M block: two
+    (max and min) per comparator of Batcher's network on the padded key count, seven per
+    greedy step (position, row and column test, two count updates, record), two per
+    key (pack magnitude and position)."""
+    P = 1
+    while P < M * M:
+        P *= 2
+    comps, p = 0, 1
+    while p < P:
+        k = p
+        while k >= 1:
+            j = k % p
+            while j + k < P:
+                comps += sum(1 for i in range(k) if i + j + k < P and (i + j) // (2 * p) == (i + j + k) // (2 * p))
+                j += 2 * k
+            k //= 2
+        p *= 2
+    return 2.0 * comps + 7.0 * M * M + 2.0 * M * M
 SPARSE_RATIO = 2.0   # 2:4 sparse tensor peak = 2x dense (dense-equivalent flops)
 
 
@@ -570,9 +595,17 @@ def main():
         unit = "GB/s"
         dom = {"ties": "nm_mask_2:4", "srste": "nm_srste_step", "scored": "nm_mask_scored",
                "transposable": "nm_mask_transposable"}[step.kind]
-        roof = {"bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": hbm, "unit": "GB/s",
-                "frac": kernels[dom]["GB/s"] / hbm, "kernel": dom,
-                "algorithmic_bytes_per_launch": step.bytes[dom]}
+        if step.kind == "transposable":
+            N_, M_ = wl["TM"]
+            ops = transposable_int_ops(M_) * (wl["R"] // M_) * (wl["K"] // M_)
+            tops = ops / (kernels[dom]["us"] * 1e-6) / 1e12
+            roof = {"bound": "alu", "achieved": tops, "peak": ALU_PEAK_TOPS, "unit": "Tint-op/s",
+                    "frac": tops / ALU_PEAK_TOPS, "kernel": dom, "algorithmic_int_ops_per_launch": ops,
+                    "algorithmic_bytes_per_launch": step.bytes[dom], "achieved_GB/s": kernels[dom]["GB/s"]}
+        else:
+            roof = {"bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": hbm, "unit": "GB/s",
+                    "frac": kernels[dom]["GB/s"] / hbm, "kernel": dom,
+                    "algorithmic_bytes_per_launch": step.bytes[dom]}
         e2e_value = world * units_per_step * args.steps / (e2e_ms * 1e-3) / 1e9
     else:
         value = world * step.flops * args.steps / (total_ms * 1e-3) / 1e12
@@ -584,7 +617,9 @@ def main():
         e2e_value = world * step.flops * args.steps / (e2e_ms * 1e-3) / 1e12
     roof["peak_source"] = ("%s: 2 x dense bf16 %s" % (peak_src, "sustained (power cap seen in the timed region)"
                                                       if dense_key.endswith("sustained") else "burst")
-                           if roof["bound"] == "tensor" else "%s: HBM copy" % peak_src)
+                           if roof["bound"] == "tensor" else
+                           "derived: 148 SMs x 64 integer lanes x 1965 MHz" if roof["bound"] == "alu" else
+                           "%s: HBM copy" % peak_src)
     roof["traffic"] = profiled_traffic(args.workload, "nm_spmm" if dom.startswith("nm_spmm") else dom)
 
     cpu = None
