@@ -292,46 +292,58 @@ class Step:
     def launches(self):
         return len(self.names)
 
-    def run(self, events=None):
-        nm, s = self.nm, torch.cuda.current_stream()
-        rec = (lambda i: events[i].record(s)) if events is not None else (lambda i: None)
-        rec(0)
+    def calls(self):
+        """The step's launches, in the order of self.names, as zero-argument callables."""
+        nm = self.nm
         if self.kind == "srste":
-            nm.nm_srste_step(self.W, self.G, 2, 4, 0.0002, W_sparse=self.WS, grad_out=self.GO, mask=self.mask)
-            rec(1)
-        elif self.kind == "scored":
-            nm.nm_mask_scored(self.W, self.D, 2, 4, mask=self.mask)
-            rec(1)
-        elif self.kind == "transposable":
-            nm.nm_mask_transposable(self.W, *self.wl["TM"], mask=self.mask)
-            rec(1)
-        elif self.kind == "ties":
-            for i, (N, M) in enumerate([(1, 4), (2, 4), (4, 8), (2, 8)]):
-                nm.nm_mask(self.W, N, M, mask=self.masks[i])
-                rec(i + 1)
-        elif self.kind == "mlp":
-            nm.nm_mask_compress(self.W, self.values, self.meta, self.img)
-            rec(1)
-            nm.nm_mask_compress(self.W2, self.v2, self.m2, self.img2)
-            rec(2)
-            nm.nm_spmm(self.values, self.img, self.X, Y=self.H, workspace=self.ws)
-            rec(3)
-            nm.nm_spmm(self.v2, self.img2, self.H, Y=self.Y, workspace=self.ws)
-            rec(4)
-        else:
-            K = self.wl["K"]
-            nm.nm_mask(self.W, 2, 4, mask=self.mask)
-            rec(1)
-            nm.nm_compress(self.W, self.mask, self.v_c, self.m_c, self.img_c)
-            rec(2)
-            nm.nm_mask_compress(self.W, self.values, self.meta, self.img)
-            rec(3)
-            nm.nm_meta_to_sm100(self.meta, self.wl["R"], K, out=self.img_r)
-            rec(4)
-            nm.nm_decompress(self.values, self.meta, K, out=self.Wd)
-            rec(5)
-            nm.nm_spmm(self.values, self.img, self.X, Y=self.Y, workspace=self.ws)
-            rec(6)
+            return [lambda: nm.nm_srste_step(self.W, self.G, 2, 4, 0.0002, W_sparse=self.WS, grad_out=self.GO,
+                                             mask=self.mask)]
+        if self.kind == "scored":
+            return [lambda: nm.nm_mask_scored(self.W, self.D, 2, 4, mask=self.mask)]
+        if self.kind == "transposable":
+            return [lambda: nm.nm_mask_transposable(self.W, *self.wl["TM"], mask=self.mask)]
+        if self.kind == "ties":
+            return [(lambda i=i, N=N, M=M: nm.nm_mask(self.W, N, M, mask=self.masks[i]))
+                    for i, (N, M) in enumerate([(1, 4), (2, 4), (4, 8), (2, 8)])]
+        if self.kind == "mlp":
+            return [lambda: nm.nm_mask_compress(self.W, self.values, self.meta, self.img),
+                    lambda: nm.nm_mask_compress(self.W2, self.v2, self.m2, self.img2),
+                    lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.H, workspace=self.ws),
+                    lambda: nm.nm_spmm(self.v2, self.img2, self.H, Y=self.Y, workspace=self.ws)]
+        K = self.wl["K"]
+        return [lambda: nm.nm_mask(self.W, 2, 4, mask=self.mask),
+                lambda: nm.nm_compress(self.W, self.mask, self.v_c, self.m_c, self.img_c),
+                lambda: nm.nm_mask_compress(self.W, self.values, self.meta, self.img),
+                lambda: nm.nm_meta_to_sm100(self.meta, self.wl["R"], K, out=self.img_r),
+                lambda: nm.nm_decompress(self.values, self.meta, K, out=self.Wd),
+                lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.Y, workspace=self.ws)]
+
+    def run(self, events=None):
+        s = torch.cuda.current_stream()
+        calls = self.calls()
+        for i, fn in enumerate(calls):
+            if events is not None:
+                events[i].record(s)
+            fn()
+        if events is not None:
+            events[len(calls)].record(s)
+
+    def capture(self):
+        """CUDA graphs of the whole step and of each launch, captured once after
+        warm-up; replaying them issues the same kernels with the same arguments
+        without the host's per-launch latency."""
+        whole = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(whole):
+            for fn in self.calls():
+                fn()
+        per = []
+        for fn in self.calls():
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn()
+            per.append(g)
+        torch.cuda.synchronize()
+        return whole, per
 
     def result(self):
         if self.kind == "srste":
@@ -341,17 +353,38 @@ class Step:
         return self.masks[1] if self.kind == "ties" else self.Y
 
 
-def timed_steps(step: Step, steps: int, flush: torch.Tensor):
-    """-> (per-step ms list, per-kernel ms lists) over exactly `steps` steps."""
+def timed_steps(step: Step, steps: int, flush: torch.Tensor, graphs=None):
+    """-> per-step ms over exactly `steps` steps (graph replays when captured)."""
+    s = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()                      # evict L2 between steps (outside the events)
+        ev[i][0].record(s)
+        if graphs is not None:
+            graphs[0].replay()
+        else:
+            step.run()
+        ev[i][1].record(s)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def kernel_breakdown(step: Step, steps: int, flush: torch.Tensor, graphs=None):
+    """-> per-kernel ms lists: the same steps again, with events around each launch."""
+    s = torch.cuda.current_stream()
     n = step.launches()
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
     for i in range(steps):
-        flush.zero_()                      # evict L2 between steps (outside the events)
-        step.run(ev[i])
+        flush.zero_()
+        if graphs is not None:
+            for j, g in enumerate(graphs[1]):
+                ev[i][j].record(s)
+                g.replay()
+            ev[i][n].record(s)
+        else:
+            step.run(ev[i])
     torch.cuda.synchronize()
-    tot = [ev[i][0].elapsed_time(ev[i][n]) for i in range(steps)]
-    per = {name: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps)] for j, name in enumerate(step.names)}
-    return tot, per
+    return {name: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps)] for j, name in enumerate(step.names)}
 
 
 def e2e_steps(step: Step, steps: int, flush: torch.Tensor):
@@ -546,6 +579,20 @@ def main():
     torch.cuda.synchronize()
     if nm.nm_last_device_status() != 0:
         raise SystemExit("device status reports a timed-out wait")
+    try:
+        eager = step.result().clone()
+        graphs = step.capture()
+        launch_mode = "CUDA graph of the step, captured once after warm-up and replayed"
+        for _ in range(warmup):
+            graphs[0].replay()
+        torch.cuda.synchronize()
+        if not torch.equal(step.result(), eager):
+            raise SystemExit("graph replay of the step differs from the eager step")
+    except SystemExit:
+        raise
+    except Exception as exc:   # capture unavailable: time eager launches instead
+        graphs = None
+        launch_mode = "eager launches (graph capture failed: %s)" % str(exc).splitlines()[0][:120]
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -554,12 +601,13 @@ def main():
         pg.barrier()
     torch.cuda.synchronize()
     clocks.mark("t_begin")
-    tot, per = timed_steps(step, args.steps, flush)
+    tot = timed_steps(step, args.steps, flush, graphs)
     torch.cuda.synchronize()
     clocks.mark("t_end")
     if pg:
         pg.barrier()
     clk = clocks.stop()
+    per = kernel_breakdown(step, args.steps, flush, graphs)
 
     total_ms = float(np.sum(tot))
     e2e_t, h2d, d2h = e2e_steps(step, args.steps, flush)
@@ -634,6 +682,7 @@ def main():
                 "config": {"workload": args.workload, "desc": wl["desc"], "R": wl["R"], "K": wl["K"], "T": wl["T"],
                            "sparsity": "2:4 along K" if step.kind != "ties" else "N:M along K",
                            "l2": "flushed: 256 MiB write between timed steps, outside the events",
+                           "launch": launch_mode,
                            "parallelism": "independent replica per GPU" if world > 1 else "single GPU"},
                 "roofline": roof, "cpu_baseline": cpu,
                 "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
