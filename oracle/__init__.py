@@ -68,6 +68,10 @@ def _load():
         f = getattr(lib, name)
         f.argtypes = [vp, i32, i64, i64, i64, i32, i32, vp, i64]
         f.restype = i32
+    lib.oracle_compress12.argtypes = [vp, vp, i32, i64, i64, vp, vp]
+    lib.oracle_compress12.restype = i32
+    lib.oracle_decompress12.argtypes = [vp, vp, i32, i64, i64, vp]
+    lib.oracle_decompress12.restype = i32
     lib.oracle_compress24.argtypes = [vp, vp, i32, i64, i64, vp, vp]
     lib.oracle_compress24.restype = i32
     lib.oracle_decompress24.argtypes = [vp, vp, i32, i64, i64, vp]
@@ -213,6 +217,31 @@ def decompress24(values: np.ndarray, meta: np.ndarray, C: int, dtype: int | None
     mt = np.ascontiguousarray(meta, dtype=np.uint8)
     _check(_load().oracle_decompress24(vb.ctypes.data, mt.ctypes.data, code, R, C, out.ctypes.data),
            "decompress24")
+    return out.view(values.dtype) if values.dtype != np.uint16 else out
+
+
+def compress12(W: np.ndarray, mask: np.ndarray, dtype: int | None = None):
+    """1:2 compression -> (values R x C/2 same bit type as W, meta R x C/16 uint8:
+    bit p%8 of byte p/8 is the kept index of pair p)."""
+    code = dtype_code(W, dtype)
+    Wb = _bits(W, code)
+    R, C = Wb.shape
+    m = np.ascontiguousarray(mask, dtype=np.uint8)
+    values = np.zeros((R, C // 2), dtype=Wb.dtype)
+    meta = np.zeros((R, C // 16), dtype=np.uint8)
+    _check(_load().oracle_compress12(Wb.ctypes.data, m.ctypes.data, code, R, C,
+                                     values.ctypes.data, meta.ctypes.data), "compress12")
+    return values.view(W.dtype) if W.dtype != np.uint16 else values, meta
+
+
+def decompress12(values: np.ndarray, meta: np.ndarray, C: int, dtype: int | None = None) -> np.ndarray:
+    code = dtype_code(values, dtype)
+    vb = _bits(values, code)
+    R = vb.shape[0]
+    out = np.zeros((R, C), dtype=vb.dtype)
+    mt = np.ascontiguousarray(meta, dtype=np.uint8)
+    _check(_load().oracle_decompress12(vb.ctypes.data, mt.ctypes.data, code, R, C, out.ctypes.data),
+           "decompress12")
     return out.view(values.dtype) if values.dtype != np.uint16 else out
 
 

@@ -441,6 +441,47 @@ int oracle_decompress24(const void *values, const uint8_t *meta, int dtype, int6
 }
 
 /* --------------------------------------------------------------------- */
+/* 1:2 compression.  [ASDNN] "Structured sparse GEMM on tensor cores":    */
+/* sparse TF32 works only with a 1:2 pattern (one of every two values).   */
+/* Layout (this library's choice, as the 2:4 one): values[r][p] is the    */
+/* kept element of pair p (columns 2p, 2p+1) of row r, bits as stored;    */
+/* its index (0 or 1) is bit p%8 of byte r*(C/16) + p/8 (LSB first).     */
+/* The mask must hold exactly one 1 per pair; otherwise OR_BAD_MASK.      */
+/* --------------------------------------------------------------------- */
+int oracle_compress12(const void *W, const uint8_t *mask, int dtype, int64_t R, int64_t C,
+                      void *values, uint8_t *meta)
+{
+    if (C % 16 != 0 || R < 0) return OR_BAD_ARG;
+    memset(meta, 0, (size_t)(R * C / 16));
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t p = 0; p < C / 2; ++p) {
+            const uint8_t m0 = mask[r * C + 2 * p], m1 = mask[r * C + 2 * p + 1];
+            if (m0 > 1 || m1 > 1 || m0 + m1 != 1) return OR_BAD_MASK;
+            const int idx = m1 ? 1 : 0;
+            store_bits(values, dtype, (size_t)(r * (C / 2) + p), load_bits(W, dtype, (size_t)(r * C + 2 * p + idx)));
+            meta[r * (C / 16) + p / 8] |= (uint8_t)(idx << (p % 8));
+        }
+    }
+    return OR_OK;
+}
+
+/* Inverse: the kept position of each pair gets its value, the other +0.0. */
+int oracle_decompress12(const void *values, const uint8_t *meta, int dtype, int64_t R, int64_t C,
+                        void *W_out)
+{
+    if (C % 16 != 0 || R < 0) return OR_BAD_ARG;
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t p = 0; p < C / 2; ++p) {
+            const int idx = (meta[r * (C / 16) + p / 8] >> (p % 8)) & 1;
+            const uint32_t b = load_bits(values, dtype, (size_t)(r * (C / 2) + p));
+            store_bits(W_out, dtype, (size_t)(r * C + 2 * p + idx), b);
+            store_bits(W_out, dtype, (size_t)(r * C + 2 * p + 1 - idx), 0u);
+        }
+    }
+    return OR_OK;
+}
+
+/* --------------------------------------------------------------------- */
 /* Tensor-core metadata layout for the sm_100 sparse MMA (.kind::f16).    */
 /* [PTX] tcgen05 sparse matrices: for an MMA of 128 rows x 32 (logical)  */
 /* K, each row's metadata is 32 bits: 8 groups of 4, a 4-bit field per   */
