@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload linear_4096|mlp_pair|decode_T16|decode_T64|decode_T256|decode_T1024|ties_mask|
-                               srste|saliency_mask|transposable_mask]
+                               srste|saliency_mask|transposable_mask|pairs_12]
 
 One step is one pass of every step of the path over one batch of synthetic
 input (default: the transformer-linear workload, bf16 W 4096x4096 pruned 2:4
@@ -125,6 +125,11 @@ def make_workload(name: str):
         return {"W": W, "D": nm_inputs.saliency_d(W.shape[1]), "X": None, "R": W.shape[0], "K": W.shape[1], "T": 0,
                 "desc": "saliency-scored 2:4 mask: bf16 W 28672x8192 ~N(0,0.02); d = diag of the upper Cholesky factor"
                         " of the inverse of a damped synthetic Gram matrix (512 calibration rows ~N(0,1))"}
+    elif name == "pairs_12":
+        W = nm_inputs.fp32_linear()
+        return {"W": W, "P12": True, "X": None, "R": W.shape[0], "K": W.shape[1], "T": 0,
+                "desc": "1:2 pattern (sparse TF32): fp32 W 8192x8192 ~N(0,0.02); mask 1:2, compress under it,"
+                        " fused mask+compress, decompress"}
     elif name == "transposable_mask":
         W, _ = nm_inputs.linear_4096()
         return {"W": W, "TM": (4, 8), "X": None, "R": 4096, "K": 4096, "T": 0,
@@ -220,8 +225,21 @@ class Step:
         self.nm, self.wl, self.dev = nm, wl, dev
         R, K, T = wl["R"], wl["K"], wl["T"]
         self.kind = "srste" if "G" in wl else "scored" if "D" in wl else "transposable" if "TM" in wl else \
+            "pairs" if "P12" in wl else \
             ("ties" if wl["X"] is None else ("mlp" if "W2" in wl else "linear"))
         self.W = wl["W"].to(dev)
+        if self.kind == "pairs":
+            self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
+            self.v1, self.m1 = nm.alloc_compressed12(R, K, self.W.dtype, dev)
+            self.v2, self.m2 = nm.alloc_compressed12(R, K, self.W.dtype, dev)
+            self.Wd = torch.empty_like(self.W)
+            es = self.W.element_size()
+            G = R * K
+            self.names = ["nm_mask_1:2", "nm_compress12", "nm_mask_compress12", "nm_decompress12"]
+            self.bytes = {"nm_mask_1:2": G * (es + 1), "nm_compress12": G * (es + 1 + es / 2 + 1 / 16),
+                          "nm_mask_compress12": G * (es + es / 2 + 1 / 16), "nm_decompress12": G * (es / 2 + 1 / 16 + es)}
+            self.flops = 0
+            return
         if self.kind == "transposable":
             self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
             self.names = ["nm_mask_transposable"]
@@ -302,6 +320,12 @@ class Step:
             return [lambda: nm.nm_mask_scored(self.W, self.D, 2, 4, mask=self.mask)]
         if self.kind == "transposable":
             return [lambda: nm.nm_mask_transposable(self.W, *self.wl["TM"], mask=self.mask)]
+        if self.kind == "pairs":
+            K = self.wl["K"]
+            return [lambda: nm.nm_mask(self.W, 1, 2, mask=self.mask),
+                    lambda: nm.nm_compress12(self.W, self.mask, self.v1, self.m1),
+                    lambda: nm.nm_mask_compress12(self.W, self.v2, self.m2),
+                    lambda: nm.nm_decompress12(self.v2, self.m2, K, out=self.Wd)]
         if self.kind == "ties":
             return [(lambda i=i, N=N, M=M: nm.nm_mask(self.W, N, M, mask=self.masks[i]))
                     for i, (N, M) in enumerate([(1, 4), (2, 4), (4, 8), (2, 8)])]
@@ -350,6 +374,8 @@ class Step:
             return self.GO
         if self.kind in ("scored", "transposable"):
             return self.mask
+        if self.kind == "pairs":
+            return self.Wd
         return self.masks[1] if self.kind == "ties" else self.Y
 
 
@@ -449,6 +475,14 @@ def oracle_step(wl, rows: int, threads: int):
         t0 = time.perf_counter()
         oracle.mask_transposable(Wb, *wl["TM"], dtype=oracle.BF16)
         return time.perf_counter() - t0, float(rows * wl["K"] * 3)
+    if "P12" in wl:               # 1:2 family on fp32
+        W = wl["W"][:rows].contiguous().numpy()
+        t0 = time.perf_counter()
+        mask = oracle.mask_rank(W, 1, 2)
+        oracle.compress12(W, mask)
+        v, m = oracle.compress12(W, mask)
+        oracle.decompress12(v, m, wl["K"])
+        return time.perf_counter() - t0, float(rows * wl["K"] * (5 + 7.0625 + 6.0625 + 6.0625))
     if "D" in wl:                 # saliency-scored mask
         Wb = _u16(wl["W"][:rows].contiguous())
         d = wl["D"].numpy()
@@ -502,6 +536,7 @@ def cpu_baseline(wl, target_s: float = 15.0):
     what = ("SR-STE step (mask, masked weight, decay gradient)" if "G" in wl else
             "saliency-scored 2:4 mask" if "D" in wl else
             "greedy transposable 4:8 mask" if "TM" in wl else
+            "1:2 mask, compress, fused compress, decompress" if "P12" in wl else
             "mask at 1:4, 2:4, 4:8, 2:8" if wl["X"] is None else
             "whole step (mask, compress, fused mask+compress, image, decompress, fp64 product)")
     return {"value": units / secs / scale, "unit": unit, "cores": threads, "kind": "oracle",
@@ -637,12 +672,12 @@ def main():
             k.update({"TFLOP/s": tf, "tensor_frac": tf / sparse_peak})
         kernels[name] = k
 
-    if step.kind in ("ties", "srste", "scored", "transposable"):
+    if step.kind in ("ties", "srste", "scored", "transposable", "pairs"):
         units_per_step = sum(step.bytes.values())
         value = world * units_per_step * args.steps / (total_ms * 1e-3) / 1e9
         unit = "GB/s"
         dom = {"ties": "nm_mask_2:4", "srste": "nm_srste_step", "scored": "nm_mask_scored",
-               "transposable": "nm_mask_transposable"}[step.kind]
+               "transposable": "nm_mask_transposable", "pairs": "nm_mask_compress12"}[step.kind]
         if step.kind == "transposable":
             N_, M_ = wl["TM"]
             ops = transposable_int_ops(M_) * (wl["R"] // M_) * (wl["K"] // M_)
@@ -680,7 +715,8 @@ def main():
                 "scaling": "weak", "vs_baseline": None, "dtype": str(wl["W"].dtype).replace("torch.", ""),
                 "data": "synthetic",
                 "config": {"workload": args.workload, "desc": wl["desc"], "R": wl["R"], "K": wl["K"], "T": wl["T"],
-                           "sparsity": "2:4 along K" if step.kind != "ties" else "N:M along K",
+                           "sparsity": {"ties": "N:M along K (1:4, 2:4, 4:8, 2:8)", "pairs": "1:2 along K",
+                                        "transposable": "4:8 transposable (8x8 blocks)"}.get(step.kind, "2:4 along K"),
                            "l2": "flushed: 256 MiB write between timed steps, outside the events",
                            "launch": launch_mode,
                            "parallelism": "independent replica per GPU" if world > 1 else "single GPU"},

@@ -157,6 +157,33 @@ NM_API nm_status nm_mask_compress(const void *W, nm_dtype dtype, int64_t R, int6
                            void *values, uint8_t *meta, uint8_t *meta_sm100, void *stream);
 
 /*
+ * 1:2 compression (one value of every pair kept).  Source: review of
+ * "Accelerating Sparse Deep Neural Networks", "Structured sparse GEMM on
+ * tensor cores": sparse TF32 supports only the 1:2 pattern.  Layout (this
+ * library's choice): values R x C/2 of W's dtype, values[r][p] = the kept
+ * element of pair p (columns 2p, 2p+1), bits copied as stored; meta R x C/16
+ * bytes, the kept index of pair p in bit p%8 of byte r*(C/16) + p/8 (LSB
+ * first).  C % 16 == 0 (else NM_ERR_SHAPE); pointers and row strides of W,
+ * values and mask 16-byte aligned (else NM_ERR_ALIGN).
+ *
+ * nm_mask_compress12 -- keep the larger magnitude of each pair (the nm_mask
+ *   order with N = 1, M = 2: ties keep the first).
+ * nm_compress12 -- keep what the uint8 mask (R x C, leading dim ldm) marks.
+ *   A pair whose two mask bytes are not exactly one 1 and one 0 is counted
+ *   into *invalid_pairs (device int32, added to atomically; NULL to skip) and
+ *   stores its first element with index 0.
+ * nm_decompress12 -- W_out (R x C, leading dim ldw): the kept element of each
+ *   pair at its index, +0.0 at the other.
+ */
+NM_API nm_status nm_mask_compress12(const void *W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw,
+                             void *values, uint8_t *meta, void *stream);
+NM_API nm_status nm_compress12(const void *W, const uint8_t *mask, nm_dtype dtype, int64_t R, int64_t C,
+                        int64_t ldw, int64_t ldm, void *values, uint8_t *meta, int32_t *invalid_pairs,
+                        void *stream);
+NM_API nm_status nm_decompress12(const void *values, const uint8_t *meta, nm_dtype dtype, int64_t R, int64_t C,
+                          void *W_out, int64_t ldw, void *stream);
+
+/*
  * nm_compress -- 2:4 compression under a caller-supplied mask (uint8, R x C,
  * leading dim ldm).  A valid group has exactly two entries equal to 1 and
  * the rest 0.  Invalid groups are counted into *invalid_groups (a device

@@ -19,6 +19,8 @@ linear/conv weights; the pages' datasets and trained weights are not used):
                       X bf16 8192xT ~N(0,1) (seed 105+T), T in {16,64,256,1024}
 * ``srste``           the linear_4096 weight and a gradient bf16(1e-3 * N(0,1))
                       of the same shape (seed 6)
+* ``fp32_linear``     W fp32 8192x8192 = fp32(0.02 * N(0,1)) (seed 8), for the
+                      1:2 pattern of sparse TF32
 * ``saliency``        the linear_4096 weight and d of length 4096: the diagonal
                       of the upper Cholesky factor of H^-1, H = (2/n) X^T X +
                       0.01 * mean(diag) * I from n = 512 synthetic calibration
@@ -38,6 +40,7 @@ SEEDS = {
     "decode_skinny.W": 5,
     "srste.grad": 6,
     "saliency.X": 7,
+    "fp32_linear.W": 8,
 }
 
 
@@ -114,3 +117,7 @@ def saliency_d(C: int = 4096, n: int = 512, seed: int | None = None) -> torch.Te
     Hinv = torch.cholesky_inverse(torch.linalg.cholesky(H))
     U = torch.linalg.cholesky(Hinv, upper=True)
     return U.diagonal().to(torch.float32).contiguous()
+
+
+def fp32_linear(R: int = 8192, C: int = 8192) -> torch.Tensor:
+    return normal((R, C), SEEDS["fp32_linear.W"], 0.02, torch.float32)

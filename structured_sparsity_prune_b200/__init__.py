@@ -49,6 +49,9 @@ def _lib():
         "nm_mask": ([vp, i32, i64, i64, i64, i32, i32, vp, i64, vp], i32),
         "nm_mask_scored": ([vp, i32, vp, i64, i64, i64, i32, i32, vp, i64, vp], i32),
         "nm_mask_transposable": ([vp, i32, i64, i64, i64, i32, i32, vp, i64, vp], i32),
+        "nm_mask_compress12": ([vp, i32, i64, i64, i64, vp, vp, vp], i32),
+        "nm_compress12": ([vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp], i32),
+        "nm_decompress12": ([vp, vp, i32, i64, i64, vp, i64, vp], i32),
         "nm_mask_compress": ([vp, i32, i64, i64, i64, vp, vp, vp, vp], i32),
         "nm_compress": ([vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp, vp], i32),
         "nm_decompress": ([vp, vp, i32, i64, i64, vp, i64, vp], i32),
@@ -145,6 +148,43 @@ def nm_mask_transposable(W: torch.Tensor, N: int, M: int, mask: torch.Tensor | N
     _check(_lib().nm_mask_transposable(_ptr(W), _dtype(W), R, C, _ld(W), N, M, _ptr(mask), _ld(mask),
                                        _stream(stream)), "nm_mask_transposable")
     return mask
+
+
+def alloc_compressed12(R: int, C: int, dtype: torch.dtype, device):
+    """Output buffers of the 1:2 compressing calls: (values R x C/2, meta R x C/16)."""
+    return (torch.empty((R, C // 2), dtype=dtype, device=device),
+            torch.empty((R, C // 16), dtype=torch.uint8, device=device))
+
+
+def nm_mask_compress12(W: torch.Tensor, values=None, meta=None, stream=None):
+    """1:2 compression keeping the larger magnitude of each pair -> (values, meta)."""
+    R, C = W.shape
+    if values is None:
+        values, meta = alloc_compressed12(R, C, W.dtype, W.device)
+    _check(_lib().nm_mask_compress12(_ptr(W), _dtype(W), R, C, _ld(W), _ptr(values), _ptr(meta), _stream(stream)),
+           "nm_mask_compress12")
+    return values, meta
+
+
+def nm_compress12(W: torch.Tensor, mask: torch.Tensor, values=None, meta=None,
+                  invalid_pairs: torch.Tensor | None = None, stream=None):
+    """1:2 compression under a mask -> (values, meta)."""
+    R, C = W.shape
+    if values is None:
+        values, meta = alloc_compressed12(R, C, W.dtype, W.device)
+    _check(_lib().nm_compress12(_ptr(W), _ptr(mask), _dtype(W), R, C, _ld(W), _ld(mask), _ptr(values), _ptr(meta),
+                                _ptr(invalid_pairs), _stream(stream)), "nm_compress12")
+    return values, meta
+
+
+def nm_decompress12(values: torch.Tensor, meta: torch.Tensor, C: int, out: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    R = values.shape[0]
+    if out is None:
+        out = torch.empty((R, C), dtype=values.dtype, device=values.device)
+    _check(_lib().nm_decompress12(_ptr(values), _ptr(meta), _dtype(values), R, C, _ptr(out), _ld(out),
+                                  _stream(stream)), "nm_decompress12")
+    return out
 
 
 def alloc_compressed(R: int, C: int, dtype: torch.dtype, device, sm100: bool = True):

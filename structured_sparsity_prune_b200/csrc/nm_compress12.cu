@@ -1,0 +1,195 @@
+// nm_compress12.cu -- 1:2 compression and decompression (one value of every
+// pair kept), the pattern the review of "Accelerating Sparse Deep Neural
+// Networks" ("Structured sparse GEMM on tensor cores") gives for sparse TF32.
+//
+// Layout (this library's choice): values[r][p] is the kept element of pair p
+// (columns 2p, 2p+1) of row r, bits as stored; its index is bit p%8 of byte
+// r*(C/16) + p/8 (LSB first).  HBM-bound streams: one thread per unit of 16
+// elements (8 pairs, one metadata byte), 16-byte vector loads and stores.
+#include "nm_internal.cuh"
+
+namespace nm {
+namespace {
+
+// 16 elements of one row, as raw bits.
+template <typename Bits> struct Row16 {
+  static constexpr int kVec = int(sizeof(Bits));   // 16-byte vectors: 2 (16-bit) or 4 (32-bit)
+  uint4 v[kVec];
+  __device__ __forceinline__ void load(const Bits* p) {
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) v[i] = __ldcs(reinterpret_cast<const uint4*>(p) + i);
+  }
+  __device__ __forceinline__ void store(Bits* p) const {
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) __stcs(reinterpret_cast<uint4*>(p) + i, v[i]);
+  }
+  __device__ __forceinline__ Bits get(int i) const { return reinterpret_cast<const Bits*>(v)[i]; }
+  __device__ __forceinline__ void set(int i, Bits b) { reinterpret_cast<Bits*>(v)[i] = b; }
+};
+
+// Eight values of one row.
+template <typename Bits> struct Row8 {
+  static constexpr int kVec = int(sizeof(Bits)) / 2;   // 1 (16-bit) or 2 (32-bit)
+  uint4 v[kVec];
+  __device__ __forceinline__ void load(const Bits* p) {
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) v[i] = __ldcs(reinterpret_cast<const uint4*>(p) + i);
+  }
+  __device__ __forceinline__ void store(Bits* p) const {
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) __stcs(reinterpret_cast<uint4*>(p) + i, v[i]);
+  }
+  __device__ __forceinline__ Bits get(int i) const { return reinterpret_cast<const Bits*>(v)[i]; }
+  __device__ __forceinline__ void set(int i, Bits b) { reinterpret_cast<Bits*>(v)[i] = b; }
+};
+
+// MODE 0: keep the larger magnitude of each pair (ties -> the first);
+// MODE 1: keep what the mask marks (exactly one 1 per pair, else the pair is
+// counted as invalid and its first element kept).
+template <typename Bits, int MODE>
+__global__ void __launch_bounds__(256) compress12_kernel(const Bits* __restrict__ W, const uint8_t* __restrict__ mask,
+                                                         int64_t R, int64_t upr, int64_t ldw, int64_t ldm,
+                                                         Bits* __restrict__ values, uint8_t* __restrict__ meta,
+                                                         int* __restrict__ invalid) {
+  const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
+  const int64_t u_step = int64_t(gridDim.x) * blockDim.x;
+  int bad = 0;
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+    for (int64_t u = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u < upr; u += u_step) {
+      Row16<Bits> e;
+      e.load(W + r * ldw + 16 * u);
+      uint4 mk = make_uint4(0u, 0u, 0u, 0u);
+      if constexpr (MODE == 1) mk = __ldcs(reinterpret_cast<const uint4*>(mask + r * ldm + 16 * u));
+      const uint8_t* mb = reinterpret_cast<const uint8_t*>(&mk);
+      Row8<Bits> out;
+      uint32_t bits = 0u;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const Bits a = e.get(2 * p), b = e.get(2 * p + 1);
+        uint32_t idx;
+        if constexpr (MODE == 0) {
+          idx = mag_key<Bits>(b) > mag_key<Bits>(a) ? 1u : 0u;
+        } else {
+          const uint32_t m0 = mb[2 * p], m1 = mb[2 * p + 1];
+          const bool ok = (m0 | m1) <= 1u && m0 + m1 == 1u;
+          bad += ok ? 0 : 1;
+          idx = ok ? m1 : 0u;
+        }
+        out.set(p, idx ? b : a);
+        bits |= idx << p;
+      }
+      out.store(values + r * (upr * 8) + 8 * u);
+      meta[r * upr + u] = uint8_t(bits);
+    }
+  }
+  if constexpr (MODE == 1) {
+    if (invalid != nullptr) {
+      bad = __reduce_add_sync(0xFFFFFFFFu, bad);
+      if ((threadIdx.x & 31) == 0 && bad != 0) atomicAdd(invalid, bad);
+    }
+  }
+}
+
+template <typename Bits>
+__global__ void __launch_bounds__(256) decompress12_kernel(const Bits* __restrict__ values,
+                                                           const uint8_t* __restrict__ meta, int64_t R, int64_t upr,
+                                                           Bits* __restrict__ out, int64_t ldo) {
+  const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
+  const int64_t u_step = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+    for (int64_t u = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u < upr; u += u_step) {
+      Row8<Bits> v;
+      v.load(values + r * (upr * 8) + 8 * u);
+      const uint32_t bits = meta[r * upr + u];
+      Row16<Bits> d;
+#pragma unroll
+      for (int p = 0; p < 8; ++p) {
+        const uint32_t idx = (bits >> p) & 1u;
+        const Bits x = v.get(p);
+        d.set(2 * p, idx ? Bits(0) : x);
+        d.set(2 * p + 1, idx ? x : Bits(0));
+      }
+      d.store(out + r * ldo + 16 * u);
+    }
+  }
+}
+
+void shape_units(int64_t R, int64_t units, dim3& grid, dim3& block) {
+  int bx = 32;
+  while (bx < 256 && bx < units) bx *= 2;
+  const int by = 256 / bx;
+  const int64_t gx = (units + bx - 1) / bx;
+  const int64_t want = int64_t(sm_count()) * 8;
+  int64_t gy = (R + by - 1) / by;
+  const int64_t cap_y = gx >= want ? 1 : want / gx;
+  if (gy > cap_y) gy = cap_y;
+  if (gy > 65535) gy = 65535;
+  grid = dim3(unsigned(gx > 2147483647 ? 2147483647 : gx), unsigned(gy < 1 ? 1 : gy), 1);
+  block = dim3(bx, by, 1);
+}
+
+nm_status check12(nm_dtype dtype, int64_t R, int64_t C) {
+  if (!dtype_ok(dtype)) return NM_ERR_DTYPE;
+  if (R < 0 || C < 0 || C % 16 != 0) return NM_ERR_SHAPE;
+  return NM_OK;
+}
+
+template <int MODE>
+nm_status run_compress12(const void* W, const uint8_t* mask, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw,
+                         int64_t ldm, void* values, uint8_t* meta, int32_t* invalid, void* stream) {
+  nm_status st = check12(dtype, R, C);
+  if (st != NM_OK) return st;
+  if (ldw < C || (MODE == 1 && ldm < C)) return NM_ERR_SHAPE;
+  if (R == 0 || C == 0) return NM_OK;
+  if (W == nullptr || values == nullptr || meta == nullptr || (MODE == 1 && mask == nullptr)) return NM_ERR_NULL;
+  const int es = esize_of(dtype);
+  if (!aligned16(W) || !aligned16(values) || !stride_ok(ldw, es) ||
+      (MODE == 1 && (!aligned16(mask) || !stride_ok(ldm, 1))))
+    return NM_ERR_ALIGN;
+  dim3 grid, block;
+  shape_units(R, C / 16, grid, block);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == NM_F32)
+    compress12_kernel<uint32_t, MODE><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(W), mask, R, C / 16, ldw,
+                                                            ldm, static_cast<uint32_t*>(values), meta, invalid);
+  else
+    compress12_kernel<uint16_t, MODE><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(W), mask, R, C / 16, ldw,
+                                                            ldm, static_cast<uint16_t*>(values), meta, invalid);
+  return launch_status();
+}
+
+}  // namespace
+}  // namespace nm
+
+extern "C" nm_status nm_mask_compress12(const void* W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw,
+                                        void* values, uint8_t* meta, void* stream) {
+  return nm::run_compress12<0>(W, nullptr, dtype, R, C, ldw, 0, values, meta, nullptr, stream);
+}
+
+extern "C" nm_status nm_compress12(const void* W, const uint8_t* mask, nm_dtype dtype, int64_t R, int64_t C,
+                                   int64_t ldw, int64_t ldm, void* values, uint8_t* meta, int32_t* invalid_pairs,
+                                   void* stream) {
+  return nm::run_compress12<1>(W, mask, dtype, R, C, ldw, ldm, values, meta, invalid_pairs, stream);
+}
+
+extern "C" nm_status nm_decompress12(const void* values, const uint8_t* meta, nm_dtype dtype, int64_t R, int64_t C,
+                                     void* W_out, int64_t ldw, void* stream) {
+  using namespace nm;
+  nm_status st = check12(dtype, R, C);
+  if (st != NM_OK) return st;
+  if (ldw < C) return NM_ERR_SHAPE;
+  if (R == 0 || C == 0) return NM_OK;
+  if (values == nullptr || meta == nullptr || W_out == nullptr) return NM_ERR_NULL;
+  const int es = esize_of(dtype);
+  if (!aligned16(values) || !aligned16(W_out) || !stride_ok(ldw, es)) return NM_ERR_ALIGN;
+  dim3 grid, block;
+  shape_units(R, C / 16, grid, block);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == NM_F32)
+    decompress12_kernel<uint32_t><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C / 16,
+                                                         static_cast<uint32_t*>(W_out), ldw);
+  else
+    decompress12_kernel<uint16_t><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(values), meta, R, C / 16,
+                                                         static_cast<uint16_t*>(W_out), ldw);
+  return launch_status();
+}
