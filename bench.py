@@ -577,6 +577,22 @@ def run_reference(args, wl, metric):
 METRIC = "nm_spmm dense-equiv TFLOP/s + mask/compress GB/s, % of B200 roofline"
 
 
+def max_over_ranks(pg, values, device):
+    """Element-wise maximum of a list of floats over every rank of the process
+    group (the slowest rank's time is the job's time); identity without one."""
+    if pg is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_rate(world: int, units_per_step: float, steps: int, ms: float, scale: float) -> float:
+    """Units every rank processed (each rank runs the full step) per second,
+    divided by `scale` (1e12 for TFLOP/s, 1e9 for GB/s)."""
+    return world * units_per_step * steps / (ms * 1e-3) / scale
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -649,10 +665,7 @@ def main():
 
     total_ms = float(np.sum(tot))
     e2e_ms, h2d, d2h = e2e_steps(step, args.steps, nm, wl, dev)
-    if pg:
-        t = torch.tensor([total_ms, e2e_ms], dtype=torch.float64, device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+    total_ms, e2e_ms = max_over_ranks(pg, [total_ms, e2e_ms], dev)
     if nm.nm_last_device_status() != 0:
         raise SystemExit("device status reports a timed-out wait")
 
@@ -676,7 +689,7 @@ def main():
 
     if step.kind in ("ties", "srste", "scored", "transposable", "pairs"):
         units_per_step = sum(step.bytes.values())
-        value = world * units_per_step * args.steps / (total_ms * 1e-3) / 1e9
+        value = whole_job_rate(world, units_per_step, args.steps, total_ms, 1e9)
         unit = "GB/s"
         dom = {"ties": "nm_mask_2:4", "srste": "nm_srste_step", "scored": "nm_mask_scored",
                "transposable": "nm_mask_transposable", "pairs": "nm_mask_compress12"}[step.kind]
@@ -691,15 +704,15 @@ def main():
             roof = {"bound": "hbm", "achieved": kernels[dom]["GB/s"], "peak": hbm, "unit": "GB/s",
                     "frac": kernels[dom]["GB/s"] / hbm, "kernel": dom,
                     "algorithmic_bytes_per_launch": step.bytes[dom]}
-        e2e_value = world * units_per_step * args.steps / (e2e_ms * 1e-3) / 1e9
+        e2e_value = whole_job_rate(world, units_per_step, args.steps, e2e_ms, 1e9)
     else:
-        value = world * step.flops * args.steps / (total_ms * 1e-3) / 1e12
+        value = whole_job_rate(world, step.flops, args.steps, total_ms, 1e12)
         unit = "TFLOP/s"
         dom = max(step.flop_k, key=lambda n: np.mean(per[n]))
         roof = {"bound": "tensor", "achieved": kernels[dom]["TFLOP/s"], "peak": sparse_peak, "unit": "TFLOP/s",
                 "frac": kernels[dom]["TFLOP/s"] / sparse_peak, "kernel": dom,
                 "algorithmic_flops_per_launch": step.flop_k[dom]}
-        e2e_value = world * step.flops * args.steps / (e2e_ms * 1e-3) / 1e12
+        e2e_value = whole_job_rate(world, step.flops, args.steps, e2e_ms, 1e12)
     roof["peak_source"] = ("%s: 2 x dense bf16 %s" % (peak_src, "sustained (power cap seen in the timed region)"
                                                       if dense_key.endswith("sustained") else "burst")
                            if roof["bound"] == "tensor" else
