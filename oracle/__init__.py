@@ -36,7 +36,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "nm_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-F32, BF16, F16 = 0, 1, 2
+F32, BF16, F16, S8 = 0, 1, 2, 3
 _OK, _BAD_ARG, _NONFINITE, _BAD_MASK = 0, 1, 2, 3
 
 _lib = None
@@ -107,11 +107,15 @@ def dtype_code(a: np.ndarray, hint: int | None = None) -> int:
         return F32
     if a.dtype == np.float16:
         return F16
+    if a.dtype in (np.int8, np.uint8):
+        return S8
     raise ValueError("pass dtype= for bf16 bit patterns (np.uint16)")
 
 
 def _bits(a: np.ndarray, code: int) -> np.ndarray:
     a = np.ascontiguousarray(a)
+    if code == S8:
+        return a.view(np.uint8)
     return a.view(np.uint32) if code == F32 else a.view(np.uint16)
 
 

@@ -57,25 +57,31 @@
 #include <math.h>
 #include <pthread.h>
 
-/* element type codes used by this file's callers (tests pass these) */
-enum { OR_F32 = 0, OR_BF16 = 1, OR_F16 = 2 };
+/* element type codes used by this file's callers (tests pass these);
+ * OR_S8 is two's-complement int8, whose magnitude is |x| */
+enum { OR_F32 = 0, OR_BF16 = 1, OR_F16 = 2, OR_S8 = 3 };
 
 /* status codes */
 enum { OR_OK = 0, OR_BAD_ARG = 1, OR_NONFINITE = 2, OR_BAD_MASK = 3 };
 
-static size_t elem_size(int dtype) { return dtype == OR_F32 ? 4 : 2; }
+static size_t elem_size(int dtype) { return dtype == OR_F32 ? 4 : (dtype == OR_S8 ? 1 : 2); }
 
 static uint32_t load_bits(const void *base, int dtype, size_t i)
 {
     if (dtype == OR_F32) return ((const uint32_t *)base)[i];
+    if (dtype == OR_S8) return ((const uint8_t *)base)[i];
     return ((const uint16_t *)base)[i];
 }
 
 static void store_bits(void *base, int dtype, size_t i, uint32_t v)
 {
     if (dtype == OR_F32) ((uint32_t *)base)[i] = v;
+    else if (dtype == OR_S8) ((uint8_t *)base)[i] = (uint8_t)v;
     else ((uint16_t *)base)[i] = (uint16_t)v;
 }
+
+/* the int8 value of an 8-bit two's-complement pattern */
+static int s8_value(uint32_t bits) { return (bits & 0x80u) ? (int)(bits & 0xFFu) - 256 : (int)(bits & 0xFFu); }
 
 /* --------------------------------------------------------------------- */
 /* IEEE-754 decoding, written from the format definitions.                */
@@ -101,6 +107,7 @@ static double decode_generic(uint32_t sign, uint32_t e, uint32_t f,
 
 double oracle_decode(uint32_t bits, int dtype)
 {
+    if (dtype == OR_S8) return (double)s8_value(bits);
     if (dtype == OR_F16)
         return decode_generic(bits >> 15, (bits >> 10) & 0x1Fu, bits & 0x3FFu, 5, 10, 15);
     if (dtype == OR_BF16) bits <<= 16;
@@ -154,6 +161,10 @@ uint32_t oracle_encode(double x, int dtype)
 /* Magnitude key: sign bit cleared, read as unsigned. */
 uint32_t oracle_mag(uint32_t bits, int dtype)
 {
+    if (dtype == OR_S8) {
+        const int v = s8_value(bits);
+        return (uint32_t)(v < 0 ? -v : v);
+    }
     return dtype == OR_F32 ? (bits & 0x7FFFFFFFu) : (bits & 0x7FFFu);
 }
 
@@ -335,6 +346,7 @@ static int big_cmp(const big_t *a, const big_t *b)
 /* |w| = m * 2^(shift-149): returns 0 on success, -1 if non-finite */
 static int exact_magnitude(uint32_t bits, int dtype, uint64_t *m, int *shift)
 {
+    if (dtype == OR_S8) { *m = oracle_mag(bits, OR_S8); *shift = 149; return 0; }   /* |x| * 2^0 */
     if (dtype == OR_BF16) { bits <<= 16; dtype = OR_F32; }
     if (dtype == OR_F32) {
         uint32_t e = (bits >> 23) & 0xFFu, f = bits & 0x7FFFFFu;
@@ -565,6 +577,7 @@ static void build_tables(void)
 
 static double decode_fast(const void *base, int dtype, size_t i)
 {
+    if (dtype == OR_S8) return (double)s8_value(((const uint8_t *)base)[i]);
     if (dtype == OR_F32) {
         float f;
         memcpy(&f, (const char *)base + 4 * i, 4);
