@@ -70,7 +70,12 @@ typedef enum {
     NM_ERR_TIMEOUT = 9       /* a bounded device-side wait gave up (see below)  */
 } nm_status;
 
-typedef enum { NM_F32 = 0, NM_BF16 = 1, NM_F16 = 2 } nm_dtype;
+/* NM_S8: two's-complement int8 weights, magnitude |x| (so -128 ranks above 127).
+ * Accepted by nm_sizes, nm_mask, nm_mask_transposable, nm_mask_compress,
+ * nm_compress and nm_decompress; the int8 sparse product is not built (nm_spmm
+ * returns NM_ERR_UNSUPPORTED for it) and the floating-point calls
+ * (nm_mask_scored, nm_srste_step, the 1:2 calls) return NM_ERR_DTYPE. */
+typedef enum { NM_F32 = 0, NM_BF16 = 1, NM_F16 = 2, NM_S8 = 3 } nm_dtype;
 
 /* Human-readable text for a status code (static string, never NULL). */
 NM_API const char *nm_status_string(int status);

@@ -19,10 +19,10 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnm.so")
 
-NM_F32, NM_BF16, NM_F16 = 0, 1, 2
+NM_F32, NM_BF16, NM_F16, NM_S8 = 0, 1, 2, 3
 STATUS = ["NM_OK", "NM_ERR_NULL", "NM_ERR_SHAPE", "NM_ERR_ALIGN", "NM_ERR_DTYPE", "NM_ERR_NM",
           "NM_ERR_UNSUPPORTED", "NM_ERR_CUDA", "NM_ERR_WORKSPACE", "NM_ERR_TIMEOUT"]
-_DT = {torch.float32: NM_F32, torch.bfloat16: NM_BF16, torch.float16: NM_F16}
+_DT = {torch.float32: NM_F32, torch.bfloat16: NM_BF16, torch.float16: NM_F16, torch.int8: NM_S8}
 
 
 class NMError(RuntimeError):

@@ -21,7 +21,7 @@ extern "C" int nm_version(void) { return 1 * 10000 + 0 * 100 + 0; }
 
 extern "C" nm_status nm_sizes(int64_t R, int64_t C, int N, int M, nm_dtype dtype, size_t* values_bytes,
                               size_t* meta_bytes, size_t* meta_sm100_bytes) {
-  if (!nm::dtype_ok(dtype)) return NM_ERR_DTYPE;
+  if (!nm::dtype_ok_int8(dtype)) return NM_ERR_DTYPE;
   if (M < 2 || M > 8 || N < 1 || N >= M) return NM_ERR_NM;
   if (R < 0 || C < 0 || C % M != 0) return NM_ERR_SHAPE;
   const bool two_four = (N == 2 && M == 4);

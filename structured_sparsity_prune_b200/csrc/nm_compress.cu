@@ -32,6 +32,11 @@ template <> struct Oct<uint16_t> {
     return uint16_t((i & 1) ? (w >> 16) : (w & 0xFFFFu));
   }
 };
+template <> struct Oct<uint8_t> {
+  uint2 v;
+  __device__ __forceinline__ void load(const uint8_t* p) { v = __ldcs(reinterpret_cast<const uint2*>(p)); }
+  __device__ __forceinline__ uint8_t operator[](int i) const { return uint8_t(((&v.x)[i >> 2] >> (8 * (i & 3))) & 0xFFu); }
+};
 template <> struct Oct<uint32_t> {
   uint4 v[2];
   __device__ __forceinline__ void load(const uint32_t* p) {
@@ -50,6 +55,11 @@ template <> struct Quad<uint16_t> {
     w = (i & 1) ? ((w & 0xFFFFu) | (uint32_t(b) << 16)) : ((w & 0xFFFF0000u) | b);
   }
   __device__ __forceinline__ void store(uint16_t* p) const { __stcs(reinterpret_cast<uint2*>(p), v); }
+};
+template <> struct Quad<uint8_t> {
+  uint32_t v;
+  __device__ __forceinline__ void set(int i, uint8_t b) { v = (v & ~(0xFFu << (8 * i))) | (uint32_t(b) << (8 * i)); }
+  __device__ __forceinline__ void store(uint8_t* p) const { __stcs(reinterpret_cast<unsigned int*>(p), v); }
 };
 template <> struct Quad<uint32_t> {
   uint4 v;
@@ -241,7 +251,18 @@ __global__ void __launch_bounds__(256) decompress_kernel(const Bits* __restrict_
     for (int64_t o = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; o < opr; o += o_step) {
       const uint32_t mb = meta[r * (C / 8) + o];
       Bits v[4], d[8];
-      if constexpr (sizeof(Bits) == 2) {
+      if constexpr (sizeof(Bits) == 1) {
+        // four int8 values in one word; each group's four outputs form one word
+        const uint32_t x = __ldcs(reinterpret_cast<const unsigned int*>(values + r * (C / 2) + 4 * o));
+        uint32_t gw[2];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const uint32_t i0 = (mb >> (4 * g)) & 3u, i1 = (mb >> (4 * g + 2)) & 3u;
+          gw[g] = (((x >> (16 * g)) & 0xFFu) << (8 * i0)) | (((x >> (16 * g + 8)) & 0xFFu) << (8 * i1));
+        }
+        __stcs(reinterpret_cast<uint2*>(out + r * ldo + 8 * o), make_uint2(gw[0], gw[1]));
+        continue;
+      } else if constexpr (sizeof(Bits) == 2) {
         const uint2 x = __ldcs(reinterpret_cast<const uint2*>(values + r * (C / 2) + 4 * o));
         v[0] = uint16_t(x.x & 0xFFFFu); v[1] = uint16_t(x.x >> 16);
         v[2] = uint16_t(x.y & 0xFFFFu); v[3] = uint16_t(x.y >> 16);
@@ -263,7 +284,7 @@ __global__ void __launch_bounds__(256) decompress_kernel(const Bits* __restrict_
         y.x = uint32_t(g01[0]); y.y = uint32_t(g01[0] >> 32);
         y.z = uint32_t(g01[1]); y.w = uint32_t(g01[1] >> 32);
         __stcs(reinterpret_cast<uint4*>(dst), y);
-      } else {
+      } else if constexpr (sizeof(Bits) == 4) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) d[i] = Bits(0);
 #pragma unroll
@@ -298,7 +319,18 @@ __global__ void __launch_bounds__(256) decompress32_kernel(const Bits* __restric
 #pragma unroll
       for (int i = 0; i < kVals; ++i) vv[i] = __ldcs(reinterpret_cast<const uint4*>(values + r * (C / 2) + 16 * u) + i);
       uint4* dst = reinterpret_cast<uint4*>(out + r * ldo + 32 * u);
-      if constexpr (sizeof(Bits) == 2) {
+      if constexpr (sizeof(Bits) == 1) {
+        const uint32_t* vw = reinterpret_cast<const uint32_t*>(vv);  // value pair of group g: bytes 2g, 2g+1
+        uint32_t o[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const uint32_t nib = (mw >> (4 * g)) & 0xFu;
+          const uint32_t w = vw[g >> 1] >> (16 * (g & 1));
+          o[g] = ((w & 0xFFu) << (8 * (nib & 3u))) | (((w >> 8) & 0xFFu) << (8 * (nib >> 2)));
+        }
+        __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+        __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+      } else if constexpr (sizeof(Bits) == 2) {
         const uint32_t* vw = reinterpret_cast<const uint32_t*>(vv);  // value pair of group g in word g
 #pragma unroll
         for (int h = 0; h < 4; ++h) {  // two groups -> one 16-byte store
@@ -336,7 +368,7 @@ int tile_grid(int64_t R, int64_t C) {
 }
 
 nm_status check_common(const void* W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw) {
-  if (!dtype_ok(dtype)) return NM_ERR_DTYPE;
+  if (!dtype_ok_int8(dtype)) return NM_ERR_DTYPE;
   if (R < 0 || C < 0 || C % 8 != 0 || ldw < C) return NM_ERR_SHAPE;
   (void)W;
   return NM_OK;
@@ -362,6 +394,10 @@ extern "C" nm_status nm_mask_compress(const void* W, nm_dtype dtype, int64_t R, 
     compress_tiles_kernel<uint32_t, 0><<<grid, kThreads, 0, s>>>(
         static_cast<const uint32_t*>(W), ldw, nullptr, 0, R, C, static_cast<uint32_t*>(values), meta,
         meta_sm100, nullptr);
+  else if (dtype == NM_S8)
+    compress_tiles_kernel<uint8_t, 0><<<grid, kThreads, 0, s>>>(
+        static_cast<const uint8_t*>(W), ldw, nullptr, 0, R, C, static_cast<uint8_t*>(values), meta,
+        meta_sm100, nullptr);
   else
     compress_tiles_kernel<uint16_t, 0><<<grid, kThreads, 0, s>>>(
         static_cast<const uint16_t*>(W), ldw, nullptr, 0, R, C, static_cast<uint16_t*>(values), meta,
@@ -386,6 +422,10 @@ extern "C" nm_status nm_compress(const void* W, const uint8_t* mask, nm_dtype dt
   if (dtype == NM_F32)
     compress_tiles_kernel<uint32_t, 1><<<grid, kThreads, 0, s>>>(
         static_cast<const uint32_t*>(W), ldw, mask, ldm, R, C, static_cast<uint32_t*>(values), meta, meta_sm100,
+        invalid_groups);
+  else if (dtype == NM_S8)
+    compress_tiles_kernel<uint8_t, 1><<<grid, kThreads, 0, s>>>(
+        static_cast<const uint8_t*>(W), ldw, mask, ldm, R, C, static_cast<uint8_t*>(values), meta, meta_sm100,
         invalid_groups);
   else
     compress_tiles_kernel<uint16_t, 1><<<grid, kThreads, 0, s>>>(
@@ -416,7 +456,14 @@ extern "C" nm_status nm_decompress(const void* values, const uint8_t* meta, nm_d
   if (gy > cap) gy = cap;
   if (gy > 65535) gy = 65535;
   dim3 grid(unsigned(gx), unsigned(gy < 1 ? 1 : gy)), block(bx, by);
-  if (dtype == NM_F32) {
+  if (dtype == NM_S8) {
+    if (wide)
+      decompress32_kernel<uint8_t><<<grid, block, 0, s>>>(static_cast<const uint8_t*>(values), meta, R, C,
+                                                          static_cast<uint8_t*>(W_out), ldw);
+    else
+      decompress_kernel<uint8_t><<<grid, block, 0, s>>>(static_cast<const uint8_t*>(values), meta, R, C,
+                                                        static_cast<uint8_t*>(W_out), ldw);
+  } else if (dtype == NM_F32) {
     if (wide)
       decompress32_kernel<uint32_t><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C,
                                                            static_cast<uint32_t*>(W_out), ldw);

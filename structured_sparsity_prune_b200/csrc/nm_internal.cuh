@@ -11,8 +11,11 @@ namespace nm {
 // ----------------------------------------------------------------- host side
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool stride_ok(int64_t ld_elems, int esize) { return ((ld_elems * esize) & 15) == 0; }
-inline int esize_of(nm_dtype d) { return d == NM_F32 ? 4 : 2; }
+inline int esize_of(nm_dtype d) { return d == NM_F32 ? 4 : (d == NM_S8 ? 1 : 2); }
+// floating-point element types
 inline bool dtype_ok(int d) { return d == NM_F32 || d == NM_BF16 || d == NM_F16; }
+// ... plus int8, for the calls that only select, move and pack elements
+inline bool dtype_ok_int8(int d) { return dtype_ok(d) || d == NM_S8; }
 
 inline nm_status launch_status() {
   cudaError_t e = cudaGetLastError();
@@ -36,6 +39,11 @@ inline int sm_count() {
 template <typename Bits> __device__ __forceinline__ uint32_t mag_key(Bits b);
 template <> __device__ __forceinline__ uint32_t mag_key<uint32_t>(uint32_t b) { return b & 0x7FFFFFFFu; }
 template <> __device__ __forceinline__ uint32_t mag_key<uint16_t>(uint16_t b) { return uint32_t(b) & 0x7FFFu; }
+// int8 (two's complement): |x|, 0..128
+template <> __device__ __forceinline__ uint32_t mag_key<uint8_t>(uint8_t b) {
+  const int v = static_cast<int8_t>(b);
+  return uint32_t(v < 0 ? -v : v);
+}
 
 // Keep-bits of one group of M keys: bit i set iff fewer than N entries beat
 // entry i (j beats i: key_j > key_i, or key_j == key_i and j < i).

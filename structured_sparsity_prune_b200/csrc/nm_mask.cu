@@ -27,6 +27,9 @@ template <> struct Chunk16<uint32_t> {
 template <> struct Chunk16<uint16_t> {
   static constexpr int kVec = 2;  // 2 x 16 B loads
 };
+template <> struct Chunk16<uint8_t> {
+  static constexpr int kVec = 1;  // 1 x 16 B load
+};
 
 template <typename Bits, int M>
 __global__ void __launch_bounds__(256) mask_vec16_kernel(const Bits* __restrict__ W, int64_t R,
@@ -301,7 +304,7 @@ void dispatch_m(const void* W, int64_t R, int64_t C, int64_t ldw, int N, int M, 
 extern "C" nm_status nm_mask(const void* W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw, int N, int M,
                              uint8_t* mask, int64_t ldm, void* stream) {
   using namespace nm;
-  if (!dtype_ok(dtype)) return NM_ERR_DTYPE;
+  if (!dtype_ok_int8(dtype)) return NM_ERR_DTYPE;
   if (M < 2 || M > 8 || N < 1 || N >= M) return NM_ERR_NM;
   if (R < 0 || C < 0 || C % M != 0 || ldw < C || ldm < C) return NM_ERR_SHAPE;
   if (R == 0 || C == 0) return NM_OK;
@@ -312,6 +315,8 @@ extern "C" nm_status nm_mask(const void* W, nm_dtype dtype, int64_t R, int64_t C
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == NM_F32)
     dispatch_m<uint32_t>(W, R, C, ldw, N, M, mask, ldm, vec, s);
+  else if (dtype == NM_S8)
+    dispatch_m<uint8_t>(W, R, C, ldw, N, M, mask, ldm, vec, s);
   else
     dispatch_m<uint16_t>(W, R, C, ldw, N, M, mask, ldm, vec, s);
   return launch_status();

@@ -1126,6 +1126,7 @@ extern "C" size_t nm_spmm_workspace_bytes(nm_dtype ab_dtype, int64_t R, int64_t 
 extern "C" nm_status nm_spmm(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X,
                              int64_t ldx, void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T,
                              float alpha, float beta, void* workspace, size_t workspace_bytes, void* stream) {
+  if (ab_dtype == NM_S8) return NM_ERR_UNSUPPORTED;  // the int8 sparse product is not built
   if (!dtype_ok(ab_dtype) || (y_dtype != NM_BF16 && y_dtype != NM_F32)) return NM_ERR_DTYPE;
   if (R < 0 || K < 0 || T < 0 || K % 16 != 0 || ldx < T || ldy < T) return NM_ERR_SHAPE;
   if (R > 0x7FFFFFFF - 256 || K > 0x7FFFFFFF - 256 || T > 0x7FFFFFFF - 256) return NM_ERR_SHAPE;

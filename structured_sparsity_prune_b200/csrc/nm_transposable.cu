@@ -85,6 +85,10 @@ template <> struct TKey<uint16_t> {
     return ((uint32_t(bits & 0x7FFFu) + 1u) << 6) | uint32_t(63 - pos);
   }
 };
+template <> struct TKey<uint8_t> {
+  using K = uint32_t;
+  __device__ static K make(uint8_t bits, int pos) { return ((mag_key<uint8_t>(bits) + 1u) << 6) | uint32_t(63 - pos); }
+};
 template <> struct TKey<uint32_t> {
   using K = unsigned long long;
   __device__ static K make(uint32_t bits, int pos) {
@@ -229,7 +233,7 @@ void dispatch_transposable(const void* W, int64_t R, int64_t C, int64_t ldw, int
 extern "C" nm_status nm_mask_transposable(const void* W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw, int N,
                                           int M, uint8_t* mask, int64_t ldm, void* stream) {
   using namespace nm;
-  if (!dtype_ok(dtype)) return NM_ERR_DTYPE;
+  if (!dtype_ok_int8(dtype)) return NM_ERR_DTYPE;
   if (M < 2 || M > 8 || N < 1 || N >= M) return NM_ERR_NM;
   if (R < 0 || C < 0 || R % M != 0 || C % M != 0 || ldw < C || ldm < C) return NM_ERR_SHAPE;
   if (R == 0 || C == 0) return NM_OK;
@@ -239,6 +243,8 @@ extern "C" nm_status nm_mask_transposable(const void* W, nm_dtype dtype, int64_t
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (dtype == NM_F32)
     dispatch_transposable<uint32_t>(W, R, C, ldw, N, M, mask, ldm, s);
+  else if (dtype == NM_S8)
+    dispatch_transposable<uint8_t>(W, R, C, ldw, N, M, mask, ldm, s);
   else
     dispatch_transposable<uint16_t>(W, R, C, ldw, N, M, mask, ldm, s);
   return launch_status();
