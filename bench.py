@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload linear_4096|mlp_pair|decode_T16|decode_T64|decode_T256|decode_T1024|ties_mask|
-                               srste|saliency_mask|transposable_mask|pairs_12]
+                               srste|saliency_mask|transposable_mask|pairs_12|int8_24]
 
 One step is one pass of every step of the path over one batch of synthetic
 input (default: the transformer-linear workload, bf16 W 4096x4096 pruned 2:4
@@ -125,6 +125,11 @@ def make_workload(name: str):
         return {"W": W, "D": nm_inputs.saliency_d(W.shape[1]), "X": None, "R": W.shape[0], "K": W.shape[1], "T": 0,
                 "desc": "saliency-scored 2:4 mask: bf16 W 28672x8192 ~N(0,0.02); d = diag of the upper Cholesky factor"
                         " of the inverse of a damped synthetic Gram matrix (512 calibration rows ~N(0,1))"}
+    elif name == "int8_24":
+        W = nm_inputs.int8_decode()
+        return {"W": W, "I8": True, "X": None, "R": W.shape[0], "K": W.shape[1], "T": 0,
+                "desc": "int8 2:4: the 28672x8192 decode weight quantised to int8; mask 2:4, fused mask+compress,"
+                        " decompress"}
     elif name == "pairs_12":
         W = nm_inputs.fp32_linear()
         return {"W": W, "P12": True, "X": None, "R": W.shape[0], "K": W.shape[1], "T": 0,
@@ -225,9 +230,19 @@ class Step:
         self.nm, self.wl, self.dev = nm, wl, dev
         R, K, T = wl["R"], wl["K"], wl["T"]
         self.kind = "srste" if "G" in wl else "scored" if "D" in wl else "transposable" if "TM" in wl else \
-            "pairs" if "P12" in wl else \
+            "pairs" if "P12" in wl else "int8" if "I8" in wl else \
             ("ties" if wl["X"] is None else ("mlp" if "W2" in wl else "linear"))
         self.W = wl["W"].to(dev)
+        if self.kind == "int8":
+            self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
+            self.values, self.meta, self.img = nm.alloc_compressed(R, K, self.W.dtype, dev)
+            self.Wd = torch.empty_like(self.W)
+            G = R * K
+            self.names = ["nm_mask_s8", "nm_mask_compress_s8", "nm_decompress_s8"]
+            self.bytes = {"nm_mask_s8": G * 2, "nm_mask_compress_s8": G * (1 + 0.5 + 0.25),
+                          "nm_decompress_s8": G * (0.5 + 0.125 + 1)}
+            self.flops = 0
+            return
         if self.kind == "pairs":
             self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
             self.v1, self.m1 = nm.alloc_compressed12(R, K, self.W.dtype, dev)
@@ -320,6 +335,11 @@ class Step:
             return [lambda: nm.nm_mask_scored(self.W, self.D, 2, 4, mask=self.mask)]
         if self.kind == "transposable":
             return [lambda: nm.nm_mask_transposable(self.W, *self.wl["TM"], mask=self.mask)]
+        if self.kind == "int8":
+            K = self.wl["K"]
+            return [lambda: nm.nm_mask(self.W, 2, 4, mask=self.mask),
+                    lambda: nm.nm_mask_compress(self.W, self.values, self.meta, self.img),
+                    lambda: nm.nm_decompress(self.values, self.meta, K, out=self.Wd)]
         if self.kind == "pairs":
             K = self.wl["K"]
             return [lambda: nm.nm_mask(self.W, 1, 2, mask=self.mask),
@@ -374,7 +394,7 @@ class Step:
             return self.GO
         if self.kind in ("scored", "transposable"):
             return self.mask
-        if self.kind == "pairs":
+        if self.kind in ("pairs", "int8"):
             return self.Wd
         return self.masks[1] if self.kind == "ties" else self.Y
 
@@ -478,6 +498,14 @@ def oracle_step(wl, rows: int, threads: int):
         t0 = time.perf_counter()
         oracle.mask_transposable(Wb, *wl["TM"], dtype=oracle.BF16)
         return time.perf_counter() - t0, float(rows * wl["K"] * 3)
+    if "I8" in wl:                # int8 2:4
+        W = wl["W"][:rows].contiguous().numpy()
+        t0 = time.perf_counter()
+        mask = oracle.mask_rank(W, 2, 4)
+        v, m = oracle.compress24(W, mask)
+        oracle.meta_sm100(m, rows, wl["K"])
+        oracle.decompress24(v, m, wl["K"])
+        return time.perf_counter() - t0, float(rows * wl["K"] * (2 + 1.75 + 1.625))
     if "P12" in wl:               # 1:2 family on fp32
         W = wl["W"][:rows].contiguous().numpy()
         t0 = time.perf_counter()
@@ -540,6 +568,7 @@ def cpu_baseline(wl, target_s: float = 15.0):
             "saliency-scored 2:4 mask" if "D" in wl else
             "greedy transposable 4:8 mask" if "TM" in wl else
             "1:2 mask, compress, fused compress, decompress" if "P12" in wl else
+            "int8 2:4 mask, fused mask+compress, decompress" if "I8" in wl else
             "mask at 1:4, 2:4, 4:8, 2:8" if wl["X"] is None else
             "whole step (mask, compress, fused mask+compress, image, decompress, fp64 product)")
     return {"value": units / secs / scale, "unit": unit, "cores": threads, "kind": "oracle",
@@ -687,12 +716,13 @@ def main():
             k.update({"TFLOP/s": tf, "tensor_frac": tf / sparse_peak})
         kernels[name] = k
 
-    if step.kind in ("ties", "srste", "scored", "transposable", "pairs"):
+    if step.kind in ("ties", "srste", "scored", "transposable", "pairs", "int8"):
         units_per_step = sum(step.bytes.values())
         value = whole_job_rate(world, units_per_step, args.steps, total_ms, 1e9)
         unit = "GB/s"
         dom = {"ties": "nm_mask_2:4", "srste": "nm_srste_step", "scored": "nm_mask_scored",
-               "transposable": "nm_mask_transposable", "pairs": "nm_mask_compress12"}[step.kind]
+               "transposable": "nm_mask_transposable", "pairs": "nm_mask_compress12",
+               "int8": "nm_mask_compress_s8"}[step.kind]
         if step.kind == "transposable":
             N_, M_ = wl["TM"]
             ops = transposable_int_ops(M_) * (wl["R"] // M_) * (wl["K"] // M_)

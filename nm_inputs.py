@@ -19,6 +19,8 @@ linear/conv weights; the pages' datasets and trained weights are not used):
                       X bf16 8192xT ~N(0,1) (seed 105+T), T in {16,64,256,1024}
 * ``srste``           the linear_4096 weight and a gradient bf16(1e-3 * N(0,1))
                       of the same shape (seed 6)
+* ``int8_decode``     the decode_skinny weight quantised to int8:
+                      clamp(round(w / 0.02 * 32), -128, 127)
 * ``fp32_linear``     W fp32 8192x8192 = fp32(0.02 * N(0,1)) (seed 8), for the
                       1:2 pattern of sparse TF32
 * ``saliency``        the linear_4096 weight and d of length 4096: the diagonal
@@ -121,3 +123,8 @@ def saliency_d(C: int = 4096, n: int = 512, seed: int | None = None) -> torch.Te
 
 def fp32_linear(R: int = 8192, C: int = 8192) -> torch.Tensor:
     return normal((R, C), SEEDS["fp32_linear.W"], 0.02, torch.float32)
+
+
+def int8_decode() -> torch.Tensor:
+    w = decode_skinny_W().float()
+    return torch.clamp(torch.round(w / 0.02 * 32), -128, 127).to(torch.int8)
