@@ -433,6 +433,39 @@ def kernel_breakdown(step: Step, steps: int, flush: torch.Tensor, graphs=None):
     return {name: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps)] for j, name in enumerate(step.names)}
 
 
+def dense_context(step: Step, reps: int, flush: torch.Tensor):
+    """Context only: the same products as dense bf16 GEMMs in cuBLAS (torch.matmul)
+    on the decompressed weights, timed like the step (L2 flushed before each rep).
+    -> {name: ms} for the product launches of the step, or None."""
+    if step.kind not in ("linear", "mlp"):
+        return None
+    nm = step.nm
+    s = torch.cuda.current_stream()
+    if step.kind == "linear":
+        Wd = nm.nm_decompress(step.values, step.meta, step.wl["K"])
+        jobs = {"nm_spmm": (Wd, step.X)}
+    else:
+        Wu = nm.nm_decompress(step.values, step.meta, step.wl["K"])
+        Wdn = nm.nm_decompress(step.v2, step.m2, step.W2.shape[1])
+        jobs = {"nm_spmm_up": (Wu, step.X), "nm_spmm_down": (Wdn, step.H)}
+    out = {}
+    for name, (A, B) in jobs.items():
+        C = torch.empty((A.shape[0], B.shape[1]), dtype=torch.bfloat16, device=A.device)
+        for _ in range(3):
+            torch.matmul(A, B, out=C)
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            torch.matmul(A, B, out=C)
+            b.record(s)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        out[name] = float(np.median(ts))
+    return out
+
+
 def e2e_steps(step: Step, steps: int, nm, wl, dev):
     """The step through the public API with host buffers, pipelined over two
     replicas of the device buffers: step i+1's inputs copy in (pinned H2D on
@@ -750,6 +783,17 @@ def main():
                            "%s: HBM copy" % peak_src)
     roof["traffic"] = profiled_traffic(args.workload, "nm_spmm" if dom.startswith("nm_spmm") else dom)
 
+    dense = dense_context(step, 20, flush)
+    dense_line = None
+    if dense:
+        dense_line = {"what": "context only: dense bf16 torch.matmul (cuBLAS) on decompress(W), same shapes, "
+                              "L2 flushed, median of 20",
+                      "kernels": {}}
+        for name, ms in dense.items():
+            tf = step.flop_k[name] / (ms * 1e-3) / 1e12
+            dense_line["kernels"][name] = {"dense_us": 1e3 * ms, "dense_TFLOP/s": tf,
+                                           "sparse_over_dense_speedup": ms / float(np.mean(per[name]))}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl)
@@ -765,7 +809,7 @@ def main():
                            "l2": "flushed: 256 MiB write between timed steps, outside the events",
                            "launch": launch_mode,
                            "parallelism": "independent replica per GPU" if world > 1 else "single GPU"},
-                "roofline": roof, "cpu_baseline": cpu,
+                "roofline": roof, "cpu_baseline": cpu, "dense_context": dense_line,
                 "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "method": "public calls with pinned host buffers; H2D, step and D2H of consecutive steps "
                                   "overlapped on three streams over two buffer replicas"},
