@@ -816,26 +816,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const uint32_t taddr = tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TOTAL + half * kc);
       if (early) {
         uint32_t packed[kCols / 2];
+        {
+          // the thread's whole segment in flight at once, one wait, and the
+          // accumulator released before the conversion (columns past kc of a
+          // half-width item are converted but never stored)
+          uint32_t v[kCols];
 #pragma unroll
-        for (int c = 0; c < kCols; c += 64) {
-          if (c >= kc) break;
-          uint32_t v0[32], v1[32];
-          tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c), v0);
-          if (c + 64 <= kCols) tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c + 32), v1);
+          for (int c = 0; c < kCols; c += 32)
+            if (c < kc) tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c), *reinterpret_cast<uint32_t(*)[32]>(&v[c]));
           tmem_ld_wait();
+          fence_before_sync();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(acc_empty_leader[buf]);
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            packed[c / 2 + j] = pack_bf16x2(p.alpha * __uint_as_float(v0[2 * j]), p.alpha * __uint_as_float(v0[2 * j + 1]));
-          if (c + 64 <= kCols) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              packed[c / 2 + 16 + j] =
-                  pack_bf16x2(p.alpha * __uint_as_float(v1[2 * j]), p.alpha * __uint_as_float(v1[2 * j + 1]));
-          }
+          for (int j = 0; j < kCols / 2; ++j)
+            packed[j] = pack_bf16x2(p.alpha * __uint_as_float(v[2 * j]), p.alpha * __uint_as_float(v[2 * j + 1]));
         }
-        fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_remote(acc_empty_leader[buf]);
         if (p.y_tma) {
           // 32 x 32 chunks through this warp's slot: lane = row, four 16-byte
           // pieces per row placed with the 64-byte swizzle (piece ^ ((row >> 1) & 3)),
