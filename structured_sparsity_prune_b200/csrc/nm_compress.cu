@@ -305,58 +305,72 @@ __global__ void __launch_bounds__(256) decompress_kernel(const Bits* __restrict_
 // Decompress, wide unit: one row x 32 columns (four canonical metadata bytes,
 // sixteen values) per thread, 16-byte loads and stores.  Needs C % 32 == 0.
 template <typename Bits>
+__device__ __forceinline__ void expand32(uint32_t mw, const uint4* vv, uint4* dst) {
+  const uint32_t* vw = reinterpret_cast<const uint32_t*>(vv);
+  if constexpr (sizeof(Bits) == 1) {
+    uint32_t o[8];  // value pair of group g: bytes 2g, 2g+1
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const uint32_t nib = (mw >> (4 * g)) & 0xFu;
+      const uint32_t w = vw[g >> 1] >> (16 * (g & 1));
+      o[g] = ((w & 0xFFu) << (8 * (nib & 3u))) | (((w >> 8) & 0xFFu) << (8 * (nib >> 2)));
+    }
+    __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+    __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+  } else if constexpr (sizeof(Bits) == 2) {
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {  // two groups -> one 16-byte store; value pair of group g in word g
+      uint64_t g2[2];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int g = 2 * h + k;
+        const uint32_t nib = (mw >> (4 * g)) & 0xFu;
+        const uint32_t w = vw[g];
+        g2[k] = (uint64_t(w & 0xFFFFu) << (16 * (nib & 3u))) | (uint64_t(w >> 16) << (16 * (nib >> 2)));
+      }
+      __stcs(dst + h, make_uint4(uint32_t(g2[0]), uint32_t(g2[0] >> 32), uint32_t(g2[1]), uint32_t(g2[1] >> 32)));
+    }
+  } else {
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {  // one group -> one 16-byte store
+      const uint32_t nib = (mw >> (4 * g)) & 0xFu;
+      const uint32_t i0 = nib & 3u, i1 = nib >> 2;
+      const uint32_t v0 = vw[2 * g], v1 = vw[2 * g + 1];
+      uint32_t o[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) o[i] = (uint32_t(i) == i0) ? v0 : ((uint32_t(i) == i1) ? v1 : 0u);
+      __stcs(dst + g, make_uint4(o[0], o[1], o[2], o[3]));
+    }
+  }
+}
+
+// A thread takes its unit in two rows (r and r + the row stride of the grid)
+// per iteration and issues both rows' loads before expanding either.
+template <typename Bits>
 __global__ void __launch_bounds__(256) decompress32_kernel(const Bits* __restrict__ values,
                                                            const uint8_t* __restrict__ meta, int64_t R,
                                                            int64_t C, Bits* __restrict__ out, int64_t ldo) {
-  constexpr int kVals = 16 * int(sizeof(Bits)) / 16;  // 16-byte loads of values per unit: 2 or 4
+  constexpr int kVals = 16 * int(sizeof(Bits)) / 16;  // 16-byte loads of values per unit: 1, 2 or 4
   const int64_t upr = C / 32;
   const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
   const int64_t u_step = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += 2 * r_step) {
+    const int64_t r2 = r + r_step;
+    const bool two = r2 < R;
     for (int64_t u = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u < upr; u += u_step) {
+      uint4 vv[kVals], vv2[kVals];
       const uint32_t mw = __ldcs(reinterpret_cast<const uint32_t*>(meta + r * (C / 8) + 4 * u));
-      uint4 vv[kVals];
 #pragma unroll
       for (int i = 0; i < kVals; ++i) vv[i] = __ldcs(reinterpret_cast<const uint4*>(values + r * (C / 2) + 16 * u) + i);
-      uint4* dst = reinterpret_cast<uint4*>(out + r * ldo + 32 * u);
-      if constexpr (sizeof(Bits) == 1) {
-        const uint32_t* vw = reinterpret_cast<const uint32_t*>(vv);  // value pair of group g: bytes 2g, 2g+1
-        uint32_t o[8];
+      uint32_t mw2 = 0;
+      if (two) {
+        mw2 = __ldcs(reinterpret_cast<const uint32_t*>(meta + r2 * (C / 8) + 4 * u));
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const uint32_t nib = (mw >> (4 * g)) & 0xFu;
-          const uint32_t w = vw[g >> 1] >> (16 * (g & 1));
-          o[g] = ((w & 0xFFu) << (8 * (nib & 3u))) | (((w >> 8) & 0xFFu) << (8 * (nib >> 2)));
-        }
-        __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
-        __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
-      } else if constexpr (sizeof(Bits) == 2) {
-        const uint32_t* vw = reinterpret_cast<const uint32_t*>(vv);  // value pair of group g in word g
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {  // two groups -> one 16-byte store
-          uint64_t g2[2];
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int g = 2 * h + k;
-            const uint32_t nib = (mw >> (4 * g)) & 0xFu;
-            const uint32_t w = vw[g];
-            g2[k] = (uint64_t(w & 0xFFFFu) << (16 * (nib & 3u))) | (uint64_t(w >> 16) << (16 * (nib >> 2)));
-          }
-          __stcs(dst + h, make_uint4(uint32_t(g2[0]), uint32_t(g2[0] >> 32), uint32_t(g2[1]), uint32_t(g2[1] >> 32)));
-        }
-      } else {
-        const uint32_t* vw = reinterpret_cast<const uint32_t*>(vv);
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {  // one group -> one 16-byte store
-          const uint32_t nib = (mw >> (4 * g)) & 0xFu;
-          const uint32_t i0 = nib & 3u, i1 = nib >> 2;
-          const uint32_t v0 = vw[2 * g], v1 = vw[2 * g + 1];
-          uint32_t o[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) o[i] = (uint32_t(i) == i0) ? v0 : ((uint32_t(i) == i1) ? v1 : 0u);
-          __stcs(dst + g, make_uint4(o[0], o[1], o[2], o[3]));
-        }
+        for (int i = 0; i < kVals; ++i)
+          vv2[i] = __ldcs(reinterpret_cast<const uint4*>(values + r2 * (C / 2) + 16 * u) + i);
       }
+      expand32<Bits>(mw, vv, reinterpret_cast<uint4*>(out + r * ldo + 32 * u));
+      if (two) expand32<Bits>(mw2, vv2, reinterpret_cast<uint4*>(out + r2 * ldo + 32 * u));
     }
   }
 }
@@ -450,7 +464,8 @@ extern "C" nm_status nm_decompress(const void* values, const uint8_t* meta, nm_d
   while (bx < 256 && bx < opr) bx *= 2;
   const int by = 256 / bx;
   const int64_t gx = (opr + bx - 1) / bx;
-  const int64_t want = int64_t(sm_count()) * 8;
+  static const int per_sm_wide = blocks_per_sm(decompress32_kernel<uint16_t>, 256);
+  const int64_t want = int64_t(sm_count()) * (wide ? per_sm_wide : 8);
   int64_t gy = (R + by - 1) / by;
   const int64_t cap = gx >= want ? 1 : want / gx;
   if (gy > cap) gy = cap;

@@ -33,6 +33,17 @@ inline int sm_count() {
   return n;
 }
 
+// Blocks of `threads` threads of kernel k that one SM holds at once (>= 1).
+template <typename Kernel>
+inline int blocks_per_sm(Kernel k, int threads, size_t smem = 0) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem) != cudaSuccess || n < 1) {
+    (void)cudaGetLastError();
+    n = 1;
+  }
+  return n;
+}
+
 // ----------------------------------------------------------------- device side
 // Magnitude key: IEEE bits with the sign cleared.  Elements are handled as raw
 // 16- or 32-bit patterns; no floating-point arithmetic touches them.

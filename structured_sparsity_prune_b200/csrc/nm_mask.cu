@@ -31,65 +31,98 @@ template <> struct Chunk16<uint8_t> {
   static constexpr int kVec = 1;  // 1 x 16 B load
 };
 
+// Keep-mask bytes of one 16-byte chunk of weights, groups of M (M | 16).
+template <typename Bits, int M>
+__device__ __forceinline__ uint4 select_chunk(const uint4 (&v)[Chunk16<Bits>::kVec], int N) {
+  const Bits* e = reinterpret_cast<const Bits*>(v);
+  uint32_t out[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int g = 0; g < 16 / M; ++g) {
+    uint32_t key[M];
+#pragma unroll
+    for (int i = 0; i < M; ++i) key[i] = mag_key<Bits>(e[g * M + i]);
+    const uint32_t kb = keep_bits<M>(key, N);
+#pragma unroll
+    for (int i = 0; i < M; ++i) {
+      const int pos = g * M + i;  // byte position in the 16-byte chunk
+      out[pos >> 2] |= ((kb >> i) & 1u) << (8 * (pos & 3));
+    }
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+// Rows r and r + the row stride of the grid per iteration, both rows' loads
+// issued before selecting in either.  For 8- and 16-bit elements in groups of
+// eight the selection arithmetic, not the loads, bounds the kernel, and the
+// second row's registers would only cost occupancy: one row at a time there.
 template <typename Bits, int M>
 __global__ void __launch_bounds__(256) mask_vec16_kernel(const Bits* __restrict__ W, int64_t R,
                                                          int64_t cpr, int64_t ldw, int N,
                                                          uint8_t* __restrict__ mask, int64_t ldm) {
   static_assert(16 % M == 0, "vector path needs M | 16");
   constexpr int kVec = Chunk16<Bits>::kVec;
+  constexpr int kRows = (sizeof(Bits) <= 2 && M == 8) ? 1 : 2;
   const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
   const int64_t c_step = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += kRows * r_step) {
+    const int64_t r2 = r + r_step;
+    const bool two = kRows == 2 && r2 < R;
     const uint4* wrow = reinterpret_cast<const uint4*>(W + r * ldw);
-    uint4* mrow = reinterpret_cast<uint4*>(mask + r * ldm);
+    const uint4* wrow2 = reinterpret_cast<const uint4*>(W + (two ? r2 : r) * ldw);
     for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < cpr; c += c_step) {
-      uint4 v[kVec];
+      uint4 v[kVec], v2[kVec];
 #pragma unroll
       for (int i = 0; i < kVec; ++i) v[i] = __ldcs(wrow + c * kVec + i);
-      const Bits* e = reinterpret_cast<const Bits*>(v);
-      uint32_t out[4] = {0u, 0u, 0u, 0u};
+      if (two) {
 #pragma unroll
-      for (int g = 0; g < 16 / M; ++g) {
-        uint32_t key[M];
-#pragma unroll
-        for (int i = 0; i < M; ++i) key[i] = mag_key<Bits>(e[g * M + i]);
-        const uint32_t kb = keep_bits<M>(key, N);
-#pragma unroll
-        for (int i = 0; i < M; ++i) {
-          const int pos = g * M + i;  // byte position in the 16-byte chunk
-          out[pos >> 2] |= ((kb >> i) & 1u) << (8 * (pos & 3));
-        }
+        for (int i = 0; i < kVec; ++i) v2[i] = __ldcs(wrow2 + c * kVec + i);
       }
-      __stcs(mrow + c, make_uint4(out[0], out[1], out[2], out[3]));
+      __stcs(reinterpret_cast<uint4*>(mask + r * ldm) + c, select_chunk<Bits, M>(v, N));
+      if (two) __stcs(reinterpret_cast<uint4*>(mask + r2 * ldm) + c, select_chunk<Bits, M>(v2, N));
     }
   }
 }
 
 // M = 4 fast path: 16 elements (four groups) per thread, the branch-free
-// selection of drop4 and the byte packing of keep_bytes4.
+// selection of drop4 and the byte packing of keep_bytes4.  A thread takes its
+// chunk of two rows (r and r + the row stride of the grid) per iteration and
+// issues both rows' loads before selecting in either; five blocks share an SM
+// (the grid is sized to exactly what the SMs hold).
 template <typename Bits, int N>
-__global__ void __launch_bounds__(256) mask4_vec16_kernel(const Bits* __restrict__ W, int64_t R, int64_t cpr,
+__device__ __forceinline__ uint4 select4_chunk(const uint4 (&v)[Chunk16<Bits>::kVec]) {
+  const Bits* e = reinterpret_cast<const Bits*>(v);
+  uint32_t out[4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint32_t x0, x1, x2, x3;
+    drop4<N>(mag_key<Bits>(e[4 * g]), mag_key<Bits>(e[4 * g + 1]), mag_key<Bits>(e[4 * g + 2]),
+             mag_key<Bits>(e[4 * g + 3]), x0, x1, x2, x3);
+    out[g] = keep_bytes4(x0, x1, x2, x3);
+  }
+  return make_uint4(out[0], out[1], out[2], out[3]);
+}
+
+template <typename Bits, int N>
+__global__ void __launch_bounds__(256, 5) mask4_vec16_kernel(const Bits* __restrict__ W, int64_t R, int64_t cpr,
                                                           int64_t ldw, uint8_t* __restrict__ mask, int64_t ldm) {
   constexpr int kVec = Chunk16<Bits>::kVec;
   const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
   const int64_t c_step = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += 2 * r_step) {
+    const int64_t r2 = r + r_step;
+    const bool two = r2 < R;
     const uint4* wrow = reinterpret_cast<const uint4*>(W + r * ldw);
-    uint4* mrow = reinterpret_cast<uint4*>(mask + r * ldm);
+    const uint4* wrow2 = reinterpret_cast<const uint4*>(W + (two ? r2 : r) * ldw);
     for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < cpr; c += c_step) {
-      uint4 v[kVec];
+      uint4 v[kVec], v2[kVec];
 #pragma unroll
       for (int i = 0; i < kVec; ++i) v[i] = __ldcs(wrow + c * kVec + i);
-      const Bits* e = reinterpret_cast<const Bits*>(v);
-      uint32_t out[4];
+      if (two) {
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        uint32_t x0, x1, x2, x3;
-        drop4<N>(mag_key<Bits>(e[4 * g]), mag_key<Bits>(e[4 * g + 1]), mag_key<Bits>(e[4 * g + 2]),
-                 mag_key<Bits>(e[4 * g + 3]), x0, x1, x2, x3);
-        out[g] = keep_bytes4(x0, x1, x2, x3);
+        for (int i = 0; i < kVec; ++i) v2[i] = __ldcs(wrow2 + c * kVec + i);
       }
-      __stcs(mrow + c, make_uint4(out[0], out[1], out[2], out[3]));
+      __stcs(reinterpret_cast<uint4*>(mask + r * ldm) + c, select4_chunk<Bits, N>(v));
+      if (two) __stcs(reinterpret_cast<uint4*>(mask + r2 * ldm) + c, select4_chunk<Bits, N>(v2));
     }
   }
 }
@@ -214,12 +247,14 @@ __global__ void __launch_bounds__(256) scored_scalar_kernel(const Bits* __restri
 
 // 2D launch shape: x over the units of a row, y over rows; about 8 blocks of
 // 256 threads per SM in total.
-void shape2d(int64_t R, int64_t units, dim3& grid, dim3& block) {
+// x over the 16-byte chunks of a row, y over rows; at most per_sm blocks per SM
+// (the kernel's occupancy), so the whole grid is resident at once.
+void shape2d(int64_t R, int64_t units, dim3& grid, dim3& block, int per_sm = 8) {
   int bx = 32;
   while (bx < 256 && bx < units) bx *= 2;
   const int by = 256 / bx;
   const int64_t gx = (units + bx - 1) / bx;
-  const int64_t want = int64_t(sm_count()) * 8;
+  const int64_t want = int64_t(sm_count()) * per_sm;
   int64_t gy = (R + by - 1) / by;
   const int64_t cap_y = gx >= want ? 1 : want / gx;
   if (gy > cap_y) gy = cap_y;
@@ -234,7 +269,8 @@ void launch_mask(const void* W, int64_t R, int64_t C, int64_t ldw, int N, uint8_
   dim3 grid, block;
   if constexpr (M == 4) {
     if (vec) {
-      shape2d(R, C / 16, grid, block);
+      static const int per_sm = blocks_per_sm(mask4_vec16_kernel<Bits, 2>, 256);
+      shape2d(R, C / 16, grid, block, per_sm);
       const Bits* w = static_cast<const Bits*>(W);
       if (N == 1) mask4_vec16_kernel<Bits, 1><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);
       else if (N == 2) mask4_vec16_kernel<Bits, 2><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);
@@ -244,7 +280,8 @@ void launch_mask(const void* W, int64_t R, int64_t C, int64_t ldw, int N, uint8_
   }
   if constexpr (16 % M == 0) {
     if (vec) {
-      shape2d(R, C / 16, grid, block);
+      static const int per_sm = blocks_per_sm(mask_vec16_kernel<Bits, M>, 256);
+      shape2d(R, C / 16, grid, block, per_sm);
       mask_vec16_kernel<Bits, M><<<grid, block, 0, s>>>(static_cast<const Bits*>(W), R, C / 16, ldw, N,
                                                         mask, ldm);
       return;
