@@ -7,13 +7,15 @@
 // values.  The hardware layout of the indices is the PTX ISA's tcgen05
 // sparse-matrix metadata (the pages do not give one).
 //
-// All kernels here are HBM-bound streams.  The compressing kernels walk the
-// matrix in 128-row x 128-column tiles (one 2048-byte block of the metadata
-// image per tile): each thread takes a (row, 32-column slice) unit, reads its
-// 32 weights with 16-byte loads, selects/compresses in registers, writes its
-// 16 values and 4 canonical metadata bytes with vector stores, and drops the
-// two 16-bit image pieces into shared memory; the block then writes the
-// finished 2048-byte image block with one coalesced 16-byte store per thread.
+// All kernels here are HBM-bound streams.  A compressing thread takes a (row,
+// 32-column) unit: it reads the unit's 32 weights with 16-byte loads,
+// selects/compresses in registers, and writes its 16 values and 4 canonical
+// metadata bytes with vector stores.  When C % 32 == 0 the units are streamed
+// row by row (two rows per thread, whose image pieces share 4-byte words that
+// the thread writes itself); otherwise a block walks 128-row x 128-column
+// tiles, drops the units' 16-bit image pieces into shared memory and writes
+// each finished 2048-byte image block with one coalesced 16-byte store per
+// thread.
 #include "nm_internal.cuh"
 
 namespace nm {
@@ -181,6 +183,106 @@ __global__ void __launch_bounds__(kThreads) compress_tiles_kernel(
         __stcs(reinterpret_cast<uint4*>(img + tile * 2048) + threadIdx.x, v);
       }
       __syncthreads();
+    }
+  }
+  if constexpr (MODE == 1) {
+    if (invalid_groups != nullptr) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) invalid += __shfl_xor_sync(0xFFFFFFFFu, invalid, off);
+      if ((threadIdx.x & 31) == 0 && invalid != 0) atomicAdd(invalid_groups, invalid);
+    }
+  }
+}
+
+// The four quads of a (row, 32-column) unit are contiguous: store them with
+// as few 16-byte stores as the element size allows.
+template <typename Bits>
+__device__ __forceinline__ void store_unit(const Quad<Bits> (&q)[4], Bits* p) {
+  uint4* d = reinterpret_cast<uint4*>(p);
+  if constexpr (sizeof(Bits) == 1) {
+    __stcs(d, make_uint4(q[0].v, q[1].v, q[2].v, q[3].v));
+  } else if constexpr (sizeof(Bits) == 2) {
+    __stcs(d, make_uint4(q[0].v.x, q[0].v.y, q[1].v.x, q[1].v.y));
+    __stcs(d + 1, make_uint4(q[2].v.x, q[2].v.y, q[3].v.x, q[3].v.y));
+  } else {
+#pragma unroll
+    for (int o = 0; o < 4; ++o) __stcs(d + o, q[o].v);
+  }
+}
+
+// Row-streaming form for C % 32 == 0.  A thread takes one 32-column unit u in
+// the two rows r and r + 8 with r % 16 < 8: the 16-bit image pieces of those
+// two rows share each 4-byte word of the image block (low half row r, high
+// half row r + 8), so the thread writes its two image words directly -- no
+// shared memory, no block barrier.  Consecutive threads take consecutive units
+// of the same rows, so a warp reads 32 contiguous units of each row.  The
+// grid covers the image's padded extent (rows up to a multiple of 128, units
+// up to a multiple of 4): threads outside the matrix write only pad pieces.
+// For 8- and 16-bit elements both rows' loads are issued before either is
+// used; fp32 (128 bytes per unit and row) takes the rows one after the other.
+// Two blocks share an SM: the kernel needs ~128 registers a thread, and a
+// tighter bound spills.
+template <typename Bits, int MODE>
+__global__ void __launch_bounds__(256, 2) compress_rows_kernel(
+    const Bits* __restrict__ W, int64_t ldw, const uint8_t* __restrict__ mask, int64_t ldm, int64_t R,
+    int64_t C, Bits* __restrict__ values, uint8_t* __restrict__ meta, uint8_t* __restrict__ img,
+    int32_t* __restrict__ invalid_groups) {
+  constexpr int kAhead = sizeof(Bits) <= 2 ? 2 : 1;  // rows whose loads are in flight together
+  const int64_t kt_count = (C + 127) / 128;
+  const int64_t units = kt_count * 4;                // padded units per row
+  const int64_t pairs = ((R + 127) / 128) * 64;      // padded row pairs
+  const int64_t p_step = int64_t(gridDim.y) * blockDim.y;
+  const int64_t u_step = int64_t(gridDim.x) * blockDim.x;
+  int invalid = 0;
+  for (int64_t p = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; p < pairs; p += p_step) {
+    const int64_t r0 = 16 * (p >> 3) + (p & 7);
+    for (int64_t u = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u < units; u += u_step) {
+      const int64_t c0 = 32 * u;
+      uint32_t piece[2][2];  // [row r0 / r0 + 8][columns c0 / c0 + 16]
+#pragma unroll
+      for (int h0 = 0; h0 < 2; h0 += kAhead) {
+        Oct<Bits> e[kAhead][4];
+        uint2 m[kAhead][4];
+        bool in[kAhead];
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k) {
+          const int64_t r = r0 + 8 * (h0 + k);
+          in[k] = r < R && c0 < C;
+          if (in[k]) {
+#pragma unroll
+            for (int o = 0; o < 4; ++o) e[k][o].load(W + r * ldw + c0 + 8 * o);
+            if constexpr (MODE == 1) {
+              const uint4* mp = reinterpret_cast<const uint4*>(mask + r * ldm + c0);
+              const uint4 a = __ldcs(mp), b = __ldcs(mp + 1);
+              m[k][0] = make_uint2(a.x, a.y); m[k][1] = make_uint2(a.z, a.w);
+              m[k][2] = make_uint2(b.x, b.y); m[k][3] = make_uint2(b.z, b.w);
+            }
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k) {
+          const int64_t r = r0 + 8 * (h0 + k);
+          uint32_t bytes[4] = {kPadByte, kPadByte, kPadByte, kPadByte};
+          if (in[k]) {
+            Quad<Bits> q[4];
+#pragma unroll
+            for (int o = 0; o < 4; ++o) bytes[o] = compress_octet<Bits, MODE>(e[k][o], m[k][o], q[o], invalid);
+            store_unit<Bits>(q, values + r * (C / 2) + c0 / 2);
+            __stcs(reinterpret_cast<uint32_t*>(meta + r * (C / 8) + c0 / 8),
+                   bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24));
+          }
+          piece[h0 + k][0] = bytes[0] | (bytes[1] << 8);
+          piece[h0 + k][1] = bytes[2] | (bytes[3] << 8);
+        }
+      }
+      if (img != nullptr) {
+        uint8_t* blk = img + ((r0 >> 7) * kt_count + (u >> 2)) * 2048;
+        const uint32_t lane0 = uint32_t(r0 & 7) + 16u * uint32_t((r0 & 127) >> 4);
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf)
+          __stcs(reinterpret_cast<uint32_t*>(blk + (lane0 + 8u * hf) * 16u + (u & 3) * 4),
+                 piece[0][hf] | (piece[1][hf] << 16));
+      }
     }
   }
   if constexpr (MODE == 1) {
@@ -381,6 +483,34 @@ int tile_grid(int64_t R, int64_t C) {
   return int(tiles < want ? tiles : want);
 }
 
+// Compressing launch: the row-streaming kernel when C % 32 == 0 (x over the
+// padded units of a row, y over padded row pairs, as many blocks as the SMs
+// hold at once), else the tile kernel.
+template <typename Bits, int MODE>
+void launch_compress(const void* W, int64_t ldw, const uint8_t* mask, int64_t ldm, int64_t R, int64_t C,
+                     void* values, uint8_t* meta, uint8_t* img, int32_t* invalid_groups, cudaStream_t s) {
+  const Bits* w = static_cast<const Bits*>(W);
+  Bits* v = static_cast<Bits*>(values);
+  if (C % 32 != 0) {
+    compress_tiles_kernel<Bits, MODE><<<tile_grid(R, C), kThreads, 0, s>>>(w, ldw, mask, ldm, R, C, v, meta, img,
+                                                                           invalid_groups);
+    return;
+  }
+  static const int per_sm = blocks_per_sm(compress_rows_kernel<Bits, MODE>, 256);
+  const int64_t units = ((C + 127) / 128) * 4, pairs = ((R + 127) / 128) * 64;
+  int bx = 32;
+  while (bx < 256 && bx < units) bx *= 2;
+  const int by = 256 / bx;
+  const int64_t gx = (units + bx - 1) / bx;
+  const int64_t cap = int64_t(per_sm) * sm_count();
+  int64_t gy = (pairs + by - 1) / by;
+  const int64_t cap_y = gx >= cap ? 1 : cap / gx;
+  if (gy > cap_y) gy = cap_y;
+  if (gy > 65535) gy = 65535;
+  dim3 grid(unsigned(gx > 2147483647 ? 2147483647 : gx), unsigned(gy < 1 ? 1 : gy)), block(bx, by);
+  compress_rows_kernel<Bits, MODE><<<grid, block, 0, s>>>(w, ldw, mask, ldm, R, C, v, meta, img, invalid_groups);
+}
+
 nm_status check_common(const void* W, nm_dtype dtype, int64_t R, int64_t C, int64_t ldw) {
   if (!dtype_ok_int8(dtype)) return NM_ERR_DTYPE;
   if (R < 0 || C < 0 || C % 8 != 0 || ldw < C) return NM_ERR_SHAPE;
@@ -403,19 +533,12 @@ extern "C" nm_status nm_mask_compress(const void* W, nm_dtype dtype, int64_t R, 
       !stride_ok(ldw, esize_of(dtype)))
     return NM_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int grid = tile_grid(R, C);
   if (dtype == NM_F32)
-    compress_tiles_kernel<uint32_t, 0><<<grid, kThreads, 0, s>>>(
-        static_cast<const uint32_t*>(W), ldw, nullptr, 0, R, C, static_cast<uint32_t*>(values), meta,
-        meta_sm100, nullptr);
+    launch_compress<uint32_t, 0>(W, ldw, nullptr, 0, R, C, values, meta, meta_sm100, nullptr, s);
   else if (dtype == NM_S8)
-    compress_tiles_kernel<uint8_t, 0><<<grid, kThreads, 0, s>>>(
-        static_cast<const uint8_t*>(W), ldw, nullptr, 0, R, C, static_cast<uint8_t*>(values), meta,
-        meta_sm100, nullptr);
+    launch_compress<uint8_t, 0>(W, ldw, nullptr, 0, R, C, values, meta, meta_sm100, nullptr, s);
   else
-    compress_tiles_kernel<uint16_t, 0><<<grid, kThreads, 0, s>>>(
-        static_cast<const uint16_t*>(W), ldw, nullptr, 0, R, C, static_cast<uint16_t*>(values), meta,
-        meta_sm100, nullptr);
+    launch_compress<uint16_t, 0>(W, ldw, nullptr, 0, R, C, values, meta, meta_sm100, nullptr, s);
   return launch_status();
 }
 
@@ -432,19 +555,12 @@ extern "C" nm_status nm_compress(const void* W, const uint8_t* mask, nm_dtype dt
       (invalid_groups && (reinterpret_cast<uintptr_t>(invalid_groups) & 3u)))
     return NM_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int grid = tile_grid(R, C);
   if (dtype == NM_F32)
-    compress_tiles_kernel<uint32_t, 1><<<grid, kThreads, 0, s>>>(
-        static_cast<const uint32_t*>(W), ldw, mask, ldm, R, C, static_cast<uint32_t*>(values), meta, meta_sm100,
-        invalid_groups);
+    launch_compress<uint32_t, 1>(W, ldw, mask, ldm, R, C, values, meta, meta_sm100, invalid_groups, s);
   else if (dtype == NM_S8)
-    compress_tiles_kernel<uint8_t, 1><<<grid, kThreads, 0, s>>>(
-        static_cast<const uint8_t*>(W), ldw, mask, ldm, R, C, static_cast<uint8_t*>(values), meta, meta_sm100,
-        invalid_groups);
+    launch_compress<uint8_t, 1>(W, ldw, mask, ldm, R, C, values, meta, meta_sm100, invalid_groups, s);
   else
-    compress_tiles_kernel<uint16_t, 1><<<grid, kThreads, 0, s>>>(
-        static_cast<const uint16_t*>(W), ldw, mask, ldm, R, C, static_cast<uint16_t*>(values), meta, meta_sm100,
-        invalid_groups);
+    launch_compress<uint16_t, 1>(W, ldw, mask, ldm, R, C, values, meta, meta_sm100, invalid_groups, s);
   return launch_status();
 }
 

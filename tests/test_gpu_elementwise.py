@@ -12,7 +12,7 @@ import structured_sparsity_prune_b200 as nm
 
 pytestmark = pytest.mark.gpu
 
-CODE = {torch.float32: oracle.F32, torch.bfloat16: oracle.BF16, torch.float16: oracle.F16}
+CODE = {torch.float32: oracle.F32, torch.bfloat16: oracle.BF16, torch.float16: oracle.F16, torch.int8: oracle.S8}
 
 
 def _bits(t: torch.Tensor) -> np.ndarray:
@@ -97,7 +97,10 @@ def _check_compressed(W, values, meta, img, code):
         assert np.array_equal(img.cpu().numpy(), oracle.meta_sm100(m_ref, R, C))
 
 
-SHAPES = [(128, 128), (256, 256), (67, 200), (300, 392), (1, 8), (129, 136), (5, 32), (250, 1000)]
+# C % 32 == 0 takes the row-streaming compressor (image padded in rows and in
+# 32-column units: 77 x 160, 300 x 96, 5 x 32); other C the tile compressor.
+SHAPES = [(128, 128), (256, 256), (67, 200), (300, 392), (1, 8), (129, 136), (5, 32), (250, 1000),
+          (77, 160), (300, 96), (1000, 384), (16, 4096)]
 
 
 @pytest.mark.parametrize("R,C", SHAPES)
@@ -116,7 +119,18 @@ def test_mask_compress_without_image_and_strided():
     _check_compressed(full[:, :C], values, meta, None, oracle.BF16)
 
 
-@pytest.mark.parametrize("R,C", [(256, 256), (67, 200), (130, 64)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.int8])
+def test_mask_compress_strided_with_image(dtype):
+    R, C = 200, 160
+    if dtype == torch.int8:
+        full = torch.randint(-128, 128, (R, C + 32), generator=torch.Generator().manual_seed(5), dtype=torch.int8)
+    else:
+        full = _rand((R, C + 32), dtype, 43, "normal")
+    values, meta, img = nm.nm_mask_compress(full.cuda()[:, :C])
+    _check_compressed(full[:, :C], values, meta, img, CODE[dtype])
+
+
+@pytest.mark.parametrize("R,C", [(256, 256), (67, 200), (130, 64), (77, 160), (1000, 384)])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_compress_with_given_mask(R, C, dtype):
     W = _rand((R, C), dtype, 7, "normal")
