@@ -341,6 +341,39 @@ __global__ void __launch_bounds__(kThreads) meta_image_kernel(const uint8_t* __r
   }
 }
 
+// Image from canonical metadata, row-pair form for C % 128 == 0.  A warp takes
+// one 16-row group of the image and four consecutive 128-column tiles; lane
+// (q, j) reads the 16 canonical bytes of rows r = 16g + q and r + 8 in tile j
+// and writes the two 16-byte image chunks those rows share: chunk lanes q and
+// q + 8 of the group, each word holding row r's piece in its low half and row
+// r + 8's in its high half.  The eight lanes of a tile write 128 contiguous
+// bytes per store; rows past R are written as pad pieces.
+__global__ void __launch_bounds__(256) meta_image_rows_kernel(const uint8_t* __restrict__ meta, int64_t R,
+                                                              int64_t C, uint8_t* __restrict__ img) {
+  const int64_t kt_count = C / 128;
+  const int64_t quads = (kt_count + 3) / 4;
+  const int64_t items = ((R + 127) / 128) * 8 * quads;
+  const int q = threadIdx.x & 7, j = (threadIdx.x >> 3) & 3;
+  const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t it = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); it < items; it += warps) {
+    const int64_t g = it / quads, kt = (it - g * quads) * 4 + j;
+    if (kt >= kt_count) continue;
+    const int64_t r = 16 * g + q;
+    const uint4 pad = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+    uint4 a = pad, b = pad;
+    if (r < R) a = __ldcs(reinterpret_cast<const uint4*>(meta + r * (C / 8) + kt * 16));
+    if (r + 8 < R) b = __ldcs(reinterpret_cast<const uint4*>(meta + (r + 8) * (C / 8) + kt * 16));
+    uint8_t* blk = img + ((r >> 7) * kt_count + kt) * 2048;
+    const uint32_t lane0 = uint32_t(r & 7) + 16u * uint32_t((r & 127) >> 4);
+    __stcs(reinterpret_cast<uint4*>(blk + lane0 * 16u),
+           make_uint4(__byte_perm(a.x, b.x, 0x5410), __byte_perm(a.y, b.y, 0x5410), __byte_perm(a.z, b.z, 0x5410),
+                      __byte_perm(a.w, b.w, 0x5410)));
+    __stcs(reinterpret_cast<uint4*>(blk + (lane0 + 8u) * 16u),
+           make_uint4(__byte_perm(a.x, b.x, 0x7632), __byte_perm(a.y, b.y, 0x7632), __byte_perm(a.z, b.z, 0x7632),
+                      __byte_perm(a.w, b.w, 0x7632)));
+  }
+}
+
 // Decompress: unit = one row x 8 columns (one metadata byte, four values).
 template <typename Bits>
 __global__ void __launch_bounds__(256) decompress_kernel(const Bits* __restrict__ values,
@@ -618,6 +651,14 @@ extern "C" nm_status nm_meta_to_sm100(const uint8_t* meta, int64_t R, int64_t C,
   if (R == 0 || C == 0) return NM_OK;
   if (meta == nullptr || meta_sm100 == nullptr) return NM_ERR_NULL;
   if (!aligned16(meta) || !aligned16(meta_sm100)) return NM_ERR_ALIGN;
-  meta_image_kernel<<<tile_grid(R, C), kThreads, 0, static_cast<cudaStream_t>(stream)>>>(meta, R, C, meta_sm100);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (C % 128 == 0) {
+    static const int per_sm = blocks_per_sm(meta_image_rows_kernel, 256);
+    const int64_t warps = ((R + 127) / 128) * 8 * ((C / 128 + 3) / 4);
+    const int64_t blocks = (warps + 7) / 8, cap = int64_t(per_sm) * sm_count();
+    meta_image_rows_kernel<<<unsigned(blocks < cap ? blocks : cap), 256, 0, s>>>(meta, R, C, meta_sm100);
+  } else {
+    meta_image_kernel<<<tile_grid(R, C), kThreads, 0, s>>>(meta, R, C, meta_sm100);
+  }
   return launch_status();
 }
