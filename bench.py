@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                     [--workload linear_4096|mlp_pair|decode_T16|decode_T64|decode_T256|decode_T1024|ties_mask|
-                               srste|saliency_mask|transposable_mask|pairs_12|int8_24]
+                               srste|saliency_mask|transposable_mask|transposable_24|pairs_12|int8_24]
 
 One step is one pass of every step of the path over one batch of synthetic
 input (default: the transformer-linear workload, bf16 W 4096x4096 pruned 2:4
@@ -139,6 +139,12 @@ def make_workload(name: str):
         W, _ = nm_inputs.linear_4096()
         return {"W": W, "TM": (4, 8), "X": None, "R": 4096, "K": 4096, "T": 0,
                 "desc": "greedy transposable 4:8 mask over 8x8 blocks: bf16 W 4096x4096 ~N(0,0.02)"}
+    elif name == "transposable_24":
+        W, X = nm_inputs.linear_4096()
+        return {"W": W, "X": X, "DY": nm_inputs.linear_4096_grad(), "T24": True, "R": 4096, "K": 4096, "T": 4096,
+                "desc": "transposable 2:4 training step of the transformer linear: bf16 W 4096x4096 ~N(0,0.02), "
+                        "X 4096x4096 and dY 4096x4096 ~N(0,1); greedy transposable 2:4 mask (4x4 blocks), "
+                        "compress W and W^T under it, Y = W X and dX = W^T dY on the sparse tensor cores"}
     elif name == "ties_mask":
         W = nm_inputs.ties_fp32()
         return {"W": W, "X": None, "R": 8192, "K": 8192, "T": 0,
@@ -230,6 +236,7 @@ class Step:
         self.nm, self.wl, self.dev = nm, wl, dev
         R, K, T = wl["R"], wl["K"], wl["T"]
         self.kind = "srste" if "G" in wl else "scored" if "D" in wl else "transposable" if "TM" in wl else \
+            "trans24" if "T24" in wl else \
             "pairs" if "P12" in wl else "int8" if "I8" in wl else \
             ("ties" if wl["X"] is None else ("mlp" if "W2" in wl else "linear"))
         self.W = wl["W"].to(dev)
@@ -288,6 +295,24 @@ class Step:
         self.X = _dev_x(wl["X"], dev)
         v, m, img = nm.alloc_compressed(R, K, self.W.dtype, dev)
         self.values, self.meta, self.img = v, m, img
+        if self.kind == "trans24":
+            self.DY = _dev_x(wl["DY"], dev)
+            self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
+            self.v_t, self.m_t, self.img_t = nm.alloc_compressed(K, R, self.W.dtype, dev)
+            self.Y = torch.empty((R, T), dtype=torch.bfloat16, device=dev)
+            self.DX = torch.empty((K, T), dtype=torch.bfloat16, device=dev)
+            ws = max(nm.nm_spmm_workspace_bytes(self.W.dtype, R, K, T), nm.nm_spmm_workspace_bytes(self.W.dtype, K, R, T))
+            self.ws = torch.empty((ws,), dtype=torch.uint8, device=dev) if ws else None
+            self.names = ["nm_mask_transposable_2:4", "nm_compress", "nm_compress_t", "nm_spmm_fwd", "nm_spmm_bwd"]
+            G = R * K
+            es = self.W.element_size()
+            self.bytes = {"nm_mask_transposable_2:4": G * (es + 1), "nm_compress": G * (es + 1 + es / 2 + 0.25),
+                          "nm_compress_t": G * (es + 1 + es / 2 + 0.25),
+                          "nm_spmm_fwd": G * (es / 2 + 0.125) + K * T * es + R * T * 2,
+                          "nm_spmm_bwd": G * (es / 2 + 0.125) + R * T * es + K * T * 2}
+            self.flop_k = {"nm_spmm_fwd": 2.0 * R * K * T, "nm_spmm_bwd": 2.0 * R * K * T}
+            self.flops = sum(self.flop_k.values())
+            return
         if self.kind == "mlp":
             self.W2 = wl["W2"].to(dev)
             R2, K2 = self.W2.shape
@@ -349,6 +374,12 @@ class Step:
         if self.kind == "ties":
             return [(lambda i=i, N=N, M=M: nm.nm_mask(self.W, N, M, mask=self.masks[i]))
                     for i, (N, M) in enumerate([(1, 4), (2, 4), (4, 8), (2, 8)])]
+        if self.kind == "trans24":
+            return [lambda: nm.nm_mask_transposable(self.W, 2, 4, mask=self.mask),
+                    lambda: nm.nm_compress(self.W, self.mask, self.values, self.meta, self.img),
+                    lambda: nm.nm_compress_t(self.W, self.mask, self.v_t, self.m_t, self.img_t),
+                    lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.Y, workspace=self.ws),
+                    lambda: nm.nm_spmm(self.v_t, self.img_t, self.DY, Y=self.DX, workspace=self.ws)]
         if self.kind == "mlp":
             return [lambda: nm.nm_mask_compress(self.W, self.values, self.meta, self.img),
                     lambda: nm.nm_mask_compress(self.W2, self.v2, self.m2, self.img2),
@@ -396,6 +427,8 @@ class Step:
             return self.mask
         if self.kind in ("pairs", "int8"):
             return self.Wd
+        if self.kind == "trans24":
+            return self.DX
         return self.masks[1] if self.kind == "ties" else self.Y
 
 
@@ -437,13 +470,16 @@ def dense_context(step: Step, reps: int, flush: torch.Tensor):
     """Context only: the same products as dense bf16 GEMMs in cuBLAS (torch.matmul)
     on the decompressed weights, timed like the step (L2 flushed before each rep).
     -> {name: ms} for the product launches of the step, or None."""
-    if step.kind not in ("linear", "mlp"):
+    if step.kind not in ("linear", "mlp", "trans24"):
         return None
     nm = step.nm
     s = torch.cuda.current_stream()
     if step.kind == "linear":
         Wd = nm.nm_decompress(step.values, step.meta, step.wl["K"])
         jobs = {"nm_spmm": (Wd, step.X)}
+    elif step.kind == "trans24":
+        Wd = nm.nm_decompress(step.values, step.meta, step.wl["K"])
+        jobs = {"nm_spmm_fwd": (Wd, step.X), "nm_spmm_bwd": (Wd.t().contiguous(), step.DY)}
     else:
         Wu = nm.nm_decompress(step.values, step.meta, step.wl["K"])
         Wdn = nm.nm_decompress(step.v2, step.m2, step.W2.shape[1])
@@ -474,7 +510,7 @@ def e2e_steps(step: Step, steps: int, nm, wl, dev):
     its inputs in and its result out.
     -> (device ms of the whole run, H2D bytes per step, D2H bytes per step)"""
     reps = [step, Step(nm, wl, dev)]
-    names = [k for k in ("W", "X", "W2", "G", "D") if wl.get(k) is not None]
+    names = [k for k in ("W", "X", "W2", "G", "D", "DY") if wl.get(k) is not None]
     host = {k: wl[k].pin_memory() for k in names}
     outs = [torch.empty(r.result().shape, dtype=r.result().dtype).pin_memory() for r in reps]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -525,6 +561,17 @@ def oracle_step(wl, rows: int, threads: int):
         t0 = time.perf_counter()
         oracle.srste(Wb, Gb, 2, 4, 0.0002, dtype=oracle.BF16)
         return time.perf_counter() - t0, float(rows * wl["K"] * 9)
+    if "T24" in wl:               # transposable 2:4 training step (whole 4-row blocks)
+        rows = max(4, rows - rows % 8)
+        Wb = _u16(wl["W"][:rows].contiguous())
+        X, DY = _u16(wl["X"]), _u16(wl["DY"][:rows].contiguous())
+        t0 = time.perf_counter()
+        mask = oracle.mask_transposable(Wb, 2, 4, dtype=oracle.BF16)
+        v, m = oracle.compress24(Wb, mask, dtype=oracle.BF16)
+        vt, mt = oracle.compress24(np.ascontiguousarray(Wb.T), np.ascontiguousarray(mask.T), dtype=oracle.BF16)
+        oracle.spmm(v, m, X, oracle.BF16, threads=threads)                  # Y rows = W rows . X
+        oracle.spmm(vt, mt, DY, oracle.BF16, threads=threads)               # dX = W^T dY over those rows
+        return time.perf_counter() - t0, 2 * 2.0 * rows * wl["K"] * wl["T"]
     if "TM" in wl:                # transposable mask (whole M-row blocks)
         rows = max(wl["TM"][1], rows - rows % wl["TM"][1])
         Wb = _u16(wl["W"][:rows].contiguous())
@@ -600,6 +647,7 @@ def cpu_baseline(wl, target_s: float = 15.0):
     what = ("SR-STE step (mask, masked weight, decay gradient)" if "G" in wl else
             "saliency-scored 2:4 mask" if "D" in wl else
             "greedy transposable 4:8 mask" if "TM" in wl else
+            "transposable 2:4 mask, compress W and W^T, fp64 forward and backward products" if "T24" in wl else
             "1:2 mask, compress, fused compress, decompress" if "P12" in wl else
             "int8 2:4 mask, fused mask+compress, decompress" if "I8" in wl else
             "mask at 1:4, 2:4, 4:8, 2:8" if wl["X"] is None else
@@ -805,7 +853,8 @@ def main():
                 "data": "synthetic",
                 "config": {"workload": args.workload, "desc": wl["desc"], "R": wl["R"], "K": wl["K"], "T": wl["T"],
                            "sparsity": {"ties": "N:M along K (1:4, 2:4, 4:8, 2:8)", "pairs": "1:2 along K",
-                                        "transposable": "4:8 transposable (8x8 blocks)"}.get(step.kind, "2:4 along K"),
+                                        "transposable": "4:8 transposable (8x8 blocks)",
+                                        "trans24": "2:4 transposable (4x4 blocks)"}.get(step.kind, "2:4 along K"),
                            "l2": "flushed: 256 MiB write between timed steps, outside the events",
                            "launch": launch_mode,
                            "parallelism": "independent replica per GPU" if world > 1 else "single GPU"},

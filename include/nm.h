@@ -190,14 +190,40 @@ NM_API nm_status nm_decompress12(const void *values, const uint8_t *meta, nm_dty
 
 /*
  * nm_compress -- 2:4 compression under a caller-supplied mask (uint8, R x C,
- * leading dim ldm).  A valid group has exactly two entries equal to 1 and
- * the rest 0.  Invalid groups are counted into *invalid_groups (a device
+ * leading dim ldm).  A valid group holds 0/1 bytes with at most two ones.
+ * A group with fewer than two ("Benefits of 2:4 sparsity": a group with more
+ * zeros still stores two values) is stored as its kept positions plus the
+ * lowest unkept ones, in ascending order, the unkept ones with value +0.0;
+ * so 1:4 masks and greedy transposable masks compress too, and decompression
+ * gives W where kept and +0.0 elsewhere.  Invalid groups (more than two ones,
+ * or a byte other than 0/1) are counted into *invalid_groups (a device
  * int32, added to atomically; pass NULL to skip); their output is the
  * pattern (0,1) with values W[4g], W[4g+1].  Outputs as nm_mask_compress.
  */
 NM_API nm_status nm_compress(const void *W, const uint8_t *mask, nm_dtype dtype, int64_t R, int64_t C,
                       int64_t ldw, int64_t ldm, void *values, uint8_t *meta, uint8_t *meta_sm100,
                       int32_t *invalid_groups, void *stream);
+
+/*
+ * nm_compress_t -- 2:4 compression of the TRANSPOSE of W under the transpose
+ * of a caller-supplied mask ("Accelerated Sparse Neural Training" review,
+ * transposable N:M masks: with a mask that is 2:4 along both rows and columns
+ * of W, W^T is itself 2:4-sparse along R, so the backward product
+ * dX = W^T dY runs on the same sparse tensor cores as Y = W X).
+ *   W, mask: R x C (leading dims ldw, ldm), R % 8 == 0, any C
+ *   Output: the canonical form of Wt = W^T (C x R) with groups of four
+ *   consecutive rows of a column of W:
+ *     values_t  C x R/2, W's dtype, row stride R/2
+ *     meta_t    C x R/8 bytes
+ *     meta_t_sm100  image of the C x R matrix (nm_sizes(C, R, ...)), or NULL
+ *   Groups are kept, filled and checked as by nm_compress (at most two ones
+ *   among four 0/1 bytes; fewer are filled with +0.0 values at the lowest
+ *   unkept positions; invalid groups are counted and stored as (0,1)).
+ *   dtype: NM_F32, NM_BF16, NM_F16 or NM_S8.  One pass over W and the mask.
+ */
+NM_API nm_status nm_compress_t(const void *W, const uint8_t *mask, nm_dtype dtype, int64_t R, int64_t C,
+                               int64_t ldw, int64_t ldm, void *values_t, uint8_t *meta_t,
+                               uint8_t *meta_t_sm100, int32_t *invalid_groups, void *stream);
 
 /*
  * nm_decompress -- dense R x C from the canonical 2:4 form: kept positions

@@ -43,6 +43,7 @@ SEEDS = {
     "srste.grad": 6,
     "saliency.X": 7,
     "fp32_linear.W": 8,
+    "linear_4096.dY": 103,
 }
 
 
@@ -80,6 +81,11 @@ def small_fp32():
 def linear_4096():
     return (normal((4096, 4096), SEEDS["linear_4096.W"], 0.02, torch.bfloat16),
             normal((4096, 4096), SEEDS["linear_4096.X"], 1.0, torch.bfloat16))
+
+
+def linear_4096_grad():
+    """Output gradient dY of the transformer linear (R x T = 4096 x 4096), bf16 ~N(0,1)."""
+    return normal((4096, 4096), SEEDS["linear_4096.dY"], 1.0, torch.bfloat16)
 
 
 def mlp_pair():

@@ -408,7 +408,12 @@ int oracle_mask_exhaustive(const void *W, int dtype, int64_t R, int64_t C, int64
 /*   values[r][2g+j] = W[r][4g+idx_j], idx_0 < idx_1, bits copied as-is   */
 /*   meta: kept entry k = 2g+j of row r -> its 2-bit idx_j in bits        */
 /*   2*(k%4) .. 2*(k%4)+1 of byte r*(C/8) + k/4 (LSB first).              */
-/* The mask must hold exactly 2 ones per group; otherwise OR_BAD_MASK.    */
+/* The mask holds 0/1 bytes with at most 2 ones per group; otherwise     */
+/* OR_BAD_MASK.  A group with fewer than 2 ones (a 1:4 mask, a greedy     */
+/* transposable mask) still stores two values, as the page says of groups */
+/* with more zeros: the pair is the kept positions plus the lowest unkept */
+/* ones, in ascending order, and an unkept position's value is +0.0, so   */
+/* decompression gives W where kept and +0.0 elsewhere.                   */
 /* --------------------------------------------------------------------- */
 int oracle_compress24(const void *W, const uint8_t *mask, int dtype, int64_t R, int64_t C,
                       void *values, uint8_t *meta)
@@ -417,18 +422,27 @@ int oracle_compress24(const void *W, const uint8_t *mask, int dtype, int64_t R, 
     memset(meta, 0, (size_t)(R * C / 8));
     for (int64_t r = 0; r < R; ++r) {
         for (int64_t g = 0; g < C / 4; ++g) {
-            int kept[4], nk = 0;
+            int keep[4], nk = 0;
             for (int i = 0; i < 4; ++i) {
                 uint8_t mv = mask[r * C + g * 4 + i];
                 if (mv > 1) return OR_BAD_MASK;
-                if (mv) { if (nk == 2) return OR_BAD_MASK; kept[nk++] = i; }
+                keep[i] = mv;
+                nk += mv;
             }
-            if (nk != 2) return OR_BAD_MASK;
-            for (int j = 0; j < 2; ++j) {
+            if (nk > 2) return OR_BAD_MASK;
+            /* fill up to two positions with the lowest unkept indices */
+            int take[4];
+            for (int i = 0; i < 4; ++i) take[i] = keep[i];
+            for (int i = 0; i < 4 && nk < 2; ++i)
+                if (!take[i]) { take[i] = 1; ++nk; }
+            int j = 0;
+            for (int i = 0; i < 4; ++i) {
+                if (!take[i]) continue;
                 int64_t k = 2 * g + j;
-                uint32_t b = load_bits(W, dtype, (size_t)(r * C + g * 4 + kept[j]));
+                uint32_t b = keep[i] ? load_bits(W, dtype, (size_t)(r * C + g * 4 + i)) : 0u;
                 store_bits(values, dtype, (size_t)(r * (C / 2) + k), b);
-                meta[r * (C / 8) + k / 4] |= (uint8_t)(kept[j] << (2 * (k % 4)));
+                meta[r * (C / 8) + k / 4] |= (uint8_t)(i << (2 * (k % 4)));
+                ++j;
             }
         }
     }

@@ -54,6 +54,7 @@ def _lib():
         "nm_decompress12": ([vp, vp, i32, i64, i64, vp, i64, vp], i32),
         "nm_mask_compress": ([vp, i32, i64, i64, i64, vp, vp, vp, vp], i32),
         "nm_compress": ([vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp, vp], i32),
+        "nm_compress_t": ([vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp, vp], i32),
         "nm_decompress": ([vp, vp, i32, i64, i64, vp, i64, vp], i32),
         "nm_meta_to_sm100": ([vp, i64, i64, vp, vp], i32),
         "nm_spmm_workspace_bytes": ([i32, i64, i64, i64], sz),
@@ -214,6 +215,17 @@ def nm_compress(W: torch.Tensor, mask: torch.Tensor, values=None, meta=None, met
         values, meta, meta_sm100 = alloc_compressed(R, C, W.dtype, W.device, sm100)
     _check(_lib().nm_compress(_ptr(W), _ptr(mask), _dtype(W), R, C, _ld(W), _ld(mask), _ptr(values), _ptr(meta),
                               _ptr(meta_sm100), _ptr(invalid_groups), _stream(stream)), "nm_compress")
+    return values, meta, meta_sm100
+
+
+def nm_compress_t(W: torch.Tensor, mask: torch.Tensor, values=None, meta=None, meta_sm100=None,
+                  sm100: bool = True, invalid_groups: torch.Tensor | None = None, stream=None):
+    """Compressed W^T (C x R, groups along R) under mask^T -> (values_t, meta_t, meta_t_sm100 or None)."""
+    R, C = W.shape
+    if values is None:
+        values, meta, meta_sm100 = alloc_compressed(C, R, W.dtype, W.device, sm100)
+    _check(_lib().nm_compress_t(_ptr(W), _ptr(mask), _dtype(W), R, C, _ld(W), _ld(mask), _ptr(values), _ptr(meta),
+                                _ptr(meta_sm100), _ptr(invalid_groups), _stream(stream)), "nm_compress_t")
     return values, meta, meta_sm100
 
 

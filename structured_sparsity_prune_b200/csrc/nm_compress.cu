@@ -91,22 +91,31 @@ __device__ __forceinline__ uint32_t compress_octet(const Oct<Bits>& e, uint2 m, 
       byte |= (i0 | (i1 << 2)) << (4 * g);
       continue;
     } else {
+      // The group keeps at most two (bytes 0/1).  With fewer, the pair is
+      // filled with the lowest unkept positions, stored as +0.0 (a group with
+      // more zeros still stores two values).  Anything else is invalid:
+      // counted, and stored as the pattern (0,1) with W's values.
       const uint32_t w = g ? m.y : m.x;  // 4 mask bytes of this group
-      uint32_t bits = 0;
-      bool ok = (w & 0xFEFEFEFEu) == 0;  // every byte is 0 or 1
+      uint32_t keep = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) bits |= ((w >> (8 * i)) & 1u) << i;
-      ok = ok && __popc(bits) == 2;
-      if (!ok) {
+      for (int i = 0; i < 4; ++i) keep |= ((w >> (8 * i)) & 1u) << i;
+      const uint32_t n = __popc(keep);
+      uint32_t take = keep;
+      if ((w & 0xFEFEFEFEu) != 0 || n > 2) {
         ++invalid;
-        bits = 0x3u;  // documented fallback: pattern (0,1)
+        take = keep = 0x3u;
+      } else if (n < 2) {
+        take |= ~take & (take + 1);                 // lowest unkept position
+        if (n == 0) take |= ~take & (take + 1);
       }
-      i0 = __ffs(bits) - 1;
-      i1 = 31 - __clz(bits);
+      i0 = __ffs(take) - 1;
+      i1 = 31 - __clz(take);
+      const Bits v0 = sel4<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3], i0);
+      const Bits v1 = sel4<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3], i1);
+      q.set(2 * g, ((keep >> i0) & 1u) ? v0 : Bits(0));
+      q.set(2 * g + 1, ((keep >> i1) & 1u) ? v1 : Bits(0));
+      byte |= (i0 | (i1 << 2)) << (4 * g);
     }
-    q.set(2 * g, sel4<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3], i0));
-    q.set(2 * g + 1, sel4<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3], i1));
-    byte |= (i0 | (i1 << 2)) << (4 * g);
   }
   return byte;
 }
@@ -510,6 +519,143 @@ __global__ void __launch_bounds__(256) decompress32_kernel(const Bits* __restric
   }
 }
 
+// ---- compression of the transpose ---------------------------------------------
+// Wt = W^T (C x R) compressed 2:4 along R under mask^T: the operand of the
+// backward product dX = W^T dY when the mask is transposable (every group of
+// four consecutive rows in a column keeps two).  A block stages a tile of
+// kTR rows x kTC columns of W and of the mask in shared memory (16-byte
+// loads along W's rows), then lane l of warp w takes column c = c0 + l of
+// the tile -- one row of Wt -- and the 32-row run w of it: eight octets
+// gathered down the column (a warp reads one row of the tile per step, so
+// the shared reads are conflict-free), compressed as by nm_compress.  Image
+// words pair rows c and c + 8 of Wt: lanes l and l ^ 8 swap their pieces and
+// each writes one word.  The grid covers the image's padded extent.
+constexpr int kTR = 256;
+constexpr int kTC = 32;
+
+template <typename Bits>
+__device__ __forceinline__ Oct<Bits> make_oct(const Bits (&a)[8]) {
+  Oct<Bits> e;
+  if constexpr (sizeof(Bits) == 1) {
+    e.v = make_uint2(uint32_t(a[0]) | (uint32_t(a[1]) << 8) | (uint32_t(a[2]) << 16) | (uint32_t(a[3]) << 24),
+                     uint32_t(a[4]) | (uint32_t(a[5]) << 8) | (uint32_t(a[6]) << 16) | (uint32_t(a[7]) << 24));
+  } else if constexpr (sizeof(Bits) == 2) {
+    e.v = make_uint4(uint32_t(a[0]) | (uint32_t(a[1]) << 16), uint32_t(a[2]) | (uint32_t(a[3]) << 16),
+                     uint32_t(a[4]) | (uint32_t(a[5]) << 16), uint32_t(a[6]) | (uint32_t(a[7]) << 16));
+  } else {
+    e.v[0] = make_uint4(a[0], a[1], a[2], a[3]);
+    e.v[1] = make_uint4(a[4], a[5], a[6], a[7]);
+  }
+  return e;
+}
+
+template <typename Bits>
+__global__ void __launch_bounds__(256) compress_t_kernel(const Bits* __restrict__ W, int64_t ldw,
+                                                         const uint8_t* __restrict__ mask, int64_t ldm, int64_t R,
+                                                         int64_t C, Bits* __restrict__ values,
+                                                         uint8_t* __restrict__ meta, uint8_t* __restrict__ img,
+                                                         int32_t* __restrict__ invalid_groups) {
+  constexpr int kEl = 16 / int(sizeof(Bits));  // elements per 16-byte chunk
+  constexpr int kWCh = kTC / kEl;              // W chunks per tile row: 2, 4 or 8
+  __shared__ __align__(16) Bits sW[kTR][kTC];
+  __shared__ __align__(16) uint8_t sM[kTR][kTC];
+  const int64_t Rp = (R + 127) / 128 * 128, Cp = (C + 127) / 128 * 128;  // padded image extents
+  const int64_t tc_count = Cp / kTC, tiles = ((Rp + kTR - 1) / kTR) * tc_count;
+  const int lane = threadIdx.x & 31, run = threadIdx.x >> 5;
+  const bool unit_vec = ((R / 2) * int64_t(sizeof(Bits))) % 16 == 0;  // Wt value rows 16-byte aligned
+  const bool meta_words = R % 32 == 0;
+  int invalid = 0;
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    const int64_t tr = tile / tc_count;
+    const int64_t r_base = tr * kTR, c_base = (tile - tr * tc_count) * kTC;
+    for (int i = threadIdx.x; i < kTR * kWCh; i += 256) {
+      const int rl = i / kWCh, k = i - rl * kWCh;
+      const int64_t r = r_base + rl, c = c_base + k * kEl;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < R && c < C) {
+        const Bits* src = W + r * ldw + c;
+        if (c + kEl <= C) {
+          v = __ldcs(reinterpret_cast<const uint4*>(src));
+        } else {
+          Bits* vb = reinterpret_cast<Bits*>(&v);
+          for (int e = 0; e < kEl && c + e < C; ++e) vb[e] = src[e];
+        }
+      }
+      *reinterpret_cast<uint4*>(&sW[rl][k * kEl]) = v;
+    }
+    for (int i = threadIdx.x; i < kTR * 2; i += 256) {
+      const int rl = i >> 1, k = i & 1;
+      const int64_t r = r_base + rl, c = c_base + 16 * k;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < R && c < C) {
+        const uint8_t* src = mask + r * ldm + c;
+        if (c + 16 <= C) {
+          v = __ldcs(reinterpret_cast<const uint4*>(src));
+        } else {
+          uint8_t* vb = reinterpret_cast<uint8_t*>(&v);
+          for (int e = 0; e < 16 && c + e < C; ++e) vb[e] = src[e];
+        }
+      }
+      *reinterpret_cast<uint4*>(&sM[rl][16 * k]) = v;
+    }
+    __syncthreads();
+    const int64_t c = c_base + lane;         // row of Wt
+    const int64_t r0 = r_base + 32 * run;    // first column of Wt in this unit
+    uint32_t bytes[4] = {kPadByte, kPadByte, kPadByte, kPadByte};
+    if (c < C && r0 < R) {
+      Quad<Bits> q[4];
+#pragma unroll
+      for (int o = 0; o < 4; ++o) {
+        if (r0 + 8 * o >= R) break;  // R % 8 == 0: octets are whole
+        Bits a[8];
+        uint32_t mlo = 0, mhi = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          a[k] = sW[32 * run + 8 * o + k][lane];
+          const uint32_t b = sM[32 * run + 8 * o + k][lane];
+          if (k < 4) mlo |= b << (8 * k);
+          else mhi |= b << (8 * (k - 4));
+        }
+        bytes[o] = compress_octet<Bits, 1>(make_oct<Bits>(a), make_uint2(mlo, mhi), q[o], invalid);
+      }
+      Bits* vrow = values + c * (R / 2) + r0 / 2;
+      if (unit_vec && r0 + 32 <= R) {
+        store_unit<Bits>(q, vrow);
+      } else {
+#pragma unroll
+        for (int o = 0; o < 4; ++o)
+          if (r0 + 8 * o < R) q[o].store(vrow + 4 * o);
+      }
+      if (meta_words) {
+        __stcs(reinterpret_cast<uint32_t*>(meta + c * (R / 8) + r0 / 8),
+               bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24));
+      } else {
+#pragma unroll
+        for (int o = 0; o < 4; ++o)
+          if (r0 + 8 * o < R) meta[c * (R / 8) + r0 / 8 + o] = uint8_t(bytes[o]);
+      }
+    }
+    if (img != nullptr) {
+      const uint32_t p0 = bytes[0] | (bytes[1] << 8), p1 = bytes[2] | (bytes[3] << 8);
+      const uint32_t o0 = __shfl_xor_sync(0xFFFFFFFFu, p0, 8), o1 = __shfl_xor_sync(0xFFFFFFFFu, p1, 8);
+      const bool upper = (lane & 8) != 0;     // this lane holds row c, its partner row c - 8
+      const uint32_t word = upper ? (o1 | (p1 << 16)) : (p0 | (o0 << 16));
+      const int64_t crow = upper ? c - 8 : c;  // the pair's row with (row % 16) < 8
+      if (r0 < Rp) {
+        uint8_t* blk = img + ((crow >> 7) * (Rp / 128) + (r0 >> 7)) * 2048;
+        const uint32_t L = uint32_t(crow & 7) + 8u * (upper ? 1u : 0u) + 16u * uint32_t((crow & 127) >> 4);
+        __stcs(reinterpret_cast<uint32_t*>(blk + L * 16u + uint32_t((r0 & 127) >> 5) * 4u), word);
+      }
+    }
+    __syncthreads();
+  }
+  if (invalid_groups != nullptr) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) invalid += __shfl_xor_sync(0xFFFFFFFFu, invalid, off);
+    if (lane == 0 && invalid != 0) atomicAdd(invalid_groups, invalid);
+  }
+}
+
 int tile_grid(int64_t R, int64_t C) {
   const int64_t tiles = ((R + 127) / 128) * ((C + 127) / 128);
   const int64_t want = int64_t(sm_count()) * 8;
@@ -594,6 +740,33 @@ extern "C" nm_status nm_compress(const void* W, const uint8_t* mask, nm_dtype dt
     launch_compress<uint8_t, 1>(W, ldw, mask, ldm, R, C, values, meta, meta_sm100, invalid_groups, s);
   else
     launch_compress<uint16_t, 1>(W, ldw, mask, ldm, R, C, values, meta, meta_sm100, invalid_groups, s);
+  return launch_status();
+}
+
+extern "C" nm_status nm_compress_t(const void* W, const uint8_t* mask, nm_dtype dtype, int64_t R, int64_t C,
+                                   int64_t ldw, int64_t ldm, void* values_t, uint8_t* meta_t, uint8_t* meta_t_sm100,
+                                   int32_t* invalid_groups, void* stream) {
+  if (!dtype_ok_int8(dtype)) return NM_ERR_DTYPE;
+  if (R < 0 || C < 0 || R % 8 != 0 || ldw < C || ldm < C) return NM_ERR_SHAPE;
+  if (R == 0 || C == 0) return NM_OK;
+  if (W == nullptr || mask == nullptr || values_t == nullptr || meta_t == nullptr) return NM_ERR_NULL;
+  if (!aligned16(W) || !aligned16(mask) || !aligned16(values_t) || !aligned16(meta_t) ||
+      (meta_t_sm100 && !aligned16(meta_t_sm100)) || !stride_ok(ldw, esize_of(dtype)) || !stride_ok(ldm, 1) ||
+      (invalid_groups && (reinterpret_cast<uintptr_t>(invalid_groups) & 3u)))
+    return NM_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t tiles = (((R + 127) / 128 * 128 + kTR - 1) / kTR) * ((C + 127) / 128 * 128 / kTC);
+  auto launch = [&](auto kernel, auto* w, auto* v) {
+    const int64_t cap = int64_t(blocks_per_sm(kernel, 256)) * sm_count();
+    kernel<<<unsigned(tiles < cap ? tiles : cap), 256, 0, s>>>(w, ldw, mask, ldm, R, C, v, meta_t, meta_t_sm100,
+                                                               invalid_groups);
+  };
+  if (dtype == NM_F32)
+    launch(compress_t_kernel<uint32_t>, static_cast<const uint32_t*>(W), static_cast<uint32_t*>(values_t));
+  else if (dtype == NM_S8)
+    launch(compress_t_kernel<uint8_t>, static_cast<const uint8_t*>(W), static_cast<uint8_t*>(values_t));
+  else
+    launch(compress_t_kernel<uint16_t>, static_cast<const uint16_t*>(W), static_cast<uint16_t*>(values_t));
   return launch_status();
 }
 

@@ -158,15 +158,43 @@ def test_compress_counts_invalid_groups():
     mask = torch.zeros((R, C), dtype=torch.uint8)
     mask[:, 0::4] = 1
     mask[:, 1::4] = 1
-    bad = [(0, 0, [1, 1, 1, 0]), (3, 5, [0, 0, 0, 0]), (63, 31, [2, 0, 1, 0]), (10, 7, [1, 0, 0, 0])]
+    # invalid: more than two ones, a byte other than 0/1.  Valid but sparser:
+    # none or one kept (stored with +0.0 fillers at the lowest unkept positions).
+    bad = [(0, 0, [1, 1, 1, 0]), (63, 31, [2, 0, 1, 0])]
+    sparse = [(3, 5, [0, 0, 0, 0]), (10, 7, [1, 0, 0, 0]), (20, 2, [0, 0, 1, 0])]
+    fixed = mask.clone()
     for r, g, pat in bad:
         mask[r, 4 * g:4 * g + 4] = torch.tensor(pat, dtype=torch.uint8)
+        fixed[r, 4 * g:4 * g + 4] = torch.tensor([1, 1, 0, 0], dtype=torch.uint8)   # fallback (0,1), W's values
+    for r, g, pat in sparse:
+        mask[r, 4 * g:4 * g + 4] = torch.tensor(pat, dtype=torch.uint8)
+        fixed[r, 4 * g:4 * g + 4] = torch.tensor(pat, dtype=torch.uint8)
     ctr = torch.zeros((1,), dtype=torch.int32, device="cuda")
-    values, meta, _ = nm.nm_compress(W.cuda(), mask.cuda(), invalid_groups=ctr)
+    values, meta, img = nm.nm_compress(W.cuda(), mask.cuda(), invalid_groups=ctr)
     assert int(ctr.item()) == len(bad)
+    v_ref, m_ref = oracle.compress24(_bits(W), fixed.numpy(), dtype=oracle.BF16)
+    assert np.array_equal(_bits(values), v_ref)
+    assert np.array_equal(meta.cpu().numpy(), m_ref)
+    assert np.array_equal(img.cpu().numpy(), oracle.meta_sm100(m_ref, R, C))
     m = meta.cpu().numpy()
-    for r, g, _ in bad:      # documented fallback: pattern (0,1)
+    for r, g, _ in bad + sparse[:2]:      # pattern (0,1)
         assert (m[r, g // 2] >> (4 * (g % 2))) & 0xF == 0x4
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("R,C", [(64, 128), (77, 208)])   # row and tile compressors
+def test_compress_sparser_masks_roundtrip(dtype, R, C):
+    """1:4 magnitude masks through nm_compress: the oracle's form, and
+    decompression gives select(mask, W, +0.0)."""
+    W = _rand((R, C), dtype, 31, "special")
+    mask = nm.nm_mask(W.cuda(), 1, 4)
+    values, meta, img = nm.nm_compress(W.cuda(), mask)
+    v_ref, m_ref = oracle.compress24(_bits(W), mask.cpu().numpy(), dtype=CODE[dtype])
+    assert np.array_equal(_bits(values), np.ascontiguousarray(v_ref).view(_bits(values).dtype))
+    assert np.array_equal(meta.cpu().numpy(), m_ref)
+    assert np.array_equal(img.cpu().numpy(), oracle.meta_sm100(m_ref, R, C))
+    back = _bits(nm.nm_decompress(values, meta, C))
+    assert np.array_equal(back, np.where(mask.cpu().numpy() == 1, _bits(W), 0))
 
 
 @pytest.mark.parametrize("R,C", SHAPES)

@@ -102,12 +102,60 @@ def test_storage_saving_36_of_64_bits():
     assert abs(1 - bits_compressed / bits_dense - 0.4375) < 1e-12
 
 
-@pytest.mark.parametrize("bad", [[1, 1, 1, 0], [1, 0, 0, 0], [0, 0, 0, 0], [2, 1, 0, 0]])
+@pytest.mark.parametrize("bad", [[1, 1, 1, 0], [1, 1, 1, 1], [2, 1, 0, 0], [0, 0, 3, 0]])
 def test_invalid_mask_rejected(bad):
+    """More than two kept, or a mask byte other than 0/1, is not a 2:4 mask."""
     W = np.ones((1, 8), dtype=np.float32)
     m = np.array([bad + [1, 1, 0, 0]], dtype=np.uint8)
     with pytest.raises(ValueError):
         oracle.compress24(W, m)
+
+
+# A group that keeps fewer than two ("Benefits of 2:4 sparsity": a group with
+# more zeros still stores two values) is stored as the kept positions plus the
+# lowest unkept ones, ascending, the unkept ones with value +0.0.  Worked by
+# hand: (mask of the group) -> (pair, stored values, nibble idx0 | idx1 << 2).
+SPARSE_GROUPS = [
+    ([0, 0, 1, 0], (0, 2), (0.0, 3.0), 0x8),
+    ([1, 0, 0, 0], (0, 1), (1.5, 0.0), 0x4),
+    ([0, 1, 0, 0], (0, 1), (0.0, -2.0), 0x4),
+    ([0, 0, 0, 1], (0, 3), (0.0, 4.0), 0xC),
+    ([0, 0, 0, 0], (0, 1), (0.0, 0.0), 0x4),
+    ([0, 0, 1, 1], (2, 3), (3.0, 4.0), 0xE),
+]
+
+
+@pytest.mark.parametrize("group,pair,vals,nib", SPARSE_GROUPS)
+def test_groups_with_fewer_than_two_kept(group, pair, vals, nib):
+    W = np.array([[1.5, -2.0, 3.0, 4.0, -1.0, -1.0, 5.0, 6.0]], dtype=np.float32)
+    m = np.array([group + [0, 1, 0, 0]], dtype=np.uint8)      # second group: keeps index 1 only
+    values, meta = oracle.compress24(W, m)
+    assert values[0, :2].tolist() == list(vals)
+    assert (meta[0, 0] & 0xF) == nib
+    # the second group [-1, -1, 5, 6] keeping index 1: pair (0, 1), values (+0.0, -1.0)
+    assert values[0, 2:].tolist() == [0.0, -1.0] and (meta[0, 0] >> 4) == 0x4
+    # stored fillers are +0.0, not -0.0, even where W is negative
+    assert values.view(np.uint32)[0, 2] == 0
+
+
+@pytest.mark.parametrize("code", [oracle.F32, oracle.BF16, oracle.F16])
+def test_sparser_masks_roundtrip_to_select(code):
+    """decompress(compress(W, mask)) == select(mask, W, +0.0) for any mask with
+    at most two ones per group: 1:4 magnitude masks and random ones."""
+    R, C = 16, 64
+    W = _random_case(code, R, C, 17)
+    rng = np.random.default_rng(3)
+    masks = [oracle.mask_rank(W, 1, 4, dtype=code)]
+    rand = np.zeros((R, C), dtype=np.uint8)
+    for r in range(R):
+        for g in range(C // 4):
+            k = rng.integers(0, 3)
+            rand[r, 4 * g + rng.choice(4, size=k, replace=False)] = 1
+    masks.append(rand)
+    for mask in masks:
+        values, meta = oracle.compress24(W, mask, dtype=code)
+        back = oracle.decompress24(values, meta, C, dtype=code)
+        assert np.array_equal(back, np.where(mask == 1, W, np.zeros_like(W)))
 
 
 # ---------------------------------------------------------------- metadata image
