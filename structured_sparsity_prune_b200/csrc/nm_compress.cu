@@ -69,55 +69,110 @@ template <> struct Quad<uint32_t> {
   __device__ __forceinline__ void store(uint32_t* p) const { __stcs(reinterpret_cast<uint4*>(p), v); }
 };
 
+// ---- one group of four -> its stored pair ----------------------------------------
+// The nibble idx0 | idx1 << 2 of every 4-bit keep pattern with at most two
+// bits set: the kept positions, filled with the lowest unkept ones (a group
+// with more zeros still stores two values).  Patterns with three or four set
+// map to 0x4, the fallback (0,1) for invalid groups.
+constexpr uint64_t make_pair_nib_lut() {
+  uint64_t lut = 0;
+  for (int k = 0; k < 16; ++k) {
+    int take = k, n = ((k >> 0) & 1) + ((k >> 1) & 1) + ((k >> 2) & 1) + ((k >> 3) & 1);
+    uint32_t nib = 0x4u;
+    if (n <= 2) {
+      for (int i = 0; i < 4 && n < 2; ++i)
+        if (!((take >> i) & 1)) { take |= 1 << i; ++n; }
+      int i0 = 0, i1 = 3;
+      while (!((take >> i0) & 1)) ++i0;
+      while (!((take >> i1) & 1)) --i1;
+      nib = uint32_t(i0 | (i1 << 2));
+    }
+    lut |= uint64_t(nib) << (4 * k);
+  }
+  return lut;
+}
+constexpr uint64_t kPairNib = make_pair_nib_lut();
+
+// Keep bits of four 0/1 mask bytes (bit k = bit 0 of byte k): one multiply
+// gathers the four byte-aligned bits into bits 28..31 without carries.
+__device__ __forceinline__ uint32_t keep_of_bytes(uint32_t w) { return ((w & 0x01010101u) * 0x10204080u) >> 28; }
+
+struct Pick {
+  uint32_t nib;   // idx0 | idx1 << 2
+  bool zlo, zhi;  // the stored value is a +0.0 filler (an unkept position)
+};
+
+// Under the caller's mask (w: the group's four mask bytes).  A valid group
+// holds 0/1 bytes with at most two ones; fewer are filled as above.  Anything
+// else is invalid: counted, and stored as (0,1) with W's values.
+__device__ __forceinline__ Pick pick_masked(uint32_t w, int& invalid) {
+  const uint32_t keep = keep_of_bytes(w), n = __popc(keep);
+  Pick p{0x4u, false, false};
+  if ((w & 0xFEFEFEFEu) != 0 || n > 2) {
+    ++invalid;
+    return p;
+  }
+  p.nib = uint32_t(kPairNib >> (4 * keep)) & 0xFu;
+  if (n < 2) {
+    p.zlo = ((keep >> (p.nib & 3u)) & 1u) == 0;
+    p.zhi = ((keep >> (p.nib >> 2)) & 1u) == 0;
+  }
+  return p;
+}
+
+// By magnitude: exactly two kept, so the first kept index is 0, 1 or 2 and
+// the second 1, 2 or 3 (read off the drop signs, cheaper than the table).
+template <typename Bits>
+__device__ __forceinline__ Pick pick_magnitude(Bits e0, Bits e1, Bits e2, Bits e3) {
+  uint32_t x0, x1, x2, x3;
+  drop4<2>(mag_key<Bits>(e0), mag_key<Bits>(e1), mag_key<Bits>(e2), mag_key<Bits>(e3), x0, x1, x2, x3);
+  const bool k0 = int32_t(x0) >= 0, k1 = int32_t(x1) >= 0, k2 = int32_t(x2) >= 0, k3 = int32_t(x3) >= 0;
+  const uint32_t i0 = k0 ? 0u : (k1 ? 1u : 2u), i1 = k3 ? 3u : (k2 ? 2u : 1u);
+  return Pick{i0 | (i1 << 2), false, false};
+}
+
+// The stored pair as packed bits.  16-bit elements: g01 holds entries 0, 1
+// and g23 entries 2, 3 (entry i = bytes 2i, 2i+1 of the pair of words); one
+// byte-permute picks both.  8-bit: the four entries in one word.
+__device__ __forceinline__ uint32_t pair16(uint32_t g01, uint32_t g23, Pick p) {
+  uint32_t v = __byte_perm(g01, g23, 34u * ((p.nib & 3u) + ((p.nib >> 2) << 8)) + 0x1010u);
+  if (p.zlo) v &= 0xFFFF0000u;
+  if (p.zhi) v &= 0x0000FFFFu;
+  return v;
+}
+__device__ __forceinline__ uint32_t pair8(uint32_t g, Pick p) {
+  uint32_t v = __byte_perm(g, 0u, (p.nib & 3u) | ((p.nib >> 2) << 4) | 0x4400u);
+  if (p.zlo) v &= 0xFF00u;
+  if (p.zhi) v &= 0x00FFu;
+  return v;
+}
+__device__ __forceinline__ uint2 pair32(uint32_t e0, uint32_t e1, uint32_t e2, uint32_t e3, Pick p) {
+  uint32_t a = sel4<uint32_t>(e0, e1, e2, e3, p.nib & 3u), b = sel4<uint32_t>(e0, e1, e2, e3, p.nib >> 2);
+  if (p.zlo) a = 0u;
+  if (p.zhi) b = 0u;
+  return make_uint2(a, b);
+}
+
 // Compress one octet (two groups).  MODE 0 selects by magnitude; MODE 1 takes
-// the caller's mask (8 bytes) and reports whether both groups were valid.
+// the caller's mask (8 bytes) and counts its invalid groups.
 template <typename Bits, int MODE>
 __device__ __forceinline__ uint32_t compress_octet(const Oct<Bits>& e, uint2 m, Quad<Bits>& q, int& invalid) {
-  uint32_t byte = 0;
+  Pick p[2];
 #pragma unroll
   for (int g = 0; g < 2; ++g) {
-    uint32_t i0, i1;
-    if constexpr (MODE == 0) {
-      // branch-free 2:4 selection; exactly two of the four are kept, so the
-      // first kept index is 0, 1 or 2 and the second 1, 2 or 3
-      uint32_t x0, x1, x2, x3;
-      drop4<2>(mag_key<Bits>(e[4 * g]), mag_key<Bits>(e[4 * g + 1]), mag_key<Bits>(e[4 * g + 2]),
-               mag_key<Bits>(e[4 * g + 3]), x0, x1, x2, x3);
-      const bool k0 = int32_t(x0) >= 0, k1 = int32_t(x1) >= 0, k2 = int32_t(x2) >= 0, k3 = int32_t(x3) >= 0;
-      i0 = k0 ? 0u : (k1 ? 1u : 2u);
-      i1 = k3 ? 3u : (k2 ? 2u : 1u);
-      q.set(2 * g, k0 ? e[4 * g] : (k1 ? e[4 * g + 1] : e[4 * g + 2]));
-      q.set(2 * g + 1, k3 ? e[4 * g + 3] : (k2 ? e[4 * g + 2] : e[4 * g + 1]));
-      byte |= (i0 | (i1 << 2)) << (4 * g);
-      continue;
-    } else {
-      // The group keeps at most two (bytes 0/1).  With fewer, the pair is
-      // filled with the lowest unkept positions, stored as +0.0 (a group with
-      // more zeros still stores two values).  Anything else is invalid:
-      // counted, and stored as the pattern (0,1) with W's values.
-      const uint32_t w = g ? m.y : m.x;  // 4 mask bytes of this group
-      uint32_t keep = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) keep |= ((w >> (8 * i)) & 1u) << i;
-      const uint32_t n = __popc(keep);
-      uint32_t take = keep;
-      if ((w & 0xFEFEFEFEu) != 0 || n > 2) {
-        ++invalid;
-        take = keep = 0x3u;
-      } else if (n < 2) {
-        take |= ~take & (take + 1);                 // lowest unkept position
-        if (n == 0) take |= ~take & (take + 1);
-      }
-      i0 = __ffs(take) - 1;
-      i1 = 31 - __clz(take);
-      const Bits v0 = sel4<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3], i0);
-      const Bits v1 = sel4<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3], i1);
-      q.set(2 * g, ((keep >> i0) & 1u) ? v0 : Bits(0));
-      q.set(2 * g + 1, ((keep >> i1) & 1u) ? v1 : Bits(0));
-      byte |= (i0 | (i1 << 2)) << (4 * g);
-    }
+    if constexpr (MODE == 0) p[g] = pick_magnitude<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3]);
+    else p[g] = pick_masked(g ? m.y : m.x, invalid);
   }
-  return byte;
+  if constexpr (sizeof(Bits) == 2) {
+    q.v = make_uint2(pair16(e.v.x, e.v.y, p[0]), pair16(e.v.z, e.v.w, p[1]));
+  } else if constexpr (sizeof(Bits) == 1) {
+    q.v = pair8(e.v.x, p[0]) | (pair8(e.v.y, p[1]) << 16);
+  } else {
+    const uint2 a = pair32(e.v[0].x, e.v[0].y, e.v[0].z, e.v[0].w, p[0]);
+    const uint2 b = pair32(e.v[1].x, e.v[1].y, e.v[1].z, e.v[1].w, p[1]);
+    q.v = make_uint4(a.x, a.y, b.x, b.y);
+  }
+  return p[0].nib | (p[1].nib << 4);
 }
 
 // One block walks 128x128 tiles (tile index = rt * kt_count + kt, the same
@@ -522,17 +577,19 @@ __global__ void __launch_bounds__(256) decompress32_kernel(const Bits* __restric
 // ---- compression of the transpose ---------------------------------------------
 // Wt = W^T (C x R) compressed 2:4 along R under mask^T: the operand of the
 // backward product dX = W^T dY when the mask is transposable (every group of
-// four consecutive rows in a column keeps two).  A block stages a tile of
-// kTR rows x kTC columns of W and of the mask in shared memory (16-byte
-// loads along W's rows), then lane l of warp w takes column c = c0 + l of
-// the tile -- one row of Wt -- and the 32-row run w of it: eight octets
-// gathered down the column (a warp reads one row of the tile per step, so
-// the shared reads are conflict-free), compressed as by nm_compress.  Image
-// words pair rows c and c + 8 of Wt: lanes l and l ^ 8 swap their pieces and
-// each writes one word.  The grid covers the image's padded extent.
-constexpr int kTR = 256;
-constexpr int kTC = 32;
-
+// four consecutive rows in a column keeps at most two).  Registers only: a
+// warp takes a tile of 32 rows x 32 columns of W, and lane (q, h) = (lane % 4,
+// lane / 4) reads columns 8q..8q+7 of the four rows 4h..4h+3 -- one group
+// down each of its eight columns -- with one 8-element load per row (a warp
+// reads 64 B, 32 B or 128 B of each of 32 rows).  It compresses the eight
+// groups in registers and stores each pair of values into row c of Wt (the
+// eight lanes of a column chunk fill 8 consecutive groups: one 32-byte run
+// of a row of Wt per store).  Three xor-shuffles give every lane of a column
+// chunk the metadata word of each of its 8 rows of Wt (8 nibbles, 32 columns
+// of Wt); lane h stores the word of row 8q + h.  Image words pair rows c and
+// c + 8 of Wt, which are lanes q and q ^ 1: one more shuffle, and lane h
+// writes the image word of row 8q + h.  The warps of a block take adjacent
+// column tiles of the same rows; the grid covers the image's padded extent.
 template <typename Bits>
 __device__ __forceinline__ Oct<Bits> make_oct(const Bits (&a)[8]) {
   Oct<Bits> e;
@@ -550,104 +607,105 @@ __device__ __forceinline__ Oct<Bits> make_oct(const Bits (&a)[8]) {
 }
 
 template <typename Bits>
-__global__ void __launch_bounds__(256) compress_t_kernel(const Bits* __restrict__ W, int64_t ldw,
+__global__ void __launch_bounds__(256, 3) compress_t_kernel(const Bits* __restrict__ W, int64_t ldw,
                                                          const uint8_t* __restrict__ mask, int64_t ldm, int64_t R,
                                                          int64_t C, Bits* __restrict__ values,
                                                          uint8_t* __restrict__ meta, uint8_t* __restrict__ img,
                                                          int32_t* __restrict__ invalid_groups) {
-  constexpr int kEl = 16 / int(sizeof(Bits));  // elements per 16-byte chunk
-  constexpr int kWCh = kTC / kEl;              // W chunks per tile row: 2, 4 or 8
-  __shared__ __align__(16) Bits sW[kTR][kTC];
-  __shared__ __align__(16) uint8_t sM[kTR][kTC];
+  const int lane = threadIdx.x & 31, q = lane & 3, h = lane >> 2;
   const int64_t Rp = (R + 127) / 128 * 128, Cp = (C + 127) / 128 * 128;  // padded image extents
-  const int64_t tc_count = Cp / kTC, tiles = ((Rp + kTR - 1) / kTR) * tc_count;
-  const int lane = threadIdx.x & 31, run = threadIdx.x >> 5;
-  const bool unit_vec = ((R / 2) * int64_t(sizeof(Bits))) % 16 == 0;  // Wt value rows 16-byte aligned
+  const int64_t ct_count = Cp / 32, tiles = (Rp / 32) * ct_count;
+  const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const bool meta_words = R % 32 == 0;
   int invalid = 0;
-  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
-    const int64_t tr = tile / tc_count;
-    const int64_t r_base = tr * kTR, c_base = (tile - tr * tc_count) * kTC;
-    for (int i = threadIdx.x; i < kTR * kWCh; i += 256) {
-      const int rl = i / kWCh, k = i - rl * kWCh;
-      const int64_t r = r_base + rl, c = c_base + k * kEl;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (r < R && c < C) {
-        const Bits* src = W + r * ldw + c;
-        if (c + kEl <= C) {
-          v = __ldcs(reinterpret_cast<const uint4*>(src));
-        } else {
-          Bits* vb = reinterpret_cast<Bits*>(&v);
-          for (int e = 0; e < kEl && c + e < C; ++e) vb[e] = src[e];
-        }
-      }
-      *reinterpret_cast<uint4*>(&sW[rl][k * kEl]) = v;
-    }
-    for (int i = threadIdx.x; i < kTR * 2; i += 256) {
-      const int rl = i >> 1, k = i & 1;
-      const int64_t r = r_base + rl, c = c_base + 16 * k;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (r < R && c < C) {
-        const uint8_t* src = mask + r * ldm + c;
-        if (c + 16 <= C) {
-          v = __ldcs(reinterpret_cast<const uint4*>(src));
-        } else {
-          uint8_t* vb = reinterpret_cast<uint8_t*>(&v);
-          for (int e = 0; e < 16 && c + e < C; ++e) vb[e] = src[e];
-        }
-      }
-      *reinterpret_cast<uint4*>(&sM[rl][16 * k]) = v;
-    }
-    __syncthreads();
-    const int64_t c = c_base + lane;         // row of Wt
-    const int64_t r0 = r_base + 32 * run;    // first column of Wt in this unit
-    uint32_t bytes[4] = {kPadByte, kPadByte, kPadByte, kPadByte};
-    if (c < C && r0 < R) {
-      Quad<Bits> q[4];
+  for (int64_t t = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < tiles; t += nwarps) {
+    const int64_t rt = t / ct_count;
+    const int64_t r0 = rt * 32, r = r0 + 4 * h;   // the lane's four rows: one group down each column
+    const int64_t c = (t - rt * ct_count) * 32 + 8 * q;
+    Oct<Bits> e[4];
+    uint2 mk[4];
 #pragma unroll
-      for (int o = 0; o < 4; ++o) {
-        if (r0 + 8 * o >= R) break;  // R % 8 == 0: octets are whole
-        Bits a[8];
-        uint32_t mlo = 0, mhi = 0;
+    for (int k = 0; k < 4; ++k) mk[k] = make_uint2(0u, 0u);
+    if (r < R && c < C) {  // R % 4 == 0: the four rows are in or out together
+      if (c + 8 <= C) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          a[k] = sW[32 * run + 8 * o + k][lane];
-          const uint32_t b = sM[32 * run + 8 * o + k][lane];
-          if (k < 4) mlo |= b << (8 * k);
-          else mhi |= b << (8 * (k - 4));
+        for (int k = 0; k < 4; ++k) {
+          e[k].load(W + (r + k) * ldw + c);
+          mk[k] = __ldcs(reinterpret_cast<const uint2*>(mask + (r + k) * ldm + c));
         }
-        bytes[o] = compress_octet<Bits, 1>(make_oct<Bits>(a), make_uint2(mlo, mhi), q[o], invalid);
-      }
-      Bits* vrow = values + c * (R / 2) + r0 / 2;
-      if (unit_vec && r0 + 32 <= R) {
-        store_unit<Bits>(q, vrow);
       } else {
 #pragma unroll
-        for (int o = 0; o < 4; ++o)
-          if (r0 + 8 * o < R) q[o].store(vrow + 4 * o);
+        for (int k = 0; k < 4; ++k) {
+          Bits a[8];
+          uint8_t b[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            a[j] = c + j < C ? W[(r + k) * ldw + c + j] : Bits(0);
+            b[j] = c + j < C ? mask[(r + k) * ldm + c + j] : uint8_t(0);
+          }
+          e[k] = make_oct<Bits>(a);
+          mk[k] = make_uint2(uint32_t(b[0]) | (uint32_t(b[1]) << 8) | (uint32_t(b[2]) << 16) | (uint32_t(b[3]) << 24),
+                             uint32_t(b[4]) | (uint32_t(b[5]) << 8) | (uint32_t(b[6]) << 16) | (uint32_t(b[7]) << 24));
+        }
       }
+    }
+    uint32_t mword = 0, iword = 0;  // this lane's metadata and image words (row 8q + h of the chunk)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint32_t nib = 0x4u;  // pad: pattern (0,1)
+      if (r < R && c + j < C) {
+        // mask byte j of rows 0..3 -> bytes 0..3 of w
+        const uint32_t sel = (j & 3) | (((j & 3) + 4) << 4);  // a constant after unrolling
+        const uint32_t lo = __byte_perm(j < 4 ? mk[0].x : mk[0].y, j < 4 ? mk[1].x : mk[1].y, sel);
+        const uint32_t hi = __byte_perm(j < 4 ? mk[2].x : mk[2].y, j < 4 ? mk[3].x : mk[3].y, sel);
+        const uint32_t w = __byte_perm(lo, hi, 0x5410);
+        const Pick pk = pick_masked(w, invalid);
+        nib = pk.nib;
+        Bits* dst = values + (c + j) * (R / 2) + r / 2;
+        if constexpr (sizeof(Bits) == 2) {
+          // entry j of rows 0..3: half j & 1 of word j / 2 of each row
+          const uint32_t hsel = (j & 1) ? 0x7632u : 0x5410u;
+          const uint32_t g01 = __byte_perm((&e[0].v.x)[j >> 1], (&e[1].v.x)[j >> 1], hsel);
+          const uint32_t g23 = __byte_perm((&e[2].v.x)[j >> 1], (&e[3].v.x)[j >> 1], hsel);
+          __stcs(reinterpret_cast<uint32_t*>(dst), pair16(g01, g23, pk));
+        } else if constexpr (sizeof(Bits) == 1) {
+          const uint32_t blo = __byte_perm(j < 4 ? e[0].v.x : e[0].v.y, j < 4 ? e[1].v.x : e[1].v.y, sel);
+          const uint32_t bhi = __byte_perm(j < 4 ? e[2].v.x : e[2].v.y, j < 4 ? e[3].v.x : e[3].v.y, sel);
+          __stcs(reinterpret_cast<unsigned short*>(dst),
+                 static_cast<unsigned short>(pair8(__byte_perm(blo, bhi, 0x5410), pk)));
+        } else {
+          __stcs(reinterpret_cast<uint2*>(dst), pair32(e[0][j], e[1][j], e[2][j], e[3][j], pk));
+        }
+      }
+      uint32_t word = nib << (4 * h);  // groups r0/4 .. r0/4 + 7 of row c + j
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 8);
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 16);
+      const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, word, 1);  // row c + j +- 8
+      if (j == h) {
+        mword = word;
+        iword = (q & 1) ? __byte_perm(other, word, 0x7632) : __byte_perm(word, other, 0x5410);
+      }
+    }
+    const int64_t crow = c + h;  // the row of Wt this lane stores for
+    if (crow < C && r0 < R) {
+      uint8_t* mrow = meta + crow * (R / 8) + r0 / 8;
       if (meta_words) {
-        __stcs(reinterpret_cast<uint32_t*>(meta + c * (R / 8) + r0 / 8),
-               bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24));
+        __stcs(reinterpret_cast<uint32_t*>(mrow), mword);
       } else {
 #pragma unroll
-        for (int o = 0; o < 4; ++o)
-          if (r0 + 8 * o < R) meta[c * (R / 8) + r0 / 8 + o] = uint8_t(bytes[o]);
+        for (int b = 0; b < 4; ++b)
+          if (r0 + 8 * b < R) mrow[b] = uint8_t(mword >> (8 * b));
       }
     }
     if (img != nullptr) {
-      const uint32_t p0 = bytes[0] | (bytes[1] << 8), p1 = bytes[2] | (bytes[3] << 8);
-      const uint32_t o0 = __shfl_xor_sync(0xFFFFFFFFu, p0, 8), o1 = __shfl_xor_sync(0xFFFFFFFFu, p1, 8);
-      const bool upper = (lane & 8) != 0;     // this lane holds row c, its partner row c - 8
-      const uint32_t word = upper ? (o1 | (p1 << 16)) : (p0 | (o0 << 16));
-      const int64_t crow = upper ? c - 8 : c;  // the pair's row with (row % 16) < 8
-      if (r0 < Rp) {
-        uint8_t* blk = img + ((crow >> 7) * (Rp / 128) + (r0 >> 7)) * 2048;
-        const uint32_t L = uint32_t(crow & 7) + 8u * (upper ? 1u : 0u) + 16u * uint32_t((crow & 127) >> 4);
-        __stcs(reinterpret_cast<uint32_t*>(blk + L * 16u + uint32_t((r0 & 127) >> 5) * 4u), word);
-      }
+      // row pair (p, p + 8), p = crow with bit 3 cleared; even q writes the
+      // half for columns r0..r0+15 of Wt, odd q the half for r0+16..r0+31
+      const int64_t prow = crow & ~int64_t(8);
+      const uint32_t L = uint32_t(prow & 7) + 8u * uint32_t(q & 1) + 16u * uint32_t((prow & 127) >> 4);
+      uint8_t* blk = img + ((prow >> 7) * (Rp / 128) + (r0 >> 7)) * 2048;
+      __stcs(reinterpret_cast<uint32_t*>(blk + L * 16u + uint32_t((r0 & 127) >> 5) * 4u), iword);
     }
-    __syncthreads();
   }
   if (invalid_groups != nullptr) {
 #pragma unroll
@@ -755,11 +813,11 @@ extern "C" nm_status nm_compress_t(const void* W, const uint8_t* mask, nm_dtype 
       (invalid_groups && (reinterpret_cast<uintptr_t>(invalid_groups) & 3u)))
     return NM_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int64_t tiles = (((R + 127) / 128 * 128 + kTR - 1) / kTR) * ((C + 127) / 128 * 128 / kTC);
+  const int64_t blocks = (((R + 127) / 128 * 4) * ((C + 127) / 128 * 4) + 7) / 8;  // eight 32x32 tiles each
   auto launch = [&](auto kernel, auto* w, auto* v) {
     const int64_t cap = int64_t(blocks_per_sm(kernel, 256)) * sm_count();
-    kernel<<<unsigned(tiles < cap ? tiles : cap), 256, 0, s>>>(w, ldw, mask, ldm, R, C, v, meta_t, meta_t_sm100,
-                                                               invalid_groups);
+    kernel<<<unsigned(blocks < cap ? blocks : cap), 256, 0, s>>>(w, ldw, mask, ldm, R, C, v, meta_t, meta_t_sm100,
+                                                                 invalid_groups);
   };
   if (dtype == NM_F32)
     launch(compress_t_kernel<uint32_t>, static_cast<const uint32_t*>(W), static_cast<uint32_t*>(values_t));
