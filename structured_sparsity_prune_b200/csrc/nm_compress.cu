@@ -160,8 +160,14 @@ __device__ __forceinline__ uint32_t compress_octet(const Oct<Bits>& e, uint2 m, 
   Pick p[2];
 #pragma unroll
   for (int g = 0; g < 2; ++g) {
-    if constexpr (MODE == 0) p[g] = pick_magnitude<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3]);
-    else p[g] = pick_masked(g ? m.y : m.x, invalid);
+    if constexpr (MODE == 0 && sizeof(Bits) == 1) {  // int8: the in-register rank rule
+      const uint32_t keep = keep_of_bytes(keep4_s8<2>(g ? e.v.y : e.v.x));
+      p[g] = Pick{uint32_t(kPairNib >> (4 * keep)) & 0xFu, false, false};
+    } else if constexpr (MODE == 0) {
+      p[g] = pick_magnitude<Bits>(e[4 * g], e[4 * g + 1], e[4 * g + 2], e[4 * g + 3]);
+    } else {
+      p[g] = pick_masked(g ? m.y : m.x, invalid);
+    }
   }
   if constexpr (sizeof(Bits) == 2) {
     q.v = make_uint2(pair16(e.v.x, e.v.y, p[0]), pair16(e.v.z, e.v.w, p[1]));
@@ -284,10 +290,14 @@ __device__ __forceinline__ void store_unit(const Quad<Bits> (&q)[4], Bits* p) {
 // up to a multiple of 4): threads outside the matrix write only pad pieces.
 // For 8- and 16-bit elements both rows' loads are issued before either is
 // used; fp32 (128 bytes per unit and row) takes the rows one after the other.
-// Two blocks share an SM: the kernel needs ~128 registers a thread, and a
-// tighter bound spills.
+// Blocks that share an SM (kRowsBlocks): two for 16- and 32-bit elements
+// (~128 registers a thread under a mask; three was slower on large weights
+// without one), more for int8, whose thread moves fewer bytes.
 template <typename Bits, int MODE>
-__global__ void __launch_bounds__(256, 2) compress_rows_kernel(
+constexpr int kRowsBlocks = sizeof(Bits) == 1 ? (MODE == 0 ? 4 : 3) : 2;
+
+template <typename Bits, int MODE>
+__global__ void __launch_bounds__(256, kRowsBlocks<Bits, MODE>) compress_rows_kernel(
     const Bits* __restrict__ W, int64_t ldw, const uint8_t* __restrict__ mask, int64_t ldm, int64_t R,
     int64_t C, Bits* __restrict__ values, uint8_t* __restrict__ meta, uint8_t* __restrict__ img,
     int32_t* __restrict__ invalid_groups) {

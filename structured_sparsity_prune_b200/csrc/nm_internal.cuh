@@ -116,6 +116,36 @@ __device__ __forceinline__ uint32_t keep_bytes4(uint32_t x0, uint32_t x1, uint32
   return (~t >> 7) & 0x01010101u;
 }
 
+// int8 groups of four, one group per 32-bit word (entry k in byte k), the
+// magnitude |x| (0..128) and the rank rule above, in-register (SWAR):
+//  - per-byte |x| without carries between bytes: (x ^ m) + s with s the sign
+//    bit of each byte and m = 0xFF where negative (|-128| = 0x80 fits);
+//  - the six pairwise tests k_i >= k_j (i < j, "i beats j"; false = "j beats
+//    i") as three 16-bit-lane subtractions (0x100 + k_i) - k_j: bit 8 of a
+//    lane is set iff k_i >= k_j, and no borrow leaves the lane;
+//  - each entry's three "beaten by" terms gathered into byte lanes (A, B, C,
+//    polarity fixed per byte), and dropped when at least N of them hold: an
+//    OR (N = 1), a majority (N = 2) or an AND (N = 3) of three 0/1 bytes.
+// Returns the keep bytes (0/1 per byte) of the group.
+template <int N>
+__device__ __forceinline__ uint32_t keep4_s8(uint32_t w) {
+  const uint32_t sgn = (w >> 7) & 0x01010101u;
+  const uint32_t a = (w ^ (sgn * 0xFFu)) + sgn;                               // |x| per byte
+  const uint32_t G = 0x01010101u;
+  const uint32_t d1 = __byte_perm(a, G, 0x4240) - __byte_perm(a, 0u, 0x4341);  // t01 (byte 1), t23 (byte 3)
+  const uint32_t x01 = __byte_perm(a, G, 0x4140);
+  const uint32_t d2 = x01 - __byte_perm(a, 0u, 0x4342);                       // t02, t13
+  const uint32_t d3 = x01 - __byte_perm(a, 0u, 0x4243);                       // t03, t12
+  const uint32_t A = __byte_perm(__byte_perm(d1, d2, 0x0511), d3, 0x5210) ^ 0x00000001u;  // t01 t01 t02 t03
+  const uint32_t B = __byte_perm(d2, d3, 0x3771) ^ 0x00000101u;                           // t02 t12 t12 t13
+  const uint32_t C = __byte_perm(__byte_perm(d3, d2, 0x0071), d1, 0x7710) ^ 0x00010101u;  // t03 t13 t23 t23
+  uint32_t drop;
+  if constexpr (N == 1) drop = A | B | C;
+  else if constexpr (N == 2) drop = (A & B) | (A & C) | (B & C);
+  else drop = A & B & C;
+  return drop ^ 0x01010101u;
+}
+
 // 2:4 specialisation: the two kept indices (ascending) of a group and the
 // 4-bit metadata field idx0 | idx1 << 2.
 struct Pick24 {

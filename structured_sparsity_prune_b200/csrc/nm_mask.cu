@@ -90,6 +90,9 @@ __global__ void __launch_bounds__(256) mask_vec16_kernel(const Bits* __restrict_
 // (the grid is sized to exactly what the SMs hold).
 template <typename Bits, int N>
 __device__ __forceinline__ uint4 select4_chunk(const uint4 (&v)[Chunk16<Bits>::kVec]) {
+  if constexpr (sizeof(Bits) == 1) {  // one int8 group per word
+    return make_uint4(keep4_s8<N>(v[0].x), keep4_s8<N>(v[0].y), keep4_s8<N>(v[0].z), keep4_s8<N>(v[0].w));
+  }
   const Bits* e = reinterpret_cast<const Bits*>(v);
   uint32_t out[4];
 #pragma unroll

@@ -38,6 +38,30 @@ def test_mask(N, M, C):
     assert np.array_equal(got, oracle.mask_rank(W.numpy(), N, M))
 
 
+def _all_groups_of_sixteen_values():
+    """Every group of four drawn from 16 values with ties, both extremes and
+    both signs of equal magnitudes: 16**4 groups, 1024 per row."""
+    vals = np.array([-128, -127, -64, -5, -3, -2, -1, 0, 1, 2, 3, 5, 63, 64, 126, 127], dtype=np.int8)
+    idx = np.indices((16, 16, 16, 16)).reshape(4, -1).T          # (65536, 4)
+    return torch.from_numpy(vals[idx].reshape(64, 4096).copy())
+
+
+@pytest.mark.parametrize("N", [1, 2, 3])
+def test_mask_every_group_of_sixteen_values(N):
+    W = _all_groups_of_sixteen_values()
+    got = nm.nm_mask(W.cuda(), N, 4).cpu().numpy()
+    assert np.array_equal(got, oracle.mask_rank(W.numpy(), N, 4))
+
+
+def test_mask_compress_every_group_of_sixteen_values():
+    W = _all_groups_of_sixteen_values()
+    v, meta, img = nm.nm_mask_compress(W.cuda())
+    rv, rm = oracle.compress24(W.numpy(), oracle.mask_rank(W.numpy(), 2, 4))
+    assert np.array_equal(v.cpu().numpy(), rv)
+    assert np.array_equal(meta.cpu().numpy(), rm)
+    assert np.array_equal(img.cpu().numpy(), oracle.meta_sm100(rm, 64, 4096))
+
+
 @pytest.mark.parametrize("R,C", [(256, 256), (200, 96), (130, 48)])
 def test_mask_compress_and_image(R, C):
     W = _int8((R, C), R + C)
