@@ -594,11 +594,11 @@ __global__ void __launch_bounds__(256) decompress32_kernel(const Bits* __restric
 // reads 64 B, 32 B or 128 B of each of 32 rows).  It compresses the eight
 // groups in registers and stores each pair of values into row c of Wt (the
 // eight lanes of a column chunk fill 8 consecutive groups: one 32-byte run
-// of a row of Wt per store).  Three xor-shuffles give every lane of a column
-// chunk the metadata word of each of its 8 rows of Wt (8 nibbles, 32 columns
-// of Wt); lane h stores the word of row 8q + h.  Image words pair rows c and
-// c + 8 of Wt, which are lanes q and q ^ 1: one more shuffle, and lane h
-// writes the image word of row 8q + h.  The warps of a block take adjacent
+// of a row of Wt per store).  The lane's eight nibbles make one word, and a
+// three-stage nibble transpose across the eight lanes of its column chunk
+// leaves lane h holding the metadata word of row c + h of Wt (8 nibbles, 32
+// columns of Wt).  Image words pair rows c and c + 8 of Wt, which are lanes q
+// and q ^ 1: one more shuffle, and lane h writes the image word of row c + h.  The warps of a block take adjacent
 // column tiles of the same rows; the grid covers the image's padded extent.
 template <typename Bits>
 __device__ __forceinline__ Oct<Bits> make_oct(const Bits (&a)[8]) {
@@ -659,7 +659,11 @@ __global__ void __launch_bounds__(256, 3) compress_t_kernel(const Bits* __restri
         }
       }
     }
-    uint32_t mword = 0, iword = 0;  // this lane's metadata and image words (row 8q + h of the chunk)
+    // This lane's eight nibbles (group h of columns c..c+7, nibble j = column j)
+    // form one word; an 8 x 8 nibble transpose across the eight lanes of the
+    // column chunk (h = lane bits 2..4) gives lane h the metadata word of row
+    // c + h of Wt (nibble g = group g).  Three masked butterfly stages.
+    uint32_t nibs = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       uint32_t nib = 0x4u;  // pad: pattern (0,1)
@@ -687,16 +691,21 @@ __global__ void __launch_bounds__(256, 3) compress_t_kernel(const Bits* __restri
           __stcs(reinterpret_cast<uint2*>(dst), pair32(e[0][j], e[1][j], e[2][j], e[3][j], pk));
         }
       }
-      uint32_t word = nib << (4 * h);  // groups r0/4 .. r0/4 + 7 of row c + j
-      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
-      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 8);
-      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 16);
-      const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, word, 1);  // row c + j +- 8
-      if (j == h) {
-        mword = word;
-        iword = (q & 1) ? __byte_perm(other, word, 0x7632) : __byte_perm(word, other, 0x5410);
+      nibs |= nib << (4 * j);
+    }
+    {
+      constexpr uint32_t kLo[3] = {0x0F0F0F0Fu, 0x00FF00FFu, 0x0000FFFFu};
+#pragma unroll
+      for (int k = 0; k < 3; ++k) {
+        const int d = 1 << k;
+        const uint32_t other = __shfl_xor_sync(0xFFFFFFFFu, nibs, 4 * d);  // lane of group h ^ d
+        nibs = (h & d) ? ((nibs & ~kLo[k]) | ((other >> (4 * d)) & kLo[k]))
+                       : ((nibs & kLo[k]) | ((other << (4 * d)) & ~kLo[k]));
       }
     }
+    const uint32_t mword = nibs;
+    const uint32_t partner = __shfl_xor_sync(0xFFFFFFFFu, mword, 1);  // row c + h +- 8 (lane q ^ 1)
+    const uint32_t iword = (q & 1) ? __byte_perm(partner, mword, 0x7632) : __byte_perm(mword, partner, 0x5410);
     const int64_t crow = c + h;  // the row of Wt this lane stores for
     if (crow < C && r0 < R) {
       uint8_t* mrow = meta + crow * (R / 8) + r0 / 8;
