@@ -15,10 +15,13 @@ roofline of the dominant kernel (nm_spmm, sparse tensor peak) and the
 bandwidth kernels' GB/s against HBM are reported beside it.
 
 Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
-events on the launching stream, with L2 flushed (a 256 MiB write) between
-steps outside the events; barrier + synchronize around the loop; the max over
-ranks.  N > 1 runs one independent copy of the workload per GPU (the path
-has no exchange step; weak scaling).
+events on the launching stream, with L2 flushed between steps outside the
+events (a 256 MiB write, then a 256 MiB read that evicts the written lines,
+so no write-back of the flush lands in a timed region); barrier + synchronize
+around the loop; the max over ranks.  The per-kernel breakdown times every
+launch on its own with the same flush before each.  N > 1 runs one
+independent copy of the workload per GPU (the path has no exchange step;
+weak scaling).
 """
 from __future__ import annotations
 
@@ -393,15 +396,9 @@ class Step:
                 lambda: nm.nm_decompress(self.values, self.meta, K, out=self.Wd),
                 lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.Y, workspace=self.ws)]
 
-    def run(self, events=None):
-        s = torch.cuda.current_stream()
-        calls = self.calls()
-        for i, fn in enumerate(calls):
-            if events is not None:
-                events[i].record(s)
+    def run(self):
+        for fn in self.calls():
             fn()
-        if events is not None:
-            events[len(calls)].record(s)
 
     def capture(self):
         """CUDA graphs of the whole step and of each launch, captured once after
@@ -432,12 +429,28 @@ class Step:
         return self.masks[1] if self.kind == "ties" else self.Y
 
 
-def timed_steps(step: Step, steps: int, flush: torch.Tensor, graphs=None):
+class L2Flush:
+    """Evicts L2 between timed iterations, outside the events: a 256 MiB write
+    (twice the L2) and then a 256 MiB read of a second buffer.  The read pushes
+    the written lines out (their write-back happens here, not in the next timed
+    kernel) and leaves L2 holding clean, unrelated lines, so the timed work
+    starts cold and pays only for its own traffic."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(32 << 20, dtype=torch.int64, device=dev)
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.sum()
+
+
+def timed_steps(step: Step, steps: int, flush, graphs=None):
     """-> per-step ms over exactly `steps` steps (graph replays when captured)."""
     s = torch.cuda.current_stream()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for i in range(steps):
-        flush.zero_()                      # evict L2 between steps (outside the events)
+        flush()                            # evict L2 between steps (outside the events)
         ev[i][0].record(s)
         if graphs is not None:
             graphs[0].replay()
@@ -448,25 +461,29 @@ def timed_steps(step: Step, steps: int, flush: torch.Tensor, graphs=None):
     return [a.elapsed_time(b) for a, b in ev]
 
 
-def kernel_breakdown(step: Step, steps: int, flush: torch.Tensor, graphs=None):
-    """-> per-kernel ms lists: the same steps again, with events around each launch."""
+def kernel_breakdown(step: Step, steps: int, flush, graphs=None):
+    """-> per-kernel ms lists: each launch of the step timed on its own, L2
+    flushed before every launch (outside its events), so every kernel starts
+    cold and its figure counts only its own traffic."""
     s = torch.cuda.current_stream()
     n = step.launches()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    calls = step.calls()
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+          for _ in range(steps)]
     for i in range(steps):
-        flush.zero_()
-        if graphs is not None:
-            for j, g in enumerate(graphs[1]):
-                ev[i][j].record(s)
-                g.replay()
-            ev[i][n].record(s)
-        else:
-            step.run(ev[i])
+        for j in range(n):
+            flush()
+            ev[i][j][0].record(s)
+            if graphs is not None:
+                graphs[1][j].replay()
+            else:
+                calls[j]()
+            ev[i][j][1].record(s)
     torch.cuda.synchronize()
-    return {name: [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(steps)] for j, name in enumerate(step.names)}
+    return {name: [ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps)] for j, name in enumerate(step.names)}
 
 
-def dense_context(step: Step, reps: int, flush: torch.Tensor):
+def dense_context(step: Step, reps: int, flush):
     """Context only: the same products as dense bf16 GEMMs in cuBLAS (torch.matmul)
     on the decompressed weights, timed like the step (L2 flushed before each rep).
     -> {name: ms} for the product launches of the step, or None."""
@@ -491,7 +508,7 @@ def dense_context(step: Step, reps: int, flush: torch.Tensor):
             torch.matmul(A, B, out=C)
         ts = []
         for _ in range(reps):
-            flush.zero_()
+            flush()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(s)
             torch.matmul(A, B, out=C)
@@ -736,7 +753,7 @@ def main():
     nm.load()                                    # fails loudly without the CUDA library
     wl = make_workload(args.workload)
     step = Step(nm, wl, dev)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
 
     for _ in range(warmup):
         step.run()
@@ -855,7 +872,8 @@ def main():
                            "sparsity": {"ties": "N:M along K (1:4, 2:4, 4:8, 2:8)", "pairs": "1:2 along K",
                                         "transposable": "4:8 transposable (8x8 blocks)",
                                         "trans24": "2:4 transposable (4x4 blocks)"}.get(step.kind, "2:4 along K"),
-                           "l2": "flushed: 256 MiB write between timed steps, outside the events",
+                           "l2": "flushed between timed steps, outside the events: a 256 MiB write, then a 256 MiB read "
+                                 "that evicts the written lines",
                            "launch": launch_mode,
                            "parallelism": "independent replica per GPU" if world > 1 else "single GPU"},
                 "roofline": roof, "cpu_baseline": cpu, "dense_context": dense_line,
