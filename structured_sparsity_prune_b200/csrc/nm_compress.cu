@@ -290,14 +290,17 @@ __device__ __forceinline__ void store_unit(const Quad<Bits> (&q)[4], Bits* p) {
 // up to a multiple of 4): threads outside the matrix write only pad pieces.
 // For 8- and 16-bit elements both rows' loads are issued before either is
 // used; fp32 (128 bytes per unit and row) takes the rows one after the other.
-// Blocks that share an SM (kRowsBlocks): two for 16- and 32-bit elements
-// (~128 registers a thread under a mask; three was slower on large weights
-// without one), more for int8, whose thread moves fewer bytes.
+// Blocks that share an SM (MINB): two for 16- and 32-bit elements (~128
+// registers a thread under a mask), more for int8, whose thread moves fewer
+// bytes.  Selection by magnitude also has a three-block form (no spills) for
+// weights under 2^25 entries: there a launch is short enough that the bytes
+// in flight, not DRAM page traffic, set its pace (three blocks were 5 %
+// slower on a 235 M-entry weight and 9 % faster on a 16.8 M one).
 template <typename Bits, int MODE>
 constexpr int kRowsBlocks = sizeof(Bits) == 1 ? (MODE == 0 ? 4 : 3) : 2;
 
-template <typename Bits, int MODE>
-__global__ void __launch_bounds__(256, kRowsBlocks<Bits, MODE>) compress_rows_kernel(
+template <typename Bits, int MODE, int MINB = kRowsBlocks<Bits, MODE>>
+__global__ void __launch_bounds__(256, MINB) compress_rows_kernel(
     const Bits* __restrict__ W, int64_t ldw, const uint8_t* __restrict__ mask, int64_t ldm, int64_t R,
     int64_t C, Bits* __restrict__ values, uint8_t* __restrict__ meta, uint8_t* __restrict__ img,
     int32_t* __restrict__ invalid_groups) {
@@ -752,7 +755,14 @@ void launch_compress(const void* W, int64_t ldw, const uint8_t* mask, int64_t ld
                                                                            invalid_groups);
     return;
   }
-  static const int per_sm = blocks_per_sm(compress_rows_kernel<Bits, MODE>, 256);
+  constexpr bool kHasSmall = MODE == 0 && sizeof(Bits) >= 2;
+  const bool small = kHasSmall && R * C < (int64_t(1) << 25);
+  static const int per_sm_big = blocks_per_sm(compress_rows_kernel<Bits, MODE>, 256);
+  int per_sm = per_sm_big;
+  if constexpr (kHasSmall) {
+    static const int per_sm_small = blocks_per_sm(compress_rows_kernel<Bits, MODE, 3>, 256);
+    if (small) per_sm = per_sm_small;
+  }
   const int64_t units = ((C + 127) / 128) * 4, pairs = ((R + 127) / 128) * 64;
   int bx = 32;
   while (bx < 256 && bx < units) bx *= 2;
@@ -764,6 +774,13 @@ void launch_compress(const void* W, int64_t ldw, const uint8_t* mask, int64_t ld
   if (gy > cap_y) gy = cap_y;
   if (gy > 65535) gy = 65535;
   dim3 grid(unsigned(gx > 2147483647 ? 2147483647 : gx), unsigned(gy < 1 ? 1 : gy)), block(bx, by);
+  if constexpr (kHasSmall) {
+    if (small) {
+      compress_rows_kernel<Bits, MODE, 3><<<grid, block, 0, s>>>(w, ldw, mask, ldm, R, C, v, meta, img,
+                                                                 invalid_groups);
+      return;
+    }
+  }
   compress_rows_kernel<Bits, MODE><<<grid, block, 0, s>>>(w, ldw, mask, ldm, R, C, v, meta, img, invalid_groups);
 }
 

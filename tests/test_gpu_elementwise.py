@@ -223,6 +223,18 @@ def test_meta_to_sm100(R, C):
     assert np.array_equal(got, oracle.meta_sm100(meta, R, C))
 
 
+@pytest.mark.parametrize("R,C,dtype", [(8192, 4096, torch.bfloat16), (4096, 8192, torch.float32)])
+def test_mask_compress_large_weights(R, C, dtype):
+    """2^25 entries: the magnitude compressor's two-block form (smaller
+    weights take the three-block form), whole matrix, bit-exact."""
+    W = nm_inputs.normal((R, C), 44, 0.02, dtype)
+    values, meta, img = nm.nm_mask_compress(W.cuda())
+    _, v_ref, m_ref = oracle.rows_parallel(1, _bits(W), 2, 4, CODE[dtype], threads=os.cpu_count() or 2)
+    assert np.array_equal(_bits(values), np.ascontiguousarray(v_ref).view(_bits(values).dtype))
+    assert np.array_equal(meta.cpu().numpy(), m_ref)
+    assert np.array_equal(img.cpu().numpy(), oracle.meta_sm100(m_ref, R, C))
+
+
 def test_linear_4096_mask_compress_full_size():
     """The 4096 x 4096 bf16 transformer-linear weight, whole matrix, bit-exact."""
     W, _ = nm_inputs.linear_4096()
