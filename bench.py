@@ -400,22 +400,68 @@ class Step:
         for fn in self.calls():
             fn()
 
+    def deps(self):
+        """For each launch of calls(), the earlier launches whose outputs it reads."""
+        n = self.launches()
+        if self.kind == "linear":     # mask -> compress; fused -> {image, decompress, product}
+            return [[], [0], [], [2], [2], [2]]
+        if self.kind == "mlp":        # two compressions; up -> down (H)
+            return [[], [], [0], [1, 2]]
+        if self.kind == "trans24":    # mask -> {compress -> forward, compress_t -> backward}
+            return [[], [0], [0], [1], [2]]
+        if self.kind == "ties":       # four masks of the same W
+            return [[] for _ in range(n)]
+        if self.kind == "int8":       # mask; fused -> decompress
+            return [[], [], [1]]
+        if self.kind == "pairs":      # mask -> compress; fused -> decompress
+            return [[], [0], [], [2]]
+        return [[i - 1] if i else [] for i in range(n)]
+
     def capture(self):
-        """CUDA graphs of the whole step and of each launch, captured once after
-        warm-up; replaying them issues the same kernels with the same arguments
-        without the host's per-launch latency."""
-        whole = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(whole):
-            for fn in self.calls():
+        """CUDA graphs captured once after warm-up: the whole step as its
+        dependency graph (a launch waits only for the launches whose outputs it
+        reads; independent chains run on forked streams), the same step as one
+        sequential chain, and each launch alone.  Replaying them issues the same
+        kernels with the same arguments without the host's per-launch latency."""
+        calls, deps = self.calls(), self.deps()
+        pool = [torch.cuda.Stream() for _ in range(4)]
+        dag = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(dag):
+            cap = torch.cuda.current_stream()
+            start = torch.cuda.Event()
+            start.record(cap)
+            done, where, last_on, used = [None] * len(calls), [None] * len(calls), {}, []
+            for i, fn in enumerate(calls):
+                # continue a dependency's chain when it is the last launch on its stream
+                st = next((where[j] for j in deps[i] if last_on.get(where[j]) == j), None)
+                if st is None:
+                    st = next(k for k in range(len(pool)) if k not in last_on or k == len(pool) - 1)
+                stream = pool[st]
+                if st not in used:
+                    stream.wait_event(start)
+                    used.append(st)
+                for j in deps[i]:
+                    if where[j] != st:
+                        stream.wait_event(done[j])
+                with torch.cuda.stream(stream):
+                    fn()
+                    ev = torch.cuda.Event()
+                    ev.record(stream)
+                done[i], where[i], last_on[st] = ev, st, i
+            for st in used:
+                cap.wait_event(done[last_on[st]])
+        seq = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(seq):
+            for fn in calls:
                 fn()
         per = []
-        for fn in self.calls():
+        for fn in calls:
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
                 fn()
             per.append(g)
         torch.cuda.synchronize()
-        return whole, per
+        return dag, per, seq
 
     def result(self):
         if self.kind == "srste":
@@ -763,12 +809,14 @@ def main():
     try:
         eager = step.result().clone()
         graphs = step.capture()
-        launch_mode = "CUDA graph of the step, captured once after warm-up and replayed"
-        for _ in range(warmup):
-            graphs[0].replay()
-        torch.cuda.synchronize()
-        if not torch.equal(step.result(), eager):
-            raise SystemExit("graph replay of the step differs from the eager step")
+        launch_mode = ("CUDA graph of the step as its dependency graph (independent launches on forked "
+                       "streams), captured once after warm-up and replayed")
+        for g in (graphs[0], graphs[2]):
+            for _ in range(warmup):
+                g.replay()
+            torch.cuda.synchronize()
+            if not torch.equal(step.result(), eager):
+                raise SystemExit("graph replay of the step differs from the eager step")
     except SystemExit:
         raise
     except Exception as exc:   # capture unavailable: time eager launches instead
@@ -789,6 +837,8 @@ def main():
         pg.barrier()
     clk = clocks.stop()
     per = kernel_breakdown(step, args.steps, flush, graphs)
+    # the same step as one sequential chain, for comparison (not the timed region)
+    seq_ms = float(np.mean(timed_steps(step, args.steps, flush, (graphs[2],) if graphs else None)))
 
     total_ms = float(np.sum(tot))
     e2e_ms, h2d, d2h = e2e_steps(step, args.steps, nm, wl, dev)
@@ -875,6 +925,7 @@ def main():
                            "l2": "flushed between timed steps, outside the events: a 256 MiB write, then a 256 MiB read "
                                  "that evicts the written lines",
                            "launch": launch_mode,
+                           "step_sequential_ms": seq_ms,
                            "parallelism": "independent replica per GPU" if world > 1 else "single GPU"},
                 "roofline": roof, "cpu_baseline": cpu, "dense_context": dense_line,
                 "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
