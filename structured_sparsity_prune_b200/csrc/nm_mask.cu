@@ -87,7 +87,9 @@ __global__ void __launch_bounds__(256) mask_vec16_kernel(const Bits* __restrict_
 // selection of drop4 and the byte packing of keep_bytes4.  A thread takes its
 // chunk of two rows (r and r + the row stride of the grid) per iteration and
 // issues both rows' loads before selecting in either; five blocks share an SM
-// (the grid is sized to exactly what the SMs hold).
+// (the grid is sized to exactly what the SMs hold).  16-bit weights under
+// 2^25 entries take four rows per iteration (four blocks per SM): on a short
+// launch the bytes in flight set the pace.
 template <typename Bits, int N>
 __device__ __forceinline__ uint4 select4_chunk(const uint4 (&v)[Chunk16<Bits>::kVec]) {
   if constexpr (sizeof(Bits) == 1) {  // one int8 group per word
@@ -105,27 +107,49 @@ __device__ __forceinline__ uint4 select4_chunk(const uint4 (&v)[Chunk16<Bits>::k
   return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-template <typename Bits, int N>
-__global__ void __launch_bounds__(256, 5) mask4_vec16_kernel(const Bits* __restrict__ W, int64_t R, int64_t cpr,
-                                                          int64_t ldw, uint8_t* __restrict__ mask, int64_t ldm) {
+template <typename Bits, int N, int ROWS = 2>
+__global__ void __launch_bounds__(256, ROWS == 2 ? 5 : 4) mask4_vec16_kernel(const Bits* __restrict__ W, int64_t R,
+                                                                          int64_t cpr, int64_t ldw,
+                                                                          uint8_t* __restrict__ mask, int64_t ldm) {
   constexpr int kVec = Chunk16<Bits>::kVec;
   const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
   const int64_t c_step = int64_t(gridDim.x) * blockDim.x;
-  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += 2 * r_step) {
-    const int64_t r2 = r + r_step;
-    const bool two = r2 < R;
-    const uint4* wrow = reinterpret_cast<const uint4*>(W + r * ldw);
-    const uint4* wrow2 = reinterpret_cast<const uint4*>(W + (two ? r2 : r) * ldw);
-    for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < cpr; c += c_step) {
-      uint4 v[kVec], v2[kVec];
+  if constexpr (ROWS == 2) {
+    for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += 2 * r_step) {
+      const int64_t r2 = r + r_step;
+      const bool two = r2 < R;
+      const uint4* wrow = reinterpret_cast<const uint4*>(W + r * ldw);
+      const uint4* wrow2 = reinterpret_cast<const uint4*>(W + (two ? r2 : r) * ldw);
+      for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < cpr; c += c_step) {
+        uint4 v[kVec], v2[kVec];
 #pragma unroll
-      for (int i = 0; i < kVec; ++i) v[i] = __ldcs(wrow + c * kVec + i);
-      if (two) {
+        for (int i = 0; i < kVec; ++i) v[i] = __ldcs(wrow + c * kVec + i);
+        if (two) {
 #pragma unroll
-        for (int i = 0; i < kVec; ++i) v2[i] = __ldcs(wrow2 + c * kVec + i);
+          for (int i = 0; i < kVec; ++i) v2[i] = __ldcs(wrow2 + c * kVec + i);
+        }
+        __stcs(reinterpret_cast<uint4*>(mask + r * ldm) + c, select4_chunk<Bits, N>(v));
+        if (two) __stcs(reinterpret_cast<uint4*>(mask + r2 * ldm) + c, select4_chunk<Bits, N>(v2));
       }
-      __stcs(reinterpret_cast<uint4*>(mask + r * ldm) + c, select4_chunk<Bits, N>(v));
-      if (two) __stcs(reinterpret_cast<uint4*>(mask + r2 * ldm) + c, select4_chunk<Bits, N>(v2));
+    }
+  } else {
+    for (int64_t r0 = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r0 < R; r0 += ROWS * r_step) {
+      for (int64_t c = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; c < cpr; c += c_step) {
+        uint4 v[ROWS][kVec];
+#pragma unroll
+        for (int k = 0; k < ROWS; ++k) {
+          const int64_t r = r0 + k * r_step;
+          if (r < R) {
+#pragma unroll
+            for (int i = 0; i < kVec; ++i) v[k][i] = __ldcs(reinterpret_cast<const uint4*>(W + r * ldw) + c * kVec + i);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < ROWS; ++k) {
+          const int64_t r = r0 + k * r_step;
+          if (r < R) __stcs(reinterpret_cast<uint4*>(mask + r * ldm) + c, select4_chunk<Bits, N>(v[k]));
+        }
+      }
     }
   }
 }
@@ -272,9 +296,19 @@ void launch_mask(const void* W, int64_t R, int64_t C, int64_t ldw, int N, uint8_
   dim3 grid, block;
   if constexpr (M == 4) {
     if (vec) {
+      const Bits* w = static_cast<const Bits*>(W);
+      if constexpr (sizeof(Bits) == 2) {  // fp32 and int8 spill with four rows
+        if (R * C < (int64_t(1) << 25)) {  // a short launch: four rows in flight per thread
+          static const int per_sm4 = blocks_per_sm(mask4_vec16_kernel<Bits, 2, 4>, 256);
+          shape2d(R, C / 16, grid, block, per_sm4);
+          if (N == 1) mask4_vec16_kernel<Bits, 1, 4><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);
+          else if (N == 2) mask4_vec16_kernel<Bits, 2, 4><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);
+          else mask4_vec16_kernel<Bits, 3, 4><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);
+          return;
+        }
+      }
       static const int per_sm = blocks_per_sm(mask4_vec16_kernel<Bits, 2>, 256);
       shape2d(R, C / 16, grid, block, per_sm);
-      const Bits* w = static_cast<const Bits*>(W);
       if (N == 1) mask4_vec16_kernel<Bits, 1><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);
       else if (N == 2) mask4_vec16_kernel<Bits, 2><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);
       else mask4_vec16_kernel<Bits, 3><<<grid, block, 0, s>>>(w, R, C / 16, ldw, mask, ldm);

@@ -223,6 +223,15 @@ def test_meta_to_sm100(R, C):
     assert np.array_equal(got, oracle.meta_sm100(meta, R, C))
 
 
+@pytest.mark.parametrize("N", [1, 2, 3])
+def test_mask_24_large_bf16(N):
+    """2^25 bf16 entries: the two-rows form of the M = 4 mask (smaller 16-bit
+    weights take the four-rows form), whole matrix, byte for byte."""
+    W = nm_inputs.normal((8192, 4096), 45, 0.02, torch.bfloat16)
+    got = nm.nm_mask(W.cuda(), N, 4).cpu().numpy()
+    assert np.array_equal(got, oracle.mask_rank(_bits(W), N, 4, dtype=oracle.BF16))
+
+
 @pytest.mark.parametrize("R,C,dtype", [(8192, 4096, torch.bfloat16), (4096, 8192, torch.float32)])
 def test_mask_compress_large_weights(R, C, dtype):
     """2^25 entries: the magnitude compressor's two-block form (smaller
