@@ -562,7 +562,7 @@ template <typename Bits>
 __global__ void __launch_bounds__(256) decompress32_kernel(const Bits* __restrict__ values,
                                                            const uint8_t* __restrict__ meta, int64_t R,
                                                            int64_t C, Bits* __restrict__ out, int64_t ldo) {
-  constexpr int kVals = 16 * int(sizeof(Bits)) / 16;  // 16-byte loads of values per unit: 1, 2 or 4
+  constexpr int kVals = 16 * int(sizeof(Bits)) / 16;  // 16-byte loads of values per unit: 1 or 2
   const int64_t upr = C / 32;
   const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
   const int64_t u_step = int64_t(gridDim.x) * blockDim.x;
@@ -898,12 +898,8 @@ extern "C" nm_status nm_decompress(const void* values, const uint8_t* meta, nm_d
       decompress_kernel<uint8_t><<<grid, block, 0, s>>>(static_cast<const uint8_t*>(values), meta, R, C,
                                                         static_cast<uint8_t*>(W_out), ldw);
   } else if (dtype == NM_F32) {
-    if (wide)
-      decompress32_kernel<uint32_t><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C,
-                                                           static_cast<uint32_t*>(W_out), ldw);
-    else
-      decompress_kernel<uint32_t><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C,
-                                                         static_cast<uint32_t*>(W_out), ldw);
+    decompress_kernel<uint32_t><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C,
+                                                       static_cast<uint32_t*>(W_out), ldw);
   } else {
     if (wide)
       decompress32_kernel<uint16_t><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(values), meta, R, C,
