@@ -7,15 +7,18 @@
 // values.  The hardware layout of the indices is the PTX ISA's tcgen05
 // sparse-matrix metadata (the pages do not give one).
 //
-// All kernels here are HBM-bound streams.  A compressing thread takes a (row,
-// 32-column) unit: it reads the unit's 32 weights with 16-byte loads,
+// All kernels here stream HBM; the int8 selections and the transposed
+// compressor are bound by integer issue first.  A compressing thread takes a
+// (row, 32-column) unit: it reads the unit's 32 weights with 16-byte loads,
 // selects/compresses in registers, and writes its 16 values and 4 canonical
 // metadata bytes with vector stores.  When C % 32 == 0 the units are streamed
 // row by row (two rows per thread, whose image pieces share 4-byte words that
 // the thread writes itself); otherwise a block walks 128-row x 128-column
 // tiles, drops the units' 16-bit image pieces into shared memory and writes
 // each finished 2048-byte image block with one coalesced 16-byte store per
-// thread.
+// thread.  Decompression expands (row, 32- or 8-column) units; the transposed
+// compressor (for the backward product) works on 32 x 32 tiles per warp in
+// registers (see its comment below).
 #include "nm_internal.cuh"
 
 namespace nm {
@@ -601,8 +604,9 @@ __global__ void __launch_bounds__(256) decompress32_kernel(const Bits* __restric
 // three-stage nibble transpose across the eight lanes of its column chunk
 // leaves lane h holding the metadata word of row c + h of Wt (8 nibbles, 32
 // columns of Wt).  Image words pair rows c and c + 8 of Wt, which are lanes q
-// and q ^ 1: one more shuffle, and lane h writes the image word of row c + h.  The warps of a block take adjacent
-// column tiles of the same rows; the grid covers the image's padded extent.
+// and q ^ 1: one more shuffle, and lane h writes the image word of row c + h.
+// The warps of a block take adjacent column tiles of the same rows; the grid
+// covers the image's padded extent.
 template <typename Bits>
 __device__ __forceinline__ Oct<Bits> make_oct(const Bits (&a)[8]) {
   Oct<Bits> e;

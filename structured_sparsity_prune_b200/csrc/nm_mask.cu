@@ -141,7 +141,8 @@ __global__ void __launch_bounds__(256, ROWS == 2 ? 5 : 4) mask4_vec16_kernel(con
           const int64_t r = r0 + k * r_step;
           if (r < R) {
 #pragma unroll
-            for (int i = 0; i < kVec; ++i) v[k][i] = __ldcs(reinterpret_cast<const uint4*>(W + r * ldw) + c * kVec + i);
+            for (int i = 0; i < kVec; ++i)
+              v[k][i] = __ldcs(reinterpret_cast<const uint4*>(W + r * ldw) + c * kVec + i);
           }
         }
 #pragma unroll
