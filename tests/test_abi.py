@@ -89,6 +89,33 @@ def test_host_validation_before_any_launch(lib):
     assert L.nm_mask_compress(fake, 1, 4, 64, 64, fake, odd, None, s) == 3
     assert L.nm_compress(fake, fake, 1, 4, 64, 64, 32, fake, fake, None, None, s) == 2  # ldm < C
     assert L.nm_compress(fake, None, 1, 4, 64, 64, 64, fake, fake, None, None, s) == 1
+    # compress of the transpose: R % 8, ldw / ldm < C, dtype, NULL, misaligned, empty
+    assert L.nm_compress_t(fake, fake, 1, 12, 64, 64, 64, fake, fake, None, None, s) == 2
+    assert L.nm_compress_t(fake, fake, 1, 16, 64, 32, 64, fake, fake, None, None, s) == 2
+    assert L.nm_compress_t(fake, fake, 1, 16, 64, 64, 32, fake, fake, None, None, s) == 2
+    assert L.nm_compress_t(fake, fake, 9, 16, 64, 64, 64, fake, fake, None, None, s) == 4
+    assert L.nm_compress_t(fake, None, 1, 16, 64, 64, 64, fake, fake, None, None, s) == 1
+    assert L.nm_compress_t(fake, fake, 1, 16, 64, 64, 64, fake, odd, None, None, s) == 3
+    assert L.nm_compress_t(fake, fake, 1, 16, 64, 68, 64, fake, fake, None, None, s) == 3   # ldw*2 not 16B
+    assert L.nm_compress_t(fake, fake, 1, 16, 64, 64, 64, fake, fake, None, ctypes.c_void_p(0x10002), s) == 3
+    assert L.nm_compress_t(fake, fake, 1, 0, 64, 64, 64, fake, fake, None, None, s) == 0    # R == 0: no-op
+    assert L.nm_compress_t(fake, fake, 1, 16, 0, 0, 0, fake, fake, None, None, s) == 0      # C == 0: no-op
+    # transposable mask: dtype, N:M, R % M, ldm < C, NULL, misaligned, empty
+    assert L.nm_mask_transposable(fake, 9, 8, 8, 8, 4, 8, fake, 8, s) == 4
+    assert L.nm_mask_transposable(fake, 1, 8, 8, 8, 8, 8, fake, 8, s) == 5
+    assert L.nm_mask_transposable(fake, 1, 12, 16, 16, 4, 8, fake, 16, s) == 2
+    assert L.nm_mask_transposable(fake, 1, 16, 16, 16, 4, 8, fake, 8, s) == 2
+    assert L.nm_mask_transposable(None, 1, 16, 16, 16, 4, 8, fake, 16, s) == 1
+    assert L.nm_mask_transposable(fake, 1, 16, 16, 16, 4, 8, odd, 16, s) == 3
+    assert L.nm_mask_transposable(fake, 1, 0, 16, 16, 4, 8, fake, 16, s) == 0
+    # saliency mask: int8 refused (floating-point call), NULL d, N:M
+    assert L.nm_mask_scored(fake, 3, fake, 4, 64, 64, 2, 4, fake, 64, s) == 4
+    assert L.nm_mask_scored(fake, 1, None, 4, 64, 64, 2, 4, fake, 64, s) == 1
+    assert L.nm_mask_scored(fake, 1, fake, 4, 64, 64, 0, 4, fake, 64, s) == 5
+    # 1:2 calls: C % 16, int8 refused
+    assert L.nm_mask_compress12(fake, 0, 4, 40, 40, fake, fake, s) == 2
+    assert L.nm_mask_compress12(fake, 3, 4, 64, 64, fake, fake, s) == 4
+    assert L.nm_decompress12(fake, fake, 0, 4, 40, fake, 40, s) == 2
     assert L.nm_decompress(fake, fake, 1, 4, 64, fake, 60, s) == 2
     assert L.nm_meta_to_sm100(fake, 4, 60, fake, s) == 2
     assert L.nm_meta_to_sm100(None, 4, 64, fake, s) == 1
