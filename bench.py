@@ -529,6 +529,24 @@ def kernel_breakdown(step: Step, steps: int, flush, graphs=None):
     return {name: [ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(steps)] for j, name in enumerate(step.names)}
 
 
+def event_floor_us(reps: int, flush) -> float:
+    """Context for the per-kernel figures: the median CUDA-event time of a
+    one-element torch kernel, timed the way each launch is (L2 flushed before,
+    outside the events).  A tiny launch cannot read below this."""
+    s = torch.cuda.current_stream()
+    t = torch.empty(1, dtype=torch.int32, device=s.device)
+    ts = []
+    for _ in range(reps):
+        flush()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        t.zero_()
+        b.record(s)
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    return 1e3 * float(np.median(ts))
+
+
 def dense_context(step: Step, reps: int, flush):
     """Context only: the same products as dense bf16 GEMMs in cuBLAS (torch.matmul)
     on the decompressed weights, timed like the step (L2 flushed before each rep).
@@ -839,6 +857,7 @@ def main():
     per = kernel_breakdown(step, args.steps, flush, graphs)
     # the same step as one sequential chain, for comparison (not the timed region)
     seq_ms = float(np.mean(timed_steps(step, args.steps, flush, (graphs[2],) if graphs else None)))
+    floor_us = event_floor_us(50, flush)
 
     total_ms = float(np.sum(tot))
     e2e_ms, h2d, d2h = e2e_steps(step, args.steps, nm, wl, dev)
@@ -926,6 +945,7 @@ def main():
                                  "that evicts the written lines",
                            "launch": launch_mode,
                            "step_sequential_ms": seq_ms,
+                           "event_floor_us": floor_us,
                            "parallelism": "independent replica per GPU" if world > 1 else "single GPU"},
                 "roofline": roof, "cpu_baseline": cpu, "dense_context": dense_line,
                 "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

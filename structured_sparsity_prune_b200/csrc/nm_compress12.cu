@@ -137,6 +137,34 @@ __global__ void __launch_bounds__(256) decompress12_kernel(const Bits* __restric
   }
 }
 
+// fp32 decompression in units of 8 elements (4 pairs, half a metadata byte):
+// 16 bytes of values in, 32 bytes out per thread, so a warp stores 1 KB of a
+// row contiguously (the 16-element unit stores 64 bytes per thread).
+__global__ void __launch_bounds__(256) decompress12_f32_kernel(const uint32_t* __restrict__ values,
+                                                               const uint8_t* __restrict__ meta, int64_t R,
+                                                               int64_t C, uint32_t* __restrict__ out, int64_t ldo) {
+  const int64_t upr = C / 8;
+  const int64_t r_step = int64_t(gridDim.y) * blockDim.y;
+  const int64_t u_step = int64_t(gridDim.x) * blockDim.x;
+  for (int64_t r = int64_t(blockIdx.y) * blockDim.y + threadIdx.y; r < R; r += r_step) {
+    for (int64_t u = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; u < upr; u += u_step) {
+      const uint4 v = __ldcs(reinterpret_cast<const uint4*>(values + r * (C / 2) + 4 * u));
+      const uint32_t bits = uint32_t(meta[r * (C / 16) + u / 2]) >> (4 * (u & 1));
+      const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+      uint32_t o[8];
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        const bool second = (bits >> p) & 1u;
+        o[2 * p] = second ? 0u : x[p];
+        o[2 * p + 1] = second ? x[p] : 0u;
+      }
+      uint4* dst = reinterpret_cast<uint4*>(out + r * ldo + 8 * u);
+      __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+      __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+    }
+  }
+}
+
 // x over the units of a row, y over rows; at most per_sm blocks per SM (the
 // kernel's occupancy), so the whole grid is resident at once.
 void shape_units(int64_t R, int64_t units, dim3& grid, dim3& block, int per_sm) {
@@ -210,13 +238,15 @@ extern "C" nm_status nm_decompress12(const void* values, const uint8_t* meta, nm
   const int es = esize_of(dtype);
   if (!aligned16(values) || !aligned16(W_out) || !stride_ok(ldw, es)) return NM_ERR_ALIGN;
   dim3 grid, block;
-  shape_units(R, C / 16, grid, block, 8);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (dtype == NM_F32)
-    decompress12_kernel<uint32_t><<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C / 16,
-                                                         static_cast<uint32_t*>(W_out), ldw);
-  else
-    decompress12_kernel<uint16_t><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(values), meta, R, C / 16,
-                                                         static_cast<uint16_t*>(W_out), ldw);
+  if (dtype == NM_F32) {
+    shape_units(R, C / 8, grid, block, 8);
+    decompress12_f32_kernel<<<grid, block, 0, s>>>(static_cast<const uint32_t*>(values), meta, R, C,
+                                                   static_cast<uint32_t*>(W_out), ldw);
+    return launch_status();
+  }
+  shape_units(R, C / 16, grid, block, 8);
+  decompress12_kernel<uint16_t><<<grid, block, 0, s>>>(static_cast<const uint16_t*>(values), meta, R, C / 16,
+                                                       static_cast<uint16_t*>(W_out), ldw);
   return launch_status();
 }
