@@ -304,8 +304,11 @@ class Step:
             self.v_t, self.m_t, self.img_t = nm.alloc_compressed(K, R, self.W.dtype, dev)
             self.Y = torch.empty((R, T), dtype=torch.bfloat16, device=dev)
             self.DX = torch.empty((K, T), dtype=torch.bfloat16, device=dev)
-            ws = max(nm.nm_spmm_workspace_bytes(self.W.dtype, R, K, T), nm.nm_spmm_workspace_bytes(self.W.dtype, K, R, T))
-            self.ws = torch.empty((ws,), dtype=torch.uint8, device=dev) if ws else None
+            # the two products run concurrently in the captured step: one scratch buffer each
+            ws_f = nm.nm_spmm_workspace_bytes(self.W.dtype, R, K, T)
+            ws_b = nm.nm_spmm_workspace_bytes(self.W.dtype, K, R, T)
+            self.ws = torch.empty((ws_f,), dtype=torch.uint8, device=dev) if ws_f else None
+            self.ws_t = torch.empty((ws_b,), dtype=torch.uint8, device=dev) if ws_b else None
             self.names = ["nm_mask_transposable_2:4", "nm_compress", "nm_compress_t", "nm_spmm_fwd", "nm_spmm_bwd"]
             G = R * K
             es = self.W.element_size()
@@ -382,7 +385,7 @@ class Step:
                     lambda: nm.nm_compress(self.W, self.mask, self.values, self.meta, self.img),
                     lambda: nm.nm_compress_t(self.W, self.mask, self.v_t, self.m_t, self.img_t),
                     lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.Y, workspace=self.ws),
-                    lambda: nm.nm_spmm(self.v_t, self.img_t, self.DY, Y=self.DX, workspace=self.ws)]
+                    lambda: nm.nm_spmm(self.v_t, self.img_t, self.DY, Y=self.DX, workspace=self.ws_t)]
         if self.kind == "mlp":
             return [lambda: nm.nm_mask_compress(self.W, self.values, self.meta, self.img),
                     lambda: nm.nm_mask_compress(self.W2, self.v2, self.m2, self.img2),
