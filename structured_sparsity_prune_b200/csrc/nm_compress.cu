@@ -623,6 +623,46 @@ __device__ __forceinline__ Oct<Bits> make_oct(const Bits (&a)[8]) {
   return e;
 }
 
+// The lane's eight columns of one tile: pick each group down a column under
+// the mask, store its pair into that column's row of Wt (vdst + j * rh), and
+// return the eight nibbles as one word (nibble j = column j; pad (0,1) for
+// columns past C).  kFull: all eight columns are in range, no per-column test.
+template <typename Bits, bool kFull>
+__device__ __forceinline__ uint32_t compress_t_columns(const Oct<Bits> (&e)[4], const uint2 (&mk)[4], int ncols,
+                                                       Bits* __restrict__ vdst, int64_t rh, int& invalid) {
+  uint32_t nibs = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    uint32_t nib = 0x4u;  // pad: pattern (0,1)
+    if (kFull || j < ncols) {
+      // mask byte j of rows 0..3 -> bytes 0..3 of w
+      const uint32_t sel = (j & 3) | (((j & 3) + 4) << 4);  // a constant after unrolling
+      const uint32_t lo = __byte_perm(j < 4 ? mk[0].x : mk[0].y, j < 4 ? mk[1].x : mk[1].y, sel);
+      const uint32_t hi = __byte_perm(j < 4 ? mk[2].x : mk[2].y, j < 4 ? mk[3].x : mk[3].y, sel);
+      const uint32_t w = __byte_perm(lo, hi, 0x5410);
+      const Pick pk = pick_masked(w, invalid);
+      nib = pk.nib;
+      Bits* dst = vdst + j * rh;
+      if constexpr (sizeof(Bits) == 2) {
+        // entry j of rows 0..3: half j & 1 of word j / 2 of each row
+        const uint32_t hsel = (j & 1) ? 0x7632u : 0x5410u;
+        const uint32_t g01 = __byte_perm((&e[0].v.x)[j >> 1], (&e[1].v.x)[j >> 1], hsel);
+        const uint32_t g23 = __byte_perm((&e[2].v.x)[j >> 1], (&e[3].v.x)[j >> 1], hsel);
+        __stcs(reinterpret_cast<uint32_t*>(dst), pair16(g01, g23, pk));
+      } else if constexpr (sizeof(Bits) == 1) {
+        const uint32_t blo = __byte_perm(j < 4 ? e[0].v.x : e[0].v.y, j < 4 ? e[1].v.x : e[1].v.y, sel);
+        const uint32_t bhi = __byte_perm(j < 4 ? e[2].v.x : e[2].v.y, j < 4 ? e[3].v.x : e[3].v.y, sel);
+        __stcs(reinterpret_cast<unsigned short*>(dst),
+               static_cast<unsigned short>(pair8(__byte_perm(blo, bhi, 0x5410), pk)));
+      } else {
+        __stcs(reinterpret_cast<uint2*>(dst), pair32(e[0][j], e[1][j], e[2][j], e[3][j], pk));
+      }
+    }
+    nibs |= nib << (4 * j);
+  }
+  return nibs;
+}
+
 template <typename Bits>
 __global__ void __launch_bounds__(256, 3) compress_t_kernel(const Bits* __restrict__ W, int64_t ldw,
                                                          const uint8_t* __restrict__ mask, int64_t ldm, int64_t R,
@@ -631,74 +671,64 @@ __global__ void __launch_bounds__(256, 3) compress_t_kernel(const Bits* __restri
                                                          int32_t* __restrict__ invalid_groups) {
   const int lane = threadIdx.x & 31, q = lane & 3, h = lane >> 2;
   const int64_t Rp = (R + 127) / 128 * 128, Cp = (C + 127) / 128 * 128;  // padded image extents
-  const int64_t ct_count = Cp / 32, tiles = (Rp / 32) * ct_count;
+  const int64_t ct_count = Cp / 32, rt_count = Rp / 32;
   const int64_t nwarps = (int64_t(gridDim.x) * blockDim.x) >> 5;
   const bool meta_words = R % 32 == 0;
+  const int64_t rh = R / 2;
   int invalid = 0;
-  for (int64_t t = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5; t < tiles; t += nwarps) {
-    const int64_t rt = t / ct_count;
+  // Tile t = rt * ct_count + ct, t stepping by nwarps: (rt, ct) advance by the
+  // quotient and remainder of nwarps, with a carry, instead of a division per tile.
+  const int64_t t0 = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  int64_t rt = t0 / ct_count, ct = t0 - rt * ct_count;
+  const int64_t d_rt = nwarps / ct_count, d_ct = nwarps - d_rt * ct_count;
+  for (; rt < rt_count; rt += d_rt, ct += d_ct) {
+    if (ct >= ct_count) {
+      ct -= ct_count;
+      ++rt;
+      if (rt >= rt_count) break;
+    }
     const int64_t r0 = rt * 32, r = r0 + 4 * h;   // the lane's four rows: one group down each column
-    const int64_t c = (t - rt * ct_count) * 32 + 8 * q;
+    const int64_t c = ct * 32 + 8 * q;
     Oct<Bits> e[4];
     uint2 mk[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) mk[k] = make_uint2(0u, 0u);
-    if (r < R && c < C) {  // R % 4 == 0: the four rows are in or out together
-      if (c + 8 <= C) {
+    const bool rows_in = r < R;  // R % 4 == 0: the four rows are in or out together
+    const bool full = rows_in && c + 8 <= C;
+    if (full) {
+      const Bits* wrow = W + r * ldw + c;
+      const uint8_t* mrow = mask + r * ldm + c;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          e[k].load(W + (r + k) * ldw + c);
-          mk[k] = __ldcs(reinterpret_cast<const uint2*>(mask + (r + k) * ldm + c));
+      for (int k = 0; k < 4; ++k) {
+        e[k].load(wrow + k * ldw);
+        mk[k] = __ldcs(reinterpret_cast<const uint2*>(mrow + k * ldm));
+      }
+    } else if (rows_in && c < C) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        Bits a[8];
+        uint8_t b[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          a[j] = c + j < C ? W[(r + k) * ldw + c + j] : Bits(0);
+          b[j] = c + j < C ? mask[(r + k) * ldm + c + j] : uint8_t(0);
         }
-      } else {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          Bits a[8];
-          uint8_t b[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            a[j] = c + j < C ? W[(r + k) * ldw + c + j] : Bits(0);
-            b[j] = c + j < C ? mask[(r + k) * ldm + c + j] : uint8_t(0);
-          }
-          e[k] = make_oct<Bits>(a);
-          mk[k] = make_uint2(uint32_t(b[0]) | (uint32_t(b[1]) << 8) | (uint32_t(b[2]) << 16) | (uint32_t(b[3]) << 24),
-                             uint32_t(b[4]) | (uint32_t(b[5]) << 8) | (uint32_t(b[6]) << 16) | (uint32_t(b[7]) << 24));
-        }
+        e[k] = make_oct<Bits>(a);
+        mk[k] = make_uint2(uint32_t(b[0]) | (uint32_t(b[1]) << 8) | (uint32_t(b[2]) << 16) | (uint32_t(b[3]) << 24),
+                           uint32_t(b[4]) | (uint32_t(b[5]) << 8) | (uint32_t(b[6]) << 16) | (uint32_t(b[7]) << 24));
       }
     }
     // This lane's eight nibbles (group h of columns c..c+7, nibble j = column j)
     // form one word; an 8 x 8 nibble transpose across the eight lanes of the
     // column chunk (h = lane bits 2..4) gives lane h the metadata word of row
     // c + h of Wt (nibble g = group g).  Three masked butterfly stages.
-    uint32_t nibs = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      uint32_t nib = 0x4u;  // pad: pattern (0,1)
-      if (r < R && c + j < C) {
-        // mask byte j of rows 0..3 -> bytes 0..3 of w
-        const uint32_t sel = (j & 3) | (((j & 3) + 4) << 4);  // a constant after unrolling
-        const uint32_t lo = __byte_perm(j < 4 ? mk[0].x : mk[0].y, j < 4 ? mk[1].x : mk[1].y, sel);
-        const uint32_t hi = __byte_perm(j < 4 ? mk[2].x : mk[2].y, j < 4 ? mk[3].x : mk[3].y, sel);
-        const uint32_t w = __byte_perm(lo, hi, 0x5410);
-        const Pick pk = pick_masked(w, invalid);
-        nib = pk.nib;
-        Bits* dst = values + (c + j) * (R / 2) + r / 2;
-        if constexpr (sizeof(Bits) == 2) {
-          // entry j of rows 0..3: half j & 1 of word j / 2 of each row
-          const uint32_t hsel = (j & 1) ? 0x7632u : 0x5410u;
-          const uint32_t g01 = __byte_perm((&e[0].v.x)[j >> 1], (&e[1].v.x)[j >> 1], hsel);
-          const uint32_t g23 = __byte_perm((&e[2].v.x)[j >> 1], (&e[3].v.x)[j >> 1], hsel);
-          __stcs(reinterpret_cast<uint32_t*>(dst), pair16(g01, g23, pk));
-        } else if constexpr (sizeof(Bits) == 1) {
-          const uint32_t blo = __byte_perm(j < 4 ? e[0].v.x : e[0].v.y, j < 4 ? e[1].v.x : e[1].v.y, sel);
-          const uint32_t bhi = __byte_perm(j < 4 ? e[2].v.x : e[2].v.y, j < 4 ? e[3].v.x : e[3].v.y, sel);
-          __stcs(reinterpret_cast<unsigned short*>(dst),
-                 static_cast<unsigned short>(pair8(__byte_perm(blo, bhi, 0x5410), pk)));
-        } else {
-          __stcs(reinterpret_cast<uint2*>(dst), pair32(e[0][j], e[1][j], e[2][j], e[3][j], pk));
-        }
-      }
-      nibs |= nib << (4 * j);
+    Bits* vdst = values + c * rh + r / 2;  // dereferenced only for columns in range
+    uint32_t nibs;
+    if (full) {
+      nibs = compress_t_columns<Bits, true>(e, mk, 8, vdst, rh, invalid);
+    } else {
+      const int ncols = rows_in && c < C ? int(C - c < 8 ? C - c : 8) : 0;
+      nibs = compress_t_columns<Bits, false>(e, mk, ncols, vdst, rh, invalid);
     }
     {
       constexpr uint32_t kLo[3] = {0x0F0F0F0Fu, 0x00FF00FFu, 0x0000FFFFu};
