@@ -435,8 +435,18 @@ __global__ void __launch_bounds__(256) meta_image_rows_kernel(const uint8_t* __r
   const int64_t items = ((R + 127) / 128) * 8 * quads;
   const int q = threadIdx.x & 7, j = (threadIdx.x >> 3) & 3;
   const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
-  for (int64_t it = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); it < items; it += warps) {
-    const int64_t g = it / quads, kt = (it - g * quads) * 4 + j;
+  // Item it = g * quads + qd, it stepping by `warps`: (g, qd) advance by the
+  // quotient and remainder of `warps`, with a carry, instead of a division per item.
+  const int64_t it0 = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t groups = items / quads, d_g = warps / quads, d_qd = warps - d_g * quads;
+  int64_t g = it0 / quads, qd = it0 - g * quads;
+  for (; g < groups; g += d_g, qd += d_qd) {
+    if (qd >= quads) {
+      qd -= quads;
+      ++g;
+      if (g >= groups) break;
+    }
+    const int64_t kt = qd * 4 + j;
     if (kt >= kt_count) continue;
     const int64_t r = 16 * g + q;
     const uint4 pad = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
