@@ -44,6 +44,7 @@ SEEDS = {
     "saliency.X": 7,
     "fp32_linear.W": 8,
     "linear_4096.dY": 103,
+    "mlp_pair.H": 104,
 }
 
 
@@ -92,6 +93,12 @@ def mlp_pair():
     return (normal((14336, 4096), SEEDS["mlp_pair.W_up"], 0.02, torch.bfloat16),
             normal((4096, 14336), SEEDS["mlp_pair.W_down"], 0.02, torch.bfloat16),
             normal((4096, 8192), SEEDS["mlp_pair.X"], 1.0, torch.bfloat16))
+
+
+def mlp_hidden():
+    """A 14336 x 8192 bf16 ~N(0,1) stand-in for the MLP pair's hidden activation
+    (the down projection's input), drawn from its own seed."""
+    return normal((14336, 8192), SEEDS["mlp_pair.H"], 1.0, torch.bfloat16)
 
 
 def ties_fp32(R: int = 8192, C: int = 8192):

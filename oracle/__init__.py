@@ -291,8 +291,9 @@ def spmm(values: np.ndarray, meta: np.ndarray, X: np.ndarray, ab_dtype: int,
 
 
 def rows_parallel(what: int, W: np.ndarray, N: int, M: int, dtype: int, threads: int):
-    """Multi-threaded mask (what=0) or 2:4 mask+compress (what=1) over rows;
-    used only to time the oracle as a CPU baseline."""
+    """Multi-threaded mask (what=0) or 2:4 mask+compress (what=1) over rows:
+    the single-row oracle run on row ranges in parallel, for the CPU baseline
+    and for the whole-matrix parity tests.  Mode 1 also fills the mask."""
     Wb = _bits(W, dtype)
     R, C = Wb.shape
     mask = np.zeros((R, C), dtype=np.uint8)

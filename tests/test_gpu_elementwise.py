@@ -244,6 +244,28 @@ def test_mask_compress_large_weights(R, C, dtype):
     assert np.array_equal(img.cpu().numpy(), oracle.meta_sm100(m_ref, R, C))
 
 
+@pytest.mark.parametrize("which", ["mlp_up", "mlp_down", "decode"])
+def test_mask_compress_decompress_full_size(which):
+    """The MLP pair's weights (14336 x 4096, 4096 x 14336) and the 28672 x 8192
+    decode weight, whole matrices, bf16: the fused mask + compress matches the
+    oracle byte for byte (values, metadata, image), and decompression returns
+    W (.) mask with +0.0 at the pruned positions."""
+    if which == "decode":
+        W = nm_inputs.decode_skinny_W()
+    else:
+        W_up, W_down, _ = nm_inputs.mlp_pair()
+        W = W_up if which == "mlp_up" else W_down
+    R, C = W.shape
+    values, meta, img = nm.nm_mask_compress(W.cuda())
+    dense = nm.nm_decompress(values, meta, C)
+    Wb = _bits(W)
+    mask_ref, v_ref, m_ref = oracle.rows_parallel(1, Wb, 2, 4, oracle.BF16, threads=os.cpu_count() or 2)
+    assert np.array_equal(_bits(values), v_ref)
+    assert np.array_equal(meta.cpu().numpy(), m_ref)
+    assert np.array_equal(img.cpu().numpy(), oracle.meta_sm100(m_ref, R, C))
+    assert np.array_equal(_bits(dense), np.where(mask_ref == 1, Wb, np.uint16(0)))
+
+
 def test_linear_4096_mask_compress_full_size():
     """The 4096 x 4096 bf16 transformer-linear weight, whole matrix, bit-exact."""
     W, _ = nm_inputs.linear_4096()

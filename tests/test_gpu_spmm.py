@@ -202,6 +202,18 @@ def test_linear_4096_full_size_sampled_rows():
     assert _nerr(Y, ref) <= 8e-3
 
 
+def test_mlp_pair_full_size_sampled_rows():
+    """The MLP pair at full size: up 14336 x 4096 x 8192, then down 4096 x
+    14336 x 8192, bf16 out, rows sampled across every row tile.  The down
+    product takes a seeded stand-in for H of the same shape and distribution,
+    so no oracle input comes from the device."""
+    W_up, W_down, X = nm_inputs.mlp_pair()
+    H, ref = _run(W_up, X, torch.bfloat16, rows=_sample_rows(W_up.shape[0], 2))
+    assert _nerr(H, ref) <= 8e-3
+    Y, ref = _run(W_down, nm_inputs.mlp_hidden(), torch.bfloat16, rows=_sample_rows(W_down.shape[0], 2))
+    assert _nerr(Y, ref) <= 8e-3
+
+
 @pytest.mark.parametrize("T", [16, 64, 256, 1024])
 def test_decode_skinny_full_size_sampled_rows(T):
     W = nm_inputs.decode_skinny_W()
