@@ -96,7 +96,8 @@ def profiled_traffic(workload: str, kernel: str):
                 k, v = line.split(":", 1)
                 fields[k.strip()] = v.strip()
     try:
-        src = open(os.path.join(ROOT, fields["source_file"]), "rb").read()
+        with open(os.path.join(ROOT, fields["source_file"]), "rb") as fh:
+            src = fh.read()
         if hashlib.sha256(src).hexdigest() != fields["source_sha256"]:
             return None
         return int(fields["traffic_bytes_per_launch"])
@@ -177,6 +178,8 @@ class ClockSampler:
                                          stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            if getattr(self, "fh", None) is not None:
+                self.fh.close()
         self.t0 = time.time()
 
     def mark(self, what: str):

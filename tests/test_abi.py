@@ -15,7 +15,8 @@ HEADER = os.path.join(ROOT, "include", "nm.h")
 
 
 def _declared():
-    text = open(HEADER).read()
+    with open(HEADER) as f:
+        text = f.read()
     return sorted(set(re.findall(r"NM_API\s+[\w\s\*]*?\b(nm_\w+)\s*\(", text)))
 
 
@@ -140,6 +141,7 @@ def test_workspace_size(lib):
 
 def test_no_cpu_fallback_in_the_binding():
     """The product binding must not reach the oracle or any CPU path."""
-    src = open(os.path.join(ROOT, "structured_sparsity_prune_b200", "__init__.py")).read()
+    with open(os.path.join(ROOT, "structured_sparsity_prune_b200", "__init__.py")) as f:
+        src = f.read()
     assert "oracle" not in src.replace("no CPU\nfallback", "")
     assert "import numpy" not in src

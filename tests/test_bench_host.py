@@ -31,7 +31,8 @@ def _fields(path):
 def test_traffic_is_read_from_the_summary_while_the_source_matches():
     rel = bench.TRAFFIC_PROFILES[("linear_4096", "nm_spmm")]
     f = _fields(os.path.join(ROOT, rel))
-    src = open(os.path.join(ROOT, f["source_file"]), "rb").read()
+    with open(os.path.join(ROOT, f["source_file"]), "rb") as fh:
+        src = fh.read()
     got = bench.profiled_traffic("linear_4096", "nm_spmm")
     if hashlib.sha256(src).hexdigest() == f["source_sha256"]:
         assert got == int(f["traffic_bytes_per_launch"])

@@ -22,7 +22,9 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "scored_cases.txt")
 
 def _cases():
     out = []
-    for line in open(GOLDEN):
+    with open(GOLDEN) as f:
+        lines = f.read().splitlines()
+    for line in lines:
         line = line.strip()
         if not line or line.startswith("#"):
             continue

@@ -26,7 +26,9 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "transposable_cases.t
 
 def _cases():
     out = []
-    for line in open(GOLDEN):
+    with open(GOLDEN) as f:
+        lines = f.read().splitlines()
+    for line in lines:
         line = line.strip()
         if not line or line.startswith("#"):
             continue
