@@ -14,6 +14,11 @@ linear/conv weights; the pages' datasets and trained weights are not used):
                       X bf16 4096x4096 ~N(0,1) (seed 101)
 * ``mlp_pair``        W_up bf16 14336x4096 (seed 2), W_down bf16 4096x14336
                       (seed 3), both bf16(0.02 * N(0,1)); X bf16 4096x8192 (seed 102)
+* ``mlp_hidden``      a bf16 14336x8192 ~N(0,1) stand-in for the MLP pair's
+                      hidden activation (seed 104), the down product's input in
+                      its full-size parity test
+* ``linear_4096_grad`` dY bf16 4096x4096 ~N(0,1) (seed 103), the backward
+                      product's input in the transposable 2:4 step
 * ``ties_fp32``       W fp32 8192x8192 = fp32(k/100), k ~ U{-8..7} (seed 4)
 * ``decode_skinny``   W bf16 28672x8192 = bf16(0.02 * N(0,1)) (seed 5),
                       X bf16 8192xT ~N(0,1) (seed 105+T), T in {16,64,256,1024}
