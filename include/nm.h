@@ -220,6 +220,12 @@ NM_API nm_status nm_compress(const void *W, const uint8_t *mask, nm_dtype dtype,
  *   among four 0/1 bytes; fewer are filled with +0.0 values at the lowest
  *   unkept positions; invalid groups are counted and stored as (0,1)).
  *   dtype: NM_F32, NM_BF16, NM_F16 or NM_S8.  One pass over W and the mask.
+ *   Errors: NM_ERR_DTYPE for another dtype; NM_ERR_SHAPE if R % 8 != 0 or
+ *   ldw, ldm < C; NM_ERR_NULL for a NULL W, mask, values_t or meta_t;
+ *   NM_ERR_ALIGN unless W, mask, values_t, meta_t (and meta_t_sm100 when
+ *   given) are 16-byte aligned, ldw * element size and ldm are multiples of
+ *   16 bytes, and invalid_groups is 4-byte aligned.  R == 0 or C == 0 does
+ *   nothing and returns NM_OK.
  */
 NM_API nm_status nm_compress_t(const void *W, const uint8_t *mask, nm_dtype dtype, int64_t R, int64_t C,
                                int64_t ldw, int64_t ldm, void *values_t, uint8_t *meta_t,
