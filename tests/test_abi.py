@@ -130,6 +130,13 @@ def test_host_validation_before_any_launch(lib):
     assert L.nm_spmm(fake, fake, 1, fake, 12, fake, 1, 16, 128, 64, 12, f(1), f(0), None, 0, s) == 3
     assert L.nm_spmm(fake, fake, 0, fake, 8, fake, 0, 8, 128, 64, 8, f(1), f(0), None, 0, s) == 8
     assert L.nm_spmm(fake, fake, 1, fake, 8, fake, 1, 8, 0, 64, 8, f(1), f(0), None, 0, s) == 0
+    # maximum sizes: tile coordinates are 32-bit, so R, K and T must stay below 2^31 - 256
+    big = 2 ** 31 - 256
+    assert L.nm_spmm(fake, fake, 1, fake, 8, fake, 1, 8, big, 64, 8, f(1), f(0), None, 0, s) == 2
+    assert L.nm_spmm(fake, fake, 1, fake, 8, fake, 1, 8, 128, big // 16 * 16 + 16, 8, f(1), f(0), None, 0, s) == 2
+    assert L.nm_spmm(fake, fake, 1, fake, big, fake, 1, big, 128, 64, big, f(1), f(0), None, 0, s) == 2
+    # K == 0 with rows and columns to write has no product to form
+    assert L.nm_spmm(fake, fake, 1, fake, 8, fake, 1, 8, 128, 0, 8, f(1), f(0), None, 0, s) == 2
 
 
 def test_workspace_size(lib):
