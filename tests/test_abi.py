@@ -56,7 +56,6 @@ def test_sizes_match_the_pages_counts(lib):
     v, m, s = nm.nm_sizes(200, 72, 2, 4, torch.float32)
     assert v == 200 * 36 * 4 and m == 200 * 9 and s == 256 * 128 // 8
     # 36 of 64 bits per four 16-bit weights
-    assert (v := nm.nm_sizes(8, 64, 2, 4, torch.float16)[0]) * 8 + m * 0 >= 0
     v16, m16, _ = nm.nm_sizes(8, 64, 2, 4, torch.float16)
     assert (v16 + m16) * 8 * 64 == 8 * 64 * 16 * 36
     # other N:M: values only
