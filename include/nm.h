@@ -250,12 +250,15 @@ NM_API nm_status nm_meta_to_sm100(const uint8_t *meta, int64_t R, int64_t C, uin
  * nm_srste_step -- one SR-STE training step, fused ("SR-STE sparse training",
  * SR-STE forward and backward): the N:M magnitude mask of W is recomputed
  * (same rule as nm_mask), and
- *   W_sparse = W where kept, +0 elsewhere                      (forward)
- *   grad_out = grad where kept, grad + decay * W elsewhere     (backward,
- *              i.e. grad + decay * (1 - mask) * W)
- * The decay term is one binary32 fused multiply-add, rounded once (nearest
- * even) to dtype; kept entries return grad bit for bit.  The page's default
- * decay is 0.0002.
+ *   W_sparse = W * mask                                   (forward)
+ *   grad_out = grad + decay * (1 - mask) * W              (backward)
+ * evaluated as PyTorch evaluates the page's listing, whose mask is float32:
+ * each product and the sum is a binary32 operation rounded on its own (no
+ * fused multiply-add), and the results are returned in dtype (one more
+ * rounding to nearest even for 16-bit types).  So kept entries return
+ * grad + (+-0) -- grad itself, except that grad = -0 with W >= +0 gives +0 --
+ * and pruned negative weights give -0 in W_sparse.  Inf and NaN inputs are
+ * outside the contract.  The page's default decay is 0.0002.
  *   W, grad, W_sparse, grad_out: R x C, dtype, common leading dim ld >= C
  *   mask: R x C uint8 with row stride ld, or NULL
  *   1 <= N < M <= 8, C % M == 0

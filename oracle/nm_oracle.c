@@ -46,9 +46,9 @@
  *  - decompress writes +0.0 at pruned positions.
  *
  * Floating point: oracle_spmm works in double from exactly-decoded
- * inputs; oracle_srste's decay term and oracle_mask_scored's scores are
- * binary32, as their sources compute them.  Magnitude masks use exact
- * integers.
+ * inputs; oracle_srste's step (one binary32 rounding per operation) and
+ * oracle_mask_scored's scores are binary32, as their sources compute
+ * them.  Magnitude masks use exact integers.
  */
 #include <stdint.h>
 #include <stddef.h>
@@ -698,19 +698,30 @@ int oracle_rows_parallel(int what, const void *W, int dtype, int64_t R, int64_t 
 
 /* --------------------------------------------------------------------- */
 /* SR-STE step.  [SRSTE] "SR-STE sparse training", SR-STE forward and     */
-/* backward: the forward keeps the N:M mask of |w| (recomputed every     */
-/* step) and returns the masked weight; the backward returns              */
-/*     grad + decay * (1 - mask) * w                                       */
-/* so pruned entries receive an extra decay * w (the page's default       */
-/* decay is 0.0002).  Readings: the masked weight is select(mask, w, +0); */
-/* the decay term is one fused multiply-add in binary32 (fmaf, correctly  */
-/* rounded), rounded once to the element type; kept entries return grad  */
-/* bit for bit.  mask may be NULL.                                         */
+/* backward.  The forward recomputes the N:M mask of |w| every step and   */
+/* returns output * w_b; the backward returns                              */
+/*     grad_output + decay * (1 - mask) * weight                           */
+/* (the page's default decay is 0.0002).  Both are evaluated here the way */
+/* PyTorch evaluates that listing: w_b is made by torch.ones with no      */
+/* dtype, so it is float32, and type promotion carries every product and  */
+/* the sum in binary32:                                                    */
+/*   forward   ws = fl32(w * m)             (exact: w, or a signed zero)   */
+/*   backward  c  = decay * (1 - m)          (decay or 0, exact)           */
+/*             t  = fl32(c * w)              rounding 1                    */
+/*             y  = fl32(g + t)              rounding 2                    */
+/* two separate roundings, never one fused multiply-add; the results are  */
+/* returned in the weight's dtype (autograd hands a parameter its         */
+/* gradient in the parameter's dtype), one more rounding to nearest even  */
+/* for 16-bit weights.  Kept entries therefore get g + (+-0): g itself,   */
+/* except that g = -0 with w >= +0 gives +0.  Pruned negative weights     */
+/* give -0 in the forward.  Inf / NaN inputs are outside the contract     */
+/* (their NaN results carry no defined payload).  mask may be NULL.       */
 /* --------------------------------------------------------------------- */
 int oracle_srste(const void *W, const void *grad, int dtype, int64_t R, int64_t C, int N, int M, float decay,
                  void *W_sparse, void *grad_out, uint8_t *mask_out)
 {
     if (M < 2 || M > 8 || N < 1 || N >= M || C % M != 0 || R < 0) return OR_BAD_ARG;
+    if (dtype == OR_S8) return OR_BAD_ARG;
     uint8_t *m = (uint8_t *)malloc((size_t)(C > 0 ? C : 1));
     for (int64_t r = 0; r < R; ++r) {
         int st = oracle_mask_rank((const char *)W + (size_t)(r * C) * elem_size(dtype), dtype, 1, C, C, N, M, m, C);
@@ -719,15 +730,15 @@ int oracle_srste(const void *W, const void *grad, int dtype, int64_t R, int64_t 
             size_t i = (size_t)(r * C + c);
             uint32_t wb = load_bits(W, dtype, i), gb = load_bits(grad, dtype, i);
             if (mask_out) mask_out[i] = m[c];
-            if (m[c]) {
-                store_bits(W_sparse, dtype, i, wb);
-                store_bits(grad_out, dtype, i, gb);
-            } else {
-                store_bits(W_sparse, dtype, i, 0u);
-                float w = (float)oracle_decode(wb, dtype), g = (float)oracle_decode(gb, dtype);
-                float y = fmaf(decay, w, g);                 /* binary32, one rounding */
-                store_bits(grad_out, dtype, i, oracle_encode((double)y, dtype));
-            }
+            float w = (float)oracle_decode(wb, dtype);   /* exact: every element type fits binary32 */
+            float g = (float)oracle_decode(gb, dtype);
+            float keep = m[c] ? 1.0f : 0.0f;              /* the listing's float32 mask */
+            float ws = w * keep;                          /* forward product */
+            float coef = decay * (1.0f - keep);           /* decay * (1 - mask) */
+            float t = coef * w;                           /* binary32, rounded once */
+            float y = g + t;                              /* binary32, rounded once */
+            store_bits(W_sparse, dtype, i, oracle_encode((double)ws, dtype));
+            store_bits(grad_out, dtype, i, oracle_encode((double)y, dtype));
         }
     }
     free(m);

@@ -7,9 +7,12 @@
 //
 // One kernel reads W and grad once and writes the masked weight, the new
 // gradient and (optionally) the mask: 2 * s bytes in and 2 * s (+1) bytes out
-// per weight.  Selection is the magnitude rule of nm_mask; the decay term is
-// one fused multiply-add in binary32 (__fmaf_rn), rounded once to the element
-// type; kept entries return grad unchanged.
+// per weight.  Selection is the magnitude rule of nm_mask.  The arithmetic is
+// the listing's as PyTorch evaluates it: its mask is float32 (torch.ones with
+// no dtype), so the forward w * m, the decay term decay * (1 - m) * w and the
+// sum with the gradient are binary32 operations, each rounded on its own
+// (never contracted into a fused multiply-add), and the results go back to the
+// element type, one more rounding to nearest even for 16-bit elements.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -39,14 +42,27 @@ __device__ __forceinline__ uint16_t f16_from_f(float x) {
   return *reinterpret_cast<const uint16_t*>(&h);
 }
 
-// new gradient of one pruned entry: round(fmaf(decay, w, g))
 template <typename Bits, bool F16>
-__device__ __forceinline__ Bits decayed(Bits w, Bits g, float decay) {
-  if constexpr (F16) {
-    return f16_from_f(__fmaf_rn(decay, f16_to_f(w), f16_to_f(g)));
-  } else {
-    return Elem<Bits>::from_f(__fmaf_rn(decay, Elem<Bits>::to_f(w), Elem<Bits>::to_f(g)));
-  }
+__device__ __forceinline__ float elem_to_f(Bits b) {
+  if constexpr (F16) return f16_to_f(b);
+  else return Elem<Bits>::to_f(b);
+}
+template <typename Bits, bool F16>
+__device__ __forceinline__ Bits elem_from_f(float x) {
+  if constexpr (F16) return f16_from_f(x);
+  else return Elem<Bits>::from_f(x);
+}
+
+// One entry of the step, in place: w <- w * m and g <- g + decay * (1 - m) * w
+// with m = 1.0 (kept) or 0.0, every product and the sum rounded to binary32 on
+// its own (__fmul_rn / __fadd_rn are never contracted), then to the element type.
+template <typename Bits, bool F16>
+__device__ __forceinline__ void srste_entry(Bits& w, Bits& g, bool keep, float decay) {
+  const float m = keep ? 1.0f : 0.0f;
+  const float wf = elem_to_f<Bits, F16>(w);
+  const float t = __fmul_rn(__fmul_rn(decay, __fsub_rn(1.0f, m)), wf);
+  g = elem_from_f<Bits, F16>(__fadd_rn(elem_to_f<Bits, F16>(g), t));
+  w = elem_from_f<Bits, F16>(__fmul_rn(wf, m));
 }
 
 // keep bits of 16 consecutive entries (groups of M, M | 16)
@@ -105,12 +121,7 @@ __global__ void __launch_bounds__(256) srste_vec16_kernel(const Bits* __restrict
         Bits* g = reinterpret_cast<Bits*>(gv[k]);
         const uint32_t kb = keep16<Bits, M, NT>(w, N);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const bool keep = (kb >> i) & 1u;
-          const Bits gd = decayed<Bits, F16>(w[i], g[i], decay);
-          g[i] = keep ? g[i] : gd;
-          w[i] = keep ? w[i] : Bits(0);
-        }
+        for (int i = 0; i < 16; ++i) srste_entry<Bits, F16>(w[i], g[i], (kb >> i) & 1u, decay);
 #pragma unroll
         for (int i = 0; i < kVec; ++i) {
           __stcs(reinterpret_cast<uint4*>(WS + r * ld) + c * kVec + i, wv[k][i]);
@@ -149,8 +160,10 @@ __global__ void __launch_bounds__(256) srste_scalar_kernel(const Bits* __restric
 #pragma unroll
       for (int i = 0; i < M; ++i) {
         const bool keep = (kb >> i) & 1u;
-        WS[r * ld + gi * M + i] = keep ? w[i] : Bits(0);
-        GO[r * ld + gi * M + i] = keep ? g[i] : decayed<Bits, F16>(w[i], g[i], decay);
+        Bits wo = w[i], go = g[i];
+        srste_entry<Bits, F16>(wo, go, keep, decay);
+        WS[r * ld + gi * M + i] = wo;
+        GO[r * ld + gi * M + i] = go;
         if (mask != nullptr) mask[r * ld + gi * M + i] = uint8_t(keep ? 1 : 0);
       }
     }
