@@ -288,7 +288,10 @@ NM_API size_t nm_spmm_workspace_bytes(nm_dtype ab_dtype, int64_t R, int64_t K, i
  *              16-byte aligned Y and ldy get vector stores
  *   X, values, meta_sm100: 16-byte aligned; ldx * element size % 16 == 0
  *   ab_dtype   NM_BF16 or NM_F16 (tensor-core path), or NM_F32 (rounded to
- *              binary16 in `workspace`, then the binary16 path)
+ *              binary16 in `workspace`, then the binary16 path; binary16
+ *              holds magnitudes up to 65504 and normal values down to
+ *              6.1e-5, so larger fp32 inputs become +-Inf and values below
+ *              about 6e-8 become zero -- scale such data first)
  *   K % 16 == 0 (the pages' rule for 16-bit sparse operands); R, T >= 1 any
  *   workspace  >= nm_spmm_workspace_bytes(...) bytes (may be NULL when 0)
  * A bounded wait inside the kernel that gives up records NM_ERR_TIMEOUT in a
@@ -313,7 +316,11 @@ NM_API nm_status nm_spmm(const void *values, const uint8_t *meta_sm100, nm_dtype
  *   return NM_ERR_WORKSPACE.  NM_BF16 / NM_F16 inputs need no scratch.
  *   The first NM_F32 call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is kept for the life of the
+ *   process: after cudaDeviceReset on a device, do not call this entry
+ *   point on that device again.
+ *   Arguments are checked as nm_spmm checks them before the size limit, so a
+ *   malformed call returns its own error rather than NM_ERR_WORKSPACE.
  *   All calls on a device share its one array, and it keeps the previous
  *   call's contents (every call overwrites what it reads, so nothing needs
  *   clearing).  Calls that may overlap on the same GPU -- issued to

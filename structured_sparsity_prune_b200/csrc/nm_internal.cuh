@@ -4,6 +4,11 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+#include <utility>
+#include <vector>
+
 #include "../../include/nm.h"
 
 namespace nm {
@@ -22,15 +27,38 @@ inline nm_status launch_status() {
   return e == cudaSuccess ? NM_OK : NM_ERR_CUDA;
 }
 
+// SMs of the current device, cached per device ordinal.
 inline int sm_count() {
-  static int n = 0;
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  const bool cached = dev >= 0 && dev < 64;
+  int n = cached ? cache[dev].load(std::memory_order_relaxed) : 0;
   if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+      (void)cudaGetLastError();
+      n = 148;
+    }
+    if (cached) cache[dev].store(n, std::memory_order_relaxed);
   }
   return n;
+}
+
+// Raises a kernel's dynamic shared-memory limit on the current device.  The
+// attribute is per device, so it is set once per (kernel, device), under a
+// lock shared by every host thread.
+inline nm_status ensure_dynamic_smem(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<const void*, int>> done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return NM_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto& d : done)
+    if (d.first == kernel && d.second == dev) return NM_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return NM_ERR_CUDA;
+  done.emplace_back(kernel, dev);
+  return NM_OK;
 }
 
 // Blocks of `threads` threads of kernel k that one SM holds at once (>= 1).

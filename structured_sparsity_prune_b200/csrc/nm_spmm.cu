@@ -33,6 +33,7 @@
 #include <cstring>
 #include <string>
 
+#include "../../include/nm_testing.h"
 #include "nm_internal.cuh"
 
 namespace nm {
@@ -87,13 +88,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait: true when the phase completed, false on timeout or abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicExch(&g_device_status, int(NM_ERR_TIMEOUT));
       return false;
@@ -345,6 +347,8 @@ struct Params {
   // partly filled wave then takes half as long).
   int split_from, num_work;
   float alpha, beta;
+  uint64_t wait_ns;  // limit of every bounded wait (kWaitLimitNs unless a test shortens it)
+  int64_t skip_it;   // test hook: the producer issues nothing for this pipeline step (-1: none)
 };
 
 // Tile order.  Tiles run in groups: with m_inner, `group` consecutive m-tiles
@@ -491,20 +495,25 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 1
 
   auto tile_coords = [&](int t, int& mt, int& nt) { grouped_tile(p, t, mt, nt); };
 
+  // last round each stage's full barrier was armed in (producer lane only),
+  // for the drain after an abort
+  uint32_t armed_round[STAGES];
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s) armed_round[s] = 0xFFFFFFFFu;
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t it = 0;
-      uint32_t armed_round[STAGES];
-      for (int s = 0; s < STAGES; ++s) armed_round[s] = 0xFFFFFFFFu;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         int mt, nt;
         tile_coords(t, mt, nt);
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          if (int64_t(it) == p.skip_it) continue;  // test hook: this step's stage is never filled
           const int s = int(it % STAGES);
           const uint32_t round = it / STAGES;
-          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
           uint8_t* st = smem + s * C::kStageBytes;
           mbar_arrive_expect_tx(&full[s], C::kStageBytes);
           armed_round[s] = round;
@@ -516,15 +525,6 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 1
           bulk_load(st + C::kABytes + C::kBBytes, esrc, 2048, &full[s]);
         }
       }
-      if (!ok) {
-        // drain: every stage armed but maybe unconsumed completes its copies
-        for (int s = 0; s < STAGES; ++s)
-          if (armed_round[s] != 0xFFFFFFFFu) {
-            const uint64_t t0 = globaltimer();
-            while (!mbar_try_wait(&full[s], armed_round[s] & 1u) && globaltimer() - t0 < 100000000ull) {
-            }
-          }
-      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -535,13 +535,13 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 1
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
         const int buf = int(local % C::kAccBufs);
         const uint32_t use = local / C::kAccBufs;
-        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
         fence_after_sync();
         const uint32_t d_tmem = tmem_base + uint32_t(buf * N_TILE);
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = int(it % STAGES);
           const uint32_t round = it / STAGES;
-          if (!mbar_wait(&full[s], round & 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&full[s], round & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
           fence_after_sync();
           uint8_t* st = smem + s * C::kStageBytes;
           const uint32_t a_addr = smem_u32(st);
@@ -586,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 1
       tile_coords(t, mt, nt);
       const int buf = int(local % C::kAccBufs);
       const uint32_t use = local / C::kAccBufs;
-      const bool ok = mbar_wait(&acc_full[buf], use & 1u, abort_flag);
+      const bool ok = mbar_wait(&acc_full[buf], use & 1u, abort_flag, p.wait_ns);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;  // warp-uniform exit keeps tcgen05.ld converged
       fence_after_sync();
       const int r = mt * kBlockM + row_in_tile;
@@ -612,6 +612,16 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 1
   // ---------------------------------------------------------------- teardown
   fence_before_sync();
   __syncthreads();
+  // After an abort some armed stages were never consumed: their copies must
+  // land before the CTA's shared memory goes away (each wait bounded).
+  if (warp == 0 && lane == 0 && *abort_flag) {
+    for (int s = 0; s < STAGES; ++s)
+      if (armed_round[s] != 0xFFFFFFFFu) {
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait(&full[s], armed_round[s] & 1u) && globaltimer() - t0 < 100000000ull) {
+        }
+      }
+  }
   if (warp == 1) {
     fence_after_sync();
     tmem_dealloc(tmem_base, C::kTmemCols);
@@ -691,12 +701,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
+  // last round each stage's full barrier was armed in (producer lane only),
+  // for the drain after an abort
+  uint32_t armed_round[STAGES];
+#pragma unroll
+  for (int s = 0; s < STAGES; ++s) armed_round[s] = 0xFFFFFFFFu;
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
       uint32_t it = 0;
-      uint32_t armed_round[STAGES];
-      for (int s = 0; s < STAGES; ++s) armed_round[s] = 0xFFFFFFFFu;
       bool ok = true;
       for (int w = pair; w < num_work && ok; w += num_pairs) {
         const PairWork wk = pair_work(p, w, N_TOTAL);
@@ -706,9 +720,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const int b_cols = wk.narrow ? 64 : C::kNHalf;
         const uint32_t tx = 2u * uint32_t(C::kABytes + b_boxes * C::kBBoxBytes + C::kEBytes);
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          if (int64_t(it) == p.skip_it) continue;  // test hook: neither CTA fills this step's stage
           const int s = int(it % STAGES);
           const uint32_t round = it / STAGES;
-          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&empty[s], (round & 1u) ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
           uint8_t* st = smem + s * C::kStageBytes;
           if (leader) mbar_arrive_expect_tx(&full[s], tx);
           armed_round[s] = round;
@@ -723,21 +738,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                            (row_tile * p.k_blocks + kb) * kBlockM);
         }
       }
-      if (!ok) {
-        // let copies already issued land before the CTA can leave
-        if (leader) {
-          for (int s = 0; s < STAGES; ++s)
-            if (armed_round[s] != 0xFFFFFFFFu) {
-              const uint64_t t0 = globaltimer();
-              while (!mbar_try_wait(&full[s], armed_round[s] & 1u) && globaltimer() - t0 < 100000000ull) {
-              }
-            }
-        } else {
-          const uint64_t t0 = globaltimer();
-          while (globaltimer() - t0 < 2000000ull) {
-          }
-        }
-      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
@@ -750,13 +750,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const uint32_t idesc = w >= p.split_from ? idesc_narrow : idesc_full;
         const int buf = int(local % C::kAccBufs);
         const uint32_t use = local / C::kAccBufs;
-        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
         fence_after_sync();
         const uint32_t d_tmem = tmem_base + uint32_t(buf * N_TOTAL);
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = int(it % STAGES);
           const uint32_t round = it / STAGES;
-          if (!mbar_wait(&full[s], round & 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&full[s], round & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
           fence_after_sync();
           uint8_t* st = smem + s * C::kStageBytes;
           const uint32_t a_addr = smem_u32(st);
@@ -808,7 +808,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const int kc = wk.narrow ? kCols / 2 : kCols;
       const int buf = int(local % C::kAccBufs);
       const uint32_t use = local / C::kAccBufs;
-      const bool ok = mbar_wait(&acc_full[buf], use & 1u, abort_flag);
+      const bool ok = mbar_wait(&acc_full[buf], use & 1u, abort_flag, p.wait_ns);
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       fence_after_sync();
       const int r = (2 * mt + int(rank)) * kBlockM + row_in_tile;
@@ -895,6 +895,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   // ---------------------------------------------------------------- teardown
   fence_before_sync();
   __syncthreads();
+  // After an abort in either CTA, copies already issued must land before the
+  // pair leaves (each wait bounded).  Both CTAs' copies complete on the even
+  // CTA's full barriers, which it waits on; the odd CTA, which owns none,
+  // waits 2 ms; the cluster barrier below keeps both CTAs alive until then.
+  if (warp == 0) {
+    if (lane == 0 && *abort_flag) {
+      if (leader) {
+        for (int s = 0; s < STAGES; ++s)
+          if (armed_round[s] != 0xFFFFFFFFu) {
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try_wait(&full[s], armed_round[s] & 1u) && globaltimer() - t0 < 100000000ull) {
+            }
+          }
+      } else {
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 2000000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  }
   cluster_sync();  // the even CTA's MMAs are done and no remote arrive is pending
   if (warp == 1) {
     fence_after_sync();
@@ -953,12 +974,7 @@ nm_status launch(const CUtensorMap& ma, const void* X, int64_t ldx, int64_t K, i
                                 : C::kBRowBytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   if (!make_map(&mb, X, BF16, K, T, ldx, C::kBoxCols, kStageK, sw)) return NM_ERR_CUDA;
   auto kern = spmm_kernel<N_TILE, STAGES, BF16>;
-  static bool attr_done = false;  // per instantiation
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
-      return NM_ERR_CUDA;
-    attr_done = true;
-  }
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes) != NM_OK) return NM_ERR_CUDA;
   const int tiles = p.m_tiles * p.n_tiles;
   const int per_sm = C::kSmemBytes <= 113 * 1024 ? 2 : 1;  // two CTAs per SM when the ring is small
   const int slots = per_sm * sm_count();
@@ -981,23 +997,12 @@ bool make_map_image(CUtensorMap* map, const uint8_t* img, int64_t rows16) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// NM_SPMM_TAIL_SPLIT=0 turns the half-width last wave off (for comparison).
-bool split_tail_enabled() {
-  const char* e = getenv("NM_SPMM_TAIL_SPLIT");
-  return !(e && e[0] == '0');
-}
-
 template <int N_TOTAL, int STAGES, bool BF16>
 nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me, const CUtensorMap& my,
-                      const Params& p, cudaStream_t s) {
+                      const Params& p, bool tail_split, cudaStream_t s) {
   using C = PairCfg<N_TOTAL, STAGES>;
   auto kern = spmm_pair_kernel<N_TOTAL, STAGES, BF16>;
-  static bool attr_done = false;  // per instantiation
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) != cudaSuccess)
-      return NM_ERR_CUDA;
-    attr_done = true;
-  }
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes) != NM_OK) return NM_ERR_CUDA;
   const int tiles = p.m_tiles * p.n_tiles;
   const int max_pairs = sm_count() / 2;
   const int pairs = tiles < max_pairs ? tiles : max_pairs;
@@ -1007,7 +1012,7 @@ nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   // A last wave that fills at most half of the pairs is done in half-width
   // items (whole 64-column B atoms per CTA, so only for 256-column tiles).
   const int rem = tiles % pairs;
-  if (N_TOTAL == 256 && tiles > pairs && rem > 0 && 2 * rem <= pairs && split_tail_enabled()) {
+  if (N_TOTAL == 256 && tiles > pairs && rem > 0 && 2 * rem <= pairs && tail_split) {
     q.split_from = tiles - rem;
     q.num_work = tiles + rem;
   }
@@ -1017,12 +1022,20 @@ nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
 
 // Kernel choice: the CTA-pair kernel when the row tiles pair up and the
 // output is wide enough to fill 128+ columns; the single-CTA kernel
-// otherwise.  NM_SPMM_KERNEL = pair256 | pair128 | single256 | single128 |
-// single64 overrides the choice (for tuning; an inapplicable override falls
-// back to the default).
+// otherwise.  A test or tuning caller may force one (nm_spmm_test); a forced
+// choice that does not apply (a pair kernel for an odd number of row tiles)
+// falls back to the default.
 enum class Kern { Pair256, Pair192, Pair128, Single256, Single128, Single64, Single64x2, Single32x2, Single16x2 };
 
-Kern choose_kernel(int64_t R, int64_t T) {
+// Options of one call: the defaults for nm_spmm, test and tuning hooks otherwise.
+struct Opts {
+  int kernel = 0;          // 0: the library's choice; 1..9: Kern value + 1
+  bool tail_split = true;  // half-width items for a partly filled last wave
+  uint64_t wait_ns = kWaitLimitNs;
+  int64_t skip_it = -1;
+};
+
+Kern choose_kernel(int64_t R, int64_t T, int forced) {
   const bool pairable = ((R + kBlockM - 1) / kBlockM) % 2 == 0;
   Kern k;
   if (pairable && T > 64) k = T > 128 ? Kern::Pair256 : Kern::Pair128;
@@ -1031,25 +1044,20 @@ Kern choose_kernel(int64_t R, int64_t T) {
   else if (T > 32) k = Kern::Single64x2;
   else if (T > 16) k = Kern::Single32x2;
   else k = Kern::Single16x2;
-  if (const char* env = getenv("NM_SPMM_KERNEL")) {
-    const std::string e(env);
-    if (e == "pair256" && pairable) k = Kern::Pair256;
-    else if (e == "pair192" && pairable) k = Kern::Pair192;
-    else if (e == "pair128" && pairable) k = Kern::Pair128;
-    else if (e == "single256") k = Kern::Single256;
-    else if (e == "single128") k = Kern::Single128;
-    else if (e == "single64") k = Kern::Single64;
-    else if (e == "single64x2") k = Kern::Single64x2;
-    else if (e == "single32x2") k = Kern::Single32x2;
-    else if (e == "single16x2") k = Kern::Single16x2;
+  if (forced >= 1 && forced <= 9) {
+    const Kern f = static_cast<Kern>(forced - 1);
+    const bool is_pair = f == Kern::Pair256 || f == Kern::Pair192 || f == Kern::Pair128;
+    if (!is_pair || pairable) k = f;
   }
   return k;
 }
 
 template <bool BF16>
 nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_t ldx, void* Y, bool y_f32,
-              int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta, cudaStream_t s) {
+              int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta, const Opts& o, cudaStream_t s) {
   Params p;
+  p.wait_ns = o.wait_ns;
+  p.skip_it = o.skip_it;
   p.y_tma = 0;
   p.meta_img = meta_img;
   p.Y = Y;
@@ -1062,7 +1070,7 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
   p.y_vec = (aligned16(Y) && stride_ok(ldy, y_f32 ? 4 : 2)) ? 1 : 0;
   p.alpha = alpha;
   p.beta = beta;
-  const Kern kern = choose_kernel(R, T);
+  const Kern kern = choose_kernel(R, T, o.kernel);
   const bool pair = kern == Kern::Pair256 || kern == Kern::Pair192 || kern == Kern::Pair128;
   const int block_m = pair ? 2 * kBlockM : kBlockM;
   const int n_tile = (kern == Kern::Pair256 || kern == Kern::Single256) ? 256
@@ -1092,9 +1100,9 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
     p.y_tma = (!y_f32 && beta == 0.0f && p.y_vec) ? 1 : 0;
     memset(&my, 0, sizeof(my));
     if (p.y_tma && !make_map(&my, Y, true, R, T, ldy, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return NM_ERR_CUDA;
-    if (kern == Kern::Pair256) return launch_pair<256, 4, BF16>(ma, mb, me, my, p, s);
-    if (kern == Kern::Pair192) return launch_pair<192, 4, BF16>(ma, mb, me, my, p, s);
-    return launch_pair<128, 6, BF16>(ma, mb, me, my, p, s);
+    if (kern == Kern::Pair256) return launch_pair<256, 4, BF16>(ma, mb, me, my, p, o.tail_split, s);
+    if (kern == Kern::Pair192) return launch_pair<192, 4, BF16>(ma, mb, me, my, p, o.tail_split, s);
+    return launch_pair<128, 6, BF16>(ma, mb, me, my, p, o.tail_split, s);
   }
   switch (kern) {
     case Kern::Single256: return launch<256, 2, BF16>(ma, X, ldx, K, T, p, s);
@@ -1119,22 +1127,39 @@ extern "C" size_t nm_spmm_workspace_bytes(nm_dtype ab_dtype, int64_t R, int64_t 
   return align256(size_t(R) * size_t(K / 2) * 2) + align256(size_t(K) * size_t(ldx_h) * 2);
 }
 
-extern "C" nm_status nm_spmm(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X,
-                             int64_t ldx, void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T,
-                             float alpha, float beta, void* workspace, size_t workspace_bytes, void* stream) {
+namespace {
+
+// Host checks of nm_spmm's arguments other than the workspace.  NM_OK with
+// *noop set means there is nothing to compute (R == 0 or T == 0).
+nm_status spmm_validate(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X,
+                        int64_t ldx, const void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T,
+                        bool* noop) {
+  *noop = false;
   if (ab_dtype == NM_S8) return NM_ERR_UNSUPPORTED;  // the int8 sparse product is not built
   if (!dtype_ok(ab_dtype) || (y_dtype != NM_BF16 && y_dtype != NM_F32)) return NM_ERR_DTYPE;
   if (R < 0 || K < 0 || T < 0 || K % 16 != 0 || ldx < T || ldy < T) return NM_ERR_SHAPE;
   if (R > 0x7FFFFFFF - 256 || K > 0x7FFFFFFF - 256 || T > 0x7FFFFFFF - 256) return NM_ERR_SHAPE;
-  if (R == 0 || T == 0) return NM_OK;
+  if (R == 0 || T == 0) {
+    *noop = true;
+    return NM_OK;
+  }
   if (values == nullptr || meta_sm100 == nullptr || X == nullptr || Y == nullptr) return NM_ERR_NULL;
   const int ab_es = esize_of(ab_dtype), y_es = esize_of(y_dtype);
   if (!aligned16(values) || !aligned16(meta_sm100) || !aligned16(X) || !stride_ok(ldx, ab_es) ||
       (reinterpret_cast<uintptr_t>(Y) % uintptr_t(y_es)) != 0)
     return NM_ERR_ALIGN;
+  if (K == 0) return NM_ERR_SHAPE;
+  return NM_OK;
+}
+
+nm_status spmm_entry(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X, int64_t ldx,
+                     void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta,
+                     void* workspace, size_t workspace_bytes, const spmm::Opts& o, void* stream) {
+  bool noop = false;
+  const nm_status v = spmm_validate(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, &noop);
+  if (v != NM_OK || noop) return v;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool y_f32 = y_dtype == NM_F32;
-  if (K == 0) return NM_ERR_SHAPE;
   if (ab_dtype == NM_F32) {
     const size_t need = nm_spmm_workspace_bytes(ab_dtype, R, K, T);
     if (workspace == nullptr || workspace_bytes < need) return NM_ERR_WORKSPACE;
@@ -1146,11 +1171,35 @@ extern "C" nm_status nm_spmm(const void* values, const uint8_t* meta_sm100, nm_d
     spmm::f32_to_f16_kernel<<<blocks, 256, 0, s>>>(static_cast<const float*>(values), R, K / 2, K / 2, vh, K / 2);
     spmm::f32_to_f16_kernel<<<blocks, 256, 0, s>>>(static_cast<const float*>(X), K, T, ldx, xh, ldx_h);
     if (launch_status() != NM_OK) return NM_ERR_CUDA;
-    return spmm::run<false>(vh, meta_sm100, xh, ldx_h, Y, y_f32, ldy, R, K, T, alpha, beta, s);
+    return spmm::run<false>(vh, meta_sm100, xh, ldx_h, Y, y_f32, ldy, R, K, T, alpha, beta, o, s);
   }
   if (ab_dtype == NM_BF16)
-    return spmm::run<true>(values, meta_sm100, X, ldx, Y, y_f32, ldy, R, K, T, alpha, beta, s);
-  return spmm::run<false>(values, meta_sm100, X, ldx, Y, y_f32, ldy, R, K, T, alpha, beta, s);
+    return spmm::run<true>(values, meta_sm100, X, ldx, Y, y_f32, ldy, R, K, T, alpha, beta, o, s);
+  return spmm::run<false>(values, meta_sm100, X, ldx, Y, y_f32, ldy, R, K, T, alpha, beta, o, s);
+}
+
+}  // namespace
+
+extern "C" nm_status nm_spmm(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X,
+                             int64_t ldx, void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T,
+                             float alpha, float beta, void* workspace, size_t workspace_bytes, void* stream) {
+  return spmm_entry(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, workspace,
+                    workspace_bytes, spmm::Opts(), stream);
+}
+
+extern "C" nm_status nm_spmm_test(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X,
+                                  int64_t ldx, void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K,
+                                  int64_t T, float alpha, float beta, void* workspace, size_t workspace_bytes,
+                                  int kernel, int tail_split, int64_t wait_limit_ns, int64_t skip_step,
+                                  void* stream) {
+  if (kernel < 0 || kernel > 9 || wait_limit_ns < 0 || skip_step < -1) return NM_ERR_SHAPE;
+  spmm::Opts o;
+  o.kernel = kernel;
+  o.tail_split = tail_split != 0;
+  if (wait_limit_ns > 0) o.wait_ns = uint64_t(wait_limit_ns);
+  o.skip_it = skip_step;
+  return spmm_entry(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, workspace,
+                    workspace_bytes, o, stream);
 }
 
 extern "C" nm_status nm_last_device_status(void* stream) {
@@ -1199,15 +1248,18 @@ nm_status noalloc_scratch(void** out) {
 extern "C" nm_status nm_spmm_noalloc(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype,
                                      const void* X, int64_t ldx, void* Y, nm_dtype y_dtype, int64_t ldy,
                                      int64_t R, int64_t K, int64_t T, float alpha, float beta, void* stream) {
+  // the same argument checks as nm_spmm first, so a malformed call reports
+  // its real fault rather than the scratch limit
+  bool noop = false;
+  const nm_status v = spmm_validate(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, &noop);
+  if (v != NM_OK || noop) return v;
   if (ab_dtype != NM_F32)  // the 16-bit paths use no scratch at all
     return nm_spmm(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, nullptr, 0, stream);
   const size_t need = nm_spmm_workspace_bytes(ab_dtype, R, K, T);
   if (need > kNoAllocScratchBytes) return NM_ERR_WORKSPACE;  // problem larger than the fixed scratch
   void* scratch = nullptr;
-  if (need > 0) {
-    const nm_status st = noalloc_scratch(&scratch);
-    if (st != NM_OK) return st;
-  }
+  const nm_status st = noalloc_scratch(&scratch);
+  if (st != NM_OK) return st;
   return nm_spmm(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, scratch,
-                 need > 0 ? kNoAllocScratchBytes : 0, stream);
+                 kNoAllocScratchBytes, stream);
 }

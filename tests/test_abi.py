@@ -1,6 +1,6 @@
-"""The C-ABI library: it builds, loads, exports every symbol include/nm.h
-declares, and validates arguments on the host (no GPU needed: every case
-here fails validation before any CUDA call)."""
+"""The C-ABI library: it builds, loads, exports every symbol the headers in
+include/ declare, and validates arguments on the host (no GPU needed: every
+case here fails validation before any CUDA call)."""
 import ctypes
 import os
 import re
@@ -11,12 +11,15 @@ import structured_sparsity_prune_b200 as nm
 from structured_sparsity_prune_b200 import build as nm_build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "nm.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in sorted(os.listdir(os.path.join(ROOT, "include")))
+           if h.endswith(".h")]
 
 
 def _declared():
-    with open(HEADER) as f:
-        text = f.read()
+    text = ""
+    for h in HEADERS:
+        with open(h) as f:
+            text += f.read()
     return sorted(set(re.findall(r"NM_API\s+[\w\s\*]*?\b(nm_\w+)\s*\(", text)))
 
 
@@ -136,6 +139,20 @@ def test_host_validation_before_any_launch(lib):
     assert L.nm_spmm(fake, fake, 1, fake, big, fake, 1, big, 128, 64, big, f(1), f(0), None, 0, s) == 2
     # K == 0 with rows and columns to write has no product to form
     assert L.nm_spmm(fake, fake, 1, fake, 8, fake, 1, 8, 128, 0, 8, f(1), f(0), None, 0, s) == 2
+    # the no-allocation product checks its arguments before its scratch limit: fp32 at 4096^3
+    # needs 48 MiB of staging, more than its 16 MiB array, yet a malformed call reports its fault
+    n = 4096
+    assert L.nm_spmm_noalloc(fake, fake, 0, fake, n, fake, 0, n, n, n + 8, n, f(1), f(0), s) == 2   # K % 16
+    assert L.nm_spmm_noalloc(fake, fake, 0, odd, n, fake, 0, n, n, n, n, f(1), f(0), s) == 3        # misaligned X
+    assert L.nm_spmm_noalloc(fake, fake, 0, fake, n - 8, fake, 0, n, n, n, n, f(1), f(0), s) == 2   # ldx < T
+    assert L.nm_spmm_noalloc(fake, fake, 0, fake, n, fake, 0, n, n, n, n, f(1), f(0), s) == 8       # too large
+    assert L.nm_spmm_noalloc(fake, fake, 0, fake, n, fake, 0, n, 0, n, n, f(1), f(0), s) == 0       # R == 0
+    # the test entry point: its own arguments, then nm_spmm's checks
+    t = lambda kern, split, wait, skip, K=64: L.nm_spmm_test(fake, fake, 1, fake, 8, fake, 1, 8, 128, K, 8, f(1),
+                                                              f(0), None, 0, kern, split, wait, skip, s)
+    assert t(10, 1, 0, -1) == 2 and t(-1, 1, 0, -1) == 2
+    assert t(0, 1, -5, -1) == 2 and t(0, 1, 0, -2) == 2
+    assert t(1, 1, 0, -1, K=40) == 2
 
 
 def test_workspace_size(lib):

@@ -53,12 +53,17 @@ def _built():
     assert torch.cuda.is_available()
 
 
-def _run(W, X, y_dtype=torch.bfloat16, alpha=1.0, beta=0.0, Y0=None, rows=None):
-    """GPU: fused compress then spmm.  Oracle: its own compress then fp64 spmm."""
+def _run(W, X, y_dtype=torch.bfloat16, alpha=1.0, beta=0.0, Y0=None, rows=None, kernel=None):
+    """GPU: fused compress then spmm (a forced tile configuration through the
+    test entry point when `kernel` is given).  Oracle: its own compress then
+    fp64 spmm."""
     ab = W.dtype
     values, meta, img = nm.nm_mask_compress(W.cuda())
     Y = None if Y0 is None else Y0.clone().cuda()
-    Y = nm.nm_spmm(values, img, _dev(X), Y=Y, y_dtype=y_dtype, alpha=alpha, beta=beta)
+    if kernel is None:
+        Y = nm.nm_spmm(values, img, _dev(X), Y=Y, y_dtype=y_dtype, alpha=alpha, beta=beta)
+    else:
+        Y = nm.nm_spmm_test(values, img, _dev(X), Y=Y, y_dtype=y_dtype, alpha=alpha, beta=beta, kernel=kernel)
     torch.cuda.synchronize()
     _ok_status()
     Wb = _bits(W)
@@ -229,55 +234,77 @@ KERNELS = ["pair256", "pair192", "pair128", "single256", "single128", "single64"
 
 
 @pytest.mark.parametrize("kern", KERNELS)
-def test_every_tile_shape_is_exact_on_integers(kern, monkeypatch):
-    """Each tile configuration, forced through NM_SPMM_KERNEL, on a shape
+def test_every_tile_shape_is_exact_on_integers(kern):
+    """Each tile configuration, forced through the test entry point, on a shape
     ragged in R (700 = 5.5 row tiles) and T (500 columns, a partial last tile
     for every width): integer inputs make the fp32 output exact and the bf16
     output its round-to-nearest-even, on both epilogue paths."""
-    monkeypatch.setenv("NM_SPMM_KERNEL", kern)
     R, K, T = 700, 384, 500
     W = nm_inputs.small_int((R, K), 81, dtype=torch.bfloat16)
     X = nm_inputs.small_int((K, T), 82, dtype=torch.bfloat16)
-    Y, ref = _run(W, X, torch.float32)
+    Y, ref = _run(W, X, torch.float32, kernel=kern)
     assert np.array_equal(Y.numpy().astype(np.float64), ref)
-    Yb, ref_b = _run(W, X, torch.bfloat16)
+    Yb, ref_b = _run(W, X, torch.bfloat16, kernel=kern)
     assert np.array_equal(_bits(Yb), oracle.encode_array(ref_b, oracle.BF16))
 
 
 @pytest.mark.parametrize("kern", KERNELS)
-def test_every_tile_shape_alpha_beta(kern, monkeypatch):
-    monkeypatch.setenv("NM_SPMM_KERNEL", kern)
+def test_every_tile_shape_alpha_beta(kern):
     R, K, T = 700, 256, 500
     W = nm_inputs.normal((R, K), 83, 0.02, torch.bfloat16)
     X = nm_inputs.normal((K, T), 84, 1.0, torch.bfloat16)
     Y0 = nm_inputs.normal((R, T), 85, 1.0, torch.bfloat16)
-    Y, ref = _run(W, X, torch.bfloat16, alpha=1.5, beta=0.5, Y0=Y0)
+    Y, ref = _run(W, X, torch.bfloat16, alpha=1.5, beta=0.5, Y0=Y0, kernel=kern)
     assert _nerr(Y, ref) <= 8e-3
 
 
 @pytest.mark.parametrize("R,T", [(2560, 2048), (2500, 2000)])
-def test_half_width_last_wave_is_exact(R, T, monkeypatch):
+def test_half_width_last_wave_is_exact(R, T):
     """80 pair tiles on 74 pairs: the last 6 tiles run as 12 half-width items
     (ragged in R and T in the second case); integer inputs make the fp32
     output exact and the bf16 output its round-to-nearest-even."""
-    monkeypatch.setenv("NM_SPMM_KERNEL", "pair256")
     K = 128
     W = nm_inputs.small_int((R, K), 91, dtype=torch.bfloat16)
     X = nm_inputs.small_int((K, T), 92, dtype=torch.bfloat16)
-    Y, ref = _run(W, X, torch.float32)
+    Y, ref = _run(W, X, torch.float32, kernel="pair256")
     assert np.array_equal(Y.numpy().astype(np.float64), ref)
-    Yb, ref_b = _run(W, X, torch.bfloat16)
+    Yb, ref_b = _run(W, X, torch.bfloat16, kernel="pair256")
     assert np.array_equal(_bits(Yb), oracle.encode_array(ref_b, oracle.BF16))
 
 
-def test_half_width_last_wave_matches_whole_tiles(monkeypatch):
+def test_half_width_last_wave_matches_whole_tiles():
     """Splitting the last wave does not change the summation order, so the
     result equals the unsplit run bit for bit."""
     W = nm_inputs.normal((4096, 1024), 93, 0.02, torch.bfloat16).cuda()
     X = nm_inputs.normal((1024, 4096), 94, 1.0, torch.bfloat16).cuda()
     values, meta, img = nm.nm_mask_compress(W)
     a = nm.nm_spmm(values, img, X)
-    monkeypatch.setenv("NM_SPMM_TAIL_SPLIT", "0")
-    b = nm.nm_spmm(values, img, X)
+    b = nm.nm_spmm_test(values, img, X, tail_split=False)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("kern,R,T", [("pair256", 1024, 1024), ("single256", 640, 512), ("single16x2", 384, 16)])
+def test_bounded_wait_runs_out_and_the_next_call_is_clean(kern, R, T):
+    """The failure path of the product kernel's bounded waits, driven without a
+    fault: through the test entry point the producer never fills its first
+    pipeline stage and every wait is limited to 5 ms, so the MMA issuer's wait
+    on that stage runs out.  The kernel must record NM_ERR_TIMEOUT, stop its
+    other roles, let its copies land, free its tensor memory and return; the
+    next ordinary call on the same stream must then run and match the oracle,
+    and leave the status word clear."""
+    K = 512
+    W = nm_inputs.normal((R, K), 97, 0.02, torch.bfloat16)
+    X = nm_inputs.normal((K, T), 98, 1.0, torch.bfloat16)
+    values, meta, img = nm.nm_mask_compress(W.cuda())
+    Xd = _dev(X)
+    assert nm.nm_last_device_status() == 0
+    nm.nm_spmm_test(values, img, Xd, y_dtype=torch.float32, kernel=kern, wait_limit_ns=5_000_000, skip_step=0)
+    assert nm.nm_last_device_status() == 9          # NM_ERR_TIMEOUT, read and cleared
+    assert nm.nm_last_device_status() == 0
+    Y, ref = _run(W, X, torch.float32)              # an ordinary call afterwards
+    assert _nerr(Y, ref) <= 1e-3
+    Y2 = nm.nm_spmm_test(values, img, Xd, y_dtype=torch.float32, kernel=kern)
+    torch.cuda.synchronize()
+    assert nm.nm_last_device_status() == 0
+    assert _nerr(Y2.cpu(), ref) <= 1e-3

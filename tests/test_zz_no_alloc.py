@@ -6,10 +6,11 @@ every device allocation (a serving engine, a plugin host with a fixed memory
 budget), or a latency-critical path that cannot take cudaMalloc's implicit
 synchronisation.  For them nm_spmm_noalloc takes the fp32 path's binary16
 staging buffers from a fixed device array inside the library instead of a
-caller workspace.  This test checks it against the workspace-taking nm_spmm,
-within the fp32-output tolerance of the other product tests, on two calls in
-a row (the second with different inputs, so stale scratch would show), and
-that a problem larger than the fixed array is refused.
+caller workspace.  This test checks it against the workspace-taking nm_spmm
+and against the fp64 CPU oracle, within the fp32-output tolerance of the
+other product tests, on two calls in a row (the second with different inputs,
+so stale scratch would show), and that a problem larger than the fixed array
+is refused.
 
 The file name sorts last so that a stop-at-first-failure run has executed
 every other test before this one."""
@@ -20,6 +21,7 @@ import pytest
 import torch
 
 import nm_inputs
+import oracle
 import structured_sparsity_prune_b200 as nm
 
 pytestmark = pytest.mark.gpu
@@ -34,10 +36,19 @@ def _nerr(a, b):
 
 
 def _case(seed_w, seed_x, R=256, K=256, T=128):
-    W = nm_inputs.normal((R, K), seed_w, 1.0, torch.float32).cuda()
-    X = nm_inputs.normal((K, T), seed_x, 1.0, torch.float32).cuda()
-    values, meta, img = nm.nm_mask_compress(W)
-    return values, img, X
+    W = nm_inputs.normal((R, K), seed_w, 1.0, torch.float32)
+    X = nm_inputs.normal((K, T), seed_x, 1.0, torch.float32)
+    values, meta, img = nm.nm_mask_compress(W.cuda())
+    return values, img, X.cuda(), W, X
+
+
+def _oracle_product(W, X):
+    """fp64 product of the oracle's own 2:4 compression of W with X."""
+    oracle.build()
+    Wn, Xn = W.numpy(), X.numpy()
+    mask = oracle.mask_rank(Wn, 2, 4)
+    v, m = oracle.compress24(Wn, mask)
+    return oracle.spmm(v, m, Xn, oracle.F32)
 
 
 def _noalloc(lib, values, img, X, Y):
@@ -52,7 +63,7 @@ def _noalloc(lib, values, img, X, Y):
 def test_noalloc_matches_workspace_entry_point_on_two_calls():
     lib = nm.load()
     for seeds in [(0, 100), (7, 107)]:
-        values, img, X = _case(*seeds)
+        values, img, X, W_host, X_host = _case(*seeds)
         ref = nm.nm_spmm(values, img, X, y_dtype=torch.float32)          # caller-provided workspace
         Y = torch.full(ref.shape, float("nan"), dtype=torch.float32, device="cuda")
         assert _noalloc(lib, values, img, X, Y) == NM_OK
@@ -60,6 +71,8 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
         assert nm.nm_last_device_status() == NM_OK
         assert torch.isfinite(Y).all()
         assert _nerr(Y, ref) <= 1e-3
+        exact = torch.from_numpy(_oracle_product(W_host, X_host))
+        assert _nerr(Y, exact) <= 1e-3
 
 
 def test_noalloc_refuses_problems_beyond_the_fixed_scratch():
