@@ -5,14 +5,17 @@
                                srste|saliency_mask|transposable_mask|transposable_24|pairs_12|int8_24]
 
 One step is one pass of every step of the path over one batch of synthetic
-input (default: the transformer-linear workload, bf16 W 4096x4096 pruned 2:4
-along K, X 4096x4096 tokens):
+input.  Default: the MLP pair, bf16 W_up 14336x4096 and W_down 4096x14336
+pruned 2:4 along K, X 4096x8192 (8192 tokens), 20 timed repetitions; on each
+weight
     nm_mask (2:4) -> nm_compress (that mask) -> nm_mask_compress (fused)
-    -> nm_meta_to_sm100 -> nm_decompress -> nm_spmm (Y = W' X, bf16 out).
-`value` is the dense-equivalent TFLOP/s of the whole step (2*R*K*T flops per
-step over the device time of the full step); the per-kernel breakdown, the
-roofline of the dominant kernel (nm_spmm, sparse tensor peak) and the
-bandwidth kernels' GB/s against HBM are reported beside it.
+    -> nm_meta_to_sm100 -> nm_decompress,
+then nm_spmm up (H = W_up' X) and down (Y = W_down' H), bf16 out.
+`value` is the dense-equivalent TFLOP/s of the whole step (2*R*K*T flops of
+both products per step over the device time of the full step); the
+per-kernel breakdown, the roofline of the dominant kernel (the longer
+product, sparse tensor peak) and the bandwidth kernels' GB/s against HBM are
+reported beside it.
 
 Timing: W untimed warm-up steps, then exactly K steps, each bracketed by CUDA
 events on the launching stream, with L2 flushed between steps outside the
@@ -323,19 +326,36 @@ class Step:
             self.flops = sum(self.flop_k.values())
             return
         if self.kind == "mlp":
+            # every row of the path on both weights, then the two products
             self.W2 = wl["W2"].to(dev)
             R2, K2 = self.W2.shape
+            es = self.W.element_size()
+            self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
+            self.mask2 = torch.empty((R2, K2), dtype=torch.uint8, device=dev)
+            self.v_c, self.m_c, self.img_c = nm.alloc_compressed(R, K, self.W.dtype, dev)
+            self.v2_c, self.m2_c, self.img2_c = nm.alloc_compressed(R2, K2, self.W2.dtype, dev)
             self.v2, self.m2, self.img2 = nm.alloc_compressed(R2, K2, self.W2.dtype, dev)
+            self.img_r = torch.empty_like(self.img)
+            self.img2_r = torch.empty_like(self.img2)
+            self.Wd = torch.empty_like(self.W)
+            self.W2d = torch.empty_like(self.W2)
             self.H = torch.empty((R, (T + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)[:, :T]
             self.Y = torch.empty((R2, T), dtype=torch.bfloat16, device=dev)
-            ws = max(nm.nm_spmm_workspace_bytes(torch.bfloat16, R, K, T),
-                     nm.nm_spmm_workspace_bytes(torch.bfloat16, R2, K2, T))
+            ws = max(nm.nm_spmm_workspace_bytes(self.W.dtype, R, K, T),
+                     nm.nm_spmm_workspace_bytes(self.W2.dtype, R2, K2, T))
+            # the two products run one after the other (down reads H), so they may share scratch
             self.ws = torch.empty((ws,), dtype=torch.uint8, device=dev) if ws else None
-            self.names = ["nm_mask_compress_up", "nm_mask_compress_down", "nm_spmm_up", "nm_spmm_down"]
-            G1, G2 = R * K, R2 * K2
-            self.bytes = {"nm_mask_compress_up": G1 * 3.25, "nm_mask_compress_down": G2 * 3.25,
-                          "nm_spmm_up": G1 * 1.125 + K * T * 2 + R * T * 2,
-                          "nm_spmm_down": G2 * 1.125 + K2 * T * 2 + R2 * T * 2}
+            self.names, self.bytes = [], {}
+            for tag, G in (("up", R * K), ("down", R2 * K2)):
+                self.names += ["nm_mask_" + tag, "nm_compress_" + tag, "nm_mask_compress_" + tag,
+                               "nm_meta_to_sm100_" + tag, "nm_decompress_" + tag]
+                self.bytes.update({"nm_mask_" + tag: G * (es + 1), "nm_compress_" + tag: G * (es + 1 + es / 2 + 0.25),
+                                   "nm_mask_compress_" + tag: G * (es + es / 2 + 0.25),
+                                   "nm_meta_to_sm100_" + tag: G * 0.25,
+                                   "nm_decompress_" + tag: G * (es / 2 + 0.125 + es)})
+            self.names += ["nm_spmm_up", "nm_spmm_down"]
+            self.bytes.update({"nm_spmm_up": R * K * (es / 2 + 0.125) + K * T * es + R * T * 2,
+                               "nm_spmm_down": R2 * K2 * (es / 2 + 0.125) + K2 * T * es + R2 * T * 2})
             self.flop_k = {"nm_spmm_up": 2.0 * R * K * T, "nm_spmm_down": 2.0 * R2 * K2 * T}
             self.flops = sum(self.flop_k.values())
             return
@@ -390,8 +410,18 @@ class Step:
                     lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.Y, workspace=self.ws),
                     lambda: nm.nm_spmm(self.v_t, self.img_t, self.DY, Y=self.DX, workspace=self.ws_t)]
         if self.kind == "mlp":
-            return [lambda: nm.nm_mask_compress(self.W, self.values, self.meta, self.img),
+            K, K2 = self.wl["K"], self.W2.shape[1]
+            R, R2 = self.wl["R"], self.W2.shape[0]
+            return [lambda: nm.nm_mask(self.W, 2, 4, mask=self.mask),
+                    lambda: nm.nm_compress(self.W, self.mask, self.v_c, self.m_c, self.img_c),
+                    lambda: nm.nm_mask_compress(self.W, self.values, self.meta, self.img),
+                    lambda: nm.nm_meta_to_sm100(self.meta, R, K, out=self.img_r),
+                    lambda: nm.nm_decompress(self.values, self.meta, K, out=self.Wd),
+                    lambda: nm.nm_mask(self.W2, 2, 4, mask=self.mask2),
+                    lambda: nm.nm_compress(self.W2, self.mask2, self.v2_c, self.m2_c, self.img2_c),
                     lambda: nm.nm_mask_compress(self.W2, self.v2, self.m2, self.img2),
+                    lambda: nm.nm_meta_to_sm100(self.m2, R2, K2, out=self.img2_r),
+                    lambda: nm.nm_decompress(self.v2, self.m2, K2, out=self.W2d),
                     lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.H, workspace=self.ws),
                     lambda: nm.nm_spmm(self.v2, self.img2, self.H, Y=self.Y, workspace=self.ws)]
         K = self.wl["K"]
@@ -411,8 +441,9 @@ class Step:
         n = self.launches()
         if self.kind == "linear":     # mask -> compress; fused -> {image, decompress, product}
             return [[], [0], [], [2], [2], [2]]
-        if self.kind == "mlp":        # two compressions; up -> down (H)
-            return [[], [], [0], [1, 2]]
+        if self.kind == "mlp":        # per weight: mask -> compress; fused -> {image, decompress}; then
+            #                               up product after the fused up call, down after fused down and up
+            return [[], [0], [], [2], [2], [], [5], [], [7], [7], [2], [7, 10]]
         if self.kind == "trans24":    # mask -> {compress -> forward, compress_t -> backward}
             return [[], [0], [0], [1], [2]]
         if self.kind == "ties":       # four masks of the same W
@@ -693,27 +724,33 @@ def oracle_step(wl, rows: int, threads: int):
         for N, M in [(1, 4), (2, 4), (4, 8), (2, 8)]:
             oracle.rows_parallel(0, W, N, M, oracle.F32, threads)
         return time.perf_counter() - t0, 4.0 * rows * W.shape[1] * 5
-    W = wl["W"][:rows].contiguous()
-    Wb = _u16(W)
     code = oracle.BF16
     X = _u16(wl["X"])
     K, T = wl["K"], wl["T"]
+
+    def six_calls(Wfull, Kw):
+        """mask, compress under it, fused mask+compress, image, decompress on the
+        first `rows` rows of one weight -> (values, meta) of the fused call"""
+        Wb = _u16(Wfull[:rows].contiguous())
+        mask, _, _ = oracle.rows_parallel(0, Wb, 2, 4, code, threads)
+        oracle.compress24(Wb, mask, dtype=code)
+        _, values, meta = oracle.rows_parallel(1, Wb, 2, 4, code, threads)
+        oracle.meta_sm100(meta, rows, Kw)
+        oracle.decompress24(values, meta, Kw, dtype=code)
+        return values, meta
+
     t0 = time.perf_counter()
-    mask, _, _ = oracle.rows_parallel(0, Wb, 2, 4, code, threads)          # mask
-    v1, m1 = oracle.compress24(Wb, mask, dtype=code)                        # compress (given mask)
-    _, values, meta = oracle.rows_parallel(1, Wb, 2, 4, code, threads)     # fused mask + compress
-    oracle.meta_sm100(meta, rows, K)                                        # metadata image
-    oracle.decompress24(values, meta, K, dtype=code)                        # decompress
+    values, meta = six_calls(wl["W"], K)
     oracle.spmm(values, meta, X, code, threads=threads)                     # product
+    units = 2.0 * rows * K * T
     if "W2" in wl:
-        # down projection on the same number of rows of W_down, fed by X's first rows
-        W2 = _u16(wl["W2"][:rows].contiguous())
-        _, v2, m2 = oracle.rows_parallel(1, W2, 2, 4, code, threads)
-        H = np.zeros((wl["W2"].shape[1], T), dtype=np.uint16)
+        # the same rows of W_down, then its product; its input H (W_up's output,
+        # 14336 x T) is a zero stand-in of that shape, which costs the oracle the same
+        K2 = wl["W2"].shape[1]
+        v2, m2 = six_calls(wl["W2"], K2)
+        H = np.zeros((K2, T), dtype=np.uint16)
         oracle.spmm(v2, m2, H, code, threads=threads)
-        units = 2.0 * rows * K * T + 2.0 * rows * wl["W2"].shape[1] * T
-    else:
-        units = 2.0 * rows * K * T
+        units += 2.0 * rows * K2 * T
     return time.perf_counter() - t0, units
 
 
@@ -738,6 +775,8 @@ def cpu_baseline(wl, target_s: float = 15.0):
             "1:2 mask, compress, fused compress, decompress" if "P12" in wl else
             "int8 2:4 mask, fused mask+compress, decompress" if "I8" in wl else
             "mask at 1:4, 2:4, 4:8, 2:8" if wl["X"] is None else
+            "whole step on the sampled rows of both weights (mask, compress, fused mask+compress, image, "
+            "decompress, fp64 product; the down product's input is a zero stand-in of H's shape)" if "W2" in wl else
             "whole step (mask, compress, fused mask+compress, image, decompress, fp64 product)")
     return {"value": units / secs / scale, "unit": unit, "cores": threads, "kind": "oracle",
             "sample": "first %d of %d rows of W, %s, %.1f s" % (rows, wl["R"], what, secs)}
@@ -793,10 +832,10 @@ def whole_job_rate(world: int, units_per_step: float, steps: int, ms: float, sca
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=20)       # the MLP-pair workload's 20 timed repetitions
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nm", choices=["nm", "reference"])
-    ap.add_argument("--workload", default="linear_4096")
+    ap.add_argument("--workload", default="mlp_pair")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
 

@@ -153,7 +153,10 @@ def test_closure_catches_a_planted_race():
     step = bench.Step(rec, WORKLOADS["mlp"], torch.device("cpu"))
     for fn in step.calls():
         fn()
-    before = _closure([[], [], [0], [1]])                 # the down product no longer waits for the up product
-    reads_down = rec.log[3][0]
-    writes_up = rec.log[2][1]
-    assert writes_up & reads_down and 2 not in before[3]
+    deps = step.deps()
+    up, down = step.names.index("nm_spmm_up"), step.names.index("nm_spmm_down")
+    planted = [d if i != down else [j for j in d if j != up] for i, d in enumerate(deps)]
+    before = _closure(planted)                            # the down product no longer waits for the up product
+    reads_down = rec.log[down][0]
+    writes_up = rec.log[up][1]
+    assert writes_up & reads_down and up not in before[down]
