@@ -21,6 +21,9 @@ What each function follows (page title and section):
   (the pages give none).
 * ``spmm`` -- same review, "Structured sparse GEMM on tensor cores":
   sparse x dense = dense; computed in double.
+* ``spmm12`` -- the 1:2 (sparse TF32) product of the same section, in double.
+* ``meta_sm100_s8`` / ``meta12_sm100`` -- PTX ISA, tcgen05 sparse metadata of
+  the .kind::i8 and .kind::tf32 MMAs.
 * ``srste`` -- "SR-STE sparse training", SR-STE forward / backward:
   masked weight and grad + decay * (1 - mask) * w.
 """
@@ -82,6 +85,13 @@ def _load():
     lib.oracle_meta_sm100.restype = i32
     lib.oracle_spmm.argtypes = [vp, vp, i32, vp, i64, vp, i32, i64, i64, dbl, dbl, vp, i64, i32, vp]
     lib.oracle_spmm.restype = i32
+    lib.oracle_spmm12.argtypes = [vp, vp, i32, vp, i64, vp, i32, i64, i64, dbl, dbl, vp, i64, i32, vp]
+    lib.oracle_spmm12.restype = i32
+    for name in ("oracle_meta_sm100_s8", "oracle_meta12_sm100"):
+        getattr(lib, name + "_bytes").argtypes = [i64, i64]
+        getattr(lib, name + "_bytes").restype = i64
+        getattr(lib, name).argtypes = [vp, i64, i64, vp]
+        getattr(lib, name).restype = i32
     lib.oracle_rows_parallel.argtypes = [i32, vp, i32, i64, i64, i32, i32, vp, vp, vp, i32]
     lib.oracle_rows_parallel.restype = i32
     lib.oracle_mask_transposable.argtypes = [vp, i32, i64, i64, i64, i32, i32, vp, i64]
@@ -260,13 +270,45 @@ def meta_sm100(meta: np.ndarray, R: int, C: int) -> np.ndarray:
     return out
 
 
+def meta_sm100_s8(meta: np.ndarray, R: int, C: int) -> np.ndarray:
+    """Tensor-core metadata image of a 2:4 int8 matrix (.kind::i8 layout)."""
+    lib = _load()
+    mt = np.ascontiguousarray(meta, dtype=np.uint8)
+    out = np.zeros(int(lib.oracle_meta_sm100_s8_bytes(R, C)), dtype=np.uint8)
+    _check(lib.oracle_meta_sm100_s8(mt.ctypes.data, R, C, out.ctypes.data), "meta_sm100_s8")
+    return out
+
+
+def meta12_sm100(meta: np.ndarray, R: int, C: int) -> np.ndarray:
+    """Tensor-core metadata image of a 1:2 fp32 matrix (.kind::tf32 layout)."""
+    lib = _load()
+    mt = np.ascontiguousarray(meta, dtype=np.uint8)
+    out = np.zeros(int(lib.oracle_meta12_sm100_bytes(R, C)), dtype=np.uint8)
+    _check(lib.oracle_meta12_sm100(mt.ctypes.data, R, C, out.ctypes.data), "meta12_sm100")
+    return out
+
+
 def spmm(values: np.ndarray, meta: np.ndarray, X: np.ndarray, ab_dtype: int,
          alpha: float = 1.0, beta: float = 0.0, Y_in: np.ndarray | None = None,
          y_dtype: int = F32, rows: np.ndarray | None = None, threads: int | None = None) -> np.ndarray:
-    """fp64 Y = alpha * (W (.) mask) X + beta * Y_in, from the compressed form.
+    """fp64 Y = alpha * (W (.) mask) X + beta * Y_in, from the compressed 2:4 form
+    (int8 inputs summed exactly in int64).
 
     values: R x K/2, meta: R x K/8 (canonical), X: K x T; returns float64
     (len(rows) or R) x T."""
+    return _spmm("oracle_spmm", 8, values, meta, X, ab_dtype, alpha, beta, Y_in, y_dtype, rows, threads)
+
+
+def spmm12(values: np.ndarray, meta: np.ndarray, X: np.ndarray, ab_dtype: int = F32,
+           alpha: float = 1.0, beta: float = 0.0, Y_in: np.ndarray | None = None,
+           y_dtype: int = F32, rows: np.ndarray | None = None, threads: int | None = None) -> np.ndarray:
+    """fp64 Y = alpha * (W (.) mask) X + beta * Y_in, from the compressed 1:2 form.
+
+    values: R x K/2, meta: R x K/16 (one index bit per pair), X: K x T."""
+    return _spmm("oracle_spmm12", 16, values, meta, X, ab_dtype, alpha, beta, Y_in, y_dtype, rows, threads)
+
+
+def _spmm(fn, meta_div, values, meta, X, ab_dtype, alpha, beta, Y_in, y_dtype, rows, threads):
     vb = _bits(values, ab_dtype)
     xb = _bits(X, ab_dtype)
     R, Kh = vb.shape
@@ -282,11 +324,12 @@ def spmm(values: np.ndarray, meta: np.ndarray, X: np.ndarray, ab_dtype: int,
     nrows = R if rows_arr is None else len(rows_arr)
     out = np.zeros((nrows, T), dtype=np.float64)
     nthr = threads or os.cpu_count() or 1
-    _check(_load().oracle_spmm(vb.ctypes.data, mt.ctypes.data, ab_dtype, xb.ctypes.data, T,
-                               None if ybits is None else ybits.ctypes.data, y_dtype, R, K,
-                               float(alpha), float(beta),
-                               None if rows_arr is None else rows_arr.ctypes.data, nrows,
-                               int(nthr), out.ctypes.data), "spmm")
+    assert mt.size == R * K // meta_div, "metadata size does not match the values"
+    _check(getattr(_load(), fn)(vb.ctypes.data, mt.ctypes.data, ab_dtype, xb.ctypes.data, T,
+                                None if ybits is None else ybits.ctypes.data, y_dtype, R, K,
+                                float(alpha), float(beta),
+                                None if rows_arr is None else rows_arr.ctypes.data, nrows,
+                                int(nthr), out.ctypes.data), fn)
     return out
 
 

@@ -559,21 +559,100 @@ int oracle_meta_sm100(const uint8_t *meta, int64_t R, int64_t C, uint8_t *out)
 }
 
 /* --------------------------------------------------------------------- */
+/* Tensor-core metadata for the int8 sparse MMA (.kind::i8).  [PTX]       */
+/* tcgen05 sparse matrices: an i8 MMA covers 64 logical K per row, 16     */
+/* groups of 4 with the same 4-bit field idx_0 | idx_1 << 2 per group,    */
+/* and its metadata fills two 32-bit tensor-memory columns of the row's   */
+/* own lane, group g at bit 4*(g%8) of column g/8 -- the canonical         */
+/* row-major order of this library's metadata, read as little-endian      */
+/* words.  The image holds, per block of 128 rows x 128 logical K, the    */
+/* 2048 bytes one 128-lane x 128-bit copy moves: lane L = r%128 gets the  */
+/* 16 canonical bytes of row r for those 128 columns.  Blocks are stored   */
+/* row-tile major, block (rt, kt) at byte (rt*nk + kt)*2048 with           */
+/* nk = 2*ceil(C/256) (K is padded to the product's 256-column stage).    */
+/* Padding rows and columns hold the valid pattern (0,1), byte 0x44.      */
+/* --------------------------------------------------------------------- */
+int64_t oracle_meta_sm100_s8_bytes(int64_t R, int64_t C)
+{
+    int64_t Rp = (R + 127) / 128 * 128, Cp = (C + 255) / 256 * 256;
+    return Rp * Cp / 8;
+}
+
+int oracle_meta_sm100_s8(const uint8_t *meta, int64_t R, int64_t C, uint8_t *out)
+{
+    if (C % 8 != 0 || R < 0) return OR_BAD_ARG;
+    int64_t nk = (C + 255) / 256 * 2;
+    memset(out, 0x44, (size_t)oracle_meta_sm100_s8_bytes(R, C));
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t b = 0; b < C / 8; ++b) {      /* canonical byte b: groups 2b, 2b+1 */
+            int64_t rt = r / 128, kt = b / 16;      /* 16 bytes = 128 logical columns */
+            out[(rt * nk + kt) * 2048 + (r % 128) * 16 + (b % 16)] = meta[r * (C / 8) + b];
+        }
+    }
+    return OR_OK;
+}
+
+/* --------------------------------------------------------------------- */
+/* Tensor-core metadata for the 1:2 TF32 sparse MMA (.kind::tf32).  [PTX] */
+/* tcgen05 sparse matrices: a tf32 MMA covers 16 logical K per row (one  */
+/* of each pair kept), and its metadata has the .kind::f16 layout for the */
+/* row seen as 16-bit halves: pair p of 32-bit elements is the group of   */
+/* four halves 4p..4p+3, and its field is 0x4 (halves 0,1: element 0      */
+/* kept) or 0xE (halves 2,3: element 1 kept).  The image is therefore the */
+/* .kind::f16 image above for the R x 2C matrix of halves: per block of   */
+/* 128 rows x 64 fp32 columns, 2048 bytes, lane L = r%8 + 8*((h%32)/16)   */
+/* + 16*((r%128)/16), bits 16*((r%16)/8) + 4*((h%16)/4) of slice          */
+/* (h%128)/32, with h = 4p the pair's first half-column.  Blocks row-tile */
+/* major, block (rt, kt) at byte (rt*ceil(C/64) + kt)*2048; padding pairs */
+/* hold 0x4.                                                               */
+/* --------------------------------------------------------------------- */
+int64_t oracle_meta12_sm100_bytes(int64_t R, int64_t C)
+{
+    return (R + 127) / 128 * ((C + 63) / 64) * 2048;
+}
+
+int oracle_meta12_sm100(const uint8_t *meta, int64_t R, int64_t C, uint8_t *out)
+{
+    if (C % 16 != 0 || R < 0) return OR_BAD_ARG;
+    int64_t Rp = (R + 127) / 128 * 128, Cp = (C + 63) / 64 * 64, kblocks = Cp / 64;
+    memset(out, 0, (size_t)oracle_meta12_sm100_bytes(R, C));
+    for (int64_t r = 0; r < Rp; ++r) {
+        for (int64_t p = 0; p < Cp / 2; ++p) {
+            uint32_t nib = 0x4u;
+            if (r < R && p < C / 2 && ((meta[r * (C / 16) + p / 8] >> (p % 8)) & 1)) nib = 0xEu;
+            int64_t h = 4 * p;                       /* first half-column of the pair */
+            int64_t rt = r / 128, kt = h / 128;
+            int64_t rr = r % 128, hh = h % 128;
+            int64_t lane = (rr % 8) + 8 * ((hh % 32) / 16) + 16 * (rr / 16);
+            int64_t slice = hh / 32;
+            int64_t bit = 16 * ((rr % 16) / 8) + 4 * ((hh % 16) / 4);
+            out[(rt * kblocks + kt) * 2048 + lane * 16 + slice * 4 + bit / 8] |= (uint8_t)(nib << (bit % 8));
+        }
+    }
+    return OR_OK;
+}
+
+/* --------------------------------------------------------------------- */
 /* Sparse x dense product in double.  [ASDNN] "Structured sparse GEMM on  */
 /* tensor cores": sparse matrix x dense matrix = dense matrix; only the  */
 /* kept values are multiplied.                                            */
-/*   Y[r][t] = alpha * sum_k values[r][k] * X[4*(k/2) + idx_k][t]         */
+/*   Y[r][t] = alpha * sum_k values[r][k] * X[col(r, k)][t]               */
 /*             + beta * Y_in[r][t]        (Y_in not read when beta == 0)  */
-/* values/meta in the canonical layout, X is K x T row-major, Y_in R x T  */
-/* row-major (y_dtype).  Only the listed rows are computed (rows == NULL  */
-/* means all R rows); Y_out is nrows x T doubles.                          */
+/* 2:4 (oracle_spmm): col(r, k) = 4*(k/2) + idx_k from the canonical 2:4  */
+/* metadata.  1:2 (oracle_spmm12): col(r, k) = 2*k + idx_k from the 1:2    */
+/* metadata (one index bit per pair).  X is K x T row-major, Y_in R x T    */
+/* row-major (y_dtype).  Floating-point inputs are decoded exactly and     */
+/* summed in double.  int8 inputs (OR_S8) are summed exactly in int64      */
+/* (every product is an integer of magnitude <= 2^14) and the sum is then  */
+/* exact in double for |sum| < 2^53.  Only the listed rows are computed    */
+/* (rows == NULL means all R rows); Y_out is nrows x T doubles.            */
 /* --------------------------------------------------------------------- */
 typedef struct {
     const void *values; const uint8_t *meta; int ab_dtype;
     const void *X; int64_t T; const void *Y_in; int y_dtype;
     int64_t R, K; double alpha, beta;
     const int64_t *rows; int64_t nrows; double *Y_out;
-    int64_t lo, hi;
+    int64_t lo, hi; int pattern;   /* 24: 2:4 metadata, 12: 1:2 metadata */
 } spmm_job;
 
 /* exact decode of one element to double: a 65536-entry table for the
@@ -600,37 +679,59 @@ static double decode_fast(const void *base, int dtype, size_t i)
     return g_tab[dtype][((const uint16_t *)base)[i]];
 }
 
+/* logical column of kept value k of row r */
+static int64_t kept_column(const spmm_job *j, int64_t r, int64_t k)
+{
+    if (j->pattern == 12) {
+        int idx = (j->meta[r * (j->K / 16) + k / 8] >> (k % 8)) & 1;
+        return 2 * k + idx;
+    }
+    int idx = (j->meta[r * (j->K / 8) + k / 4] >> (2 * (k % 4))) & 3;
+    return 4 * (k / 2) + idx;
+}
+
 static void *spmm_worker(void *arg)
 {
     spmm_job *j = (spmm_job *)arg;
-    double *acc = (double *)malloc(sizeof(double) * (size_t)(j->T > 0 ? j->T : 1));
+    size_t n = (size_t)(j->T > 0 ? j->T : 1);
+    double *acc = (double *)malloc(sizeof(double) * n);
+    int64_t *iacc = (int64_t *)malloc(sizeof(int64_t) * n);
+    const int ints = j->ab_dtype == OR_S8;
     for (int64_t i = j->lo; i < j->hi; ++i) {
         int64_t r = j->rows ? j->rows[i] : i;
-        for (int64_t t = 0; t < j->T; ++t) acc[t] = 0.0;
+        for (int64_t t = 0; t < j->T; ++t) { acc[t] = 0.0; iacc[t] = 0; }
         for (int64_t k = 0; k < j->K / 2; ++k) {
-            int idx = (j->meta[r * (j->K / 8) + k / 4] >> (2 * (k % 4))) & 3;
-            int64_t kk = 4 * (k / 2) + idx;            /* logical column of this value */
-            double v = decode_fast(j->values, j->ab_dtype, (size_t)(r * (j->K / 2) + k));
-            for (int64_t t = 0; t < j->T; ++t)
-                acc[t] += v * decode_fast(j->X, j->ab_dtype, (size_t)(kk * j->T + t));
+            int64_t kk = kept_column(j, r, k);
+            size_t vi = (size_t)(r * (j->K / 2) + k);
+            if (ints) {
+                int64_t v = s8_value(((const uint8_t *)j->values)[vi]);
+                const uint8_t *xrow = (const uint8_t *)j->X + kk * j->T;
+                for (int64_t t = 0; t < j->T; ++t) iacc[t] += v * s8_value(xrow[t]);
+            } else {
+                double v = decode_fast(j->values, j->ab_dtype, vi);
+                for (int64_t t = 0; t < j->T; ++t)
+                    acc[t] += v * decode_fast(j->X, j->ab_dtype, (size_t)(kk * j->T + t));
+            }
         }
         for (int64_t t = 0; t < j->T; ++t) {
-            double y = j->alpha * acc[t];
+            double sum = ints ? (double)iacc[t] : acc[t];
+            double y = j->alpha * sum;
             if (j->beta != 0.0)
                 y += j->beta * decode_fast(j->Y_in, j->y_dtype, (size_t)(r * j->T + t));
             j->Y_out[i * j->T + t] = y;
         }
     }
     free(acc);
+    free(iacc);
     return NULL;
 }
 
-int oracle_spmm(const void *values, const uint8_t *meta, int ab_dtype,
-                const void *X, int64_t T, const void *Y_in, int y_dtype,
-                int64_t R, int64_t K, double alpha, double beta,
-                const int64_t *rows, int64_t nrows, int nthreads, double *Y_out)
+static int spmm_run(int pattern, const void *values, const uint8_t *meta, int ab_dtype,
+                    const void *X, int64_t T, const void *Y_in, int y_dtype,
+                    int64_t R, int64_t K, double alpha, double beta,
+                    const int64_t *rows, int64_t nrows, int nthreads, double *Y_out)
 {
-    if (K % 8 != 0 || R < 0 || T < 0) return OR_BAD_ARG;
+    if (K % (pattern == 12 ? 16 : 8) != 0 || R < 0 || T < 0) return OR_BAD_ARG;
     if (rows == NULL) nrows = R;
     for (int64_t i = 0; rows && i < nrows; ++i) if (rows[i] < 0 || rows[i] >= R) return OR_BAD_ARG;
     pthread_once(&g_tab_once, build_tables);
@@ -641,13 +742,31 @@ int oracle_spmm(const void *values, const uint8_t *meta, int ab_dtype,
     pthread_t th[256];
     for (int i = 0; i < nthreads; ++i) {
         spmm_job j = { values, meta, ab_dtype, X, T, Y_in, y_dtype, R, K, alpha, beta,
-                       rows, nrows, Y_out, nrows * i / nthreads, nrows * (i + 1) / nthreads };
+                       rows, nrows, Y_out, nrows * i / nthreads, nrows * (i + 1) / nthreads, pattern };
         jobs[i] = j;
     }
     if (nthreads == 1) { spmm_worker(&jobs[0]); return OR_OK; }
     for (int i = 0; i < nthreads; ++i) pthread_create(&th[i], NULL, spmm_worker, &jobs[i]);
     for (int i = 0; i < nthreads; ++i) pthread_join(th[i], NULL);
     return OR_OK;
+}
+
+int oracle_spmm(const void *values, const uint8_t *meta, int ab_dtype,
+                const void *X, int64_t T, const void *Y_in, int y_dtype,
+                int64_t R, int64_t K, double alpha, double beta,
+                const int64_t *rows, int64_t nrows, int nthreads, double *Y_out)
+{
+    return spmm_run(24, values, meta, ab_dtype, X, T, Y_in, y_dtype, R, K, alpha, beta, rows, nrows,
+                    nthreads, Y_out);
+}
+
+int oracle_spmm12(const void *values, const uint8_t *meta, int ab_dtype,
+                  const void *X, int64_t T, const void *Y_in, int y_dtype,
+                  int64_t R, int64_t K, double alpha, double beta,
+                  const int64_t *rows, int64_t nrows, int nthreads, double *Y_out)
+{
+    return spmm_run(12, values, meta, ab_dtype, X, T, Y_in, y_dtype, R, K, alpha, beta, rows, nrows,
+                    nthreads, Y_out);
 }
 
 /* --------------------------------------------------------------------- */
