@@ -72,10 +72,11 @@ typedef enum {
 
 /* NM_S8: two's-complement int8 weights, magnitude |x| (so -128 ranks above 127).
  * Accepted by nm_sizes, nm_mask, nm_mask_transposable, nm_mask_compress,
- * nm_compress and nm_decompress; the int8 sparse product is not built (nm_spmm
- * returns NM_ERR_UNSUPPORTED for it) and the floating-point calls
- * (nm_mask_scored, nm_srste_step, the 1:2 calls) return NM_ERR_DTYPE. */
-typedef enum { NM_F32 = 0, NM_BF16 = 1, NM_F16 = 2, NM_S8 = 3 } nm_dtype;
+ * nm_compress, nm_decompress, nm_meta_to_sm100_s8 and nm_spmm (the int8 2:4
+ * product); the floating-point calls (nm_mask_scored, nm_srste_step, the 1:2
+ * calls) return NM_ERR_DTYPE.
+ * NM_S32: two's-complement int32, only as the output of the int8 product. */
+typedef enum { NM_F32 = 0, NM_BF16 = 1, NM_F16 = 2, NM_S8 = 3, NM_S32 = 4 } nm_dtype;
 
 /* Human-readable text for a status code (static string, never NULL). */
 NM_API const char *nm_status_string(int status);
@@ -247,6 +248,40 @@ NM_API nm_status nm_meta_to_sm100(const uint8_t *meta, int64_t R, int64_t C, uin
                            void *stream);
 
 /*
+ * nm_meta_to_sm100_s8 -- canonical 2:4 metadata of an int8 matrix (R x C/8
+ * bytes) -> the tensor-core metadata image the int8 product reads
+ * (.kind::i8; PTX ISA, tcgen05 sparse matrices: an int8 instruction covers 64
+ * logical columns and reads their 16 group fields from two 32-bit columns of
+ * the row's own lane, in the canonical order).  Layout: per block of 128 rows
+ * x 128 logical columns, 2048 bytes, lane L = r%128 holding the 16 canonical
+ * bytes of row r for those columns; blocks row-tile major, block (rt, kt) at
+ * byte (rt*nk + kt)*2048 with nk = 2*ceil(C/256); padding rows and columns
+ * hold the pattern (0,1), byte 0x44.  Size: nm_meta_s8_image_bytes(R, C)
+ * = ceil(R/128)*128 * ceil(C/256)*256 / 8.  C % 8 == 0 (else NM_ERR_SHAPE);
+ * meta_s8_sm100 16-byte aligned (else NM_ERR_ALIGN).
+ */
+NM_API size_t nm_meta_s8_image_bytes(int64_t R, int64_t C);
+NM_API nm_status nm_meta_to_sm100_s8(const uint8_t *meta, int64_t R, int64_t C, uint8_t *meta_s8_sm100,
+                                     void *stream);
+
+/*
+ * nm_meta12_to_sm100 -- canonical 1:2 metadata (R x C/16 bytes, from
+ * nm_mask_compress12 / nm_compress12) -> the tensor-core metadata image the
+ * TF32 1:2 product reads (.kind::tf32; PTX ISA, tcgen05 sparse matrices: the
+ * .kind::f16 layout of the row seen as 16-bit halves, pair p being the group
+ * of halves 4p..4p+3 with field 0x4 when element 0 is kept and 0xE when
+ * element 1 is).  Layout: per block of 128 rows x 64 fp32 columns, 2048
+ * bytes; lane L = r%8 + 8*((h%32)/16) + 16*((r%128)/16), bit
+ * 16*((r%16)/8) + 4*((h%16)/4) of the 32-bit slice (h%128)/32, h = 4p; blocks
+ * row-tile major, (rt, kt) at byte (rt*ceil(C/64) + kt)*2048; padding pairs
+ * hold 0x4.  Size: nm_meta12_image_bytes(R, C) = ceil(R/128)*ceil(C/64)*2048.
+ * C % 16 == 0 (else NM_ERR_SHAPE); meta12_sm100 16-byte aligned.
+ */
+NM_API size_t nm_meta12_image_bytes(int64_t R, int64_t C);
+NM_API nm_status nm_meta12_to_sm100(const uint8_t *meta, int64_t R, int64_t C, uint8_t *meta12_sm100,
+                                    void *stream);
+
+/*
  * nm_srste_step -- one SR-STE training step, fused ("SR-STE sparse training",
  * SR-STE forward and backward): the N:M magnitude mask of W is recomputed
  * (same rule as nm_mask), and
@@ -287,13 +322,21 @@ NM_API size_t nm_spmm_workspace_bytes(nm_dtype ab_dtype, int64_t R, int64_t K, i
  *              read only when beta != 0.  Y needs only element alignment;
  *              16-byte aligned Y and ldy get vector stores
  *   X, values, meta_sm100: 16-byte aligned; ldx * element size % 16 == 0
- *   ab_dtype   NM_BF16 or NM_F16 (tensor-core path), or NM_F32 (rounded to
+ *   ab_dtype   NM_BF16 or NM_F16 (tensor-core path), NM_S8 (the int8 2:4
+ *              tensor-core path, below), or NM_F32 (rounded to
  *              binary16 in `workspace`, then the binary16 path; binary16
  *              holds magnitudes up to 65504 and normal values down to
  *              6.1e-5, so larger fp32 inputs become +-Inf and values below
  *              about 6e-8 become zero -- scale such data first)
  *   K % 16 == 0 (the pages' rule for 16-bit sparse operands); R, T >= 1 any
  *   workspace  >= nm_spmm_workspace_bytes(...) bytes (may be NULL when 0)
+ * int8 (ab_dtype NM_S8; review, "Structured sparse GEMM on tensor cores":
+ * INT8 at 2:4, dimensions multiples of 32): values and X int8, meta_sm100 the
+ * .kind::i8 image of nm_meta_to_sm100_s8 (NOT the nm_meta_to_sm100 image),
+ * K % 32 == 0, exact s32 accumulation.  y_dtype NM_S32 stores the exact sum
+ * (requires alpha == 1 and beta == 0, else NM_ERR_UNSUPPORTED; no overflow
+ * while K <= 262144, since |sum| <= K/2 * 2^14); NM_F32 / NM_BF16 store
+ * alpha * float(sum) + beta * Y (the conversion of sums beyond 2^24 rounds).
  * A bounded wait inside the kernel that gives up records NM_ERR_TIMEOUT in a
  * device status word, read and cleared by nm_last_device_status().
  */
@@ -301,6 +344,23 @@ NM_API nm_status nm_spmm(const void *values, const uint8_t *meta_sm100, nm_dtype
                   const void *X, int64_t ldx, void *Y, nm_dtype y_dtype, int64_t ldy,
                   int64_t R, int64_t K, int64_t T, float alpha, float beta,
                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * nm_spmm12 -- Y = alpha * (W (.) mask) X + beta * Y for a 1:2-sparse fp32 W
+ * on the TF32 sparse tensor cores (review of "Accelerating Sparse Deep Neural
+ * Networks", "Structured sparse GEMM on tensor cores": sparse TF32 only with
+ * the 1:2 pattern), fp32 accumulation.
+ *   values       R x K/2 fp32, the kept element of each pair (nm_mask_compress12
+ *                / nm_compress12), row stride K/2
+ *   meta12_sm100 the .kind::tf32 image of the 1:2 metadata (nm_meta12_to_sm100)
+ *   X            K x T fp32, leading dim ldx >= T, ldx % 4 == 0
+ *   Y            R x T, y_dtype NM_F32 or NM_BF16, leading dim ldy >= T
+ *   K % 16 == 0; R, T any.  The tensor cores read values and X as TF32 (10
+ *   fraction bits), so results carry that precision.  Errors as nm_spmm.
+ */
+NM_API nm_status nm_spmm12(const float *values, const uint8_t *meta12_sm100, const float *X, int64_t ldx,
+                           void *Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T,
+                           float alpha, float beta, void *stream);
 
 /*
  * nm_spmm_noalloc -- nm_spmm that allocates nothing and takes no workspace.

@@ -35,7 +35,10 @@ enum {
  * nm_spmm_test -- nm_spmm (same arguments, same results, same errors) with
  * four hooks:
  *   kernel         NM_SPMM_KERNEL_*; a CTA-pair kernel asked for on an odd
- *                  number of 128-row tiles falls back to the default choice.
+ *                  number of 128-row tiles falls back to the default choice;
+ *                  for int8 operands the 192- and 128-column pair kernels
+ *                  become the 256-column one, and for int8 and tf32 operands
+ *                  the 16-column kernel the 32-column one.
  *                  Every tile configuration computes the same sums in the same
  *                  order per output, so results do not depend on it.
  *   tail_split     1: a last wave that fills at most half of the CTA pairs is
@@ -60,6 +63,14 @@ NM_API nm_status nm_spmm_test(const void *values, const uint8_t *meta_sm100, nm_
                               void *workspace, size_t workspace_bytes,
                               int kernel, int tail_split, int64_t wait_limit_ns, int64_t skip_step,
                               void *stream);
+
+/*
+ * nm_spmm12_test -- nm_spmm12 with a forced tile configuration (`kernel`, as
+ * above) and the half-width last wave on (1) or off (0).
+ */
+NM_API nm_status nm_spmm12_test(const float *values, const uint8_t *meta12_sm100, const float *X, int64_t ldx,
+                                void *Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T,
+                                float alpha, float beta, int kernel, int tail_split, void *stream);
 
 #ifdef __cplusplus
 }

@@ -26,8 +26,12 @@ linear/conv weights; the pages' datasets and trained weights are not used):
                       of the same shape (seed 6)
 * ``int8_decode``     the decode_skinny weight quantised to int8:
                       clamp(round(w / 0.02 * 32), -128, 127)
+* ``decode_X_int8``   the decode_skinny X (8192xT, seed 105+T) quantised to
+                      int8: clamp(round(x * 32), -128, 127), the int8 product's
+                      activations
 * ``fp32_linear``     W fp32 8192x8192 = fp32(0.02 * N(0,1)) (seed 8), for the
-                      1:2 pattern of sparse TF32
+                      1:2 pattern of sparse TF32; X fp32 8192xT ~N(0,1)
+                      (seed 109), the TF32 product's activations
 * ``saliency``        the linear_4096 weight and d of length 4096: the diagonal
                       of the upper Cholesky factor of H^-1, H = (2/n) X^T X +
                       0.01 * mean(diag) * I from n = 512 synthetic calibration
@@ -50,6 +54,7 @@ SEEDS = {
     "fp32_linear.W": 8,
     "linear_4096.dY": 103,
     "mlp_pair.H": 104,
+    "fp32_linear.X": 109,
 }
 
 
@@ -146,3 +151,17 @@ def fp32_linear(R: int = 8192, C: int = 8192) -> torch.Tensor:
 def int8_decode() -> torch.Tensor:
     w = decode_skinny_W().float()
     return torch.clamp(torch.round(w / 0.02 * 32), -128, 127).to(torch.int8)
+
+
+def decode_X_int8(T: int) -> torch.Tensor:
+    x = decode_skinny_X(T).float()
+    return torch.clamp(torch.round(x * 32), -128, 127).to(torch.int8)
+
+
+def fp32_linear_X(T: int = 4096, K: int = 8192) -> torch.Tensor:
+    return normal((K, T), SEEDS["fp32_linear.X"], 1.0, torch.float32)
+
+
+def small_int8(shape, seed: int, lo: int = -128, hi: int = 127) -> torch.Tensor:
+    """int8 values uniform on the integers lo..hi."""
+    return torch.randint(lo, hi + 1, shape, generator=_gen(seed), dtype=torch.int64).to(torch.int8)

@@ -7,7 +7,8 @@ straight through, and a non-zero status raises ``NMError``.  There is no CPU
 fallback: if ``libnm.so`` is missing or fails to load, every call raises.
 
 Element types: torch.float32 -> NM_F32, torch.bfloat16 -> NM_BF16,
-torch.float16 -> NM_F16.
+torch.float16 -> NM_F16, torch.int8 -> NM_S8, torch.int32 -> NM_S32 (the
+int8 product's exact output).
 """
 from __future__ import annotations
 
@@ -19,10 +20,11 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnm.so")
 
-NM_F32, NM_BF16, NM_F16, NM_S8 = 0, 1, 2, 3
+NM_F32, NM_BF16, NM_F16, NM_S8, NM_S32 = 0, 1, 2, 3, 4
 STATUS = ["NM_OK", "NM_ERR_NULL", "NM_ERR_SHAPE", "NM_ERR_ALIGN", "NM_ERR_DTYPE", "NM_ERR_NM",
           "NM_ERR_UNSUPPORTED", "NM_ERR_CUDA", "NM_ERR_WORKSPACE", "NM_ERR_TIMEOUT"]
-_DT = {torch.float32: NM_F32, torch.bfloat16: NM_BF16, torch.float16: NM_F16, torch.int8: NM_S8}
+_DT = {torch.float32: NM_F32, torch.bfloat16: NM_BF16, torch.float16: NM_F16, torch.int8: NM_S8,
+       torch.int32: NM_S32}
 
 
 class NMError(RuntimeError):
@@ -57,6 +59,12 @@ def _lib():
         "nm_compress_t": ([vp, vp, i32, i64, i64, i64, i64, vp, vp, vp, vp, vp], i32),
         "nm_decompress": ([vp, vp, i32, i64, i64, vp, i64, vp], i32),
         "nm_meta_to_sm100": ([vp, i64, i64, vp, vp], i32),
+        "nm_meta_s8_image_bytes": ([i64, i64], sz),
+        "nm_meta_to_sm100_s8": ([vp, i64, i64, vp, vp], i32),
+        "nm_meta12_image_bytes": ([i64, i64], sz),
+        "nm_meta12_to_sm100": ([vp, i64, i64, vp, vp], i32),
+        "nm_spmm12": ([vp, vp, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp], i32),
+        "nm_spmm12_test": ([vp, vp, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, i32, i32, vp], i32),
         "nm_spmm_workspace_bytes": ([i32, i64, i64, i64], sz),
         "nm_spmm": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp, sz, vp], i32),
         "nm_spmm_noalloc": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp], i32),
@@ -248,6 +256,22 @@ def nm_meta_to_sm100(meta: torch.Tensor, R: int, C: int, out: torch.Tensor | Non
     return out
 
 
+def nm_meta_to_sm100_s8(meta: torch.Tensor, R: int, C: int, out: torch.Tensor | None = None, stream=None):
+    """Canonical 2:4 metadata of an int8 matrix -> the image the int8 product reads."""
+    if out is None:
+        out = torch.empty((int(_lib().nm_meta_s8_image_bytes(R, C)),), dtype=torch.uint8, device=meta.device)
+    _check(_lib().nm_meta_to_sm100_s8(_ptr(meta), R, C, _ptr(out), _stream(stream)), "nm_meta_to_sm100_s8")
+    return out
+
+
+def nm_meta12_to_sm100(meta: torch.Tensor, R: int, C: int, out: torch.Tensor | None = None, stream=None):
+    """Canonical 1:2 metadata -> the image the TF32 1:2 product reads."""
+    if out is None:
+        out = torch.empty((int(_lib().nm_meta12_image_bytes(R, C)),), dtype=torch.uint8, device=meta.device)
+    _check(_lib().nm_meta12_to_sm100(_ptr(meta), R, C, _ptr(out), _stream(stream)), "nm_meta12_to_sm100")
+    return out
+
+
 def nm_spmm_workspace_bytes(ab_dtype: torch.dtype, R: int, K: int, T: int) -> int:
     return int(_lib().nm_spmm_workspace_bytes(_DT[ab_dtype], R, K, T))
 
@@ -255,7 +279,9 @@ def nm_spmm_workspace_bytes(ab_dtype: torch.dtype, R: int, K: int, T: int) -> in
 def nm_spmm(values: torch.Tensor, meta_sm100: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = None,
             y_dtype: torch.dtype = torch.bfloat16, alpha: float = 1.0, beta: float = 0.0,
             workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """Y = alpha * (W (.) mask) X + beta * Y from the compressed W (values, meta_sm100)."""
+    """Y = alpha * (W (.) mask) X + beta * Y from the compressed W (values, meta_sm100).
+    int8 values and X take the .kind::i8 image (nm_meta_to_sm100_s8) and may
+    write torch.int32 (the exact sum)."""
     R, Kh = values.shape
     K = 2 * Kh
     Kx, T = X.shape
@@ -298,6 +324,29 @@ def nm_spmm_test(values: torch.Tensor, meta_sm100: torch.Tensor, X: torch.Tensor
                                _ld(Y), R, K, T, float(alpha), float(beta), _ptr(workspace), ws_bytes,
                                SPMM_KERNELS[kernel], 1 if tail_split else 0, int(wait_limit_ns), int(skip_step),
                                _stream(stream)), "nm_spmm_test")
+    return Y
+
+
+def nm_spmm12(values: torch.Tensor, meta12_sm100: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = None,
+              y_dtype: torch.dtype = torch.float32, alpha: float = 1.0, beta: float = 0.0, kernel: str | None = None,
+              tail_split: bool = True, stream=None) -> torch.Tensor:
+    """Y = alpha * (W (.) mask) X + beta * Y for a 1:2-sparse fp32 W (values R x K/2,
+    the nm_meta12_to_sm100 image) on the TF32 sparse tensor cores.  `kernel` /
+    `tail_split` go through the test entry point."""
+    R, Kh = values.shape
+    K = 2 * Kh
+    Kx, T = X.shape
+    assert Kx == K, "X must be K x T"
+    if Y is None:
+        Y = torch.empty((R, T), dtype=y_dtype, device=values.device)
+    lib = _lib()
+    args = (_ptr(values), _ptr(meta12_sm100), _ptr(X), _ld(X), _ptr(Y), _dtype(Y), _ld(Y), R, K, T, float(alpha),
+            float(beta))
+    if kernel is None and tail_split:
+        _check(lib.nm_spmm12(*args, _stream(stream)), "nm_spmm12")
+    else:
+        _check(lib.nm_spmm12_test(*args, SPMM_KERNELS[kernel or "default"], 1 if tail_split else 0,
+                                  _stream(stream)), "nm_spmm12_test")
     return Y
 
 

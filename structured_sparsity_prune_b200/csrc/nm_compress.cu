@@ -972,3 +972,63 @@ extern "C" nm_status nm_meta_to_sm100(const uint8_t* meta, int64_t R, int64_t C,
   }
   return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// 2:4 metadata image for the int8 sparse MMA (.kind::i8; PTX ISA, tcgen05
+// sparse matrices).  An i8 instruction covers 64 logical K of a row and reads
+// its 16 group fields from two 32-bit tensor-memory columns of the row's own
+// lane, group g at bit 4*(g%8) of column g/8: the canonical row-major order.
+// The image holds, per block of 128 rows x 128 logical columns, the 2048 bytes
+// one 128-lane x 128-bit copy moves: lane L gets the 16 canonical bytes of row
+// 128*rt + L for those columns.  Blocks are row-tile major with
+// nk = 2 * ceil(C / 256) per row tile (the product's stage is 256 columns);
+// padding holds the pattern (0,1), byte 0x44.  One thread per lane row.
+namespace nm {
+namespace {
+
+__global__ void __launch_bounds__(256) meta_image_s8_kernel(const uint8_t* __restrict__ meta, int64_t R, int64_t C,
+                                                            int64_t nk, int64_t nrows16, uint4* __restrict__ out) {
+  const int64_t bpr = C / 8;  // canonical bytes per row
+  const bool rows_vec = (bpr % 16) == 0 && (reinterpret_cast<uintptr_t>(meta) & 15u) == 0;
+  for (int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; t < nrows16;
+       t += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t blk = t >> 7;
+    const int64_t rt = blk / nk, kb = blk - rt * nk;
+    const int64_t r = rt * 128 + (t & 127);
+    const int64_t b0 = kb * 16;
+    uint4 v = make_uint4(0x44444444u, 0x44444444u, 0x44444444u, 0x44444444u);
+    if (r < R && b0 < bpr) {
+      const uint8_t* src = meta + r * bpr + b0;
+      if (rows_vec) {
+        v = __ldg(reinterpret_cast<const uint4*>(src));
+      } else {
+        uint8_t* vb = reinterpret_cast<uint8_t*>(&v);
+        for (int j = 0; j < 16 && b0 + j < bpr; ++j) vb[j] = src[j];
+      }
+    }
+    out[t] = v;
+  }
+}
+
+}  // namespace
+}  // namespace nm
+
+extern "C" size_t nm_meta_s8_image_bytes(int64_t R, int64_t C) {
+  if (R <= 0 || C <= 0) return 0;
+  return size_t((R + 127) / 128) * 128 * size_t((C + 255) / 256) * 256 / 8;
+}
+
+extern "C" nm_status nm_meta_to_sm100_s8(const uint8_t* meta, int64_t R, int64_t C, uint8_t* meta_s8_sm100,
+                                         void* stream) {
+  using namespace nm;
+  if (R < 0 || C < 0 || C % 8 != 0) return NM_ERR_SHAPE;
+  if (R == 0 || C == 0) return NM_OK;
+  if (meta == nullptr || meta_s8_sm100 == nullptr) return NM_ERR_NULL;
+  if (!aligned16(meta_s8_sm100)) return NM_ERR_ALIGN;
+  const int64_t nk = (C + 255) / 256 * 2;
+  const int64_t rows16 = (R + 127) / 128 * nk * 128;
+  const int64_t want = (rows16 + 255) / 256, cap = int64_t(sm_count()) * 8;
+  meta_image_s8_kernel<<<unsigned(want < cap ? want : cap), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      meta, R, C, nk, rows16, reinterpret_cast<uint4*>(meta_s8_sm100));
+  return launch_status();
+}

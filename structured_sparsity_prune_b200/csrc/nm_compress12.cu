@@ -250,3 +250,68 @@ extern "C" nm_status nm_decompress12(const void* values, const uint8_t* meta, nm
                                                        static_cast<uint16_t*>(W_out), ldw);
   return launch_status();
 }
+
+// ---------------------------------------------------------------------------
+// 1:2 metadata image for the .kind::tf32 sparse MMA (PTX ISA, tcgen05 sparse
+// matrices).  A tf32 instruction reads its metadata in the .kind::f16 layout
+// of the row seen as 16-bit halves: pair p (fp32 columns 2p, 2p+1) is the
+// group of halves 4p..4p+3, whose 4-bit field is 0x4 when element 0 is kept
+// and 0xE when element 1 is.  Per block of 128 rows x 64 fp32 columns the
+// image holds the 2048 bytes one 128-lane x 128-bit copy moves into tensor
+// memory: lane L, 32-bit slice s, field at bit 16*h8 + 4*q holds row
+// 16*(L/16) + 8*h8 + L%8 and half-column 32*s + 16*((L/8)%2) + 4*q.  Blocks are
+// row-tile major; padding rows and pairs hold 0x4.  One thread per lane row
+// (16 bytes) of a block.
+namespace nm {
+namespace {
+
+__global__ void __launch_bounds__(256) meta12_image_kernel(const uint8_t* __restrict__ meta, int64_t R, int64_t C,
+                                                           int64_t kblocks, int64_t nrows16,
+                                                           uint4* __restrict__ out) {
+  const int64_t bpr = C / 16;  // metadata bytes per row
+  for (int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; t < nrows16;
+       t += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t blk = t >> 7;
+    const int L = int(t & 127);
+    const int64_t rt = blk / kblocks, kt = blk - rt * kblocks;
+    uint32_t w[4];
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        const int h8 = n >> 2, q = n & 3;
+        const int64_t r = rt * 128 + 16 * (L >> 4) + 8 * h8 + (L & 7);
+        const int64_t p = kt * 32 + (32 * sl + 16 * ((L >> 3) & 1) + 4 * q) / 4;
+        uint32_t nib = 0x4u;
+        if (r < R && p < C / 2 && ((meta[r * bpr + (p >> 3)] >> (p & 7)) & 1u)) nib = 0xEu;
+        word |= nib << (16 * h8 + 4 * q);
+      }
+      w[sl] = word;
+    }
+    out[t] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+}  // namespace
+}  // namespace nm
+
+extern "C" size_t nm_meta12_image_bytes(int64_t R, int64_t C) {
+  if (R <= 0 || C <= 0) return 0;
+  return size_t((R + 127) / 128) * size_t((C + 63) / 64) * 2048;
+}
+
+extern "C" nm_status nm_meta12_to_sm100(const uint8_t* meta, int64_t R, int64_t C, uint8_t* meta12_sm100,
+                                        void* stream) {
+  using namespace nm;
+  if (R < 0 || C < 0 || C % 16 != 0) return NM_ERR_SHAPE;
+  if (R == 0 || C == 0) return NM_OK;
+  if (meta == nullptr || meta12_sm100 == nullptr) return NM_ERR_NULL;
+  if (!aligned16(meta12_sm100)) return NM_ERR_ALIGN;
+  const int64_t kblocks = (C + 63) / 64;
+  const int64_t rows16 = (R + 127) / 128 * kblocks * 128;
+  const int64_t want = (rows16 + 255) / 256, cap = int64_t(sm_count()) * 8;
+  meta12_image_kernel<<<unsigned(want < cap ? want : cap), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      meta, R, C, kblocks, rows16, reinterpret_cast<uint4*>(meta12_sm100));
+  return launch_status();
+}

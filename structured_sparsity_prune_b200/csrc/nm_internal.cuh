@@ -16,7 +16,7 @@ namespace nm {
 // ----------------------------------------------------------------- host side
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool stride_ok(int64_t ld_elems, int esize) { return ((ld_elems * esize) & 15) == 0; }
-inline int esize_of(nm_dtype d) { return d == NM_F32 ? 4 : (d == NM_S8 ? 1 : 2); }
+inline int esize_of(nm_dtype d) { return (d == NM_F32 || d == NM_S32) ? 4 : (d == NM_S8 ? 1 : 2); }
 // floating-point element types
 inline bool dtype_ok(int d) { return d == NM_F32 || d == NM_BF16 || d == NM_F16; }
 // ... plus int8, for the calls that only select, move and pack elements

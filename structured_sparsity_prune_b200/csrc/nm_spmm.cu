@@ -44,9 +44,37 @@ __device__ int g_device_status = 0;
 namespace spmm {
 
 constexpr int kBlockM = 128;     // rows of W per tile = TMEM lanes
-constexpr int kStageK = 128;     // logical K per pipeline stage
-constexpr int kStageKPhys = 64;  // compressed values per row per stage (128 B)
-constexpr int kMmaK = 32;        // logical K per sparse MMA instruction
+
+// Operand kinds of the sparse MMA.  Every kind moves 128 bytes of compressed
+// A per row per pipeline stage and 32 bytes per instruction, so the A tile,
+// its swizzle and its descriptor walk are shared; what differs is the logical
+// K those bytes cover, the instruction's kind and formats, and the metadata:
+//   F16 / BF16  2:4, 16-bit, 32 logical K per MMA, one 2 KB image block per
+//               stage (.kind::f16, one tensor-memory column per MMA);
+//   TF32        1:2, 32-bit, 16 logical K per MMA, one 2 KB block per stage
+//               (.kind::tf32: the .kind::f16 layout over 16-bit halves);
+//   S8          2:4, int8, 64 logical K per MMA, two 2 KB blocks per stage
+//               (.kind::i8: two columns per MMA, canonical row order);
+//               s32 accumulation.
+enum class Kind : int { F16 = 0, BF16 = 1, TF32 = 2, S8 = 3 };
+
+template <Kind KD>
+struct KT {
+  static constexpr int kEsize = KD == Kind::TF32 ? 4 : KD == Kind::S8 ? 1 : 2;
+  static constexpr int kStageK = KD == Kind::TF32 ? 64 : KD == Kind::S8 ? 256 : 128;  // logical K per stage
+  static constexpr int kMmaK = kStageK / 4;            // logical K per instruction (4 per stage)
+  static constexpr int kStageKPhys = 128 / kEsize;     // compressed values per row per stage (128 B)
+  static constexpr int kAtomCols = 128 / kEsize;       // X columns in one 128-byte swizzle row
+  static constexpr int kEBytes = KD == Kind::S8 ? 4096 : 2048;  // metadata image bytes per stage
+  static constexpr int kECols = kEBytes / 512;         // tensor-memory columns they fill (128 lanes x 4 B)
+  static constexpr bool kAccS32 = KD == Kind::S8;
+  // X (the MN-major B operand) of a tf32 instruction must sit in the 128-byte
+  // swizzle with 32-byte atoms (rows of 128 bytes, 32-byte granules XORed with
+  // the row index mod 4, so the pattern repeats every 4 rows): descriptor
+  // layout type 1, TMA swizzle 128B_ATOM_32B.  The other kinds use the usual
+  // swizzles with 16-byte granules.
+  static constexpr bool kB32Atom = KD == Kind::TF32;
+};
 constexpr int kThreads = 192;    // 6 warps (single-CTA kernel)
 constexpr int kPairThreads = 320;  // 10 warps: producer, MMA, 8 epilogue warps (CTA-pair kernel)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
@@ -143,20 +171,37 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
   d |= uint64_t(layout & 7u) << 61;
   return d;
 }
-constexpr uint32_t kLayoutNone = 0, kLayoutSW128 = 2, kLayoutSW64 = 4, kLayoutSW32 = 6;
+constexpr uint32_t kLayoutNone = 0, kLayoutSW128_32B = 1, kLayoutSW128 = 2, kLayoutSW64 = 4, kLayoutSW32 = 6;
 
 __device__ __forceinline__ void tmem_cp_128x128b(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+template <Kind KD>
 __device__ __forceinline__ void mma_sp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t e_tmem,
                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if constexpr (KD == Kind::TF32) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::tf32 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else if constexpr (KD == Kind::S8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::1.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -244,14 +289,31 @@ __device__ __forceinline__ void tmem_cp_pair_128x128b(uint32_t taddr, uint64_t s
   asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+template <Kind KD>
 __device__ __forceinline__ void mma_sp_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t e_tmem,
                                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
-      : "memory");
+  if constexpr (KD == Kind::TF32) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::tf32 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else if constexpr (KD == Kind::S8) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::i8 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::f16 [%0], %1, %2, [%3], %4, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(e_tmem), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
 }
 
 // completion of this thread's earlier tcgen05 ops arrives on the mbarrier at
@@ -290,45 +352,75 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Instruction descriptor, .kind::f16 with sparsity: D fp32, A/B fp16 or bf16,
-// A K-major, B N-major (X is K x T with T contiguous), M = 128, N = n.
-__host__ __device__ constexpr uint32_t make_idesc(bool bf16, int n, int m = kBlockM) {
-  return (1u << 2)                    // sparse
-         | (1u << 4)                  // D format fp32
-         | ((bf16 ? 1u : 0u) << 7)    // A format
-         | ((bf16 ? 1u : 0u) << 10)   // B format
-         | (0u << 15)                 // A K-major
-         | (1u << 16)                 // B MN-major
-         | (uint32_t(n >> 3) << 17)   // N / 8
-         | (uint32_t(m >> 4) << 24);  // M / 16
+// Instruction descriptor of a sparse MMA: bit 2 sparse; bits 4-5 the
+// accumulator format (1 fp32, 2 s32); bits 7-9 and 10-12 the A and B formats
+// (.kind::f16: 0 f16, 1 bf16; .kind::tf32: 2; .kind::i8: 1 signed); bit 15 A
+// K-major (0); bit 16 B MN-major (1: X is K x T with T contiguous); N / 8 at
+// bit 17; M / 16 at bit 24.
+template <Kind KD>
+__host__ __device__ constexpr uint32_t make_idesc(int n, int m = kBlockM) {
+  constexpr uint32_t fmt = KD == Kind::BF16 ? 1u : KD == Kind::TF32 ? 2u : KD == Kind::S8 ? 1u : 0u;
+  constexpr uint32_t acc = KD == Kind::S8 ? 2u : 1u;
+  return (1u << 2) | (acc << 4) | (fmt << 7) | (fmt << 10) | (0u << 15) | (1u << 16) |
+         (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
+}
+
+// Metadata operand of instruction k2 (0..3) of a stage whose metadata starts
+// at tensor-memory column e_tmem: the column address (even) and the selector
+// that goes into the descriptor's low bits.  .kind::f16 / tf32 instructions use
+// one column each (an even base plus the selector); .kind::i8 ones use two.
+template <Kind KD>
+__device__ __forceinline__ void meta_operand(uint32_t e_tmem, int k2, uint32_t& e_col, uint32_t& sel) {
+  if constexpr (KD == Kind::S8) {
+    e_col = e_tmem + uint32_t(2 * k2);
+    sel = 0;
+  } else {
+    e_col = e_tmem + uint32_t(k2 & ~1);
+    sel = uint32_t(k2 & 1);
+  }
+}
+
+// Accumulator word -> fp32 for the epilogue.
+template <Kind KD>
+__device__ __forceinline__ float acc_to_f(uint32_t v) {
+  if constexpr (KT<KD>::kAccS32) return __int2float_rn(static_cast<int>(v));
+  else return __uint_as_float(v);
 }
 
 // ----------------------------------------------------------------- kernel
-template <int N_TILE, int STAGES>
+template <int N_TILE, int STAGES, Kind KD>
 struct Cfg {
-  static constexpr int kABytes = kBlockM * kStageKPhys * 2;   // 16 KB
-  // X tile: N_TILE >= 64 -> 64-column boxes with 128-byte rows; narrower tiles
-  // (16 or 32 columns) use one box whose 32- or 64-byte rows carry only the
-  // columns the MMA reads, with the matching swizzle.
-  static constexpr int kBoxCols = N_TILE < 64 ? N_TILE : 64;
-  static constexpr int kBRowBytes = kBoxCols * 2;             // 32, 64 or 128
-  static constexpr int kBBoxes = N_TILE < 64 ? 1 : N_TILE / 64;
-  static constexpr int kBBoxBytes = kStageK * kBRowBytes;
+  using K_ = KT<KD>;
+  static constexpr int kABytes = kBlockM * 128;                // 16 KB: 128 B of compressed A per row
+  // X tile: N_TILE >= one swizzle row's worth of columns -> boxes of kAtomCols
+  // columns with 128-byte rows; narrower tiles use one box whose 32- or
+  // 64-byte rows carry only the columns the MMA reads, with the matching swizzle.
+  static constexpr int kBoxCols = N_TILE < K_::kAtomCols ? N_TILE : K_::kAtomCols;
+  static constexpr int kBRowBytes = kBoxCols * K_::kEsize;      // 32, 64 or 128
+  static constexpr int kBBoxes = N_TILE < K_::kAtomCols ? 1 : N_TILE / K_::kAtomCols;
+  static constexpr int kBBoxBytes = K_::kStageK * kBRowBytes;
   static constexpr int kBBytes = kBBoxes * kBBoxBytes;
-  static constexpr uint32_t kBLayout = kBRowBytes == 128 ? kLayoutSW128 : (kBRowBytes == 64 ? kLayoutSW64 : kLayoutSW32);
-  static constexpr int kEBytes = 2048;
+  static constexpr uint32_t kBLayout = K_::kB32Atom ? kLayoutSW128_32B
+                                       : kBRowBytes == 128 ? kLayoutSW128 : (kBRowBytes == 64 ? kLayoutSW64 : kLayoutSW32);
+  // stride between groups of K rows that one swizzle pattern spans (8 rows;
+  // 4 with 32-byte atoms)
+  static constexpr uint32_t kBSbo = K_::kB32Atom ? 4 * 128 : 8 * kBRowBytes;
+  static constexpr int kEBytes = K_::kEBytes;
   static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
   static constexpr int kAccCols = N_TILE;
-  static constexpr int kAccBufs = (2 * N_TILE + 4 * STAGES <= 512) ? 2 : 1;
+  static constexpr int kAccBufs = (2 * N_TILE + K_::kECols * STAGES <= 512) ? 2 : 1;
   static constexpr int kECol0 = kAccBufs * N_TILE;
-  static constexpr int kTmemNeed = kECol0 + 4 * STAGES;
+  static constexpr int kTmemNeed = kECol0 + K_::kECols * STAGES;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
   static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 /* align */ + 256 /* barriers, flags */;
   static constexpr int kChunk = N_TILE < 32 ? N_TILE : 32;      // epilogue columns per TMEM load
-  static_assert((N_TILE % 64 == 0 || N_TILE == 16 || N_TILE == 32) && N_TILE <= 256, "N_TILE");
+  static_assert(N_TILE % K_::kAtomCols == 0 || (N_TILE < K_::kAtomCols && kBRowBytes >= 32 &&
+                                                (kBRowBytes & (kBRowBytes - 1)) == 0), "N_TILE");
+  static_assert(N_TILE <= 256 && N_TILE >= 16, "N_TILE");
+  static_assert(!K_::kB32Atom || kBRowBytes == 128, "tf32 X rows must be whole 128-byte swizzle rows");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
-  static_assert(kECol0 + 4 * STAGES <= 512, "TMEM budget");
+  static_assert(kECol0 + K_::kECols * STAGES <= 512, "TMEM budget");
 };
 
 struct Params {
@@ -339,7 +431,8 @@ struct Params {
   int m_tiles, n_tiles, k_blocks;
   int m_inner;  // tile order: 1 -> m fastest inside a group of `group` m-tiles, 0 -> n fastest
   int group;    // tiles of the slow operand kept together (sized so the group stays in L2)
-  int y_f32;    // 1: fp32 output, 0: bf16 output
+  int y_f32;    // 1: fp32 output, 0: bf16 output (or s32, below)
+  int y_s32;    // 1: the raw s32 accumulator (int8 products; alpha == 1, beta == 0)
   int y_vec;    // 1: Y and ldy allow 16-byte vector stores
   int y_tma;    // 1: bf16 output with beta == 0 leaves through staged bulk tensor stores (pair kernel)
   // Pair kernel work list: items [0, split_from) are whole tiles; the tiles
@@ -389,14 +482,25 @@ __device__ __forceinline__ PairWork pair_work(const Params& p, int w, int n_tota
 }
 
 // Epilogue of one 32-column chunk of one output row: y = alpha * acc (+ beta * y_old),
-// rounded to the output type; vector stores when Y allows them, scalar at the T edge.
-template <int CW>
+// rounded to the output type (or the raw s32 accumulator); vector stores when Y
+// allows them, scalar at the T edge.
+template <int CW, Kind KD>
 __device__ __forceinline__ void store_chunk_n(const Params& p, int r, int col0, const uint32_t (&v)[CW]) {
   if (r < p.R && col0 < p.T) {
     const bool full_chunk = p.y_vec && col0 + CW <= p.T;
+    if (KT<KD>::kAccS32 && p.y_s32) {
+      uint32_t* yrow = static_cast<uint32_t*>(p.Y) + size_t(r) * p.ldy + col0;
+      if (full_chunk) {
+#pragma unroll
+        for (int j = 0; j < CW; j += 4) *reinterpret_cast<uint4*>(yrow + j) = make_uint4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      } else {
+        for (int j = 0; j < CW && col0 + j < p.T; ++j) yrow[j] = v[j];
+      }
+      return;
+    }
     float y[CW];
 #pragma unroll
-    for (int j = 0; j < CW; ++j) y[j] = p.alpha * __uint_as_float(v[j]);
+    for (int j = 0; j < CW; ++j) y[j] = p.alpha * acc_to_f<KD>(v[j]);
     if (p.y_f32) {
       float* yrow = static_cast<float*>(p.Y) + size_t(r) * p.ldy + col0;
       if (full_chunk) {
@@ -451,14 +555,16 @@ __device__ __forceinline__ void store_chunk_n(const Params& p, int r, int col0, 
     }
   }
 }
+template <Kind KD>
 __device__ __forceinline__ void store_chunk(const Params& p, int r, int col0, const uint32_t (&v)[32]) {
-  store_chunk_n<32>(p, r, col0, v);
+  store_chunk_n<32, KD>(p, r, col0, v);
 }
 
-template <int N_TILE, int STAGES, bool BF16>
-__global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 113 * 1024 ? 2 : 1)
+template <int N_TILE, int STAGES, Kind KD>
+__global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES, KD>::kSmemBytes <= 113 * 1024 ? 2 : 1)
     spmm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, Params p) {
-  using C = Cfg<N_TILE, STAGES>;
+  using C = Cfg<N_TILE, STAGES, KD>;
+  using K_ = KT<KD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
@@ -517,19 +623,20 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 1
           uint8_t* st = smem + s * C::kStageBytes;
           mbar_arrive_expect_tx(&full[s], C::kStageBytes);
           armed_round[s] = round;
-          tma_load_2d(st, &map_a, &full[s], kb * kStageKPhys, mt * kBlockM);
+          tma_load_2d(st, &map_a, &full[s], kb * K_::kStageKPhys, mt * kBlockM);
 #pragma unroll
           for (int j = 0; j < C::kBBoxes; ++j)
-            tma_load_2d(st + C::kABytes + j * C::kBBoxBytes, &map_b, &full[s], nt * N_TILE + 64 * j, kb * kStageK);
-          const uint8_t* esrc = p.meta_img + (size_t(mt) * p.k_blocks + kb) * 2048;
-          bulk_load(st + C::kABytes + C::kBBytes, esrc, 2048, &full[s]);
+            tma_load_2d(st + C::kABytes + j * C::kBBoxBytes, &map_b, &full[s], nt * N_TILE + K_::kAtomCols * j,
+                        kb * K_::kStageK);
+          const uint8_t* esrc = p.meta_img + (size_t(mt) * p.k_blocks + kb) * C::kEBytes;
+          bulk_load(st + C::kABytes + C::kBBytes, esrc, C::kEBytes, &full[s]);
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = make_idesc(BF16, N_TILE);
+      const uint32_t idesc = make_idesc<KD>(N_TILE);
       uint32_t it = 0, local = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
@@ -547,22 +654,24 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 1
           const uint32_t a_addr = smem_u32(st);
           const uint32_t b_addr = smem_u32(st + C::kABytes);
           const uint32_t e_addr = smem_u32(st + C::kABytes + C::kBBytes);
-          const uint32_t e_tmem = tmem_base + uint32_t(C::kECol0 + 4 * s);
-          // metadata: 128 lanes x 16 bytes, rows contiguous (8-row groups 128 B apart)
-          tmem_cp_128x128b(e_tmem, smem_desc(e_addr, 0, 128, kLayoutNone));
+          const uint32_t e_tmem = tmem_base + uint32_t(C::kECol0 + K_::kECols * s);
+          // metadata: per 2 KB block, 128 lanes x 16 bytes, rows contiguous
+          // (8-row groups 128 B apart); int8 stages carry two blocks
 #pragma unroll
-          for (int k2 = 0; k2 < kStageK / kMmaK; ++k2) {
+          for (int j = 0; j < C::kEBytes / 2048; ++j)
+            tmem_cp_128x128b(e_tmem + uint32_t(4 * j), smem_desc(e_addr + uint32_t(2048 * j), 0, 128, kLayoutNone));
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) {
             // A: K-major, 128B swizzle, rows 128 B apart, 8-row atoms 1024 B apart;
-            //    32 logical K = 16 compressed values = 32 bytes further per MMA.
+            //    32 bytes of compressed values (kMmaK logical K) further per MMA.
             const uint64_t adesc = smem_desc(a_addr + 32u * k2, 16, 1024, kLayoutSW128);
-            // B: N-major, 128B swizzle: 64-column atoms LBO apart, 8-row K groups 1024 B apart;
-            //    32 logical K rows = 4096 bytes further per MMA.
-            const uint64_t bdesc = smem_desc(b_addr + uint32_t(32 * C::kBRowBytes) * k2, C::kBBoxBytes,
-                                             uint32_t(8 * C::kBRowBytes), C::kBLayout);
-            // metadata column of this MMA: even base + selector bit
-            const uint32_t e_col = e_tmem + uint32_t(k2 & ~1);
-            const uint32_t id = idesc | uint32_t(k2 & 1);
-            mma_sp(d_tmem, adesc, bdesc, e_col, id, (kb > 0 || k2 > 0) ? 1u : 0u);
+            // B: N-major, swizzled rows of kBRowBytes: atoms LBO apart, 8-row K
+            //    groups SBO apart; kMmaK rows further per MMA.
+            const uint64_t bdesc = smem_desc(b_addr + uint32_t(K_::kMmaK * C::kBRowBytes) * k2, C::kBBoxBytes,
+                                             C::kBSbo, C::kBLayout);
+            uint32_t e_col, sel;
+            meta_operand<KD>(e_tmem, k2, e_col, sel);
+            mma_sp<KD>(d_tmem, adesc, bdesc, e_col, idesc | sel, (kb > 0 || k2 > 0) ? 1u : 0u);
           }
           mma_commit(&empty[s]);
         }
@@ -594,13 +703,13 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 1
       if constexpr (C::kChunk == 16) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TILE), v);
-        store_chunk_n<16>(p, r, c_base, v);
+        store_chunk_n<16, KD>(p, r, c_base, v);
       } else {
 #pragma unroll 1
         for (int c = 0; c < N_TILE; c += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TILE + c), v);
-          store_chunk(p, r, c_base + c, v);
+          store_chunk<KD>(p, r, c_base + c, v);
         }
       }
       fence_before_sync();
@@ -635,35 +744,39 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES>::kSmemBytes <= 1
 // issued by the even CTA reads both halves, so each SM's shared memory feeds
 // only half of B.  Both CTAs' TMA loads complete on the even CTA's full
 // barrier; the even CTA's commits arrive on both CTAs' barriers.
-template <int N_TOTAL, int STAGES>
+template <int N_TOTAL, int STAGES, Kind KD>
 struct PairCfg {
+  using K_ = KT<KD>;
   static constexpr int kNHalf = N_TOTAL / 2;
-  static constexpr int kABytes = kBlockM * kStageKPhys * 2;   // 16 KB
-  static constexpr int kBBoxes = (kNHalf + 63) / 64;           // the last box may be partly unused
-  static constexpr int kBBoxBytes = kStageK * 64 * 2;         // 16 KB
+  static constexpr int kABytes = kBlockM * 128;                               // 16 KB
+  static constexpr int kBBoxes = (kNHalf + K_::kAtomCols - 1) / K_::kAtomCols;  // the last may be partly unused
+  static constexpr int kBBoxBytes = K_::kStageK * 128;                        // 8, 16 or 32 KB
   static constexpr int kBBytes = kBBoxes * kBBoxBytes;
-  static constexpr int kEBytes = 2048;
+  static constexpr int kEBytes = K_::kEBytes;
   static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;
-  static constexpr int kAccBufs = (2 * N_TOTAL + 4 * STAGES <= 512) ? 2 : 1;
+  static constexpr int kAccBufs = (2 * N_TOTAL + K_::kECols * STAGES <= 512) ? 2 : 1;
   static constexpr int kECol0 = kAccBufs * N_TOTAL;
-  static constexpr int kTmemCols = (kECol0 + 4 * STAGES) <= 256 ? 256 : 512;
+  static constexpr int kTmemCols = (kECol0 + K_::kECols * STAGES) <= 256 ? 256 : 512;
   // One 2 KB output slot (32 rows x 32 bf16 columns, 64-byte swizzle) per
   // epilogue warp, 1024-byte aligned after the barriers.
   static constexpr int kOutSlotBytes = 2048;
   static constexpr int kOutOff = STAGES * kStageBytes + 1024;
   static constexpr int kSmemBytes = kOutOff + 8 * kOutSlotBytes + 1024 /* base alignment */;
+  // a half-width last-wave item stages one 64-column half per CTA in whole atoms
+  static constexpr bool kCanSplit = N_TOTAL == 256 && K_::kAtomCols <= 64;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kNHalf % 32 == 0 && N_TOTAL <= 256, "N_TOTAL");
-  static_assert(kECol0 + 4 * STAGES <= 512, "TMEM budget");
+  static_assert(kECol0 + K_::kECols * STAGES <= 512, "TMEM budget");
 };
 
-template <int N_TOTAL, int STAGES, bool BF16>
+template <int N_TOTAL, int STAGES, Kind KD>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     spmm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                      const __grid_constant__ CUtensorMap map_e, const __grid_constant__ CUtensorMap map_y,
                      Params p) {
-  using C = PairCfg<N_TOTAL, STAGES>;
+  using C = PairCfg<N_TOTAL, STAGES, KD>;
+  using K_ = KT<KD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * C::kStageBytes);
@@ -715,9 +828,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       for (int w = pair; w < num_work && ok; w += num_pairs) {
         const PairWork wk = pair_work(p, w, N_TOTAL);
         const int row_tile = 2 * wk.mt + int(rank);  // this CTA's 128-row tile
-        // a half-width item stages one 64-column B atom per CTA
-        const int b_boxes = wk.narrow ? 1 : C::kBBoxes;
-        const int b_cols = wk.narrow ? 64 : C::kNHalf;
+        // a half-width item stages 64 columns (whole atoms) per CTA
+        const int b_boxes = (C::kCanSplit && wk.narrow) ? 64 / K_::kAtomCols : C::kBBoxes;
+        const int b_cols = (C::kCanSplit && wk.narrow) ? 64 : C::kNHalf;
         const uint32_t tx = 2u * uint32_t(C::kABytes + b_boxes * C::kBBoxBytes + C::kEBytes);
         for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           if (int64_t(it) == p.skip_it) continue;  // test hook: neither CTA fills this step's stage
@@ -728,22 +841,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (leader) mbar_arrive_expect_tx(&full[s], tx);
           armed_round[s] = round;
           const uint32_t bar = mapa(smem_u32(&full[s]), 0);
-          tma_load_2d_pair(st, &map_a, bar, kb * kStageKPhys, row_tile * kBlockM);
+          tma_load_2d_pair(st, &map_a, bar, kb * K_::kStageKPhys, row_tile * kBlockM);
 #pragma unroll
           for (int j = 0; j < C::kBBoxes; ++j)
             if (j < b_boxes)
               tma_load_2d_pair(st + C::kABytes + j * C::kBBoxBytes, &map_b, bar,
-                               wk.col0 + int(rank) * b_cols + 64 * j, kb * kStageK);
+                               wk.col0 + int(rank) * b_cols + K_::kAtomCols * j, kb * K_::kStageK);
+          // the stage's image: kEBytes / 16 rows of 16 bytes
           tma_load_2d_pair(st + C::kABytes + C::kBBytes, &map_e, bar, 0,
-                           (row_tile * p.k_blocks + kb) * kBlockM);
+                           (row_tile * p.k_blocks + kb) * (C::kEBytes / 16));
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && leader) {
-      const uint32_t idesc_full = make_idesc(BF16, N_TOTAL, 2 * kBlockM);
-      const uint32_t idesc_narrow = make_idesc(BF16, N_TOTAL / 2, 2 * kBlockM);
+      const uint32_t idesc_full = make_idesc<KD>(N_TOTAL, 2 * kBlockM);
+      const uint32_t idesc_narrow = make_idesc<KD>(N_TOTAL / 2, 2 * kBlockM);
       uint32_t it = 0, local = 0;
       bool ok = true;
       for (int w = pair; w < num_work && ok; w += num_pairs, ++local) {
@@ -762,14 +876,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           const uint32_t a_addr = smem_u32(st);
           const uint32_t b_addr = smem_u32(st + C::kABytes);
           const uint32_t e_addr = smem_u32(st + C::kABytes + C::kBBytes);
-          const uint32_t e_tmem = tmem_base + uint32_t(C::kECol0 + 4 * s);
-          tmem_cp_pair_128x128b(e_tmem, smem_desc(e_addr, 0, 128, kLayoutNone));
+          const uint32_t e_tmem = tmem_base + uint32_t(C::kECol0 + K_::kECols * s);
 #pragma unroll
-          for (int k2 = 0; k2 < kStageK / kMmaK; ++k2) {
+          for (int j = 0; j < C::kEBytes / 2048; ++j)
+            tmem_cp_pair_128x128b(e_tmem + uint32_t(4 * j),
+                                  smem_desc(e_addr + uint32_t(2048 * j), 0, 128, kLayoutNone));
+#pragma unroll
+          for (int k2 = 0; k2 < 4; ++k2) {
             const uint64_t adesc = smem_desc(a_addr + 32u * k2, 16, 1024, kLayoutSW128);
-            const uint64_t bdesc = smem_desc(b_addr + 4096u * k2, C::kBBoxBytes, 1024, kLayoutSW128);
-            mma_sp_pair(d_tmem, adesc, bdesc, e_tmem + uint32_t(k2 & ~1), idesc | uint32_t(k2 & 1),
-                        (kb > 0 || k2 > 0) ? 1u : 0u);
+            const uint64_t bdesc = smem_desc(b_addr + uint32_t(K_::kMmaK * 128) * k2, C::kBBoxBytes,
+                                             K_::kB32Atom ? 512u : 1024u, K_::kB32Atom ? kLayoutSW128_32B : kLayoutSW128);
+            uint32_t e_col, sel;
+            meta_operand<KD>(e_tmem, k2, e_col, sel);
+            mma_sp_pair<KD>(d_tmem, adesc, bdesc, e_col, idesc | sel, (kb > 0 || k2 > 0) ? 1u : 0u);
           }
           mma_commit_pair(&empty[s]);
         }
@@ -796,7 +915,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int half = (warp - 2) >> 2;
     const int row_in_tile = 32 * q + lane;
     const uint32_t acc_empty_leader[2] = {mapa(smem_u32(&acc_empty[0]), 0), mapa(smem_u32(&acc_empty[1]), 0)};
-    const bool early = !p.y_f32 && p.beta == 0.0f && p.y_vec;
+    const bool early = !p.y_f32 && !p.y_s32 && p.beta == 0.0f && p.y_vec;
     const uint32_t out_slot = smem_u32(smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes);
     uint32_t local = 0;
     for (int w = pair; w < num_work; w += num_pairs, ++local) {
@@ -830,7 +949,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (lane == 0) mbar_arrive_remote(acc_empty_leader[buf]);
 #pragma unroll
           for (int j = 0; j < kCols / 2; ++j)
-            packed[j] = pack_bf16x2(p.alpha * __uint_as_float(v[2 * j]), p.alpha * __uint_as_float(v[2 * j + 1]));
+            packed[j] = pack_bf16x2(p.alpha * acc_to_f<KD>(v[2 * j]), p.alpha * acc_to_f<KD>(v[2 * j + 1]));
         }
         if (p.y_tma) {
           // 32 x 32 chunks through this warp's slot: lane = row, four 16-byte
@@ -882,7 +1001,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         for (int c = 0; c < kc; c += 32) {
           uint32_t v[32];
           tmem_ld_32x32b_x32(taddr + uint32_t(c), v);
-          store_chunk(p, r, c_base + c, v);
+          store_chunk<KD>(p, r, c_base + c, v);
         }
         fence_before_sync();
         __syncwarp();
@@ -951,29 +1070,43 @@ EncodeFn get_encode() {
   return fn;
 }
 
-// 2D tile map over a row-major [rows x cols] 16-bit matrix, box = box_cols x box_rows, 128B swizzle.
-bool make_map(CUtensorMap* map, const void* base, bool bf16, int64_t rows, int64_t cols, int64_t ld_elems,
-              int box_cols, int box_rows, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
+// TMA element type of each operand kind.
+template <Kind KD>
+constexpr CUtensorMapDataType tma_type() {
+  return KD == Kind::BF16   ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+         : KD == Kind::F16  ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+         : KD == Kind::TF32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                            : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+}
+
+CUtensorMapSwizzle swizzle_for(int row_bytes) {
+  return row_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+         : row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+}
+
+// 2D tile map over a row-major [rows x cols] matrix of esize-byte elements,
+// box = box_cols x box_rows.
+bool make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize, int64_t rows, int64_t cols,
+              int64_t ld_elems, int box_cols, int box_rows, CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeFn enc = get_encode();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(ld_elems) * 2};
+  const cuuint64_t strides[1] = {cuuint64_t(ld_elems) * cuuint64_t(esize)};
   const cuuint32_t box[2] = {cuuint32_t(box_cols), cuuint32_t(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-             const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  return enc(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
              swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N_TILE, int STAGES, bool BF16>
+template <int N_TILE, int STAGES, Kind KD>
 nm_status launch(const CUtensorMap& ma, const void* X, int64_t ldx, int64_t K, int64_t T, const Params& p,
                  cudaStream_t s) {
-  using C = Cfg<N_TILE, STAGES>;
+  using C = Cfg<N_TILE, STAGES, KD>;
   CUtensorMap mb;
-  const CUtensorMapSwizzle sw = C::kBRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-                                : C::kBRowBytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-  if (!make_map(&mb, X, BF16, K, T, ldx, C::kBoxCols, kStageK, sw)) return NM_ERR_CUDA;
-  auto kern = spmm_kernel<N_TILE, STAGES, BF16>;
+  if (!make_map(&mb, X, tma_type<KD>(), KT<KD>::kEsize, K, T, ldx, C::kBoxCols, KT<KD>::kStageK,
+                KT<KD>::kB32Atom ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : swizzle_for(C::kBRowBytes)))
+    return NM_ERR_CUDA;
+  auto kern = spmm_kernel<N_TILE, STAGES, KD>;
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes) != NM_OK) return NM_ERR_CUDA;
   const int tiles = p.m_tiles * p.n_tiles;
   const int per_sm = C::kSmemBytes <= 113 * 1024 ? 2 : 1;  // two CTAs per SM when the ring is small
@@ -984,24 +1117,24 @@ nm_status launch(const CUtensorMap& ma, const void* X, int64_t ldx, int64_t K, i
 }
 
 // 2D byte map over the metadata image seen as rows of 16 bytes (one row per
-// tensor-memory lane), box = 128 rows = one 2048-byte block.
-bool make_map_image(CUtensorMap* map, const uint8_t* img, int64_t rows16) {
+// tensor-memory lane), box = one stage's image (128 or 256 rows).
+bool make_map_image(CUtensorMap* map, const uint8_t* img, int64_t rows16, int box_rows) {
   EncodeFn enc = get_encode();
   if (!enc) return false;
   const cuuint64_t dims[2] = {16, cuuint64_t(rows16)};
   const cuuint64_t strides[1] = {16};
-  const cuuint32_t box[2] = {16, 128};
+  const cuuint32_t box[2] = {16, cuuint32_t(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(img), dims, strides, box, estr,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N_TOTAL, int STAGES, bool BF16>
+template <int N_TOTAL, int STAGES, Kind KD>
 nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me, const CUtensorMap& my,
                       const Params& p, bool tail_split, cudaStream_t s) {
-  using C = PairCfg<N_TOTAL, STAGES>;
-  auto kern = spmm_pair_kernel<N_TOTAL, STAGES, BF16>;
+  using C = PairCfg<N_TOTAL, STAGES, KD>;
+  auto kern = spmm_pair_kernel<N_TOTAL, STAGES, KD>;
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes) != NM_OK) return NM_ERR_CUDA;
   const int tiles = p.m_tiles * p.n_tiles;
   const int max_pairs = sm_count() / 2;
@@ -1010,9 +1143,10 @@ nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   q.split_from = tiles;
   q.num_work = tiles;
   // A last wave that fills at most half of the pairs is done in half-width
-  // items (whole 64-column B atoms per CTA, so only for 256-column tiles).
+  // items (whole B atoms per CTA, so only for 256-column tiles of 16- and
+  // 32-bit operands).
   const int rem = tiles % pairs;
-  if (N_TOTAL == 256 && tiles > pairs && rem > 0 && 2 * rem <= pairs && tail_split) {
+  if (C::kCanSplit && tiles > pairs && rem > 0 && 2 * rem <= pairs && tail_split) {
     q.split_from = tiles - rem;
     q.num_work = tiles + rem;
   }
@@ -1024,7 +1158,8 @@ nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
 // output is wide enough to fill 128+ columns; the single-CTA kernel
 // otherwise.  A test or tuning caller may force one (nm_spmm_test); a forced
 // choice that does not apply (a pair kernel for an odd number of row tiles)
-// falls back to the default.
+// falls back to the default.  int8 operands have 128-column swizzle atoms, so
+// their pair kernel is the 256-column one and their narrowest tile 32 columns.
 enum class Kern { Pair256, Pair192, Pair128, Single256, Single128, Single64, Single64x2, Single32x2, Single16x2 };
 
 // Options of one call: the defaults for nm_spmm, test and tuning hooks otherwise.
@@ -1035,26 +1170,33 @@ struct Opts {
   int64_t skip_it = -1;
 };
 
+template <Kind KD>
 Kern choose_kernel(int64_t R, int64_t T, int forced) {
   const bool pairable = ((R + kBlockM - 1) / kBlockM) % 2 == 0;
+  const bool s8 = KD == Kind::S8;
+  const bool no16 = s8 || KD == Kind::TF32;  // X rows of a 16-column tile would be narrower than the swizzle
   Kern k;
-  if (pairable && T > 64) k = T > 128 ? Kern::Pair256 : Kern::Pair128;
+  if (pairable && T > (s8 ? 128 : 64)) k = (T > 128 || s8) ? Kern::Pair256 : Kern::Pair128;
   else if (T > 128) k = Kern::Single256;
   else if (T > 64) k = Kern::Single128;
   else if (T > 32) k = Kern::Single64x2;
-  else if (T > 16) k = Kern::Single32x2;
+  else if (T > 16 || no16) k = Kern::Single32x2;
   else k = Kern::Single16x2;
   if (forced >= 1 && forced <= 9) {
-    const Kern f = static_cast<Kern>(forced - 1);
+    Kern f = static_cast<Kern>(forced - 1);
+    if (s8 && (f == Kern::Pair192 || f == Kern::Pair128)) f = Kern::Pair256;
+    if (no16 && f == Kern::Single16x2) f = Kern::Single32x2;
     const bool is_pair = f == Kern::Pair256 || f == Kern::Pair192 || f == Kern::Pair128;
     if (!is_pair || pairable) k = f;
   }
   return k;
 }
 
-template <bool BF16>
-nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_t ldx, void* Y, bool y_f32,
+// y_kind: 0 bf16, 1 fp32, 2 s32 (int8 operands only)
+template <Kind KD>
+nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_t ldx, void* Y, int y_kind,
               int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta, const Opts& o, cudaStream_t s) {
+  using K_ = KT<KD>;
   Params p;
   p.wait_ns = o.wait_ns;
   p.skip_it = o.skip_it;
@@ -1065,12 +1207,13 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
   p.R = int(R);
   p.T = int(T);
   p.K = int(K);
-  p.k_blocks = int((K + kStageK - 1) / kStageK);
-  p.y_f32 = y_f32 ? 1 : 0;
-  p.y_vec = (aligned16(Y) && stride_ok(ldy, y_f32 ? 4 : 2)) ? 1 : 0;
+  p.k_blocks = int((K + K_::kStageK - 1) / K_::kStageK);
+  p.y_f32 = y_kind == 1 ? 1 : 0;
+  p.y_s32 = y_kind == 2 ? 1 : 0;
+  p.y_vec = (aligned16(Y) && stride_ok(ldy, y_kind == 0 ? 2 : 4)) ? 1 : 0;
   p.alpha = alpha;
   p.beta = beta;
-  const Kern kern = choose_kernel(R, T, o.kernel);
+  const Kern kern = choose_kernel<KD>(R, T, o.kernel);
   const bool pair = kern == Kern::Pair256 || kern == Kern::Pair192 || kern == Kern::Pair128;
   const int block_m = pair ? 2 * kBlockM : kBlockM;
   const int n_tile = (kern == Kern::Pair256 || kern == Kern::Single256) ? 256
@@ -1083,34 +1226,46 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
   // Tile order: the operand with fewer bytes is swept fastest, so consecutive
   // tiles (running at the same time) share a slice of the larger one.
   {
-    const double a_bytes = double(R) * double(K);          // compressed values, 2 B x K/2
-    const double b_bytes = double(K) * double(T) * 2.0;
+    const double a_bytes = double(R) * double(K) * 0.5 * K_::kEsize;   // compressed values
+    const double b_bytes = double(K) * double(T) * K_::kEsize;
     p.m_inner = a_bytes < b_bytes ? 1 : 0;
     p.group = p.m_inner ? p.m_tiles : p.n_tiles;
   }
 
   CUtensorMap ma, mb;
-  if (!make_map(&ma, values, BF16, R, K / 2, K / 2, kStageKPhys, kBlockM)) return NM_ERR_CUDA;
-  if (!make_map(&mb, X, BF16, K, T, ldx, 64, kStageK)) return NM_ERR_CUDA;
+  if (!make_map(&ma, values, tma_type<KD>(), K_::kEsize, R, K / 2, K / 2, K_::kStageKPhys, kBlockM))
+    return NM_ERR_CUDA;
+  if (!make_map(&mb, X, tma_type<KD>(), K_::kEsize, K, T, ldx, K_::kAtomCols, K_::kStageK,
+                K_::kB32Atom ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B))
+    return NM_ERR_CUDA;
   if (pair) {
     CUtensorMap me, my;
-    const int64_t rows16 = ((R + 127) / 128) * int64_t(p.k_blocks) * 128;
-    if (!make_map_image(&me, meta_img, rows16)) return NM_ERR_CUDA;
+    constexpr int e_rows = K_::kEBytes / 16;
+    const int64_t rows16 = ((R + 127) / 128) * int64_t(p.k_blocks) * e_rows;
+    if (!make_map_image(&me, meta_img, rows16, e_rows)) return NM_ERR_CUDA;
     // bf16 output without beta leaves through bulk tensor stores (32 x 32 boxes)
-    p.y_tma = (!y_f32 && beta == 0.0f && p.y_vec) ? 1 : 0;
+    p.y_tma = (y_kind == 0 && beta == 0.0f && p.y_vec) ? 1 : 0;
     memset(&my, 0, sizeof(my));
-    if (p.y_tma && !make_map(&my, Y, true, R, T, ldy, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return NM_ERR_CUDA;
-    if (kern == Kern::Pair256) return launch_pair<256, 4, BF16>(ma, mb, me, my, p, o.tail_split, s);
-    if (kern == Kern::Pair192) return launch_pair<192, 4, BF16>(ma, mb, me, my, p, o.tail_split, s);
-    return launch_pair<128, 6, BF16>(ma, mb, me, my, p, o.tail_split, s);
+    if (p.y_tma && !make_map(&my, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, T, ldy, 32, 32,
+                             CU_TENSOR_MAP_SWIZZLE_64B))
+      return NM_ERR_CUDA;
+    if constexpr (KD == Kind::S8) {
+      return launch_pair<256, 4, KD>(ma, mb, me, my, p, o.tail_split, s);
+    } else {
+      if (kern == Kern::Pair256) return launch_pair<256, 4, KD>(ma, mb, me, my, p, o.tail_split, s);
+      if (kern == Kern::Pair192) return launch_pair<192, 4, KD>(ma, mb, me, my, p, o.tail_split, s);
+      return launch_pair<128, 6, KD>(ma, mb, me, my, p, o.tail_split, s);
+    }
   }
   switch (kern) {
-    case Kern::Single256: return launch<256, 2, BF16>(ma, X, ldx, K, T, p, s);
-    case Kern::Single128: return launch<128, 4, BF16>(ma, X, ldx, K, T, p, s);
-    case Kern::Single64x2: return launch<64, 3, BF16>(ma, X, ldx, K, T, p, s);
-    case Kern::Single32x2: return launch<32, 4, BF16>(ma, X, ldx, K, T, p, s);
-    case Kern::Single16x2: return launch<16, 5, BF16>(ma, X, ldx, K, T, p, s);
-    default: return launch<64, 6, BF16>(ma, X, ldx, K, T, p, s);
+    case Kern::Single256: return launch<256, 2, KD>(ma, X, ldx, K, T, p, s);
+    case Kern::Single128: return launch<128, 4, KD>(ma, X, ldx, K, T, p, s);
+    case Kern::Single64x2: return launch<64, 3, KD>(ma, X, ldx, K, T, p, s);
+    case Kern::Single32x2: return launch<32, (KD == Kind::S8 ? 3 : 4), KD>(ma, X, ldx, K, T, p, s);
+    case Kern::Single16x2:
+      if constexpr (KD == Kind::S8 || KD == Kind::TF32) return NM_ERR_UNSUPPORTED;  // never chosen (above)
+      else return launch<16, 5, KD>(ma, X, ldx, K, T, p, s);
+    default: return launch<64, 6, KD>(ma, X, ldx, K, T, p, s);
   }
 }
 
@@ -1133,12 +1288,20 @@ namespace {
 // *noop set means there is nothing to compute (R == 0 or T == 0).
 nm_status spmm_validate(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X,
                         int64_t ldx, const void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T,
-                        bool* noop) {
+                        float alpha, float beta, bool* noop) {
   *noop = false;
-  if (ab_dtype == NM_S8) return NM_ERR_UNSUPPORTED;  // the int8 sparse product is not built
-  if (!dtype_ok(ab_dtype) || (y_dtype != NM_BF16 && y_dtype != NM_F32)) return NM_ERR_DTYPE;
-  if (R < 0 || K < 0 || T < 0 || K % 16 != 0 || ldx < T || ldy < T) return NM_ERR_SHAPE;
+  if (!dtype_ok_int8(ab_dtype)) return NM_ERR_DTYPE;
+  if (ab_dtype == NM_S8) {
+    if (y_dtype != NM_BF16 && y_dtype != NM_F32 && y_dtype != NM_S32) return NM_ERR_DTYPE;
+  } else if (y_dtype != NM_BF16 && y_dtype != NM_F32) {
+    return NM_ERR_DTYPE;
+  }
+  // int8: the compressed rows (K/2 bytes) must be whole 16-byte units, the
+  // pages' "multiples of 32" for INT8 sparse operands
+  const int k_mult = ab_dtype == NM_S8 ? 32 : 16;
+  if (R < 0 || K < 0 || T < 0 || K % k_mult != 0 || ldx < T || ldy < T) return NM_ERR_SHAPE;
   if (R > 0x7FFFFFFF - 256 || K > 0x7FFFFFFF - 256 || T > 0x7FFFFFFF - 256) return NM_ERR_SHAPE;
+  if (y_dtype == NM_S32 && (alpha != 1.0f || beta != 0.0f)) return NM_ERR_UNSUPPORTED;
   if (R == 0 || T == 0) {
     *noop = true;
     return NM_OK;
@@ -1152,14 +1315,18 @@ nm_status spmm_validate(const void* values, const uint8_t* meta_sm100, nm_dtype 
   return NM_OK;
 }
 
+int y_kind_of(nm_dtype y) { return y == NM_BF16 ? 0 : y == NM_F32 ? 1 : 2; }
+
 nm_status spmm_entry(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X, int64_t ldx,
                      void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta,
                      void* workspace, size_t workspace_bytes, const spmm::Opts& o, void* stream) {
   bool noop = false;
-  const nm_status v = spmm_validate(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, &noop);
+  const nm_status v =
+      spmm_validate(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, &noop);
   if (v != NM_OK || noop) return v;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const bool y_f32 = y_dtype == NM_F32;
+  const int yk = y_kind_of(y_dtype);
+  using spmm::Kind;
   if (ab_dtype == NM_F32) {
     const size_t need = nm_spmm_workspace_bytes(ab_dtype, R, K, T);
     if (workspace == nullptr || workspace_bytes < need) return NM_ERR_WORKSPACE;
@@ -1171,11 +1338,29 @@ nm_status spmm_entry(const void* values, const uint8_t* meta_sm100, nm_dtype ab_
     spmm::f32_to_f16_kernel<<<blocks, 256, 0, s>>>(static_cast<const float*>(values), R, K / 2, K / 2, vh, K / 2);
     spmm::f32_to_f16_kernel<<<blocks, 256, 0, s>>>(static_cast<const float*>(X), K, T, ldx, xh, ldx_h);
     if (launch_status() != NM_OK) return NM_ERR_CUDA;
-    return spmm::run<false>(vh, meta_sm100, xh, ldx_h, Y, y_f32, ldy, R, K, T, alpha, beta, o, s);
+    return spmm::run<Kind::F16>(vh, meta_sm100, xh, ldx_h, Y, yk, ldy, R, K, T, alpha, beta, o, s);
   }
+  if (ab_dtype == NM_S8)
+    return spmm::run<Kind::S8>(values, meta_sm100, X, ldx, Y, yk, ldy, R, K, T, alpha, beta, o, s);
   if (ab_dtype == NM_BF16)
-    return spmm::run<true>(values, meta_sm100, X, ldx, Y, y_f32, ldy, R, K, T, alpha, beta, o, s);
-  return spmm::run<false>(values, meta_sm100, X, ldx, Y, y_f32, ldy, R, K, T, alpha, beta, o, s);
+    return spmm::run<Kind::BF16>(values, meta_sm100, X, ldx, Y, yk, ldy, R, K, T, alpha, beta, o, s);
+  return spmm::run<Kind::F16>(values, meta_sm100, X, ldx, Y, yk, ldy, R, K, T, alpha, beta, o, s);
+}
+
+nm_status spmm12_entry(const float* values, const uint8_t* meta12_img, const float* X, int64_t ldx, void* Y,
+                       nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta,
+                       const spmm::Opts& o, void* stream) {
+  if (y_dtype != NM_BF16 && y_dtype != NM_F32) return NM_ERR_DTYPE;
+  if (R < 0 || K < 0 || T < 0 || K % 16 != 0 || ldx < T || ldy < T) return NM_ERR_SHAPE;
+  if (R > 0x7FFFFFFF - 256 || K > 0x7FFFFFFF - 256 || T > 0x7FFFFFFF - 256) return NM_ERR_SHAPE;
+  if (R == 0 || T == 0) return NM_OK;
+  if (values == nullptr || meta12_img == nullptr || X == nullptr || Y == nullptr) return NM_ERR_NULL;
+  if (!aligned16(values) || !aligned16(meta12_img) || !aligned16(X) || !stride_ok(ldx, 4) ||
+      (reinterpret_cast<uintptr_t>(Y) % uintptr_t(esize_of(y_dtype))) != 0)
+    return NM_ERR_ALIGN;
+  if (K == 0) return NM_ERR_SHAPE;
+  return spmm::run<spmm::Kind::TF32>(values, meta12_img, X, ldx, Y, y_kind_of(y_dtype), ldy, R, K, T, alpha, beta,
+                                     o, static_cast<cudaStream_t>(stream));
 }
 
 }  // namespace
@@ -1200,6 +1385,22 @@ extern "C" nm_status nm_spmm_test(const void* values, const uint8_t* meta_sm100,
   o.skip_it = skip_step;
   return spmm_entry(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, workspace,
                     workspace_bytes, o, stream);
+}
+
+extern "C" nm_status nm_spmm12(const float* values, const uint8_t* meta12_sm100, const float* X, int64_t ldx,
+                               void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha,
+                               float beta, void* stream) {
+  return spmm12_entry(values, meta12_sm100, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, spmm::Opts(), stream);
+}
+
+extern "C" nm_status nm_spmm12_test(const float* values, const uint8_t* meta12_sm100, const float* X, int64_t ldx,
+                                    void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K, int64_t T,
+                                    float alpha, float beta, int kernel, int tail_split, void* stream) {
+  if (kernel < 0 || kernel > 9) return NM_ERR_SHAPE;
+  spmm::Opts o;
+  o.kernel = kernel;
+  o.tail_split = tail_split != 0;
+  return spmm12_entry(values, meta12_sm100, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, o, stream);
 }
 
 extern "C" nm_status nm_last_device_status(void* stream) {
@@ -1251,9 +1452,10 @@ extern "C" nm_status nm_spmm_noalloc(const void* values, const uint8_t* meta_sm1
   // the same argument checks as nm_spmm first, so a malformed call reports
   // its real fault rather than the scratch limit
   bool noop = false;
-  const nm_status v = spmm_validate(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, &noop);
+  const nm_status v =
+      spmm_validate(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, &noop);
   if (v != NM_OK || noop) return v;
-  if (ab_dtype != NM_F32)  // the 16-bit paths use no scratch at all
+  if (ab_dtype != NM_F32)  // the 16-bit and int8 paths use no scratch at all
     return nm_spmm(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, nullptr, 0, stream);
   const size_t need = nm_spmm_workspace_bytes(ab_dtype, R, K, T);
   if (need > kNoAllocScratchBytes) return NM_ERR_WORKSPACE;  // problem larger than the fixed scratch

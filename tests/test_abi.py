@@ -148,11 +148,43 @@ def test_host_validation_before_any_launch(lib):
     assert L.nm_spmm_noalloc(fake, fake, 0, fake, n, fake, 0, n, n, n, n, f(1), f(0), s) == 8       # too large
     assert L.nm_spmm_noalloc(fake, fake, 0, fake, n, fake, 0, n, 0, n, n, f(1), f(0), s) == 0       # R == 0
     # the test entry point: its own arguments, then nm_spmm's checks
+    # int8 product: K % 32, output types, exact s32 output only with alpha 1 and beta 0
+    assert L.nm_spmm(fake, fake, 3, fake, 16, fake, 4, 16, 128, 48, 16, f(1), f(0), None, 0, s) == 2
+    assert L.nm_spmm(fake, fake, 3, fake, 16, fake, 2, 16, 128, 64, 16, f(1), f(0), None, 0, s) == 4
+    assert L.nm_spmm(fake, fake, 3, fake, 16, fake, 4, 16, 128, 64, 16, f(2), f(0), None, 0, s) == 6
+    assert L.nm_spmm(fake, fake, 3, fake, 16, fake, 4, 16, 128, 64, 16, f(1), f(1), None, 0, s) == 6
+    assert L.nm_spmm(fake, fake, 3, fake, 8, fake, 4, 16, 128, 64, 8, f(1), f(0), None, 0, s) == 3   # ldx bytes % 16
+    assert L.nm_spmm(fake, fake, 1, fake, 8, fake, 4, 8, 128, 64, 8, f(1), f(0), None, 0, s) == 4    # s32 out of bf16
+    assert L.nm_spmm(fake, fake, 3, fake, 16, fake, 4, 16, 0, 64, 16, f(1), f(0), None, 0, s) == 0
+    # TF32 1:2 product: K % 16, output types, X row stride, NULL, empty
+    assert L.nm_spmm12(fake, fake, fake, 8, fake, 0, 8, 128, 40, 8, f(1), f(0), s) == 2
+    assert L.nm_spmm12(fake, fake, fake, 8, fake, 3, 8, 128, 64, 8, f(1), f(0), s) == 4
+    assert L.nm_spmm12(fake, fake, fake, 6, fake, 0, 8, 128, 64, 6, f(1), f(0), s) == 3
+    assert L.nm_spmm12(fake, None, fake, 8, fake, 0, 8, 128, 64, 8, f(1), f(0), s) == 1
+    assert L.nm_spmm12(fake, fake, fake, 8, fake, 0, 8, 128, 64, 0, f(1), f(0), s) == 0
+    assert L.nm_spmm12_test(fake, fake, fake, 8, fake, 0, 8, 128, 64, 8, f(1), f(0), 10, 1, s) == 2
+    # the two metadata images
+    assert L.nm_meta_to_sm100_s8(fake, 4, 60, fake, s) == 2
+    assert L.nm_meta_to_sm100_s8(None, 4, 64, fake, s) == 1
+    assert L.nm_meta_to_sm100_s8(fake, 4, 64, odd, s) == 3
+    assert L.nm_meta12_to_sm100(fake, 4, 40, fake, s) == 2
+    assert L.nm_meta12_to_sm100(fake, 4, 64, None, s) == 1
+    assert L.nm_meta12_to_sm100(fake, 0, 64, fake, s) == 0
     t = lambda kern, split, wait, skip, K=64: L.nm_spmm_test(fake, fake, 1, fake, 8, fake, 1, 8, 128, K, 8, f(1),
                                                               f(0), None, 0, kern, split, wait, skip, s)
     assert t(10, 1, 0, -1) == 2 and t(-1, 1, 0, -1) == 2
     assert t(0, 1, -5, -1) == 2 and t(0, 1, 0, -2) == 2
     assert t(1, 1, 0, -1, K=40) == 2
+
+
+def test_image_sizes(lib):
+    """.kind::i8: 128-row x 256-column stages, one bit per column; .kind::tf32:
+    2048 bytes per 128 rows x 64 fp32 columns."""
+    assert lib.nm_meta_s8_image_bytes(200, 300) == 256 * 512 // 8
+    assert lib.nm_meta_s8_image_bytes(128, 256) == 128 * 256 // 8
+    assert lib.nm_meta12_image_bytes(200, 100) == 2 * 2 * 2048
+    assert lib.nm_meta12_image_bytes(128, 64) == 2048
+    assert lib.nm_meta12_image_bytes(0, 64) == 0
 
 
 def test_workspace_size(lib):

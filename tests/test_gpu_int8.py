@@ -106,16 +106,19 @@ def test_full_size_decode_weight_quantised():
     assert np.array_equal(v.cpu().numpy(), rv) and np.array_equal(meta.cpu().numpy(), rm)
 
 
-def test_product_and_float_only_calls_refuse_int8():
+def test_float_only_calls_refuse_int8():
+    """int8 weights go to the selection, compression and product calls, not to
+    the floating-point ones; the int8 product takes no 16-bit output type
+    (host checks, nothing is launched)."""
     lib = nm.load()
     s = torch.cuda.current_stream().cuda_stream
     W = torch.zeros((128, 128), dtype=torch.int8, device="cuda")
     v, meta, img = nm.nm_mask_compress(W)
     X = torch.zeros((128, 64), dtype=torch.int8, device="cuda")
-    Y = torch.empty((128, 64), dtype=torch.float32, device="cuda")
-    st = lib.nm_spmm(v.data_ptr(), img.data_ptr(), 3, X.data_ptr(), 64, Y.data_ptr(), 0, 64, 128, 128, 64,
+    Y = torch.empty((128, 64), dtype=torch.float16, device="cuda")
+    st = lib.nm_spmm(v.data_ptr(), img.data_ptr(), 3, X.data_ptr(), 64, Y.data_ptr(), 2, 64, 128, 128, 64,
                      1.0, 0.0, None, 0, s)
-    assert st == 6                                                     # NM_ERR_UNSUPPORTED
+    assert st == 4                                                     # NM_ERR_DTYPE: no fp16 output
     d = torch.ones(128, dtype=torch.float32, device="cuda")
     m = torch.empty((128, 128), dtype=torch.uint8, device="cuda")
     assert lib.nm_mask_scored(W.data_ptr(), 3, d.data_ptr(), 128, 128, 128, 2, 4, m.data_ptr(), 128, s) == 4
