@@ -70,6 +70,10 @@ def transposable_int_ops(M: int) -> float:
         p *= 2
     return 2.0 * comps + 7.0 * M * M + 2.0 * M * M
 SPARSE_RATIO = 2.0   # 2:4 sparse tensor peak = 2x dense (dense-equivalent flops)
+# dense throughput of the int8 and tf32 tensor-core kinds relative to bf16 (nominal B200 figures:
+# 4.5 POPS int8, 1.1 PFLOPS tf32 against 2.25 PFLOPS bf16); applied to the measured bf16 peak
+KIND_RATIO = {"int8": 2.0, "pairs": 0.5}
+KIND_NOTE = {"int8": " x 2 (nominal int8/bf16 ratio)", "pairs": " x 0.5 (nominal tf32/bf16 ratio)"}
 
 
 def load_peaks():
@@ -134,14 +138,17 @@ def make_workload(name: str):
                         " of the inverse of a damped synthetic Gram matrix (512 calibration rows ~N(0,1))"}
     elif name == "int8_24":
         W = nm_inputs.int8_decode()
-        return {"W": W, "I8": True, "X": None, "R": W.shape[0], "K": W.shape[1], "T": 0,
-                "desc": "int8 2:4: the 28672x8192 decode weight quantised to int8; mask 2:4, fused mask+compress,"
-                        " decompress"}
+        X = nm_inputs.decode_X_int8(1024)
+        return {"W": W, "I8": True, "X": X, "R": W.shape[0], "K": W.shape[1], "T": X.shape[1],
+                "desc": "int8 2:4: the 28672x8192 decode weight quantised to int8, X its 8192x1024 activations"
+                        " quantised to int8; mask 2:4, fused mask+compress, .kind::i8 image, decompress, int8"
+                        " sparse product with exact int32 output"}
     elif name == "pairs_12":
         W = nm_inputs.fp32_linear()
-        return {"W": W, "P12": True, "X": None, "R": W.shape[0], "K": W.shape[1], "T": 0,
-                "desc": "1:2 pattern (sparse TF32): fp32 W 8192x8192 ~N(0,0.02); mask 1:2, compress under it,"
-                        " fused mask+compress, decompress"}
+        X = nm_inputs.fp32_linear_X(4096)
+        return {"W": W, "P12": True, "X": X, "R": W.shape[0], "K": W.shape[1], "T": X.shape[1],
+                "desc": "1:2 pattern (sparse TF32): fp32 W 8192x8192 ~N(0,0.02), X fp32 8192x4096 ~N(0,1); mask 1:2,"
+                        " compress under it, fused mask+compress, .kind::tf32 image, decompress, TF32 sparse product"}
     elif name == "transposable_mask":
         W, _ = nm_inputs.linear_4096()
         return {"W": W, "TM": (4, 8), "X": None, "R": 4096, "K": 4096, "T": 0,
@@ -230,10 +237,10 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- GPU arm
-def _dev_x(X: torch.Tensor, dev) -> torch.Tensor:
-    """X on the device in a buffer whose rows are 16-byte aligned."""
+def _dev_x(X: torch.Tensor, dev, mult: int = 8) -> torch.Tensor:
+    """X on the device in a buffer whose rows are 16-byte aligned (mult elements)."""
     K, T = X.shape
-    buf = torch.zeros((K, (T + 7) // 8 * 8), dtype=X.dtype, device=dev)
+    buf = torch.zeros((K, (T + mult - 1) // mult * mult), dtype=X.dtype, device=dev)
     buf[:, :T].copy_(X)
     return buf[:, :T]
 
@@ -250,26 +257,39 @@ class Step:
             ("ties" if wl["X"] is None else ("mlp" if "W2" in wl else "linear"))
         self.W = wl["W"].to(dev)
         if self.kind == "int8":
+            self.X = _dev_x(wl["X"], dev, 16)
             self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
-            self.values, self.meta, self.img = nm.alloc_compressed(R, K, self.W.dtype, dev)
+            self.values, self.meta, _ = nm.alloc_compressed(R, K, self.W.dtype, dev, sm100=False)
+            self.img = torch.empty((nm.nm_meta_s8_image_bytes(R, K),), dtype=torch.uint8, device=dev)
             self.Wd = torch.empty_like(self.W)
+            self.Y = torch.empty((R, T), dtype=torch.int32, device=dev)
             G = R * K
-            self.names = ["nm_mask_s8", "nm_mask_compress_s8", "nm_decompress_s8"]
-            self.bytes = {"nm_mask_s8": G * 2, "nm_mask_compress_s8": G * (1 + 0.5 + 0.25),
-                          "nm_decompress_s8": G * (0.5 + 0.125 + 1)}
-            self.flops = 0
+            self.names = ["nm_mask_s8", "nm_mask_compress_s8", "nm_meta_to_sm100_s8", "nm_decompress_s8",
+                          "nm_spmm_s8"]
+            self.bytes = {"nm_mask_s8": G * 2, "nm_mask_compress_s8": G * (1 + 0.5 + 0.125),
+                          "nm_meta_to_sm100_s8": G * 0.25, "nm_decompress_s8": G * (0.5 + 0.125 + 1),
+                          "nm_spmm_s8": G * (0.5 + 0.125) + K * T + R * T * 4}
+            self.flop_k = {"nm_spmm_s8": 2.0 * R * K * T}
+            self.flops = self.flop_k["nm_spmm_s8"]
             return
         if self.kind == "pairs":
+            self.X = _dev_x(wl["X"], dev, 4)
             self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
             self.v1, self.m1 = nm.alloc_compressed12(R, K, self.W.dtype, dev)
             self.v2, self.m2 = nm.alloc_compressed12(R, K, self.W.dtype, dev)
+            self.img = torch.empty((nm.nm_meta12_image_bytes(R, K),), dtype=torch.uint8, device=dev)
             self.Wd = torch.empty_like(self.W)
+            self.Y = torch.empty((R, T), dtype=torch.float32, device=dev)
             es = self.W.element_size()
             G = R * K
-            self.names = ["nm_mask_1:2", "nm_compress12", "nm_mask_compress12", "nm_decompress12"]
+            self.names = ["nm_mask_1:2", "nm_compress12", "nm_mask_compress12", "nm_meta12_to_sm100",
+                          "nm_decompress12", "nm_spmm12"]
             self.bytes = {"nm_mask_1:2": G * (es + 1), "nm_compress12": G * (es + 1 + es / 2 + 1 / 16),
-                          "nm_mask_compress12": G * (es + es / 2 + 1 / 16), "nm_decompress12": G * (es / 2 + 1 / 16 + es)}
-            self.flops = 0
+                          "nm_mask_compress12": G * (es + es / 2 + 1 / 16), "nm_meta12_to_sm100": G * (1 / 16 + 1 / 8),
+                          "nm_decompress12": G * (es / 2 + 1 / 16 + es),
+                          "nm_spmm12": G * (es / 2 + 1 / 8) + K * T * es + R * T * 4}
+            self.flop_k = {"nm_spmm12": 2.0 * R * K * T}
+            self.flops = self.flop_k["nm_spmm12"]
             return
         if self.kind == "transposable":
             self.mask = torch.empty((R, K), dtype=torch.uint8, device=dev)
@@ -390,16 +410,20 @@ class Step:
         if self.kind == "transposable":
             return [lambda: nm.nm_mask_transposable(self.W, *self.wl["TM"], mask=self.mask)]
         if self.kind == "int8":
-            K = self.wl["K"]
+            R, K = self.wl["R"], self.wl["K"]
             return [lambda: nm.nm_mask(self.W, 2, 4, mask=self.mask),
-                    lambda: nm.nm_mask_compress(self.W, self.values, self.meta, self.img),
-                    lambda: nm.nm_decompress(self.values, self.meta, K, out=self.Wd)]
+                    lambda: nm.nm_mask_compress(self.W, self.values, self.meta, None, sm100=False),
+                    lambda: nm.nm_meta_to_sm100_s8(self.meta, R, K, out=self.img),
+                    lambda: nm.nm_decompress(self.values, self.meta, K, out=self.Wd),
+                    lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.Y)]
         if self.kind == "pairs":
-            K = self.wl["K"]
+            R, K = self.wl["R"], self.wl["K"]
             return [lambda: nm.nm_mask(self.W, 1, 2, mask=self.mask),
                     lambda: nm.nm_compress12(self.W, self.mask, self.v1, self.m1),
                     lambda: nm.nm_mask_compress12(self.W, self.v2, self.m2),
-                    lambda: nm.nm_decompress12(self.v2, self.m2, K, out=self.Wd)]
+                    lambda: nm.nm_meta12_to_sm100(self.m2, R, K, out=self.img),
+                    lambda: nm.nm_decompress12(self.v2, self.m2, K, out=self.Wd),
+                    lambda: nm.nm_spmm12(self.v2, self.img, self.X, Y=self.Y)]
         if self.kind == "ties":
             return [(lambda i=i, N=N, M=M: nm.nm_mask(self.W, N, M, mask=self.masks[i]))
                     for i, (N, M) in enumerate([(1, 4), (2, 4), (4, 8), (2, 8)])]
@@ -448,10 +472,10 @@ class Step:
             return [[], [0], [0], [1], [2]]
         if self.kind == "ties":       # four masks of the same W
             return [[] for _ in range(n)]
-        if self.kind == "int8":       # mask; fused -> decompress
-            return [[], [], [1]]
-        if self.kind == "pairs":      # mask -> compress; fused -> decompress
-            return [[], [0], [], [2]]
+        if self.kind == "int8":       # mask; fused -> {image -> product, decompress}
+            return [[], [], [1], [1], [1, 2]]
+        if self.kind == "pairs":      # mask -> compress; fused -> {image -> product, decompress}
+            return [[], [0], [], [2], [2], [2, 3]]
         return [[i - 1] if i else [] for i in range(n)]
 
     def capture(self):
@@ -505,8 +529,6 @@ class Step:
             return self.GO
         if self.kind in ("scored", "transposable"):
             return self.mask
-        if self.kind in ("pairs", "int8"):
-            return self.Wd
         if self.kind == "trans24":
             return self.DX
         return self.masks[1] if self.kind == "ties" else self.Y
@@ -588,11 +610,19 @@ def dense_context(step: Step, reps: int, flush):
     """Context only: the same products as dense bf16 GEMMs in cuBLAS (torch.matmul)
     on the decompressed weights, timed like the step (L2 flushed before each rep).
     -> {name: ms} for the product launches of the step, or None."""
-    if step.kind not in ("linear", "mlp", "trans24"):
+    if step.kind not in ("linear", "mlp", "trans24", "int8", "pairs"):
         return None
     nm = step.nm
     s = torch.cuda.current_stream()
-    if step.kind == "linear":
+    mm = torch.matmul
+    if step.kind == "int8":          # cuBLAS int8 GEMM with int32 output
+        Wd = nm.nm_decompress(step.values, step.meta, step.wl["K"])
+        jobs = {"nm_spmm_s8": (Wd, step.X.contiguous())}
+        mm = torch._int_mm
+    elif step.kind == "pairs":       # cuBLAS fp32 GEMM on the TF32 tensor cores
+        Wd = nm.nm_decompress12(step.v2, step.m2, step.wl["K"])
+        jobs = {"nm_spmm12": (Wd, step.X.contiguous())}
+    elif step.kind == "linear":
         Wd = nm.nm_decompress(step.values, step.meta, step.wl["K"])
         jobs = {"nm_spmm": (Wd, step.X)}
     elif step.kind == "trans24":
@@ -603,20 +633,26 @@ def dense_context(step: Step, reps: int, flush):
         Wdn = nm.nm_decompress(step.v2, step.m2, step.W2.shape[1])
         jobs = {"nm_spmm_up": (Wu, step.X), "nm_spmm_down": (Wdn, step.H)}
     out = {}
-    for name, (A, B) in jobs.items():
-        C = torch.empty((A.shape[0], B.shape[1]), dtype=torch.bfloat16, device=A.device)
-        for _ in range(3):
-            torch.matmul(A, B, out=C)
-        ts = []
-        for _ in range(reps):
-            flush()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(s)
-            torch.matmul(A, B, out=C)
-            b.record(s)
-            b.synchronize()
-            ts.append(a.elapsed_time(b))
-        out[name] = float(np.median(ts))
+    tf32 = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = step.kind == "pairs"
+    try:
+        for name, (A, B) in jobs.items():
+            cdt = torch.int32 if step.kind == "int8" else (torch.float32 if step.kind == "pairs" else torch.bfloat16)
+            C = torch.empty((A.shape[0], B.shape[1]), dtype=cdt, device=A.device)
+            for _ in range(3):
+                mm(A, B, out=C)
+            ts = []
+            for _ in range(reps):
+                flush()
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record(s)
+                mm(A, B, out=C)
+                b.record(s)
+                b.synchronize()
+                ts.append(a.elapsed_time(b))
+            out[name] = float(np.median(ts))
+    finally:
+        torch.backends.cuda.matmul.allow_tf32 = tf32
     return out
 
 
@@ -696,22 +732,27 @@ def oracle_step(wl, rows: int, threads: int):
         t0 = time.perf_counter()
         oracle.mask_transposable(Wb, *wl["TM"], dtype=oracle.BF16)
         return time.perf_counter() - t0, float(rows * wl["K"] * 3)
-    if "I8" in wl:                # int8 2:4
+    if "I8" in wl:                # int8 2:4 with its product
         W = wl["W"][:rows].contiguous().numpy()
+        X = wl["X"].numpy()
         t0 = time.perf_counter()
         mask = oracle.mask_rank(W, 2, 4)
         v, m = oracle.compress24(W, mask)
-        oracle.meta_sm100(m, rows, wl["K"])
+        oracle.meta_sm100_s8(m, rows, wl["K"])
         oracle.decompress24(v, m, wl["K"])
-        return time.perf_counter() - t0, float(rows * wl["K"] * (2 + 1.75 + 1.625))
-    if "P12" in wl:               # 1:2 family on fp32
+        oracle.spmm(v, m, X, oracle.S8, threads=threads)
+        return time.perf_counter() - t0, 2.0 * rows * wl["K"] * wl["T"]
+    if "P12" in wl:               # 1:2 family on fp32 with the TF32 product
         W = wl["W"][:rows].contiguous().numpy()
+        X = wl["X"].numpy()
         t0 = time.perf_counter()
         mask = oracle.mask_rank(W, 1, 2)
         oracle.compress12(W, mask)
         v, m = oracle.compress12(W, mask)
+        oracle.meta12_sm100(m, rows, wl["K"])
         oracle.decompress12(v, m, wl["K"])
-        return time.perf_counter() - t0, float(rows * wl["K"] * (5 + 7.0625 + 6.0625 + 6.0625))
+        oracle.spmm12(v, m, X, threads=threads)
+        return time.perf_counter() - t0, 2.0 * rows * wl["K"] * wl["T"]
     if "D" in wl:                 # saliency-scored mask
         Wb = _u16(wl["W"][:rows].contiguous())
         d = wl["D"].numpy()
@@ -767,13 +808,13 @@ def cpu_baseline(wl, target_s: float = 15.0):
     threads = os.cpu_count() or 1
     rows = size_oracle_sample(wl, threads, target_s)
     secs, units = oracle_step(wl, rows, threads)
-    scale, unit = (1e12, "TFLOP/s") if wl["X"] is not None else (1e9, "GB/s")
+    scale, unit = ((1e12, "TOP/s" if "I8" in wl else "TFLOP/s") if wl["X"] is not None else (1e9, "GB/s"))
     what = ("SR-STE step (mask, masked weight, decay gradient)" if "G" in wl else
             "saliency-scored 2:4 mask" if "D" in wl else
             "greedy transposable 4:8 mask" if "TM" in wl else
             "transposable 2:4 mask, compress W and W^T, fp64 forward and backward products" if "T24" in wl else
-            "1:2 mask, compress, fused compress, decompress" if "P12" in wl else
-            "int8 2:4 mask, fused mask+compress, decompress" if "I8" in wl else
+            "1:2 mask, compress, fused compress, image, decompress, fp64 1:2 product" if "P12" in wl else
+            "int8 2:4 mask, compress, image, decompress, exact int8 product" if "I8" in wl else
             "mask at 1:4, 2:4, 4:8, 2:8" if wl["X"] is None else
             "whole step on the sampled rows of both weights (mask, compress, fused mask+compress, image, "
             "decompress, fp64 product; the down product's input is a zero stand-in of H's shape)" if "W2" in wl else
@@ -794,14 +835,15 @@ def run_reference(args, wl, metric):
         s, u = oracle_step(wl, rows, threads)
         tot_s += s
         tot_u += u
-    scale, unit = (1e12, "TFLOP/s") if wl["X"] is not None else (1e9, "GB/s")
+    scale, unit = ((1e12, "TOP/s" if "I8" in wl else "TFLOP/s") if wl["X"] is not None else (1e9, "GB/s"))
     value = tot_u / tot_s / scale
     sample = "first %d of %d rows of W per step, whole step on the CPU oracle" % (rows, wl["R"])
     line = {"metric": metric, "value": value, "unit": unit, "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * tot_s / max(1, args.steps), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "data": "synthetic",
             # the oracle's arithmetic: fp64 product, binary32 decay term / scores, integer magnitude keys
-            "dtype": "f64" if wl["X"] is not None else ("f32" if ("G" in wl or "D" in wl) else "u32"),
+            "dtype": ("int64" if "I8" in wl else "f64") if wl["X"] is not None else
+                     ("f32" if ("G" in wl or "D" in wl) else "u32"),
             "config": {"workload": args.workload, "desc": wl["desc"], "R": wl["R"], "K": wl["K"], "T": wl["T"]},
             "impl": "reference",
             "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle", "sample": sample},
@@ -928,13 +970,12 @@ def main():
             k.update({"TFLOP/s": tf, "tensor_frac": tf / sparse_peak})
         kernels[name] = k
 
-    if step.kind in ("ties", "srste", "scored", "transposable", "pairs", "int8"):
+    if step.kind in ("ties", "srste", "scored", "transposable"):
         units_per_step = sum(step.bytes.values())
         value = whole_job_rate(world, units_per_step, args.steps, total_ms, 1e9)
         unit = "GB/s"
         dom = {"ties": "nm_mask_2:4", "srste": "nm_srste_step", "scored": "nm_mask_scored",
-               "transposable": "nm_mask_transposable", "pairs": "nm_mask_compress12",
-               "int8": "nm_mask_compress_s8"}[step.kind]
+               "transposable": "nm_mask_transposable"}[step.kind]
         if step.kind == "transposable":
             N_, M_ = wl["TM"]
             ops = transposable_int_ops(M_) * (wl["R"] // M_) * (wl["K"] // M_)
@@ -949,14 +990,21 @@ def main():
         e2e_value = whole_job_rate(world, units_per_step, args.steps, e2e_ms, 1e9)
     else:
         value = whole_job_rate(world, step.flops, args.steps, total_ms, 1e12)
-        unit = "TFLOP/s"
+        unit = "TOP/s" if step.kind == "int8" else "TFLOP/s"
         dom = max(step.flop_k, key=lambda n: np.mean(per[n]))
-        roof = {"bound": "tensor", "achieved": kernels[dom]["TFLOP/s"], "peak": sparse_peak, "unit": "TFLOP/s",
-                "frac": kernels[dom]["TFLOP/s"] / sparse_peak, "kernel": dom,
+        # the product's own tensor peak: 2:4 (or 1:2) sparse = 2 x dense of its
+        # operand type; int8 and tf32 dense taken as the measured bf16 figure
+        # times the nominal B200 ratios (int8 2x, tf32 0.5x bf16)
+        ratio = KIND_RATIO.get(step.kind, 1.0)
+        peak = sparse_peak * ratio
+        roof = {"bound": "tensor", "achieved": kernels[dom]["TFLOP/s"], "peak": peak, "unit": unit,
+                "frac": kernels[dom]["TFLOP/s"] / peak, "kernel": dom,
                 "algorithmic_flops_per_launch": step.flop_k[dom]}
+        kernels[dom]["tensor_frac"] = kernels[dom]["TFLOP/s"] / peak
         e2e_value = whole_job_rate(world, step.flops, args.steps, e2e_ms, 1e12)
-    roof["peak_source"] = ("%s: 2 x dense bf16 %s" % (peak_src, "sustained (power cap seen in the timed region)"
-                                                      if dense_key.endswith("sustained") else "burst")
+    roof["peak_source"] = ("%s: 2 x dense bf16 %s%s" % (peak_src, "sustained (power cap seen in the timed region)"
+                                                        if dense_key.endswith("sustained") else "burst",
+                                                        KIND_NOTE.get(step.kind, ""))
                            if roof["bound"] == "tensor" else
                            "derived: 148 SMs x 64 integer lanes x 1965 MHz" if roof["bound"] == "alu" else
                            "%s: HBM copy" % peak_src)
@@ -965,8 +1013,9 @@ def main():
     dense = dense_context(step, 20, flush)
     dense_line = None
     if dense:
-        dense_line = {"what": "context only: dense bf16 torch.matmul (cuBLAS) on decompress(W), same shapes, "
-                              "L2 flushed, median of 20",
+        dense_line = {"what": "context only: the dense cuBLAS GEMM of the same operand type on decompress(W) "
+                              "(bf16 torch.matmul; int8 torch._int_mm; fp32 torch.matmul on the TF32 tensor cores), "
+                              "same shapes, L2 flushed, median of 20",
                       "kernels": {}}
         for name, ms in dense.items():
             tf = step.flop_k[name] / (ms * 1e-3) / 1e12

@@ -36,7 +36,7 @@ class _Recorder:
         self.log.append(({_key(t) for t in reads if t is not None}, {_key(t) for t in writes if t is not None}))
 
     # allocation and sizing
-    def alloc_compressed(self, R, K, dtype, dev):
+    def alloc_compressed(self, R, K, dtype, dev, sm100=True):
         return (torch.empty((R, K // 2), dtype=dtype, device=dev), torch.empty((R, K // 4), dtype=torch.uint8, device=dev),
                 torch.empty((128, 128), dtype=torch.uint8, device=dev))
 
@@ -65,8 +65,23 @@ class _Recorder:
     def nm_compress_t(self, W, mask, values, meta, img):
         self._rec([W, mask], [values, meta, img])
 
-    def nm_mask_compress(self, W, values, meta, img):
+    def nm_mask_compress(self, W, values, meta, img, sm100=True):
         self._rec([W], [values, meta, img])
+
+    def nm_meta_s8_image_bytes(self, R, K):
+        return 256
+
+    def nm_meta12_image_bytes(self, R, K):
+        return 256
+
+    def nm_meta_to_sm100_s8(self, meta, R, K, out):
+        self._rec([meta], [out])
+
+    def nm_meta12_to_sm100(self, meta, R, K, out):
+        self._rec([meta], [out])
+
+    def nm_spmm12(self, values, img, X, Y):
+        self._rec([values, img, X], [Y])
 
     def nm_meta_to_sm100(self, meta, R, K, out):
         self._rec([meta], [out])
@@ -83,7 +98,7 @@ class _Recorder:
     def nm_decompress12(self, values, meta, K, out):
         self._rec([values, meta], [out])
 
-    def nm_spmm(self, values, img, X, Y, workspace):
+    def nm_spmm(self, values, img, X, Y, workspace=None):
         self._rec([values, img, X], [Y, workspace])
 
 
@@ -97,9 +112,10 @@ WORKLOADS = {
     "mlp": {"W": _bf16(R, K), "W2": _bf16(K, R), "X": _bf16(K, T), "R": R, "K": K, "T": T},
     "trans24": {"W": _bf16(R, K), "X": _bf16(K, T), "DY": _bf16(R, T), "T24": True, "R": R, "K": K, "T": T},
     "ties": {"W": torch.randn(R, K), "X": None, "R": R, "K": K, "T": 0},
-    "int8": {"W": torch.randint(-128, 128, (R, K), dtype=torch.int16).to(torch.int8), "I8": True, "X": None,
+    "int8": {"W": torch.randint(-128, 128, (R, K), dtype=torch.int16).to(torch.int8), "I8": True,
+             "X": torch.randint(-128, 128, (K, T), dtype=torch.int16).to(torch.int8),
              "R": R, "K": K, "T": 0},
-    "pairs": {"W": torch.randn(R, K), "P12": True, "X": None, "R": R, "K": K, "T": 0},
+    "pairs": {"W": torch.randn(R, K), "P12": True, "X": torch.randn(K, T), "R": R, "K": K, "T": T},
     "transposable": {"W": _bf16(R, K), "TM": (4, 8), "X": None, "R": R, "K": K, "T": 0},
     "scored": {"W": _bf16(R, K), "D": torch.rand(K), "X": None, "R": R, "K": K, "T": 0},
     "srste": {"W": _bf16(R, K), "G": _bf16(R, K), "X": None, "R": R, "K": K, "T": 0},
