@@ -256,10 +256,18 @@ def nm_meta_to_sm100(meta: torch.Tensor, R: int, C: int, out: torch.Tensor | Non
     return out
 
 
+def nm_meta_s8_image_bytes(R: int, C: int) -> int:
+    return int(_lib().nm_meta_s8_image_bytes(R, C))
+
+
+def nm_meta12_image_bytes(R: int, C: int) -> int:
+    return int(_lib().nm_meta12_image_bytes(R, C))
+
+
 def nm_meta_to_sm100_s8(meta: torch.Tensor, R: int, C: int, out: torch.Tensor | None = None, stream=None):
     """Canonical 2:4 metadata of an int8 matrix -> the image the int8 product reads."""
     if out is None:
-        out = torch.empty((int(_lib().nm_meta_s8_image_bytes(R, C)),), dtype=torch.uint8, device=meta.device)
+        out = torch.empty((nm_meta_s8_image_bytes(R, C),), dtype=torch.uint8, device=meta.device)
     _check(_lib().nm_meta_to_sm100_s8(_ptr(meta), R, C, _ptr(out), _stream(stream)), "nm_meta_to_sm100_s8")
     return out
 
@@ -267,7 +275,7 @@ def nm_meta_to_sm100_s8(meta: torch.Tensor, R: int, C: int, out: torch.Tensor | 
 def nm_meta12_to_sm100(meta: torch.Tensor, R: int, C: int, out: torch.Tensor | None = None, stream=None):
     """Canonical 1:2 metadata -> the image the TF32 1:2 product reads."""
     if out is None:
-        out = torch.empty((int(_lib().nm_meta12_image_bytes(R, C)),), dtype=torch.uint8, device=meta.device)
+        out = torch.empty((nm_meta12_image_bytes(R, C),), dtype=torch.uint8, device=meta.device)
     _check(_lib().nm_meta12_to_sm100(_ptr(meta), R, C, _ptr(out), _stream(stream)), "nm_meta12_to_sm100")
     return out
 
@@ -327,26 +335,49 @@ def nm_spmm_test(values: torch.Tensor, meta_sm100: torch.Tensor, X: torch.Tensor
     return Y
 
 
-def nm_spmm12(values: torch.Tensor, meta12_sm100: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = None,
-              y_dtype: torch.dtype = torch.float32, alpha: float = 1.0, beta: float = 0.0, kernel: str | None = None,
-              tail_split: bool = True, stream=None) -> torch.Tensor:
-    """Y = alpha * (W (.) mask) X + beta * Y for a 1:2-sparse fp32 W (values R x K/2,
-    the nm_meta12_to_sm100 image) on the TF32 sparse tensor cores.  `kernel` /
-    `tail_split` go through the test entry point."""
+def _spmm12_args(values, meta12_sm100, X, Y, y_dtype, alpha, beta):
     R, Kh = values.shape
     K = 2 * Kh
     Kx, T = X.shape
     assert Kx == K, "X must be K x T"
     if Y is None:
         Y = torch.empty((R, T), dtype=y_dtype, device=values.device)
-    lib = _lib()
-    args = (_ptr(values), _ptr(meta12_sm100), _ptr(X), _ld(X), _ptr(Y), _dtype(Y), _ld(Y), R, K, T, float(alpha),
-            float(beta))
-    if kernel is None and tail_split:
-        _check(lib.nm_spmm12(*args, _stream(stream)), "nm_spmm12")
-    else:
-        _check(lib.nm_spmm12_test(*args, SPMM_KERNELS[kernel or "default"], 1 if tail_split else 0,
-                                  _stream(stream)), "nm_spmm12_test")
+    return Y, (_ptr(values), _ptr(meta12_sm100), _ptr(X), _ld(X), _ptr(Y), _dtype(Y), _ld(Y), R, K, T,
+               float(alpha), float(beta))
+
+
+def nm_spmm12(values: torch.Tensor, meta12_sm100: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = None,
+              y_dtype: torch.dtype = torch.float32, alpha: float = 1.0, beta: float = 0.0, stream=None) -> torch.Tensor:
+    """Y = alpha * (W (.) mask) X + beta * Y for a 1:2-sparse fp32 W (values R x K/2,
+    the nm_meta12_to_sm100 image) on the TF32 sparse tensor cores."""
+    Y, args = _spmm12_args(values, meta12_sm100, X, Y, y_dtype, alpha, beta)
+    _check(_lib().nm_spmm12(*args, _stream(stream)), "nm_spmm12")
+    return Y
+
+
+def nm_spmm12_test(values: torch.Tensor, meta12_sm100: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = None,
+                   y_dtype: torch.dtype = torch.float32, alpha: float = 1.0, beta: float = 0.0,
+                   kernel: str = "default", tail_split: bool = True, stream=None) -> torch.Tensor:
+    """nm_spmm12 with a forced tile configuration and the half-width last wave on or off."""
+    Y, args = _spmm12_args(values, meta12_sm100, X, Y, y_dtype, alpha, beta)
+    _check(_lib().nm_spmm12_test(*args, SPMM_KERNELS[kernel], 1 if tail_split else 0, _stream(stream)),
+           "nm_spmm12_test")
+    return Y
+
+
+def nm_spmm_noalloc(values: torch.Tensor, meta_sm100: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = None,
+                    y_dtype: torch.dtype = torch.bfloat16, alpha: float = 1.0, beta: float = 0.0,
+                    stream=None) -> torch.Tensor:
+    """nm_spmm without a workspace: fp32 inputs are staged in the library's fixed device array."""
+    R, Kh = values.shape
+    K = 2 * Kh
+    Kx, T = X.shape
+    assert Kx == K, "X must be K x T"
+    if Y is None:
+        Y = torch.empty((R, T), dtype=y_dtype, device=values.device)
+    _check(_lib().nm_spmm_noalloc(_ptr(values), _ptr(meta_sm100), _dtype(values), _ptr(X), _ld(X), _ptr(Y),
+                                  _dtype(Y), _ld(Y), R, K, T, float(alpha), float(beta), _stream(stream)),
+           "nm_spmm_noalloc")
     return Y
 
 

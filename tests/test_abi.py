@@ -200,3 +200,9 @@ def test_no_cpu_fallback_in_the_binding():
         src = f.read()
     assert "oracle" not in src.replace("no CPU\nfallback", "")
     assert "import numpy" not in src
+
+
+def test_binding_has_every_declared_call():
+    """The Python binding keeps the C names: one function per declared call."""
+    missing = [name for name in _declared() if not callable(getattr(nm, name, None))]
+    assert missing == []

@@ -160,7 +160,11 @@ def _tf32_gpu(W, X, y_dtype=torch.float32, kernel=None, alpha=1.0, beta=0.0, Y0=
     values, meta = nm.nm_mask_compress12(W.cuda())
     img = nm.nm_meta12_to_sm100(meta, R, K)
     Y = None if Y0 is None else Y0.clone().cuda()
-    Y = nm.nm_spmm12(values, img, _dev_x(X, 4), Y=Y, y_dtype=y_dtype, alpha=alpha, beta=beta, kernel=kernel)
+    if kernel is None:
+        Y = nm.nm_spmm12(values, img, _dev_x(X, 4), Y=Y, y_dtype=y_dtype, alpha=alpha, beta=beta)
+    else:
+        Y = nm.nm_spmm12_test(values, img, _dev_x(X, 4), Y=Y, y_dtype=y_dtype, alpha=alpha, beta=beta,
+                              kernel=kernel)
     torch.cuda.synchronize()
     assert nm.nm_last_device_status() == 0
     return Y.cpu()
