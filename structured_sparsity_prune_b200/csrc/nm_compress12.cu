@@ -265,31 +265,50 @@ extern "C" nm_status nm_decompress12(const void* values, const uint8_t* meta, nm
 namespace nm {
 namespace {
 
+// A lane row holds two rows (r0 = 16*(L/16) + L%8 and r0 + 8), and for each
+// row the pairs kt*32 + 8*s + 4*((L/8)%2) + q, s, q in 0..3: all inside the
+// row's 32-bit metadata word kt.  So a thread reads two words and spreads
+// their bits; with C % 64 == 0 (whole words per block) the words are loaded
+// whole, otherwise byte by byte.
 __global__ void __launch_bounds__(256) meta12_image_kernel(const uint8_t* __restrict__ meta, int64_t R, int64_t C,
                                                            int64_t kblocks, int64_t nrows16,
                                                            uint4* __restrict__ out) {
   const int64_t bpr = C / 16;  // metadata bytes per row
+  const bool words = (C % 64) == 0 && (reinterpret_cast<uintptr_t>(meta) & 3u) == 0;
   for (int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; t < nrows16;
        t += int64_t(gridDim.x) * blockDim.x) {
     const int64_t blk = t >> 7;
     const int L = int(t & 127);
     const int64_t rt = blk / kblocks, kt = blk - rt * kblocks;
-    uint32_t w[4];
+    uint32_t w[2];
+#pragma unroll
+    for (int h8 = 0; h8 < 2; ++h8) {
+      const int64_t r = rt * 128 + 16 * (L >> 4) + 8 * h8 + (L & 7);
+      uint32_t v = 0;                      // index bits of pairs kt*32 .. kt*32+31 (0 past the matrix: 0x4)
+      if (r < R) {
+        const uint8_t* src = meta + r * bpr + kt * 4;
+        if (words) {
+          v = __ldg(reinterpret_cast<const uint32_t*>(src));
+        } else {
+          for (int j = 0; j < 4 && kt * 4 + j < bpr; ++j) v |= uint32_t(src[j]) << (8 * j);
+        }
+      }
+      w[h8] = v;
+    }
+    const int half = (L >> 3) & 1;
+    uint32_t o[4];
 #pragma unroll
     for (int sl = 0; sl < 4; ++sl) {
       uint32_t word = 0;
 #pragma unroll
       for (int n = 0; n < 8; ++n) {
         const int h8 = n >> 2, q = n & 3;
-        const int64_t r = rt * 128 + 16 * (L >> 4) + 8 * h8 + (L & 7);
-        const int64_t p = kt * 32 + (32 * sl + 16 * ((L >> 3) & 1) + 4 * q) / 4;
-        uint32_t nib = 0x4u;
-        if (r < R && p < C / 2 && ((meta[r * bpr + (p >> 3)] >> (p & 7)) & 1u)) nib = 0xEu;
-        word |= nib << (16 * h8 + 4 * q);
+        const uint32_t bit = (w[h8] >> (8 * sl + 4 * half + q)) & 1u;
+        word |= (bit ? 0xEu : 0x4u) << (16 * h8 + 4 * q);
       }
-      w[sl] = word;
+      o[sl] = word;
     }
-    out[t] = make_uint4(w[0], w[1], w[2], w[3]);
+    out[t] = make_uint4(o[0], o[1], o[2], o[3]);
   }
 }
 
