@@ -359,7 +359,20 @@ class Step:
             self.img2_r = torch.empty_like(self.img2)
             self.Wd = torch.empty_like(self.W)
             self.W2d = torch.empty_like(self.W2)
-            self.H = torch.empty((R, (T + 7) // 8 * 8), dtype=torch.bfloat16, device=dev)[:, :T]
+            Tp = (T + 7) // 8 * 8
+            self.gather = wl.get("gather")
+            if self.gather is None:
+                self.H = torch.empty((R, Tp), dtype=torch.bfloat16, device=dev)[:, :T]
+                self.H_down = self.H
+            else:
+                # the up product writes this rank's rows into a slice-sized buffer; the
+                # all-gather assembles every rank's rows; the down product reads them all
+                dist_, per, R_full = self.gather
+                world_ = dist_.get_world_size()
+                self.H_local = torch.zeros((per, Tp), dtype=torch.bfloat16, device=dev)
+                self.H_all = torch.empty((world_ * per, Tp), dtype=torch.bfloat16, device=dev)
+                self.H = self.H_local[:R, :T]
+                self.H_down = self.H_all[:R_full, :T]
             self.Y = torch.empty((R2, T), dtype=torch.bfloat16, device=dev)
             ws = max(nm.nm_spmm_workspace_bytes(self.W.dtype, R, K, T),
                      nm.nm_spmm_workspace_bytes(self.W2.dtype, R2, K2, T))
@@ -373,9 +386,11 @@ class Step:
                                    "nm_mask_compress_" + tag: G * (es + es / 2 + 0.25),
                                    "nm_meta_to_sm100_" + tag: G * 0.25,
                                    "nm_decompress_" + tag: G * (es / 2 + 0.125 + es)})
-            self.names += ["nm_spmm_up", "nm_spmm_down"]
+            self.names += ["nm_spmm_up"] + (["all_gather_H"] if self.gather else []) + ["nm_spmm_down"]
             self.bytes.update({"nm_spmm_up": R * K * (es / 2 + 0.125) + K * T * es + R * T * 2,
                                "nm_spmm_down": R2 * K2 * (es / 2 + 0.125) + K2 * T * es + R2 * T * 2})
+            if self.gather:
+                self.bytes["all_gather_H"] = self.H_all.numel() * self.H_all.element_size()
             self.flop_k = {"nm_spmm_up": 2.0 * R * K * T, "nm_spmm_down": 2.0 * R2 * K2 * T}
             self.flops = sum(self.flop_k.values())
             return
@@ -446,8 +461,9 @@ class Step:
                     lambda: nm.nm_mask_compress(self.W2, self.v2, self.m2, self.img2),
                     lambda: nm.nm_meta_to_sm100(self.m2, R2, K2, out=self.img2_r),
                     lambda: nm.nm_decompress(self.v2, self.m2, K2, out=self.W2d),
-                    lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.H, workspace=self.ws),
-                    lambda: nm.nm_spmm(self.v2, self.img2, self.H, Y=self.Y, workspace=self.ws)]
+                    lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.H, workspace=self.ws)] + \
+                ([lambda: gather_rows(self.gather[0], self.H_all, self.H_local)] if self.gather else []) + \
+                [lambda: nm.nm_spmm(self.v2, self.img2, self.H_down, Y=self.Y, workspace=self.ws)]
         K = self.wl["K"]
         return [lambda: nm.nm_mask(self.W, 2, 4, mask=self.mask),
                 lambda: nm.nm_compress(self.W, self.mask, self.v_c, self.m_c, self.img_c),
@@ -467,6 +483,9 @@ class Step:
             return [[], [0], [], [2], [2], [2]]
         if self.kind == "mlp":        # per weight: mask -> compress; fused -> {image, decompress}; then
             #                               up product after the fused up call, down after fused down and up
+            #                               (split by rows: up -> all-gather of H -> down)
+            if self.gather:
+                return [[], [0], [], [2], [2], [], [5], [], [7], [7], [2], [10], [7, 11]]
             return [[], [0], [], [2], [2], [], [5], [], [7], [7], [2], [7, 10]]
         if self.kind == "trans24":    # mask -> {compress -> forward, compress_t -> backward}
             return [[], [0], [0], [1], [2]]
@@ -631,7 +650,7 @@ def dense_context(step: Step, reps: int, flush):
     else:
         Wu = nm.nm_decompress(step.values, step.meta, step.wl["K"])
         Wdn = nm.nm_decompress(step.v2, step.m2, step.W2.shape[1])
-        jobs = {"nm_spmm_up": (Wu, step.X), "nm_spmm_down": (Wdn, step.H)}
+        jobs = {"nm_spmm_up": (Wu, step.X), "nm_spmm_down": (Wdn, step.H_down)}
     out = {}
     tf32 = torch.backends.cuda.matmul.allow_tf32
     torch.backends.cuda.matmul.allow_tf32 = step.kind == "pairs"
@@ -865,6 +884,50 @@ def max_over_ranks(pg, values, device):
     return [float(v) for v in t.tolist()]
 
 
+def shard_rows(R: int, world: int, rank: int, align: int = 256):
+    """Rows [lo, hi) of an R-row weight that `rank` holds when the rows are split
+    over `world` ranks in slices of one common size `per` (a multiple of `align`,
+    so every slice is whole CTA-pair tiles); the last slices may be short or
+    empty.  -> (lo, hi, per)"""
+    per = -(-R // world)
+    per = -(-per // align) * align
+    lo = min(R, rank * per)
+    return lo, min(R, lo + per), per
+
+
+def gather_rows(dist, out: torch.Tensor, local: torch.Tensor):
+    """All-gather of equal row slices: rank i's `local` (per x T) lands in rows
+    [i*per, (i+1)*per) of `out` (world*per x T) on every rank.  NCCL gathers into
+    the tensor directly; other backends (gloo, in the CPU tests) through a list."""
+    if dist.get_backend() == "nccl":
+        dist.all_gather_into_tensor(out, local)
+    else:
+        parts = list(out.split(local.shape[0]))
+        dist.all_gather(parts, local.contiguous())
+        for dst, src in zip(out.split(local.shape[0]), parts):
+            if dst.data_ptr() != src.data_ptr():
+                dst.copy_(src)
+
+
+def split_workload(wl, world: int, rank: int, dist):
+    """The rank's share of a product workload split by output rows: its rows of
+    W (and of W_down for the MLP pair), all of X.  The MLP pair's hidden
+    activation H = W_up X is row-split too and all-gathered before the down
+    product, the path's one exchange; the transformer linear needs none."""
+    lo, hi, per = shard_rows(wl["R"], world, rank)
+    out = dict(wl)
+    out["W"] = wl["W"][lo:hi]
+    out["R"] = hi - lo
+    out["rows"] = (lo, hi)
+    if "W2" in wl:
+        R2 = wl["W2"].shape[0]
+        lo2, hi2, _ = shard_rows(R2, world, rank)
+        out["W2"] = wl["W2"][lo2:hi2]
+        out["rows2"] = (lo2, hi2)
+        out["gather"] = (dist, per, wl["R"])       # H slices of `per` rows, R_up rows in all
+    return out
+
+
 def whole_job_rate(world: int, units_per_step: float, steps: int, ms: float, scale: float) -> float:
     """Units every rank processed (each rank runs the full step) per second,
     divided by `scale` (1e12 for TFLOP/s, 1e9 for GB/s)."""
@@ -879,6 +942,9 @@ def main():
     ap.add_argument("--impl", default="nm", choices=["nm", "reference"])
     ap.add_argument("--workload", default="mlp_pair")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "rows"],
+                    help="N > 1: an independent replica of the workload per GPU (weak scaling), or one problem "
+                         "split by output rows over the GPUs (strong scaling; linear_4096 and mlp_pair)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -902,8 +968,15 @@ def main():
 
     import structured_sparsity_prune_b200 as nm
     nm.load()                                    # fails loudly without the CUDA library
-    wl = make_workload(args.workload)
+    wl_full = make_workload(args.workload)
+    split = args.split == "rows" and world > 1
+    if split and args.workload not in ("linear_4096", "mlp_pair"):
+        raise SystemExit("--split rows applies to the product workloads linear_4096 and mlp_pair")
+    wl = split_workload(wl_full, world, rank, pg) if split else wl_full
     step = Step(nm, wl, dev)
+    # work of the whole job per step: every rank's replica, or the one split problem
+    full_flops = 2.0 * wl_full["R"] * wl_full["K"] * wl_full["T"] + \
+        (2.0 * wl_full["W2"].shape[0] * wl_full["W2"].shape[1] * wl_full["T"] if "W2" in wl_full else 0.0)
     flush = L2Flush(dev)
 
     for _ in range(warmup):
@@ -912,6 +985,8 @@ def main():
     if nm.nm_last_device_status() != 0:
         raise SystemExit("device status reports a timed-out wait")
     try:
+        if split:   # the all-gather stays outside CUDA graphs: the split step is timed as eager launches
+            raise RuntimeError("row-split step with a collective, timed eagerly")
         eager = step.result().clone()
         graphs = step.capture()
         launch_mode = ("CUDA graph of the step as its dependency graph (independent launches on forked "
@@ -989,7 +1064,8 @@ def main():
                     "algorithmic_bytes_per_launch": step.bytes[dom]}
         e2e_value = whole_job_rate(world, units_per_step, args.steps, e2e_ms, 1e9)
     else:
-        value = whole_job_rate(world, step.flops, args.steps, total_ms, 1e12)
+        value = (full_flops * args.steps / (total_ms * 1e-3) / 1e12 if split
+                 else whole_job_rate(world, step.flops, args.steps, total_ms, 1e12))
         unit = "TOP/s" if step.kind == "int8" else "TFLOP/s"
         dom = max(step.flop_k, key=lambda n: np.mean(per[n]))
         # the product's own tensor peak: 2:4 (or 1:2) sparse = 2 x dense of its
@@ -1001,7 +1077,8 @@ def main():
                 "frac": kernels[dom]["TFLOP/s"] / peak, "kernel": dom,
                 "algorithmic_flops_per_launch": step.flop_k[dom]}
         kernels[dom]["tensor_frac"] = kernels[dom]["TFLOP/s"] / peak
-        e2e_value = whole_job_rate(world, step.flops, args.steps, e2e_ms, 1e12)
+        e2e_value = (full_flops * args.steps / (e2e_ms * 1e-3) / 1e12 if split
+                     else whole_job_rate(world, step.flops, args.steps, e2e_ms, 1e12))
     roof["peak_source"] = ("%s: 2 x dense bf16 %s%s" % (peak_src, "sustained (power cap seen in the timed region)"
                                                         if dense_key.endswith("sustained") else "burst",
                                                         KIND_NOTE.get(step.kind, ""))
@@ -1029,9 +1106,10 @@ def main():
     if rank == 0:
         line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
                 "warmup": warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": str(wl["W"].dtype).replace("torch.", ""),
+                "scaling": "strong" if split else "weak", "vs_baseline": None,
+                "dtype": str(wl["W"].dtype).replace("torch.", ""),
                 "data": "synthetic",
-                "config": {"workload": args.workload, "desc": wl["desc"], "R": wl["R"], "K": wl["K"], "T": wl["T"],
+                "config": {"workload": args.workload, "desc": wl["desc"], "R": wl_full["R"], "K": wl["K"], "T": wl["T"],
                            "sparsity": {"ties": "N:M along K (1:4, 2:4, 4:8, 2:8)", "pairs": "1:2 along K",
                                         "transposable": "4:8 transposable (8x8 blocks)",
                                         "trans24": "2:4 transposable (4x4 blocks)"}.get(step.kind, "2:4 along K"),
@@ -1040,7 +1118,10 @@ def main():
                            "launch": launch_mode,
                            "step_sequential_ms": seq_ms,
                            "event_floor_us": floor_us,
-                           "parallelism": "independent replica per GPU" if world > 1 else "single GPU"},
+                           "parallelism": ("rows of W split over the GPUs, X replicated%s" %
+                                           (", H all-gathered (NCCL) before the down product"
+                                            if step.kind == "mlp" else ", no exchange")) if split else
+                                          ("independent replica per GPU" if world > 1 else "single GPU")},
                 "roofline": roof, "cpu_baseline": cpu, "dense_context": dense_line,
                 "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "method": "public calls with pinned host buffers; H2D, step and D2H of consecutive steps "

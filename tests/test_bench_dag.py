@@ -156,6 +156,46 @@ def test_dependency_graph_covers_the_data_flow(kind):
                     kind, j, step.names[j], i, step.names[i])
 
 
+class _FakeDist:
+    """Stands in for torch.distributed in the row-split MLP step: the all-gather
+    of H is recorded like a launch (reads this rank's H rows, writes all of H)."""
+
+    def __init__(self, rec):
+        self.rec = rec
+
+    def get_world_size(self):
+        return 2
+
+    def get_backend(self):
+        return "nccl"
+
+    def all_gather_into_tensor(self, out, local):
+        self.rec._rec([local], [out])
+
+
+def test_row_split_mlp_step_orders_the_all_gather():
+    """--split rows: up product -> all-gather of H -> down product, and every
+    buffer shared between launches ordered by the graph."""
+    rec = _Recorder()
+    wl = bench.split_workload(WORKLOADS["mlp"], 2, 0, _FakeDist(rec))
+    step = bench.Step(rec, wl, torch.device("cpu"))
+    calls, deps = step.calls(), step.deps()
+    assert "all_gather_H" in step.names and len(calls) == len(deps) == len(step.names)
+    for fn in calls:
+        fn()
+    before = _closure(deps)
+    for i, d in enumerate(deps):
+        reads_i, writes_i = rec.log[i]
+        for j in d:
+            assert rec.log[j][1] & reads_i
+        for j in range(i):
+            reads_j, writes_j = rec.log[j]
+            if (writes_j & reads_i) or (reads_j & writes_i) or (writes_j & writes_i):
+                assert j in before[i], (step.names[j], step.names[i])
+    up, ag, down = (step.names.index(n) for n in ("nm_spmm_up", "all_gather_H", "nm_spmm_down"))
+    assert up in before[ag] and ag in before[down]
+
+
 def test_the_linear_step_forks():
     """The default step is not a chain: after the fused mask+compress, the
     image reorder, the decompression and the product are independent."""
