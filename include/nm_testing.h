@@ -54,15 +54,23 @@ enum {
  *                  other roles, lets the copies it issued land, frees its
  *                  tensor memory and returns.  Y is then undefined.  Every
  *                  later call runs normally.
+ *   raster_group, raster_m_inner
+ *                  0, 0: the library's tile order.  raster_group > 0: tiles
+ *                  run in groups of raster_group tiles of the operand named
+ *                  by raster_m_inner (1: row tiles of W, swept fastest across
+ *                  every column tile of X; 0: column tiles of X, swept across
+ *                  every row tile), for tuning the order against the L2.
+ *                  Results do not depend on it.
  * Errors: as nm_spmm, plus NM_ERR_SHAPE for kernel outside 0..9, a negative
- * wait_limit_ns or skip_step < -1.
+ * wait_limit_ns, skip_step < -1, a negative raster_group or raster_m_inner
+ * outside 0..1.
  */
 NM_API nm_status nm_spmm_test(const void *values, const uint8_t *meta_sm100, nm_dtype ab_dtype,
                               const void *X, int64_t ldx, void *Y, nm_dtype y_dtype, int64_t ldy,
                               int64_t R, int64_t K, int64_t T, float alpha, float beta,
                               void *workspace, size_t workspace_bytes,
                               int kernel, int tail_split, int64_t wait_limit_ns, int64_t skip_step,
-                              void *stream);
+                              int raster_group, int raster_m_inner, void *stream);
 
 /*
  * nm_spmm12_test -- nm_spmm12 with a forced tile configuration (`kernel`, as

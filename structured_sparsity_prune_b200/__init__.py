@@ -69,7 +69,7 @@ def _lib():
         "nm_spmm": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp, sz, vp], i32),
         "nm_spmm_noalloc": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp], i32),
         "nm_spmm_test": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, f32, f32, vp, sz,
-                          i32, i32, i64, i64, vp], i32),
+                          i32, i32, i64, i64, i32, i32, vp], i32),
         "nm_srste_step": ([vp, vp, i32, i64, i64, i64, i32, i32, f32, vp, vp, vp, vp], i32),
         "nm_last_device_status": ([vp], i32),
     }
@@ -314,7 +314,8 @@ SPMM_KERNELS = {"default": 0, "pair256": 1, "pair192": 2, "pair128": 3, "single2
 def nm_spmm_test(values: torch.Tensor, meta_sm100: torch.Tensor, X: torch.Tensor, Y: torch.Tensor | None = None,
                  y_dtype: torch.dtype = torch.bfloat16, alpha: float = 1.0, beta: float = 0.0,
                  workspace: torch.Tensor | None = None, kernel: str = "default", tail_split: bool = True,
-                 wait_limit_ns: int = 0, skip_step: int = -1, stream=None) -> torch.Tensor:
+                 wait_limit_ns: int = 0, skip_step: int = -1, raster_group: int = 0, raster_m_inner: int = 0,
+                 stream=None) -> torch.Tensor:
     """nm_spmm with the test hooks of include/nm_testing.h: a forced tile
     configuration, the half-width last wave on or off, a shorter limit for the
     kernel's bounded waits, and a pipeline step the producer never fills."""
@@ -331,7 +332,7 @@ def nm_spmm_test(values: torch.Tensor, meta_sm100: torch.Tensor, X: torch.Tensor
     _check(_lib().nm_spmm_test(_ptr(values), _ptr(meta_sm100), _dtype(values), _ptr(X), _ld(X), _ptr(Y), _dtype(Y),
                                _ld(Y), R, K, T, float(alpha), float(beta), _ptr(workspace), ws_bytes,
                                SPMM_KERNELS[kernel], 1 if tail_split else 0, int(wait_limit_ns), int(skip_step),
-                               _stream(stream)), "nm_spmm_test")
+                               int(raster_group), int(raster_m_inner), _stream(stream)), "nm_spmm_test")
     return Y
 
 

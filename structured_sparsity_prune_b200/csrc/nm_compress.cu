@@ -600,6 +600,152 @@ __global__ void __launch_bounds__(256) decompress32_kernel(const Bits* __restric
   }
 }
 
+// ---- decompression with staged reads ----------------------------------------
+// The compressed inputs are packed (values R x C/2, metadata R x C/8), so the
+// matrix is one stream of 8192-element units: unit u covers logical elements
+// [8192u, 8192u + 8192) of the row-major R x C matrix.  One thread per CTA
+// keeps kRingStages units' values and metadata in flight with bulk copies
+// (cp.async.bulk, this GPU's own memory, no multicast) into a shared-memory
+// ring, so the reads are never queued behind the CTA's own output stream;
+// the 256 threads expand a unit from shared memory in 16-byte output chunks,
+// consecutive threads on consecutive chunks, with 16-byte streaming stores.
+// Needs every chunk inside one row (C % 8 == 0 for 16-bit, C % 16 for 8-bit
+// elements) and R*C % 128 == 0 (whole 16-byte copies).
+constexpr int kRingElems = 8192;
+constexpr int kRingStages = 6;
+constexpr uint64_t kRingWaitNs = 2000000000ull;  // bounded waits: 2 s
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 16 bytes of decompressed output from 8 bytes of values and the groups'
+// nibbles: 16-bit elements, 2 groups (4 values, nibbles in bits 0-7); 8-bit
+// elements, 4 groups (8 values, nibbles in bits 0-15).  Unkept positions +0.
+template <typename Bits>
+__device__ __forceinline__ uint4 expand_chunk(uint2 vals, uint32_t nibs) {
+  if constexpr (sizeof(Bits) == 2) {
+    uint64_t g[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t nib = (nibs >> (4 * k)) & 0xFu;
+      const uint32_t w = k ? vals.y : vals.x;
+      g[k] = (uint64_t(w & 0xFFFFu) << (16 * (nib & 3u))) | (uint64_t(w >> 16) << (16 * (nib >> 2)));
+    }
+    return make_uint4(uint32_t(g[0]), uint32_t(g[0] >> 32), uint32_t(g[1]), uint32_t(g[1] >> 32));
+  } else {
+    uint32_t o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t nib = (nibs >> (4 * k)) & 0xFu;
+      const uint32_t w = ((k < 2 ? vals.x : vals.y) >> (16 * (k & 1))) & 0xFFFFu;
+      o[k] = ((w & 0xFFu) << (8 * (nib & 3u))) | ((w >> 8) << (8 * (nib >> 2)));
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+template <typename Bits>
+__global__ void __launch_bounds__(256) decompress_ring_kernel(const Bits* __restrict__ values,
+                                                              const uint8_t* __restrict__ meta, int64_t R,
+                                                              int64_t C, Bits* __restrict__ out, int64_t ldo,
+                                                              int* __restrict__ status) {
+  constexpr int kValBytes = kRingElems / 2 * int(sizeof(Bits));
+  constexpr int kMetaBytes = kRingElems / 8;
+  constexpr int kStageBytes = kValBytes + kMetaBytes;
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ __align__(8) uint64_t full[kRingStages];
+  const int64_t total = R * C;
+  const int64_t units = (total + kRingElems - 1) / kRingElems;
+  const int tid = threadIdx.x;
+
+  auto issue = [&](int64_t u, int st) {
+    const int64_t e0 = u * kRingElems;
+    const int64_t n = (total - e0) < kRingElems ? (total - e0) : kRingElems;
+    const uint32_t vb = uint32_t(n / 2) * uint32_t(sizeof(Bits)), mb = uint32_t(n / 8);
+    const uint32_t bar = smem_addr(&full[st]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(vb + mb) : "memory");
+    uint8_t* dst = ring + st * kStageBytes;
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst)),
+                 "l"(reinterpret_cast<const uint8_t*>(values) + (e0 / 2) * int64_t(sizeof(Bits))), "r"(vb), "r"(bar)
+                 : "memory");
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst + kValBytes)),
+                 "l"(meta + e0 / 8), "r"(mb), "r"(bar)
+                 : "memory");
+  };
+
+  if (tid == 0) {
+    for (int st = 0; st < kRingStages; ++st)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&full[st])));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int st = 0;
+    for (int64_t u = blockIdx.x; u < units && st < kRingStages; u += gridDim.x, ++st) issue(u, st);
+  }
+
+  int64_t it = 0;
+  for (int64_t u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+    const int st = int(it % kRingStages);
+    const uint32_t parity = uint32_t(it / kRingStages) & 1u;
+    // bounded wait for this unit's copies (uniform: every thread waits on the same phase)
+    bool ok = false;
+    {
+      const uint32_t bar = smem_addr(&full[st]);
+      uint64_t t0 = 0;
+      for (uint32_t spin = 0;; ++spin) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done) { ok = true; break; }
+        uint64_t now;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+        if (spin == 0) t0 = now;
+        else if (now - t0 > kRingWaitNs) break;
+      }
+    }
+    if (!__syncthreads_and(ok ? 1 : 0)) {  // one decision for the whole CTA
+      if (tid == 0 && status != nullptr) atomicExch(status, int(NM_ERR_TIMEOUT));
+      break;
+    }
+    // 16 bytes of output per chunk (8 bf16 / 16 int8 columns: 2 or 4 groups),
+    // chunk j of the unit handled by thread j % 256, so each warp store covers
+    // 512 contiguous bytes; a chunk's 8 bytes of values and 2/es bytes of
+    // metadata sit at 8j and (2/es)j in the stage
+    const int64_t e0 = u * kRingElems;
+    const uint8_t* src = ring + st * kStageBytes;
+    constexpr int kChunks = kRingElems * int(sizeof(Bits)) / 16;
+    constexpr int kCols = 16 / int(sizeof(Bits));
+#pragma unroll
+    for (int h = 0; h < kChunks / 256; ++h) {
+      const int j = h * 256 + tid;
+      const int64_t e = e0 + int64_t(j) * kCols;
+      if (e < total) {
+        const uint2 vals = *reinterpret_cast<const uint2*>(src + 8 * j);
+        uint32_t nibs;
+        if constexpr (sizeof(Bits) == 2) nibs = src[kValBytes + j];
+        else nibs = *reinterpret_cast<const uint16_t*>(src + kValBytes + 2 * j);
+        const int64_t r = e / C, c = e - r * C;
+        __stcs(reinterpret_cast<uint4*>(out + r * ldo + c), expand_chunk<Bits>(vals, nibs));
+      }
+    }
+    __syncthreads();  // every thread has read this stage
+    if (tid == 0) {
+      const int64_t un = u + int64_t(kRingStages) * gridDim.x;
+      if (un < units) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic reads before the async refill
+        issue(un, st);
+      }
+    }
+  }
+}
+
 // ---- compression of the transpose ---------------------------------------------
 // Wt = W^T (C x R) compressed 2:4 along R under mask^T: the operand of the
 // backward product dX = W^T dY when the mask is transposable (every group of
@@ -917,6 +1063,27 @@ extern "C" nm_status nm_decompress(const void* values, const uint8_t* meta, nm_d
   if (!aligned16(values) || !aligned16(meta) || !aligned16(W_out) || !stride_ok(ldw, esize_of(dtype)))
     return NM_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype != NM_F32 && C % (dtype == NM_S8 ? 16 : 8) == 0 && (R * C) % 128 == 0) {
+    // staged reads: a bulk-copy ring per CTA, several CTAs per SM
+    const int es = esize_of(dtype);
+    const int smem = kRingStages * (kRingElems / 2 * es + kRingElems / 8);
+    const int64_t units = (R * C + kRingElems - 1) / kRingElems;
+    auto k16 = decompress_ring_kernel<uint16_t>;
+    auto k8 = decompress_ring_kernel<uint8_t>;
+    const void* kp = es == 2 ? reinterpret_cast<const void*>(k16) : reinterpret_cast<const void*>(k8);
+    if (ensure_dynamic_smem(kp, smem) != NM_OK) return NM_ERR_CUDA;
+    const int per_sm = es == 2 ? blocks_per_sm(k16, 256, smem) : blocks_per_sm(k8, 256, smem);
+    const int64_t cap = int64_t(sm_count()) * per_sm;
+    const unsigned grid = unsigned(units < cap ? units : cap);
+    int* status = device_status_word();
+    if (es == 2)
+      k16<<<grid, 256, smem, s>>>(static_cast<const uint16_t*>(values), meta, R, C, static_cast<uint16_t*>(W_out),
+                                  ldw, status);
+    else
+      k8<<<grid, 256, smem, s>>>(static_cast<const uint8_t*>(values), meta, R, C, static_cast<uint8_t*>(W_out), ldw,
+                                 status);
+    return launch_status();
+  }
   // x over the units of a row, y over rows
   // 32-column units for 8- and 16-bit elements; fp32 takes 8-column units,
   // whose warp stores 1 KB of a row contiguously (the 32-column form's fp32

@@ -44,6 +44,11 @@ inline int sm_count() {
   return n;
 }
 
+// Device address of the status word that bounded device-side waits write
+// NM_ERR_TIMEOUT into (read and cleared by nm_last_device_status), for the
+// current device; nullptr if it cannot be found.  Defined in nm_spmm.cu.
+int* device_status_word();
+
 // Raises a kernel's dynamic shared-memory limit on the current device.  The
 // attribute is per device, so it is set once per (kernel, device), under a
 // lock shared by every host thread.

@@ -41,6 +41,25 @@ namespace nm {
 // Device word written by kernels whose bounded waits give up (NM_ERR_TIMEOUT).
 __device__ int g_device_status = 0;
 
+// Its device address per device, looked up once (kernels of other source
+// files take it as an argument).
+int* device_status_word() {
+  static std::mutex mu;
+  static int* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = static_cast<int*>(p);
+  }
+  return addr[dev];
+}
+
 namespace spmm {
 
 constexpr int kBlockM = 128;     // rows of W per tile = TMEM lanes
@@ -1168,6 +1187,7 @@ struct Opts {
   bool tail_split = true;  // half-width items for a partly filled last wave
   uint64_t wait_ns = kWaitLimitNs;
   int64_t skip_it = -1;
+  int raster = 0;          // 0: the library's tile order; else 1 + 2*group + m_inner (tuning)
 };
 
 template <Kind KD>
@@ -1230,6 +1250,20 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
     const double b_bytes = double(K) * double(T) * K_::kEsize;
     p.m_inner = a_bytes < b_bytes ? 1 : 0;
     p.group = p.m_inner ? p.m_tiles : p.n_tiles;
+    if (p.m_inner) {
+      // sweep groups of row tiles whose slice of W (values + image) is about
+      // 32 MB, so the slice stays in L2 while X streams past it: measured on
+      // the MLP up product (56 row tiles) 8 % faster than sweeping all rows
+      const double tile_a = double(block_m) * (double(K) * 0.5 * K_::kEsize + double(K) / 8.0);
+      const int g = int(32.0e6 / tile_a + 0.5);
+      p.group = g < 1 ? 1 : (g > p.m_tiles ? p.m_tiles : g);
+    }
+    if (o.raster > 0) {  // a forced order: `group` tiles of the fast operand, m or n fastest
+      p.m_inner = (o.raster - 1) & 1;
+      const int g = (o.raster - 1) >> 1;
+      const int lim = p.m_inner ? p.m_tiles : p.n_tiles;
+      p.group = g < 1 ? 1 : (g > lim ? lim : g);
+    }
   }
 
   CUtensorMap ma, mb;
@@ -1376,13 +1410,16 @@ extern "C" nm_status nm_spmm_test(const void* values, const uint8_t* meta_sm100,
                                   int64_t ldx, void* Y, nm_dtype y_dtype, int64_t ldy, int64_t R, int64_t K,
                                   int64_t T, float alpha, float beta, void* workspace, size_t workspace_bytes,
                                   int kernel, int tail_split, int64_t wait_limit_ns, int64_t skip_step,
-                                  void* stream) {
-  if (kernel < 0 || kernel > 9 || wait_limit_ns < 0 || skip_step < -1) return NM_ERR_SHAPE;
+                                  int raster_group, int raster_m_inner, void* stream) {
+  if (kernel < 0 || kernel > 9 || wait_limit_ns < 0 || skip_step < -1 || raster_group < 0 ||
+      raster_m_inner < 0 || raster_m_inner > 1)
+    return NM_ERR_SHAPE;
   spmm::Opts o;
   o.kernel = kernel;
   o.tail_split = tail_split != 0;
   if (wait_limit_ns > 0) o.wait_ns = uint64_t(wait_limit_ns);
   o.skip_it = skip_step;
+  if (raster_group > 0) o.raster = 1 + 2 * raster_group + raster_m_inner;
   return spmm_entry(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, workspace,
                     workspace_bytes, o, stream);
 }

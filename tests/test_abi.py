@@ -170,11 +170,12 @@ def test_host_validation_before_any_launch(lib):
     assert L.nm_meta12_to_sm100(fake, 4, 40, fake, s) == 2
     assert L.nm_meta12_to_sm100(fake, 4, 64, None, s) == 1
     assert L.nm_meta12_to_sm100(fake, 0, 64, fake, s) == 0
-    t = lambda kern, split, wait, skip, K=64: L.nm_spmm_test(fake, fake, 1, fake, 8, fake, 1, 8, 128, K, 8, f(1),
-                                                              f(0), None, 0, kern, split, wait, skip, s)
+    t = lambda kern, split, wait, skip, K=64, rg=0, rm=0: L.nm_spmm_test(
+        fake, fake, 1, fake, 8, fake, 1, 8, 128, K, 8, f(1), f(0), None, 0, kern, split, wait, skip, rg, rm, s)
     assert t(10, 1, 0, -1) == 2 and t(-1, 1, 0, -1) == 2
     assert t(0, 1, -5, -1) == 2 and t(0, 1, 0, -2) == 2
     assert t(1, 1, 0, -1, K=40) == 2
+    assert t(0, 1, 0, -1, rg=-1) == 2 and t(0, 1, 0, -1, rg=4, rm=2) == 2
 
 
 def test_image_sizes(lib):

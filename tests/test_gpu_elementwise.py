@@ -197,7 +197,12 @@ def test_compress_sparser_masks_roundtrip(dtype, R, C):
     assert np.array_equal(back, np.where(mask.cpu().numpy() == 1, _bits(W), 0))
 
 
-@pytest.mark.parametrize("R,C", SHAPES)
+# staged-read decompression (C % 32 == 0, R*C % 128 == 0): a partial last
+# 8192-element unit, rows that straddle units, one row, a single unit
+RING_SHAPES = [(67, 256), (7, 2176), (1, 128), (3, 8192), (129, 4096), (516, 96)]
+
+
+@pytest.mark.parametrize("R,C", SHAPES + RING_SHAPES)
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
 def test_decompress(R, C, dtype):
     W = _rand((R, C), dtype, 3 * R + C, "special")
