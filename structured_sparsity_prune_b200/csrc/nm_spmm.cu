@@ -789,7 +789,9 @@ struct PairCfg {
   static_assert(kECol0 + K_::kECols * STAGES <= 512, "TMEM budget");
 };
 
-template <int N_TOTAL, int STAGES, Kind KD>
+// Y4: the output is a 4-byte type (fp32 or s32); each instantiation carries
+// only its own early-release epilogue, which keeps the register budget.
+template <int N_TOTAL, int STAGES, Kind KD, bool Y4>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     spmm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                      const __grid_constant__ CUtensorMap map_e, const __grid_constant__ CUtensorMap map_y,
@@ -934,7 +936,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int half = (warp - 2) >> 2;
     const int row_in_tile = 32 * q + lane;
     const uint32_t acc_empty_leader[2] = {mapa(smem_u32(&acc_empty[0]), 0), mapa(smem_u32(&acc_empty[1]), 0)};
-    const bool early = !p.y_f32 && !p.y_s32 && p.beta == 0.0f && p.y_vec;
+    const bool early = !Y4 && p.beta == 0.0f && p.y_vec;
+    // 4-byte outputs (fp32, s32) without beta: the same early release and
+    // staged bulk stores, in 32-row x 16-column chunks
+    const bool early4 = Y4 && p.beta == 0.0f && p.y_vec && p.y_tma;
     const uint32_t out_slot = smem_u32(smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes);
     uint32_t local = 0;
     for (int w = pair; w < num_work; w += num_pairs, ++local) {
@@ -952,7 +957,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       const int r = (2 * mt + int(rank)) * kBlockM + row_in_tile;
       const int c_base = wk.col0 + half * kc;
       const uint32_t taddr = tmem_base + (uint32_t(32 * q) << 16) + uint32_t(buf * N_TOTAL + half * kc);
-      if (early) {
+      if (early4) {
+        uint32_t v[kCols];
+#pragma unroll
+        for (int c = 0; c < kCols; c += 32)
+          if (c < kc) tmem_ld_32x32b_x32_nowait(taddr + uint32_t(c), *reinterpret_cast<uint32_t(*)[32]>(&v[c]));
+        tmem_ld_wait();
+        fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader[buf]);
+        if (p.y_f32) {
+#pragma unroll
+          for (int j = 0; j < kCols; ++j) v[j] = __float_as_uint(p.alpha * acc_to_f<KD>(v[j]));
+        }
+        const uint32_t slot = out_slot + uint32_t(lane) * 64u;
+        const uint32_t sw = (uint32_t(lane) >> 1) & 3u;
+        const int row0 = (2 * mt + int(rank)) * kBlockM + 32 * q;
+#pragma unroll
+        for (int c = 0; c < kCols; c += 16) {
+          if (c >= kc) break;
+          if (lane == 0) bulk_wait_read_all();  // the slot's previous store has read it
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            st_shared_v4(slot + 16u * (uint32_t(j) ^ sw), v[c + 4 * j], v[c + 4 * j + 1], v[c + 4 * j + 2],
+                         v[c + 4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0 && row0 < p.R && c_base + c < p.T) {  // boxes start inside Y
+            tma_store_2d(&map_y, smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes, c_base + c, row0);
+            bulk_commit();
+          }
+        }
+      } else if (early) {
         uint32_t packed[kCols / 2];
         {
           // the thread's whole segment in flight at once, one wait, and the
@@ -1153,7 +1190,8 @@ template <int N_TOTAL, int STAGES, Kind KD>
 nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me, const CUtensorMap& my,
                       const Params& p, bool tail_split, cudaStream_t s) {
   using C = PairCfg<N_TOTAL, STAGES, KD>;
-  auto kern = spmm_pair_kernel<N_TOTAL, STAGES, KD>;
+  auto kern = (p.y_f32 || p.y_s32) ? spmm_pair_kernel<N_TOTAL, STAGES, KD, true>
+                                   : spmm_pair_kernel<N_TOTAL, STAGES, KD, false>;
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes) != NM_OK) return NM_ERR_CUDA;
   const int tiles = p.m_tiles * p.n_tiles;
   const int max_pairs = sm_count() / 2;
@@ -1277,12 +1315,18 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
     constexpr int e_rows = K_::kEBytes / 16;
     const int64_t rows16 = ((R + 127) / 128) * int64_t(p.k_blocks) * e_rows;
     if (!make_map_image(&me, meta_img, rows16, e_rows)) return NM_ERR_CUDA;
-    // bf16 output without beta leaves through bulk tensor stores (32 x 32 boxes)
-    p.y_tma = (y_kind == 0 && beta == 0.0f && p.y_vec) ? 1 : 0;
+    // output without beta leaves through bulk tensor stores: 32-row boxes of
+    // 64-byte rows (32 bf16 or 16 fp32 / s32 columns)
+    p.y_tma = (beta == 0.0f && p.y_vec) ? 1 : 0;
     memset(&my, 0, sizeof(my));
-    if (p.y_tma && !make_map(&my, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, T, ldy, 32, 32,
-                             CU_TENSOR_MAP_SWIZZLE_64B))
-      return NM_ERR_CUDA;
+    if (p.y_tma) {
+      const bool ok = y_kind == 0 ? make_map(&my, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, T, ldy, 32, 32,
+                                             CU_TENSOR_MAP_SWIZZLE_64B)
+                                  : make_map(&my, Y, y_kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                                                 : CU_TENSOR_MAP_DATA_TYPE_INT32,
+                                             4, R, T, ldy, 16, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+      if (!ok) return NM_ERR_CUDA;
+    }
     if constexpr (KD == Kind::S8) {
       return launch_pair<256, 4, KD>(ma, mb, me, my, p, o.tail_split, s);
     } else {
