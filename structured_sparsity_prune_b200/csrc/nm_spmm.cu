@@ -165,6 +165,12 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
                : "memory");
 }
 
+// Pull a tensor map (a __grid_constant__ kernel parameter) into the TMA unit's
+// descriptor cache ahead of its first use.
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 __device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -612,6 +618,10 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES, KD>::kSmemBytes 
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&map_a);
+    prefetch_tmap(&map_b);
+  }
   if (warp == 1) tmem_alloc(tmem_slot, C::kTmemCols);
   fence_before_sync();
   __syncthreads();
@@ -827,6 +837,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&map_a);
+    prefetch_tmap(&map_b);
+    prefetch_tmap(&map_e);
+    if (p.y_tma) prefetch_tmap(&map_y);
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, C::kTmemCols);
   fence_before_sync();
