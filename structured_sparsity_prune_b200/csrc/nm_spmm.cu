@@ -1297,21 +1297,28 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
                      : kern == Kern::Single16x2                              ? 16 : 64;
   p.m_tiles = int((R + block_m - 1) / block_m);
   p.n_tiles = int((T + n_tile - 1) / n_tile);
-  // Tile order: the operand with fewer bytes is swept fastest, so consecutive
-  // tiles (running at the same time) share a slice of the larger one.
+  // Tile order.  Tiles run in groups: `group` row tiles of W swept across every
+  // column tile of X (m_inner), or `group` column tiles of X swept across every
+  // row tile.  A group's slice of the grouped operand is sized to about 32 MB,
+  // so it stays in L2 while the other operand streams past it once per group;
+  // of the two orders, the one with the smaller estimated DRAM traffic (the
+  // grouped operand once, the other once per group) is taken, row groups
+  // within 10 %.  On the MLP up
+  // product this cut DRAM reads from 661 to 316 MB; on the TF32 8192^2 x 4096
+  // product the whole-row sweep had read 1117 MB.
   {
-    const double a_bytes = double(R) * double(K) * 0.5 * K_::kEsize;   // compressed values
+    const double a_bytes = double(R) * (double(K) * 0.5 * K_::kEsize + double(K) / 8.0);  // values + image
     const double b_bytes = double(K) * double(T) * K_::kEsize;
-    p.m_inner = a_bytes < b_bytes ? 1 : 0;
-    p.group = p.m_inner ? p.m_tiles : p.n_tiles;
-    if (p.m_inner) {
-      // sweep groups of row tiles whose slice of W (values + image) is about
-      // 32 MB, so the slice stays in L2 while X streams past it: measured on
-      // the MLP up product (56 row tiles) 8 % faster than sweeping all rows
-      const double tile_a = double(block_m) * (double(K) * 0.5 * K_::kEsize + double(K) / 8.0);
-      const int g = int(32.0e6 / tile_a + 0.5);
-      p.group = g < 1 ? 1 : (g > p.m_tiles ? p.m_tiles : g);
-    }
+    const double a_tile = a_bytes / p.m_tiles, b_tile = b_bytes / p.n_tiles;
+    auto groups = [](double tile, int tiles) {
+      const int g = int(32.0e6 / tile + 0.5);
+      return g < 1 ? 1 : (g > tiles ? tiles : g);
+    };
+    const int gm = groups(a_tile, p.m_tiles), gn = groups(b_tile, p.n_tiles);
+    const double est_m = a_bytes + double((p.m_tiles + gm - 1) / gm) * b_bytes;
+    const double est_n = b_bytes + double((p.n_tiles + gn - 1) / gn) * a_bytes;
+    p.m_inner = est_m <= 1.1 * est_n ? 1 : 0;  // near-ties: row groups (measured better on the MLP up shape)
+    p.group = p.m_inner ? gm : gn;
     if (o.raster > 0) {  // a forced order: `group` tiles of the fast operand, m or n fastest
       p.m_inner = (o.raster - 1) & 1;
       const int g = (o.raster - 1) >> 1;
