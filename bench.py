@@ -88,7 +88,13 @@ def load_peaks():
 # ncu summaries that carry a per-launch DRAM traffic figure for the dominant
 # kernel of a workload; the figure is reported only while the kernel source is
 # unchanged since the capture (its sha256 is recorded in the summary).
-TRAFFIC_PROFILES = {("linear_4096", "nm_spmm"): "profiles/spmm_pair_linear_4096.md"}
+TRAFFIC_PROFILES = {
+    ("linear_4096", "nm_spmm"): "profiles/spmm_pair_linear_4096.md",
+    ("mlp_pair", "nm_spmm_up"): "profiles/spmm_pair_mlp_up.md",
+    ("mlp_pair", "nm_spmm_down"): "profiles/spmm_pair_mlp_down.md",
+    ("int8_24", "nm_spmm_s8"): "profiles/spmm_pair_int8_decode_28672x8192x1024.md",
+    ("pairs_12", "nm_spmm12"): "profiles/spmm_pair_tf32_8192x8192x4096.md",
+}
 
 
 def profiled_traffic(workload: str, kernel: str):
@@ -1085,7 +1091,7 @@ def main():
                            if roof["bound"] == "tensor" else
                            "derived: 148 SMs x 64 integer lanes x 1965 MHz" if roof["bound"] == "alu" else
                            "%s: HBM copy" % peak_src)
-    roof["traffic"] = profiled_traffic(args.workload, "nm_spmm" if dom.startswith("nm_spmm") else dom)
+    roof["traffic"] = profiled_traffic(args.workload, dom)
 
     dense = dense_context(step, 20, flush)
     dense_line = None

@@ -29,17 +29,17 @@ def _fields(path):
 
 
 def test_traffic_is_read_from_the_summary_while_the_source_matches():
-    rel = bench.TRAFFIC_PROFILES[("linear_4096", "nm_spmm")]
-    f = _fields(os.path.join(ROOT, rel))
-    with open(os.path.join(ROOT, f["source_file"]), "rb") as fh:
-        src = fh.read()
-    got = bench.profiled_traffic("linear_4096", "nm_spmm")
-    if hashlib.sha256(src).hexdigest() == f["source_sha256"]:
-        assert got == int(f["traffic_bytes_per_launch"])
-    else:
-        assert got is None
+    for (workload, kernel), rel in bench.TRAFFIC_PROFILES.items():
+        f = _fields(os.path.join(ROOT, rel))
+        with open(os.path.join(ROOT, f["source_file"]), "rb") as fh:
+            src = fh.read()
+        got = bench.profiled_traffic(workload, kernel)
+        if hashlib.sha256(src).hexdigest() == f["source_sha256"]:
+            assert got == int(f["traffic_bytes_per_launch"])
+        else:
+            assert got is None
     assert bench.profiled_traffic("linear_4096", "nm_mask") is None
-    assert bench.profiled_traffic("mlp_pair", "nm_spmm_up") is None
+    assert bench.profiled_traffic("mlp_pair", "nm_mask_up") is None
 
 
 def test_traffic_is_dropped_when_the_kernel_changes(tmp_path, monkeypatch):

@@ -80,7 +80,8 @@ def _s8_ref(W, X, rows=None, alpha=1.0, beta=0.0, Y0=None):
                        Y_in=None if Y0 is None else Y0.numpy(), y_dtype=oracle.F32, rows=rows, threads=THREADS)
 
 
-S8_CASES = [(128, 64, 8), (256, 256, 256), (300, 160, 100), (700, 512, 500), (129, 96, 33), (512, 1024, 1000)]
+S8_CASES = [(128, 64, 8), (256, 256, 256), (300, 160, 100), (700, 512, 500), (129, 96, 33), (512, 1024, 1000),
+            (1, 32, 1), (257, 32, 130), (384, 288, 1), (2, 4096, 7)]
 
 
 @pytest.mark.parametrize("R,K,T", S8_CASES)
@@ -177,7 +178,8 @@ def _tf32_ref(W, X, rows=None, alpha=1.0, beta=0.0, Y0=None):
                          rows=rows, threads=THREADS)
 
 
-TF32_CASES = [(128, 64, 8), (256, 256, 256), (300, 160, 100), (700, 512, 500), (129, 96, 33), (40, 16, 3)]
+TF32_CASES = [(128, 64, 8), (256, 256, 256), (300, 160, 100), (700, 512, 500), (129, 96, 33), (40, 16, 3),
+              (1, 16, 1), (257, 48, 129), (384, 80, 2)]
 
 
 @pytest.mark.parametrize("R,K,T", TF32_CASES)
