@@ -954,8 +954,7 @@ void launch_compress(const void* W, int64_t ldw, const uint8_t* mask, int64_t ld
     if (small) per_sm = per_sm_small;
   }
   const int64_t units = ((C + 127) / 128) * 4, pairs = ((R + 127) / 128) * 64;
-  int bx = 32;
-  while (bx < 256 && bx < units) bx *= 2;
+  const int bx = row_block_x(units);
   const int by = 256 / bx;
   const int64_t gx = (units + bx - 1) / bx;
   const int64_t cap = int64_t(per_sm) * sm_count();
@@ -1090,8 +1089,7 @@ extern "C" nm_status nm_decompress(const void* values, const uint8_t* meta, nm_d
   // stores are 16-byte pieces 128 bytes apart: 2.6 against 4.3 TB/s).
   const bool wide = (C % 32) == 0 && dtype != NM_F32;
   const int64_t opr = wide ? C / 32 : C / 8;
-  int bx = 32;
-  while (bx < 256 && bx < opr) bx *= 2;
+  const int bx = row_block_x(opr);
   const int by = 256 / bx;
   const int64_t gx = (opr + bx - 1) / bx;
   static const int per_sm_wide = blocks_per_sm(decompress32_kernel<uint16_t>, 256);

@@ -22,6 +22,25 @@ inline bool dtype_ok(int d) { return d == NM_F32 || d == NM_BF16 || d == NM_F16;
 // ... plus int8, for the calls that only select, move and pack elements
 inline bool dtype_ok_int8(int d) { return dtype_ok(d) || d == NM_S8; }
 
+// x width of a 256-thread block laid over `units` work items of a row (y
+// takes the rest of the block, over rows): the widest of 32..256 that leaves
+// the fewest threads of a row's last x-block idle.  A power of two at or
+// above `units` when a row has fewer than 256 items; 14336 bf16 columns in
+// 16-element chunks (896) take 128, not 256, which would idle 1/8 of them.
+inline int row_block_x(int64_t units) {
+  int best = 32;
+  int64_t best_idle = -1;
+  for (int bx = 32; bx <= 256; bx *= 2) {
+    const int64_t idle = (units + bx - 1) / bx * bx - units;
+    if (best_idle < 0 || idle <= best_idle) {
+      best = bx;
+      best_idle = idle;
+    }
+    if (bx >= units) break;
+  }
+  return best;
+}
+
 inline nm_status launch_status() {
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? NM_OK : NM_ERR_CUDA;

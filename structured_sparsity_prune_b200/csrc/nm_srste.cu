@@ -173,8 +173,7 @@ __global__ void __launch_bounds__(256) srste_scalar_kernel(const Bits* __restric
 // x over the units of a row, y over rows; at most per_sm blocks per SM (the
 // kernel's occupancy), so the whole grid is resident at once.
 void shape2d(int64_t R, int64_t units, dim3& grid, dim3& block, int per_sm = 8) {
-  int bx = 32;
-  while (bx < 256 && bx < units) bx *= 2;
+  const int bx = row_block_x(units);
   const int by = 256 / bx;
   const int64_t gx = (units + bx - 1) / bx;
   const int64_t want = int64_t(sm_count()) * per_sm;
