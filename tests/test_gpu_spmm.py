@@ -308,3 +308,22 @@ def test_bounded_wait_runs_out_and_the_next_call_is_clean(kern, R, T):
     torch.cuda.synchronize()
     assert nm.nm_last_device_status() == 0
     assert _nerr(Y2.cpu(), ref) <= 1e-3
+
+
+@pytest.mark.skipif(torch.cuda.device_count() < 2, reason="needs two visible GPUs")
+def test_second_device_after_the_first():
+    """The kernels' shared-memory attributes, the SM count and the scratch address
+    are cached per device: products on device 1 after products on device 0 (the
+    CTA-pair kernel and the skinny one, both above 48 KB of shared memory) run
+    and stay exact on integer inputs."""
+    prev = torch.cuda.current_device()
+    try:
+        for dev in (0, 1, 0):
+            torch.cuda.set_device(dev)
+            for R, K, T in [(512, 256, 512), (384, 256, 16)]:
+                W = nm_inputs.small_int((R, K), 91 + T, dtype=torch.bfloat16)
+                X = nm_inputs.small_int((K, T), 92 + T, dtype=torch.bfloat16)
+                Y, ref = _run(W, X, torch.float32)
+                assert np.array_equal(Y.numpy().astype(np.float64), ref)
+    finally:
+        torch.cuda.set_device(prev)
