@@ -64,7 +64,7 @@ typedef enum {
     NM_ERR_ALIGN = 3,        /* pointer or row stride not 16-byte aligned       */
     NM_ERR_DTYPE = 4,        /* dtype not supported by this call                */
     NM_ERR_NM = 5,           /* N, M outside 1 <= N < M <= 8                     */
-    NM_ERR_UNSUPPORTED = 6,  /* valid request this build does not implement     */
+    NM_ERR_UNSUPPORTED = 6,  /* valid request the library does not implement   */
     NM_ERR_CUDA = 7,         /* a CUDA runtime / driver call failed             */
     NM_ERR_WORKSPACE = 8,    /* workspace NULL or smaller than required         */
     NM_ERR_TIMEOUT = 9       /* a bounded device-side wait gave up (see below)  */
