@@ -97,6 +97,15 @@ TRAFFIC_PROFILES = {
 }
 
 
+def compute_dtype(wl, kind: str) -> str:
+    """The arithmetic type of the step's dominant work: the product's operand
+    type where the step has a product (TF32 for the 1:2 product on fp32 W),
+    else the element type the masks and compressors read."""
+    if kind == "pairs":
+        return "tf32"
+    return {torch.bfloat16: "bf16", torch.float16: "f16", torch.float32: "f32", torch.int8: "s8"}[wl["W"].dtype]
+
+
 def profiled_traffic(workload: str, kernel: str):
     import hashlib
     rel = TRAFFIC_PROFILES.get((workload, kernel))
@@ -1113,7 +1122,7 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
                 "warmup": warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
                 "scaling": "strong" if split else "weak", "vs_baseline": None,
-                "dtype": str(wl["W"].dtype).replace("torch.", ""),
+                "dtype": compute_dtype(wl, step.kind),
                 "data": "synthetic",
                 "config": {"workload": args.workload, "desc": wl["desc"], "R": wl_full["R"], "K": wl["K"], "T": wl["T"],
                            "sparsity": {"ties": "N:M along K (1:4, 2:4, 4:8, 2:8)", "pairs": "1:2 along K",
