@@ -19,6 +19,10 @@
 // thread.  Decompression expands (row, 32- or 8-column) units; the transposed
 // compressor (for the backward product) works on 32 x 32 tiles per warp in
 // registers (see its comment below).
+#include <cuda.h>
+
+#include <mutex>
+
 #include "nm_internal.cuh"
 
 namespace nm {
@@ -746,6 +750,165 @@ __global__ void __launch_bounds__(256) decompress_ring_kernel(const Bits* __rest
   }
 }
 
+// ---- fused magnitude mask + compression with staged reads ----------------------
+// nm_mask_compress on 16-bit weights with C % 256 == 0.  W comes in through a
+// three-stage shared-memory ring of 64-row x 256-column tiles: four TMA boxes
+// of 64 x 64 in the 128-byte swizzle per stage, issued by one thread per CTA
+// (this GPU's own memory, no multicast), so the selection never waits on its
+// own loads.  The threads then work as the row kernel does -- one (row pair r,
+// r + 8; 32-column unit) each, the same selection, stores and image words --
+// reading the unit from shared memory.  With the swizzle, the 32 threads of a
+// warp (four row pairs x eight units) read eight distinct 16-byte bank groups
+// per load, four deep: the minimum for 512 bytes.  Tiles cover the image's
+// padded rows (a multiple of 128); rows past R arrive as zeros and only their
+// image pieces (the pad pattern) are written.  Every wait is bounded and
+// reports NM_ERR_TIMEOUT in the status word.
+constexpr int kCRingStages = 3;
+constexpr int kCRingRows = 64, kCRingCols = 256;
+constexpr int kCRingBoxBytes = 64 * 128;                   // one 64 x 64 box of 16-bit weights
+constexpr int kCRingStageBytes = 4 * kCRingBoxBytes;       // 32 KB
+constexpr int kCRingSmem = kCRingStages * kCRingStageBytes + 1024;  // + alignment slack
+
+__global__ void __launch_bounds__(256, 2) compress_ring_kernel(const __grid_constant__ CUtensorMap map_w,
+                                                               int64_t R, int64_t C, uint16_t* __restrict__ values,
+                                                               uint8_t* __restrict__ meta, uint8_t* __restrict__ img,
+                                                               int* __restrict__ status) {
+  extern __shared__ uint8_t cring_raw[];
+  __shared__ __align__(8) uint64_t full[kCRingStages];
+  // 128-byte swizzled boxes need 1024-byte aligned destinations
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(cring_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int64_t kt_count = C / 128;
+  const int64_t ncb = C / kCRingCols;
+  const int64_t tiles = ((R + 127) / 128) * (128 / kCRingRows) * ncb;
+
+  auto issue = [&](int64_t t, int st) {
+    const int64_t rb = t / ncb, cb = t - rb * ncb;
+    const uint32_t bar = smem_addr(&full[st]);
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(kCRingStageBytes)
+                 : "memory");
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+      asm volatile(
+          "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+              "r"(smem_addr(ring + st * kCRingStageBytes + b * kCRingBoxBytes)),
+          "l"(reinterpret_cast<uint64_t>(&map_w)), "r"(bar), "r"(int(cb * kCRingCols + 64 * b)),
+          "r"(int(rb * kCRingRows))
+          : "memory");
+  };
+
+  if (tid == 0) {
+    for (int st = 0; st < kCRingStages; ++st)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&full[st])));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int st = 0;
+    for (int64_t t = blockIdx.x; t < tiles && st < kCRingStages; t += gridDim.x, ++st) issue(t, st);
+  }
+
+  // this thread's item inside a tile: 16-row group g, row pair p (rows 16g + p
+  // and + 8), unit u (32 columns) = half h of box b
+  const int g = tid >> 6, p = (tid >> 3) & 7, u = tid & 7, b = u >> 1, h = u & 1;
+  const int rl = 16 * g + p;
+  int64_t it = 0;
+  for (int64_t t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+    const int st = int(it % kCRingStages);
+    const uint32_t parity = uint32_t(it / kCRingStages) & 1u;
+    bool ok = false;
+    {
+      const uint32_t bar = smem_addr(&full[st]);
+      uint64_t t0 = 0;
+      for (uint32_t spin = 0;; ++spin) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done) { ok = true; break; }
+        uint64_t now;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+        if (spin == 0) t0 = now;
+        else if (now - t0 > kRingWaitNs) break;
+      }
+    }
+    if (!__syncthreads_and(ok ? 1 : 0)) {  // one decision for the whole CTA
+      if (tid == 0 && status != nullptr) atomicExch(status, int(NM_ERR_TIMEOUT));
+      break;
+    }
+    const int64_t rb = t / ncb, cb = t - rb * ncb;
+    const int64_t r0 = rb * kCRingRows + rl;
+    const int64_t c0 = cb * kCRingCols + 32 * u;
+    const uint8_t* box = ring + st * kCRingStageBytes + b * kCRingBoxBytes;
+    uint32_t piece[2][2];
+    int invalid = 0;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int row = rl + 8 * k;
+      const int64_t r = r0 + 8 * k;
+      Oct<uint16_t> e[4];
+#pragma unroll
+      for (int o = 0; o < 4; ++o)  // chunk 4h + o of the row sits at (4h + o) ^ (row % 8)
+        e[o].v = *reinterpret_cast<const uint4*>(box + row * 128 + (((4 * h + o) ^ (row & 7)) << 4));
+      uint32_t bytes[4] = {kPadByte, kPadByte, kPadByte, kPadByte};
+      if (r < R) {
+        Quad<uint16_t> q[4];
+#pragma unroll
+        for (int o = 0; o < 4; ++o) bytes[o] = compress_octet<uint16_t, 0>(e[o], make_uint2(0u, 0u), q[o], invalid);
+        store_unit<uint16_t>(q, values + r * (C / 2) + c0 / 2);
+        __stcs(reinterpret_cast<uint32_t*>(meta + r * (C / 8) + c0 / 8),
+               bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24));
+      }
+      piece[k][0] = bytes[0] | (bytes[1] << 8);
+      piece[k][1] = bytes[2] | (bytes[3] << 8);
+    }
+    if (img != nullptr) {
+      uint8_t* blk = img + ((r0 >> 7) * kt_count + (c0 >> 7)) * 2048;
+      const uint32_t lane0 = uint32_t(r0 & 7) + 16u * uint32_t((r0 & 127) >> 4);
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+        __stcs(reinterpret_cast<uint32_t*>(blk + (lane0 + 8u * hf) * 16u + ((c0 >> 5) & 3) * 4),
+               piece[0][hf] | (piece[1][hf] << 16));
+    }
+    __syncthreads();  // every thread has read this stage
+    if (tid == 0) {
+      const int64_t tn = t + int64_t(kCRingStages) * gridDim.x;
+      if (tn < tiles) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic reads before the async refill
+        issue(tn, st);
+      }
+    }
+  }
+  // a CTA that stopped early lets its copies in flight land before leaving
+  // (bounded): they complete on its barriers
+  if (tid == 0) {
+    const uint64_t lim = kRingWaitNs;
+    uint64_t t0;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+    for (int64_t k = it; k < it + kCRingStages; ++k) {
+      const int64_t t = blockIdx.x + k * int64_t(gridDim.x);
+      if (t >= tiles) break;
+      const uint32_t bar = smem_addr(&full[int(k % kCRingStages)]);
+      const uint32_t parity = uint32_t(k / kCRingStages) & 1u;
+      for (;;) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred q;\n\tmbarrier.try_wait.parity.shared::cta.b64 q, [%1], %2;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        uint64_t now;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(now));
+        if (done || now - t0 > lim) break;
+      }
+    }
+  }
+  __syncthreads();
+}
+
 // ---- compression of the transpose ---------------------------------------------
 // Wt = W^T (C x R) compressed 2:4 along R under mask^T: the operand of the
 // backward product dX = W^T dY when the mask is transposable (every group of
@@ -932,14 +1095,67 @@ int tile_grid(int64_t R, int64_t C) {
   return int(tiles < want ? tiles : want);
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda at link time)
+using TensorMapEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                       const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                       CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+TensorMapEncodeFn tensor_map_encoder() {
+  static TensorMapEncodeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<TensorMapEncodeFn>(ptr);
+  });
+  return fn;
+}
+
+// The staged fused compressor (compress_ring_kernel) from this many weights
+// on.  Measured on bf16 (the row kernel -> staged): 28672 x 8192, 133.1 ->
+// 125.0 us; 14336 x 4096 and 4096 x 14336, 36.9 -> 38.9 us (12 tiles a CTA:
+// the ring's fill and the uneven last tiles cost more than it saves); 4096^2
+// no better.
+constexpr int64_t kCRingMinWeights = int64_t(1) << 27;
+
+// true when it launched the staged fused compressor (16-bit W, C % 256 == 0,
+// 16-byte aligned rows); false leaves the call to the row kernel
+bool launch_compress_ring(const uint16_t* w, int64_t ldw, int64_t R, int64_t C, uint16_t* v, uint8_t* meta,
+                          uint8_t* img, cudaStream_t s) {
+  if (C % kCRingCols != 0 || R * C < kCRingMinWeights || !aligned16(w) || !stride_ok(ldw, 2)) return false;
+  TensorMapEncodeFn enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {cuuint64_t(C), cuuint64_t(R)};
+  const cuuint64_t strides[1] = {cuuint64_t(ldw) * 2};
+  const cuuint32_t box[2] = {64, cuuint32_t(kCRingRows)};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(w), dims, strides, box, estr,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(compress_ring_kernel), kCRingSmem) != NM_OK) return false;
+  static const int per_sm = blocks_per_sm(compress_ring_kernel, 256, kCRingSmem);
+  const int64_t tiles = ((R + 127) / 128) * (128 / kCRingRows) * (C / kCRingCols);
+  const int64_t cap = int64_t(sm_count()) * (per_sm > 0 ? per_sm : 1);
+  const unsigned grid = unsigned(tiles < cap ? tiles : cap);
+  compress_ring_kernel<<<grid, 256, kCRingSmem, s>>>(map, R, C, v, meta, img, device_status_word());
+  return true;
+}
+
 // Compressing launch: the row-streaming kernel when C % 32 == 0 (x over the
 // padded units of a row, y over padded row pairs, as many blocks as the SMs
-// hold at once), else the tile kernel.
+// hold at once), else the tile kernel; selection by magnitude on 16-bit
+// weights with C % 256 == 0 takes the staged fused compressor instead.
 template <typename Bits, int MODE>
 void launch_compress(const void* W, int64_t ldw, const uint8_t* mask, int64_t ldm, int64_t R, int64_t C,
                      void* values, uint8_t* meta, uint8_t* img, int32_t* invalid_groups, cudaStream_t s) {
   const Bits* w = static_cast<const Bits*>(W);
   Bits* v = static_cast<Bits*>(values);
+  if constexpr (MODE == 0 && sizeof(Bits) == 2) {
+    if (launch_compress_ring(w, ldw, R, C, v, meta, img, s)) return;
+  }
   if (C % 32 != 0) {
     compress_tiles_kernel<Bits, MODE><<<tile_grid(R, C), kThreads, 0, s>>>(w, ldw, mask, ldm, R, C, v, meta, img,
                                                                            invalid_groups);

@@ -130,6 +130,26 @@ def test_mask_compress_strided_with_image(dtype):
     _check_compressed(full[:, :C], values, meta, img, CODE[dtype])
 
 
+# 16-bit weights with C % 256 == 0 and at least 2^27 entries take the staged
+# fused compressor (64-row x 256-column tiles through a shared-memory ring):
+# ragged R (not a multiple of 64 or 128), strided rows, and no image; the
+# whole matrix is compared.
+RING_CASES = [(16449, 8192, 0), (16384, 8448, 256), (134217, 1024, 0)]
+
+
+@pytest.mark.parametrize("R,C,pad", RING_CASES)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_mask_compress_staged(R, C, pad, dtype):
+    full = _rand((R, C + pad), dtype, R + C + pad, "special")
+    Wd = full.cuda()[:, :C]
+    values, meta, img = nm.nm_mask_compress(Wd)
+    _check_compressed(full[:, :C], values, meta, img, CODE[dtype])
+    v2, m2, none = nm.nm_mask_compress(Wd, sm100=False)
+    assert none is None
+    assert torch.equal(v2.view(torch.int16), values.view(torch.int16)) and torch.equal(m2, meta)
+    assert nm.nm_last_device_status() == 0
+
+
 @pytest.mark.parametrize("R,C", [(256, 256), (67, 200), (130, 64), (77, 160), (1000, 384)])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_compress_with_given_mask(R, C, dtype):
