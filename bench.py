@@ -70,6 +70,7 @@ def transposable_int_ops(M: int) -> float:
         p *= 2
     return 2.0 * comps + 7.0 * M * M + 2.0 * M * M
 SPARSE_RATIO = 2.0   # 2:4 sparse tensor peak = 2x dense (dense-equivalent flops)
+PEER_WAIT_NS = 2_000_000_000   # limit of the row-split step's wait for every GPU's rows of H
 # dense throughput of the int8 and tf32 tensor-core kinds relative to bf16 (nominal B200 figures:
 # 4.5 POPS int8, 1.1 PFLOPS tf32 against 2.25 PFLOPS bf16); applied to the measured bf16 peak
 KIND_RATIO = {"int8": 2.0, "pairs": 0.5}
@@ -376,9 +377,12 @@ class Step:
             self.W2d = torch.empty_like(self.W2)
             Tp = (T + 7) // 8 * 8
             self.gather = wl.get("gather")
+            self.fused = self.gather is not None and wl.get("gather_mode") == "fused"
             if self.gather is None:
                 self.H = torch.empty((R, Tp), dtype=torch.bfloat16, device=dev)[:, :T]
                 self.H_down = self.H
+            elif self.fused:
+                self._init_fused_gather(nm, wl, Tp, dev)
             else:
                 # the up product writes this rank's rows into a slice-sized buffer; the
                 # all-gather assembles every rank's rows; the down product reads them all
@@ -401,10 +405,14 @@ class Step:
                                    "nm_mask_compress_" + tag: G * (es + es / 2 + 0.25),
                                    "nm_meta_to_sm100_" + tag: G * 0.25,
                                    "nm_decompress_" + tag: G * (es / 2 + 0.125 + es)})
-            self.names += ["nm_spmm_up"] + (["all_gather_H"] if self.gather else []) + ["nm_spmm_down"]
-            self.bytes.update({"nm_spmm_up": R * K * (es / 2 + 0.125) + K * T * es + R * T * 2,
+            exchange = (["peer_signal", "peer_wait"] if self.fused else ["all_gather_H"]) if self.gather else []
+            self.names += ["nm_spmm_up"] + exchange + ["nm_spmm_down"]
+            n_dest = len(self.peer_H[0]) if self.fused else 1     # the up product's output copies
+            self.bytes.update({"nm_spmm_up": R * K * (es / 2 + 0.125) + K * T * es + n_dest * R * T * 2,
                                "nm_spmm_down": R2 * K2 * (es / 2 + 0.125) + K2 * T * es + R2 * T * 2})
-            if self.gather:
+            if self.fused:
+                self.bytes.update({"peer_signal": 8 * n_dest, "peer_wait": 8 * n_dest})
+            elif self.gather:
                 self.bytes["all_gather_H"] = self.H_all.numel() * self.H_all.element_size()
             self.flop_k = {"nm_spmm_up": 2.0 * R * K * T, "nm_spmm_down": 2.0 * R2 * K2 * T}
             self.flops = sum(self.flop_k.values())
@@ -426,8 +434,57 @@ class Step:
         self.flop_k = {"nm_spmm": 2.0 * R * K * T}
         self.flops = self.flop_k["nm_spmm"]
 
+    def _init_fused_gather(self, nm, wl, Tp, dev):
+        """The exchange of the row-split MLP pair without a collective library:
+        every rank's up product stores its rows of H straight into every rank's
+        H (nm_spmm_peers over CUDA IPC mappings), raises its flag on every rank
+        (nm_peer_signal) and waits for all flags (nm_peer_wait) before the down
+        product.  H is double-buffered by step parity: a rank that runs ahead
+        writes step s+1's rows into the buffer its peers last read at step s-1,
+        which they finished before signalling step s."""
+        dist_, per, R_full = self.gather
+        world_, rank_ = dist_.get_world_size(), dist_.get_rank()
+        T = wl["T"]
+        self.rank, self.epoch, self.row0, self.ldh = rank_, 0, wl["rows"][0], Tp
+        self.H_bufs = [torch.zeros((world_ * per, Tp), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+        self.flags = torch.zeros(world_, dtype=torch.int64, device=dev)
+        mine = [nm.nm_ipc_handle(t) for t in (self.H_bufs[0], self.H_bufs[1], self.flags)]
+        if self.flags.is_cuda:
+            torch.cuda.synchronize()              # zeroed before any peer can write
+        every = [None] * world_
+        dist_.all_gather_object(every, mine)
+        self.peer_H, self.peer_F, self._opened = [[], []], [], []
+        for j in range(world_):
+            if j == rank_:
+                self.peer_H[0].append(self.H_bufs[0])
+                self.peer_H[1].append(self.H_bufs[1])
+                self.peer_F.append(self.flags)
+                continue
+            addrs = []
+            for h, off in every[j]:
+                addrs.append(nm.nm_ipc_open(h, off))
+                self._opened.append((addrs[-1], off))
+            self.peer_H[0].append(addrs[0])
+            self.peer_H[1].append(addrs[1])
+            self.peer_F.append(addrs[2])
+        self.H = self.H_bufs[0][self.row0:self.row0 + wl["R"], :T]
+        self.H_down = self.H_bufs[0][:R_full, :T]
+        dist_.barrier()                           # every rank has mapped every buffer
+
+    def _up_fused(self):
+        nm = self.nm
+        self.epoch += 1
+        b = self.epoch % 2
+        R_full, T = self.gather[2], self.wl["T"]
+        self.H_down = self.H_bufs[b][:R_full, :T]
+        nm.nm_spmm_peers(self.values, self.img, self.X, self.peer_H[b], self.row0, self.ldh)
+
     def launches(self):
         return len(self.names)
+
+    def own_launches(self):
+        """Launches of the library's own kernels per step (a collective library's are not counted)."""
+        return len([n for n in self.names if n != "all_gather_H"])
 
     def calls(self):
         """The step's launches, in the order of self.names, as zero-argument callables."""
@@ -475,9 +532,12 @@ class Step:
                     lambda: nm.nm_compress(self.W2, self.mask2, self.v2_c, self.m2_c, self.img2_c),
                     lambda: nm.nm_mask_compress(self.W2, self.v2, self.m2, self.img2),
                     lambda: nm.nm_meta_to_sm100(self.m2, R2, K2, out=self.img2_r),
-                    lambda: nm.nm_decompress(self.v2, self.m2, K2, out=self.W2d),
-                    lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.H, workspace=self.ws)] + \
-                ([lambda: gather_rows(self.gather[0], self.H_all, self.H_local)] if self.gather else []) + \
+                    lambda: nm.nm_decompress(self.v2, self.m2, K2, out=self.W2d)] + \
+                ([self._up_fused,
+                  lambda: nm.nm_peer_signal(self.peer_F, self.rank, self.epoch),
+                  lambda: nm.nm_peer_wait(self.flags, self.epoch, timeout_ns=PEER_WAIT_NS)] if self.fused else
+                 [lambda: nm.nm_spmm(self.values, self.img, self.X, Y=self.H, workspace=self.ws)] +
+                 ([lambda: gather_rows(self.gather[0], self.H_all, self.H_local)] if self.gather else [])) + \
                 [lambda: nm.nm_spmm(self.v2, self.img2, self.H_down, Y=self.Y, workspace=self.ws)]
         K = self.wl["K"]
         return [lambda: nm.nm_mask(self.W, 2, 4, mask=self.mask),
@@ -499,6 +559,8 @@ class Step:
         if self.kind == "mlp":        # per weight: mask -> compress; fused -> {image, decompress}; then
             #                               up product after the fused up call, down after fused down and up
             #                               (split by rows: up -> all-gather of H -> down)
+            if self.fused:            # up (peer stores) -> signal -> wait -> down
+                return [[], [0], [], [2], [2], [], [5], [], [7], [7], [2], [10], [11], [7, 12]]
             if self.gather:
                 return [[], [0], [], [2], [2], [], [5], [], [7], [7], [2], [10], [7, 11]]
             return [[], [0], [], [2], [2], [], [5], [], [7], [7], [2], [7, 10]]
@@ -924,11 +986,13 @@ def gather_rows(dist, out: torch.Tensor, local: torch.Tensor):
                 dst.copy_(src)
 
 
-def split_workload(wl, world: int, rank: int, dist):
+def split_workload(wl, world: int, rank: int, dist, gather: str = "nccl"):
     """The rank's share of a product workload split by output rows: its rows of
     W (and of W_down for the MLP pair), all of X.  The MLP pair's hidden
-    activation H = W_up X is row-split too and all-gathered before the down
-    product, the path's one exchange; the transformer linear needs none."""
+    activation H = W_up X is row-split too and gathered on every rank before
+    the down product, the path's one exchange: an NCCL all-gather ("nccl"), or
+    the up product's own stores into every rank's H followed by completion
+    flags ("fused").  The transformer linear needs none."""
     lo, hi, per = shard_rows(wl["R"], world, rank)
     out = dict(wl)
     out["W"] = wl["W"][lo:hi]
@@ -940,6 +1004,7 @@ def split_workload(wl, world: int, rank: int, dist):
         out["W2"] = wl["W2"][lo2:hi2]
         out["rows2"] = (lo2, hi2)
         out["gather"] = (dist, per, wl["R"])       # H slices of `per` rows, R_up rows in all
+        out["gather_mode"] = gather
     return out
 
 
@@ -960,6 +1025,9 @@ def main():
     ap.add_argument("--split", default="replicas", choices=["replicas", "rows"],
                     help="N > 1: an independent replica of the workload per GPU (weak scaling), or one problem "
                          "split by output rows over the GPUs (strong scaling; linear_4096 and mlp_pair)")
+    ap.add_argument("--gather", default="nccl", choices=["nccl", "fused"],
+                    help="--split rows, mlp_pair: assemble H with an NCCL all-gather, or by the up product's "
+                         "own stores into every GPU's H (CUDA IPC) and completion flags")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -987,7 +1055,9 @@ def main():
     split = args.split == "rows" and world > 1
     if split and args.workload not in ("linear_4096", "mlp_pair"):
         raise SystemExit("--split rows applies to the product workloads linear_4096 and mlp_pair")
-    wl = split_workload(wl_full, world, rank, pg) if split else wl_full
+    if args.gather == "fused" and not (split and args.workload == "mlp_pair"):
+        raise SystemExit("--gather fused applies to --split rows of mlp_pair on more than one GPU")
+    wl = split_workload(wl_full, world, rank, pg, args.gather) if split else wl_full
     step = Step(nm, wl, dev)
     # work of the whole job per step: every rank's replica, or the one split problem
     full_flops = 2.0 * wl_full["R"] * wl_full["K"] * wl_full["T"] + \
@@ -1100,7 +1170,8 @@ def main():
                            if roof["bound"] == "tensor" else
                            "derived: 148 SMs x 64 integer lanes x 1965 MHz" if roof["bound"] == "alu" else
                            "%s: HBM copy" % peak_src)
-    roof["traffic"] = profiled_traffic(args.workload, dom)
+    # the committed DRAM counters were taken on the whole problem on one GPU
+    roof["traffic"] = None if split else profiled_traffic(args.workload, dom)
 
     dense = dense_context(step, 20, flush)
     dense_line = None
@@ -1134,14 +1205,17 @@ def main():
                            "step_sequential_ms": seq_ms,
                            "event_floor_us": floor_us,
                            "parallelism": ("rows of W split over the GPUs, X replicated%s" %
-                                           (", H all-gathered (NCCL) before the down product"
+                                           ((", H gathered by the up product's stores into every GPU's H "
+                                             "(CUDA IPC) and completion flags before the down product"
+                                             if args.gather == "fused" else
+                                             ", H all-gathered (NCCL) before the down product")
                                             if step.kind == "mlp" else ", no exchange")) if split else
                                           ("independent replica per GPU" if world > 1 else "single GPU")},
                 "roofline": roof, "cpu_baseline": cpu, "dense_context": dense_line,
                 "e2e": {"value": e2e_value, "unit": unit, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                         "method": "public calls with pinned host buffers; H2D, step and D2H of consecutive steps "
                                   "overlapped on three streams over two buffer replicas"},
-                "gpu_launches": step.launches() * args.steps,
+                "gpu_launches": step.own_launches() * args.steps,
                 "clocks": clk, "kernels": kernels}
         print(json.dumps(line), flush=True)
     if pg:

@@ -320,7 +320,9 @@ NM_API size_t nm_spmm_workspace_bytes(nm_dtype ab_dtype, int64_t R, int64_t K, i
  *   X          K x T, ab_dtype, leading dim ldx >= T
  *   Y          R x T, y_dtype (NM_BF16 or NM_F32), leading dim ldy >= T;
  *              read only when beta != 0.  Y needs only element alignment;
- *              16-byte aligned Y and ldy get vector stores
+ *              16-byte aligned Y and ldy get vector stores.  Nothing outside
+ *              the R x T block is written (elements between T and ldy
+ *              included)
  *   X, values, meta_sm100: 16-byte aligned; ldx * element size % 16 == 0
  *   ab_dtype   NM_BF16 or NM_F16 (tensor-core path), NM_S8 (the int8 2:4
  *              tensor-core path, below), or NM_F32 (rounded to
@@ -390,6 +392,86 @@ NM_API nm_status nm_spmm12(const float *values, const uint8_t *meta12_sm100, con
 NM_API nm_status nm_spmm_noalloc(const void *values, const uint8_t *meta_sm100, nm_dtype ab_dtype,
                                  const void *X, int64_t ldx, void *Y, nm_dtype y_dtype, int64_t ldy,
                                  int64_t R, int64_t K, int64_t T, float alpha, float beta, void *stream);
+
+/*
+ * Row-split product over several GPUs.  The pages describe the product on one
+ * GPU only; these calls are this library's way of splitting it by output rows
+ * (each GPU holds some rows of W and all of X) when the next step needs the
+ * whole output on every GPU, as the down projection of an MLP needs all of
+ * H = W_up X.  Each GPU stores its rows of the output straight into every
+ * GPU's copy from the product's epilogue, then raises a flag on every GPU;
+ * a GPU that needs the whole output waits for every flag.  One process per
+ * GPU; the other GPUs' buffers are reached through CUDA IPC mappings.
+ */
+#define NM_IPC_HANDLE_BYTES 64
+#define NM_MAX_PEERS 8
+
+/*
+ * nm_spmm_peers -- nm_spmm with beta = 0 and a bf16 output written into
+ * rows [row0, row0 + R) of each of n_peers buffers.
+ *   values, meta_sm100, X, ldx, R, K, T, alpha: as nm_spmm; ab_dtype NM_BF16
+ *              or NM_F16 only (else NM_ERR_DTYPE)
+ *   peer_Y     HOST array of n_peers device pointers (1 <= n_peers <= 8,
+ *              else NM_ERR_SHAPE), each the start of a bf16 buffer with
+ *              leading dim ldy >= T and at least row0 + R rows: this GPU's
+ *              own buffer or another GPU's, mapped with nm_ipc_open; the
+ *              caller owns them.  Every peer_Y[j] + row0 * ldy element must be
+ *              16-byte aligned and ldy * 2 % 16 == 0 (else NM_ERR_ALIGN).
+ *              Nothing outside those rows and the first T columns is written.
+ *   row0 >= 0  the first output row of this GPU's slice.
+ * Only the 256-column CTA-pair kernel does this: R must span an even number
+ * of 128-row tiles, T > 128 and T % 8 == 0 (rows of whole 16-byte units:
+ * a bulk tensor store writes the whole 16-byte unit holding a row's last
+ * column), else NM_ERR_UNSUPPORTED.  Each output tile
+ * leaves shared memory once per destination (bulk tensor stores, no
+ * multicast).  The stores into other GPUs' buffers are complete when the
+ * kernel ends; follow the call with nm_peer_signal on the same stream.
+ * Errors otherwise as nm_spmm.
+ */
+NM_API nm_status nm_spmm_peers(const void *values, const uint8_t *meta_sm100, nm_dtype ab_dtype,
+                               const void *X, int64_t ldx, void *const *peer_Y, int n_peers,
+                               int64_t row0, int64_t ldy, int64_t R, int64_t K, int64_t T,
+                               float alpha, void *stream);
+
+/*
+ * nm_peer_signal -- once the work issued to `stream` before it has finished,
+ * stores `epoch` into slot `rank` of every GPU's flag array, with a
+ * system-scope release (so a GPU that reads the flag sees every write that
+ * work made to its memory).
+ *   peer_flags HOST array of n_peers device pointers, 8-byte aligned, each
+ *              GPU j's array of n_peers uint64 slots (own or IPC-mapped)
+ *   0 <= rank < n_peers <= 8 (else NM_ERR_SHAPE)
+ *   epoch      raised by the caller for every new round of stores; slots are
+ *              compared with >=, so they never need resetting
+ */
+NM_API nm_status nm_peer_signal(uint64_t *const *peer_flags, int n_peers, int rank, uint64_t epoch,
+                                void *stream);
+
+/*
+ * nm_peer_wait -- makes `stream` wait until every slot of this GPU's flag
+ * array holds at least `epoch`: a one-warp kernel spins on the slots with
+ * system-scope acquire loads.  The wait is bounded: after timeout_ns (> 0,
+ * else NM_ERR_SHAPE) it gives up, records NM_ERR_TIMEOUT in the device status
+ * word (nm_last_device_status) and lets the stream go on, so work after it
+ * may then read rows that never arrived; check the status.
+ *   flags      device array of n_peers uint64 slots, 8-byte aligned
+ */
+NM_API nm_status nm_peer_wait(const uint64_t *flags, int n_peers, uint64_t epoch, int64_t timeout_ns,
+                              void *stream);
+
+/*
+ * nm_ipc_handle -- the CUDA IPC handle (NM_IPC_HANDLE_BYTES bytes written to
+ * `handle`) of the device allocation holding dev_ptr, and dev_ptr's byte
+ * offset in it.  nm_ipc_open(handle, offset, &p) in ANOTHER process (CUDA
+ * refuses the process's own handles) maps the allocation and returns the
+ * same byte in p; nm_ipc_close(p, offset) unmaps it.  The exporter keeps the
+ * allocation alive while any importer has it mapped.  NM_ERR_CUDA when CUDA
+ * refuses (not device memory, an allocation that cannot be exported, no
+ * peer access).
+ */
+NM_API nm_status nm_ipc_handle(const void *dev_ptr, void *handle, int64_t *offset);
+NM_API nm_status nm_ipc_open(const void *handle, int64_t offset, void **dev_ptr);
+NM_API nm_status nm_ipc_close(void *dev_ptr, int64_t offset);
 
 /*
  * nm_last_device_status -- synchronises `stream`, then returns and clears the

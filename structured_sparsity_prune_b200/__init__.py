@@ -72,6 +72,12 @@ def _lib():
                           i32, i32, i64, i64, i32, i32, vp], i32),
         "nm_srste_step": ([vp, vp, i32, i64, i64, i64, i32, i32, f32, vp, vp, vp, vp], i32),
         "nm_last_device_status": ([vp], i32),
+        "nm_spmm_peers": ([vp, vp, i32, vp, i64, vp, i32, i64, i64, i64, i64, i64, f32, vp], i32),
+        "nm_peer_signal": ([vp, i32, i32, ctypes.c_uint64, vp], i32),
+        "nm_peer_wait": ([vp, i32, ctypes.c_uint64, i64, vp], i32),
+        "nm_ipc_handle": ([vp, vp, vp], i32),
+        "nm_ipc_open": ([vp, i64, vp], i32),
+        "nm_ipc_close": ([vp, i64], i32),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -380,6 +386,70 @@ def nm_spmm_noalloc(values: torch.Tensor, meta_sm100: torch.Tensor, X: torch.Ten
                                   _dtype(Y), _ld(Y), R, K, T, float(alpha), float(beta), _stream(stream)),
            "nm_spmm_noalloc")
     return Y
+
+
+# ---------------------------------------------------------------------------
+# Row-split product over several GPUs (include/nm.h: nm_spmm_peers,
+# nm_peer_signal, nm_peer_wait, nm_ipc_*).  Destination buffers and flag
+# arrays are given as torch tensors (this process's memory) or as integer
+# device addresses (another process's memory, mapped with nm_ipc_open).
+NM_IPC_HANDLE_BYTES = 64
+NM_MAX_PEERS = 8
+
+
+def _addr(x) -> int:
+    return x.data_ptr() if isinstance(x, torch.Tensor) else int(x)
+
+
+def _ptr_array(xs):
+    return (ctypes.c_void_p * len(xs))(*[_addr(x) for x in xs])
+
+
+def nm_spmm_peers(values: torch.Tensor, meta_sm100: torch.Tensor, X: torch.Tensor, peer_Y, row0: int, ldy: int,
+                  alpha: float = 1.0, stream=None) -> None:
+    """(W (.) mask) X * alpha in bf16, written into rows [row0, row0 + R) of
+    every buffer of peer_Y (leading dim ldy)."""
+    R, Kh = values.shape
+    K = 2 * Kh
+    Kx, T = X.shape
+    assert Kx == K, "X must be K x T"
+    ys = list(peer_Y)
+    _check(_lib().nm_spmm_peers(_ptr(values), _ptr(meta_sm100), _dtype(values), _ptr(X), _ld(X), _ptr_array(ys),
+                                len(ys), int(row0), int(ldy), R, K, T, float(alpha), _stream(stream)),
+           "nm_spmm_peers")
+
+
+def nm_peer_signal(peer_flags, rank: int, epoch: int, stream=None) -> None:
+    """Store epoch into slot `rank` of every flag array of peer_flags."""
+    fs = list(peer_flags)
+    _check(_lib().nm_peer_signal(_ptr_array(fs), len(fs), int(rank), int(epoch), _stream(stream)), "nm_peer_signal")
+
+
+def nm_peer_wait(flags: torch.Tensor, epoch: int, timeout_ns: int = 2_000_000_000, stream=None) -> None:
+    """Make the stream wait (bounded) until every slot of flags holds >= epoch."""
+    assert flags.dtype in (torch.int64, torch.uint64) and flags.dim() == 1
+    _check(_lib().nm_peer_wait(_ptr(flags), flags.numel(), int(epoch), int(timeout_ns), _stream(stream)),
+           "nm_peer_wait")
+
+
+def nm_ipc_handle(t: torch.Tensor):
+    """-> (64-byte handle, byte offset of t's first element in its allocation)."""
+    h = ctypes.create_string_buffer(NM_IPC_HANDLE_BYTES)
+    off = ctypes.c_int64()
+    _check(_lib().nm_ipc_handle(_ptr(t), h, ctypes.byref(off)), "nm_ipc_handle")
+    return h.raw, off.value
+
+
+def nm_ipc_open(handle: bytes, offset: int) -> int:
+    """Map another process's buffer; -> its device address in this process."""
+    assert len(handle) == NM_IPC_HANDLE_BYTES
+    p = ctypes.c_void_p()
+    _check(_lib().nm_ipc_open(ctypes.c_char_p(handle), int(offset), ctypes.byref(p)), "nm_ipc_open")
+    return int(p.value)
+
+
+def nm_ipc_close(addr: int, offset: int) -> None:
+    _check(_lib().nm_ipc_close(ctypes.c_void_p(addr), int(offset)), "nm_ipc_close")
 
 
 def nm_last_device_status(stream=None) -> int:

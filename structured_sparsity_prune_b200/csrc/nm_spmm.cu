@@ -96,6 +96,7 @@ struct KT {
 };
 constexpr int kThreads = 192;    // 6 warps (single-CTA kernel)
 constexpr int kPairThreads = 320;  // 10 warps: producer, MMA, 8 epilogue warps (CTA-pair kernel)
+constexpr int kMaxPeers = 8;       // destination GPUs of the peer-store product
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 
 // ----------------------------------------------------------------- PTX helpers
@@ -473,6 +474,7 @@ struct Params {
   // from split_from on are each done as two half-width items (the last,
   // partly filled wave then takes half as long).
   int split_from, num_work;
+  int n_ymaps;  // output tensor maps the staged stores go through (1, or one per destination GPU)
   float alpha, beta;
   uint64_t wait_ns;  // limit of every bounded wait (kWaitLimitNs unless a test shortens it)
   int64_t skip_it;   // test hook: the producer issues nothing for this pipeline step (-1: none)
@@ -782,6 +784,15 @@ __global__ void __launch_bounds__(kThreads, Cfg<N_TILE, STAGES, KD>::kSmemBytes 
 // issued by the even CTA reads both halves, so each SM's shared memory feeds
 // only half of B.  Both CTAs' TMA loads complete on the even CTA's full
 // barrier; the even CTA's commits arrive on both CTAs' barriers.
+// Output tensor maps of the pair kernel: one over the call's Y, or, for the
+// peer-store product, one per destination GPU, each over the same rows of that
+// GPU's buffer. Every staged output chunk is stored through each map with the
+// same coordinates, so each copy is clipped at the same R and T.
+template <int NMAP>
+struct YMaps {
+  CUtensorMap m[NMAP];
+};
+
 template <int N_TOTAL, int STAGES, Kind KD>
 struct PairCfg {
   using K_ = KT<KD>;
@@ -810,11 +821,12 @@ struct PairCfg {
 
 // Y4: the output is a 4-byte type (fp32 or s32); each instantiation carries
 // only its own early-release epilogue, which keeps the register budget.
-template <int N_TOTAL, int STAGES, Kind KD, bool Y4>
+template <int N_TOTAL, int STAGES, Kind KD, bool Y4, int NMAP = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     spmm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                     const __grid_constant__ CUtensorMap map_e, const __grid_constant__ CUtensorMap map_y,
+                     const __grid_constant__ CUtensorMap map_e, const __grid_constant__ YMaps<NMAP> ymaps,
                      Params p) {
+  const int n_ymaps = NMAP == 1 ? 1 : p.n_ymaps;
   using C = PairCfg<N_TOTAL, STAGES, KD>;
   using K_ = KT<KD>;
   extern __shared__ uint8_t smem_raw[];
@@ -851,7 +863,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     prefetch_tmap(&map_a);
     prefetch_tmap(&map_b);
     prefetch_tmap(&map_e);
-    if (p.y_tma) prefetch_tmap(&map_y);
+    if (p.y_tma)
+      for (int j = 0; j < n_ymaps; ++j) prefetch_tmap(&ymaps.m[j]);
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, C::kTmemCols);
   fence_before_sync();
@@ -1010,7 +1023,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && row0 < p.R && c_base + c < p.T) {  // boxes start inside Y
-            tma_store_2d(&map_y, smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes, c_base + c, row0);
+            for (int j = 0; j < n_ymaps; ++j)
+              tma_store_2d(&ymaps.m[j], smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes, c_base + c, row0);
             bulk_commit();
           }
         }
@@ -1052,7 +1066,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0 && row0 < p.R && c_base + c < p.T) {  // boxes start inside Y
-              tma_store_2d(&map_y, smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes, c_base + c, row0);
+              for (int j = 0; j < n_ymaps; ++j)
+                tma_store_2d(&ymaps.m[j], smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes, c_base + c, row0);
               bulk_commit();
             }
           }
@@ -1211,12 +1226,12 @@ bool make_map_image(CUtensorMap* map, const uint8_t* img, int64_t rows16, int bo
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int N_TOTAL, int STAGES, Kind KD>
-nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me, const CUtensorMap& my,
+template <int N_TOTAL, int STAGES, Kind KD, int NMAP = 1>
+nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me, const YMaps<NMAP>& my,
                       const Params& p, bool tail_split, cudaStream_t s) {
   using C = PairCfg<N_TOTAL, STAGES, KD>;
-  auto kern = (p.y_f32 || p.y_s32) ? spmm_pair_kernel<N_TOTAL, STAGES, KD, true>
-                                   : spmm_pair_kernel<N_TOTAL, STAGES, KD, false>;
+  auto kern = (p.y_f32 || p.y_s32) ? spmm_pair_kernel<N_TOTAL, STAGES, KD, true, NMAP>
+                                   : spmm_pair_kernel<N_TOTAL, STAGES, KD, false, NMAP>;
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes) != NM_OK) return NM_ERR_CUDA;
   const int tiles = p.m_tiles * p.n_tiles;
   const int max_pairs = sm_count() / 2;
@@ -1275,12 +1290,20 @@ Kern choose_kernel(int64_t R, int64_t T, int forced) {
   return k;
 }
 
-// y_kind: 0 bf16, 1 fp32, 2 s32 (int8 operands only)
+// y_kind: 0 bf16, 1 fp32, 2 s32 (int8 operands only).
+// peer_y / n_peers / row0 (the peer-store product): when n_peers > 0, rows
+// [row0, row0 + R) of every buffer peer_y[j] (ldy elements per row) receive
+// the bf16 output and Y is ignored.  Only the 256-column CTA-pair kernel with
+// bulk tensor stores does this (bf16 or fp16 operands, bf16 output, beta == 0,
+// 16-byte aligned rows); any other case is NM_ERR_UNSUPPORTED.
 template <Kind KD>
 nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_t ldx, void* Y, int y_kind,
-              int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta, const Opts& o, cudaStream_t s) {
+              int64_t ldy, int64_t R, int64_t K, int64_t T, float alpha, float beta, const Opts& o, cudaStream_t s,
+              void* const* peer_y = nullptr, int n_peers = 0, int64_t row0 = 0) {
   using K_ = KT<KD>;
+  if (n_peers > 0) Y = static_cast<uint8_t*>(peer_y[0]) + size_t(row0) * size_t(ldy) * 2;
   Params p;
+  p.n_ymaps = 1;
   p.wait_ns = o.wait_ns;
   p.skip_it = o.skip_it;
   p.y_tma = 0;
@@ -1343,19 +1366,43 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
                 K_::kB32Atom ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B))
     return NM_ERR_CUDA;
   if (pair) {
-    CUtensorMap me, my;
+    CUtensorMap me;
+    YMaps<1> my;
     constexpr int e_rows = K_::kEBytes / 16;
     const int64_t rows16 = ((R + 127) / 128) * int64_t(p.k_blocks) * e_rows;
     if (!make_map_image(&me, meta_img, rows16, e_rows)) return NM_ERR_CUDA;
     // output without beta leaves through bulk tensor stores: 32-row boxes of
-    // 64-byte rows (32 bf16 or 16 fp32 / s32 columns)
-    p.y_tma = (beta == 0.0f && p.y_vec) ? 1 : 0;
+    // 64-byte rows (32 bf16 or 16 fp32 / s32 columns).  Only when a row of Y
+    // is whole 16-byte units: measured on B200, a bulk tensor store clips rows
+    // exactly but writes the whole 16-byte unit that holds a row's last
+    // column, i.e. up to 7 bf16 (3 fp32) elements past T inside ldy.  A
+    // ragged T takes the plain stores, which stop at T.
+    const int y_es = y_kind == 0 ? 2 : 4;
+    p.y_tma = (beta == 0.0f && p.y_vec && (int64_t(T) * y_es) % 16 == 0) ? 1 : 0;
     memset(&my, 0, sizeof(my));
+    if (n_peers > 0) {
+      if constexpr (KD == Kind::BF16 || KD == Kind::F16) {
+        if (kern != Kern::Pair256 || y_kind != 0 || !p.y_tma || n_peers > kMaxPeers) return NM_ERR_UNSUPPORTED;
+        YMaps<kMaxPeers> ym;
+        memset(&ym, 0, sizeof(ym));
+        for (int j = 0; j < n_peers; ++j) {
+          void* dst = static_cast<uint8_t*>(peer_y[j]) + size_t(row0) * size_t(ldy) * 2;
+          if (!aligned16(dst)) return NM_ERR_UNSUPPORTED;
+          if (!make_map(&ym.m[j], dst, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, T, ldy, 32, 32,
+                        CU_TENSOR_MAP_SWIZZLE_64B))
+            return NM_ERR_CUDA;
+        }
+        p.n_ymaps = n_peers;
+        return launch_pair<256, 4, KD, kMaxPeers>(ma, mb, me, ym, p, o.tail_split, s);
+      } else {
+        return NM_ERR_UNSUPPORTED;
+      }
+    }
     if (p.y_tma) {
-      const bool ok = y_kind == 0 ? make_map(&my, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, T, ldy, 32, 32,
+      const bool ok = y_kind == 0 ? make_map(&my.m[0], Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, R, T, ldy, 32, 32,
                                              CU_TENSOR_MAP_SWIZZLE_64B)
-                                  : make_map(&my, Y, y_kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
-                                                                 : CU_TENSOR_MAP_DATA_TYPE_INT32,
+                                  : make_map(&my.m[0], Y, y_kind == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                                                      : CU_TENSOR_MAP_DATA_TYPE_INT32,
                                              4, R, T, ldy, 16, 32, CU_TENSOR_MAP_SWIZZLE_64B);
       if (!ok) return NM_ERR_CUDA;
     }
@@ -1367,6 +1414,7 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
       return launch_pair<128, 6, KD>(ma, mb, me, my, p, o.tail_split, s);
     }
   }
+  if (n_peers > 0) return NM_ERR_UNSUPPORTED;  // the single-CTA kernels store through plain pointers
   switch (kern) {
     case Kern::Single256: return launch<256, 2, KD>(ma, X, ldx, K, T, p, s);
     case Kern::Single128: return launch<128, 4, KD>(ma, X, ldx, K, T, p, s);
@@ -1480,6 +1528,31 @@ extern "C" nm_status nm_spmm(const void* values, const uint8_t* meta_sm100, nm_d
                              float alpha, float beta, void* workspace, size_t workspace_bytes, void* stream) {
   return spmm_entry(values, meta_sm100, ab_dtype, X, ldx, Y, y_dtype, ldy, R, K, T, alpha, beta, workspace,
                     workspace_bytes, spmm::Opts(), stream);
+}
+
+extern "C" nm_status nm_spmm_peers(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X,
+                                   int64_t ldx, void* const* peer_Y, int n_peers, int64_t row0, int64_t ldy,
+                                   int64_t R, int64_t K, int64_t T, float alpha, void* stream) {
+  if (ab_dtype != NM_BF16 && ab_dtype != NM_F16) return NM_ERR_DTYPE;
+  if (n_peers < 1 || n_peers > spmm::kMaxPeers || row0 < 0) return NM_ERR_SHAPE;
+  if (peer_Y == nullptr) return NM_ERR_NULL;
+  for (int j = 0; j < n_peers; ++j)
+    if (peer_Y[j] == nullptr) return NM_ERR_NULL;
+  if (row0 > 0x7FFFFFFF) return NM_ERR_SHAPE;
+  bool noop = false;
+  void* y0 = static_cast<uint8_t*>(peer_Y[0]) + size_t(row0) * size_t(ldy < 0 ? 0 : ldy) * 2;
+  const nm_status v =
+      spmm_validate(values, meta_sm100, ab_dtype, X, ldx, y0, NM_BF16, ldy, R, K, T, alpha, 0.0f, &noop);
+  if (v != NM_OK || noop) return v;
+  if (!stride_ok(ldy, 2)) return NM_ERR_ALIGN;
+  for (int j = 0; j < n_peers; ++j)
+    if (!aligned16(static_cast<uint8_t*>(peer_Y[j]) + size_t(row0) * size_t(ldy) * 2)) return NM_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (ab_dtype == NM_BF16)
+    return spmm::run<spmm::Kind::BF16>(values, meta_sm100, X, ldx, y0, 0, ldy, R, K, T, alpha, 0.0f, spmm::Opts(),
+                                       s, peer_Y, n_peers, row0);
+  return spmm::run<spmm::Kind::F16>(values, meta_sm100, X, ldx, y0, 0, ldy, R, K, T, alpha, 0.0f, spmm::Opts(), s,
+                                    peer_Y, n_peers, row0);
 }
 
 extern "C" nm_status nm_spmm_test(const void* values, const uint8_t* meta_sm100, nm_dtype ab_dtype, const void* X,

@@ -207,3 +207,51 @@ def test_binding_has_every_declared_call():
     """The Python binding keeps the C names: one function per declared call."""
     missing = [name for name in _declared() if not callable(getattr(nm, name, None))]
     assert missing == []
+
+
+def test_peer_calls_validate_on_the_host(lib):
+    """nm_spmm_peers, nm_peer_signal, nm_peer_wait and the IPC calls reject
+    malformed arguments before any CUDA call."""
+    fake = 0x10000
+    s = ctypes.c_void_p(0)
+    vp = ctypes.c_void_p
+    f = ctypes.c_float
+
+    def arr(*xs):
+        return (ctypes.c_void_p * len(xs))(*xs)
+
+    def peers(ptrs, n, row0=0, ldy=256, dtype=1, R=256, K=64, T=256, n_override=None):
+        return lib.nm_spmm_peers(vp(fake), vp(fake), dtype, vp(fake), 256, arr(*ptrs) if ptrs is not None else None,
+                                 n if n_override is None else n_override, row0, ldy, R, K, T, f(1), s)
+
+    assert peers([fake], 1, dtype=0) == 4                     # fp32 operands: no peer path
+    assert peers([fake], 1, dtype=3) == 4                     # int8 operands: no peer path
+    assert peers([fake], 0, n_override=0) == 2                # no destination
+    assert peers([fake] * 9, 9) == 2                          # more than NM_MAX_PEERS
+    assert peers([fake], 1, row0=-1) == 2
+    assert peers(None, 1) == 1                                # NULL array
+    assert peers([fake, 0], 2) == 1                           # NULL destination
+    assert peers([fake], 1, K=40) == 2                        # K % 16
+    assert peers([fake], 1, ldy=200) == 2                     # ldy < T
+    assert peers([fake], 1, ldy=260) == 3                     # ldy * 2 not a multiple of 16
+    assert peers([fake, fake + 8], 2) == 3                    # destination rows not 16-byte aligned
+    assert peers([fake], 1, R=0) == 0                         # nothing to compute
+    assert lib.nm_peer_signal(arr(fake, fake), 2, 2, 1, s) == 2       # rank outside [0, n)
+    assert lib.nm_peer_signal(arr(fake), 0, 0, 1, s) == 2
+    assert lib.nm_peer_signal(arr(*([fake] * 9)), 9, 0, 1, s) == 2
+    assert lib.nm_peer_signal(None, 2, 0, 1, s) == 1
+    assert lib.nm_peer_signal(arr(fake, 0), 2, 0, 1, s) == 1
+    assert lib.nm_peer_signal(arr(fake, fake + 4), 2, 0, 1, s) == 3   # flags not 8-byte aligned
+    assert lib.nm_peer_wait(vp(fake), 2, 1, 0, s) == 2                # no time limit
+    assert lib.nm_peer_wait(vp(fake), 9, 1, 1000, s) == 2
+    assert lib.nm_peer_wait(None, 2, 1, 1000, s) == 1
+    assert lib.nm_peer_wait(vp(fake + 4), 2, 1, 1000, s) == 3
+    h = ctypes.create_string_buffer(64)
+    off = ctypes.c_int64()
+    assert lib.nm_ipc_handle(None, h, ctypes.byref(off)) == 1
+    assert lib.nm_ipc_handle(vp(fake), None, ctypes.byref(off)) == 1
+    p = ctypes.c_void_p()
+    assert lib.nm_ipc_open(None, 0, ctypes.byref(p)) == 1
+    assert lib.nm_ipc_open(h, -1, ctypes.byref(p)) == 2
+    assert lib.nm_ipc_close(None, 0) == 1
+    assert lib.nm_ipc_close(vp(fake), -1) == 2

@@ -216,3 +216,78 @@ def test_closure_catches_a_planted_race():
     reads_down = rec.log[down][0]
     writes_up = rec.log[up][1]
     assert writes_up & reads_down and up not in before[down]
+
+
+class _FusedRecorder(_Recorder):
+    """The recorder plus the peer calls: nm_spmm_peers writes every destination
+    that is a tensor of this process (other ranks' buffers are addresses), the
+    signal writes every flag array of this process and the wait reads them."""
+
+    def __init__(self):
+        super().__init__()
+        self.peers_calls, self.epochs = [], []
+
+    def nm_ipc_handle(self, t):
+        return bytes(64), 0
+
+    def nm_ipc_open(self, handle, offset):
+        return 0x7000_0000 + offset
+
+    def nm_spmm_peers(self, values, img, X, dests, row0, ldy):
+        own = [d for d in dests if isinstance(d, torch.Tensor)]
+        self.peers_calls.append((own, row0, ldy, len(dests)))
+        self._rec([values, img, X], own)
+
+    def nm_peer_signal(self, flags, rank, epoch):
+        self.epochs.append((rank, epoch))
+        self._rec([], [f for f in flags if isinstance(f, torch.Tensor)])
+
+    def nm_peer_wait(self, flags, epoch, timeout_ns):
+        self._rec([flags], [])
+
+
+class _FakeDist2(_FakeDist):
+    def get_rank(self):
+        return 0          # the rank that holds rows (slices are whole 256-row tiles)
+
+    def all_gather_object(self, out, obj):
+        for i in range(len(out)):
+            out[i] = obj
+
+    def barrier(self):
+        pass
+
+
+def test_row_split_mlp_fused_exchange():
+    """--split rows --gather fused: up product (stores into every rank's H)
+    -> signal -> wait -> down product, ordered by the graph; H alternates
+    between two buffers by step, and the down product reads the buffer its
+    step's up product wrote."""
+    rec = _FusedRecorder()
+    wl = bench.split_workload(WORKLOADS["mlp"], 2, 0, _FakeDist2(rec), gather="fused")
+    step = bench.Step(rec, wl, torch.device("cpu"))
+    assert step.fused
+    names = step.names
+    up, sig, wait, down = (names.index(n) for n in ("nm_spmm_up", "peer_signal", "peer_wait", "nm_spmm_down"))
+    assert up < sig < wait < down and "all_gather_H" not in names
+    deps = step.deps()
+    assert len(step.calls()) == len(deps) == len(names) == step.own_launches()
+    before = _closure(deps)
+    assert up in before[sig] and sig in before[wait] and wait in before[down]
+    for s in range(2):
+        rec.log.clear()
+        for fn in step.calls():
+            fn()
+        own, row0, ldy, n_dest = rec.peers_calls[-1]
+        assert n_dest == 2 and row0 == wl["rows"][0] and len(own) == 1
+        assert own[0].data_ptr() == step.H_bufs[(s + 1) % 2].data_ptr()
+        assert _key(step.H_down) == _key(own[0])                  # the down product reads what up wrote
+        assert rec.epochs[-1] == (0, s + 1)
+        reads_down = rec.log[down][0]
+        assert _key(own[0]) in reads_down
+        for i in range(len(names)):
+            reads_i, writes_i = rec.log[i]
+            for j in range(i):
+                reads_j, writes_j = rec.log[j]
+                if (writes_j & reads_i) or (reads_j & writes_i) or (writes_j & writes_i):
+                    assert j in before[i], (names[j], names[i])

@@ -327,3 +327,43 @@ def test_second_device_after_the_first():
                 assert np.array_equal(Y.numpy().astype(np.float64), ref)
     finally:
         torch.cuda.set_device(prev)
+
+
+# (R, K, T, ldy, y_dtype, beta, kernel): outputs that are views with ldy > T
+VIEW_CASES = [
+    (1000, 512, 333, 344, torch.bfloat16, 0.0, "default"),   # ragged T: plain stores
+    (1024, 512, 330, 344, torch.float32, 0.0, "default"),
+    (1000, 512, 328, 344, torch.bfloat16, 0.0, "default"),   # whole 16-byte rows: staged bulk stores
+    (1024, 512, 332, 344, torch.float32, 0.0, "default"),
+    (1000, 512, 333, 344, torch.bfloat16, 0.5, "default"),   # beta != 0 reads and writes Y in place
+    (256, 256, 77, 80, torch.bfloat16, 0.0, "pair128"),
+    (384, 256, 333, 344, torch.bfloat16, 0.0, "single256"),
+    (384, 256, 45, 48, torch.float32, 0.0, "single64x2"),
+]
+
+
+@pytest.mark.parametrize("R,K,T,ldy,y_dtype,beta,kernel", VIEW_CASES)
+def test_output_view_writes_nothing_outside(R, K, T, ldy, y_dtype, beta, kernel):
+    """Y a view (R x T, leading dim ldy > T) of a larger buffer whose other
+    elements hold a sentinel: every element outside the view keeps it, for
+    each epilogue (staged bulk stores, plain vector stores, element stores)."""
+    S = -3.0
+    W = nm_inputs.normal((R, K), 401 + T, 0.02, torch.bfloat16)
+    X = nm_inputs.normal((K, T), 402 + T, 1.0, torch.bfloat16)
+    Y0 = nm_inputs.normal((R, T), 403, 1.0, y_dtype) if beta else None
+    values, meta, img = nm.nm_mask_compress(W.cuda())
+    big = torch.full((R + 40, ldy), S, dtype=y_dtype, device="cuda")
+    Yv = big[:R, :T]
+    if Y0 is not None:
+        Yv.copy_(Y0.cuda())
+    nm.nm_spmm_test(values, img, _dev(X), Y=Yv, y_dtype=y_dtype, beta=beta, kernel=kernel)
+    torch.cuda.synchronize()
+    _ok_status()
+    outside = torch.ones(big.shape, dtype=torch.bool, device="cuda")
+    outside[:R, :T] = False
+    assert bool((big[outside] == S).all()), "stores outside the R x T view"
+    Wb = _bits(W)
+    _, v_ref, m_ref = oracle.rows_parallel(1, Wb, 2, 4, oracle.BF16, threads=THREADS)
+    ref = oracle.spmm(v_ref, m_ref, _bits(X), oracle.BF16, beta=beta, Y_in=None if Y0 is None else _bits(Y0),
+                      y_dtype=CODE[y_dtype], threads=THREADS)
+    assert _nerr(Yv, ref) <= TOL[y_dtype]
