@@ -367,3 +367,29 @@ def test_output_view_writes_nothing_outside(R, K, T, ldy, y_dtype, beta, kernel)
     ref = oracle.spmm(v_ref, m_ref, _bits(X), oracle.BF16, beta=beta, Y_in=None if Y0 is None else _bits(Y0),
                       y_dtype=CODE[y_dtype], threads=THREADS)
     assert _nerr(Yv, ref) <= TOL[y_dtype]
+
+
+def test_mlp_chain_against_an_fp64_chain():
+    """The MLP pair's chain at a reduced size: the up product, H kept in bf16
+    on the GPU, the down product; against the oracle's chain with H in fp64
+    (the down weight decompressed by the oracle, one fp64 matmul).  The only
+    error beyond each product's own is H's bf16 rounding (at most 2^-9
+    relative per element, about 2^-9 / sqrt(3) RMS), so the chain stays within
+    the bf16-output bound."""
+    R, K, T = 2048, 512, 1024
+    Wu = nm_inputs.normal((R, K), 511, 0.02, torch.bfloat16)
+    Wd = nm_inputs.normal((K, R), 512, 0.02, torch.bfloat16)
+    X = nm_inputs.normal((K, T), 513, 1.0, torch.bfloat16)
+    vu, mu, iu = nm.nm_mask_compress(Wu.cuda())
+    vd, md, idn = nm.nm_mask_compress(Wd.cuda())
+    H = nm.nm_spmm(vu, iu, X.cuda())
+    Y = nm.nm_spmm(vd, idn, H)
+    torch.cuda.synchronize()
+    _ok_status()
+    _, vu_r, mu_r = oracle.rows_parallel(1, _bits(Wu), 2, 4, oracle.BF16, threads=THREADS)
+    H_ref = oracle.spmm(vu_r, mu_r, _bits(X), oracle.BF16, threads=THREADS)
+    _, vd_r, md_r = oracle.rows_parallel(1, _bits(Wd), 2, 4, oracle.BF16, threads=THREADS)
+    Wd_m = oracle.decode_array(oracle.decompress24(vd_r, md_r, R, dtype=oracle.BF16), oracle.BF16)
+    err = _nerr(Y, Wd_m @ H_ref)
+    print("MLP chain (bf16 H) against the fp64 chain: normalised error %.3e" % err)
+    assert err <= 8e-3
