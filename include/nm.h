@@ -339,10 +339,6 @@ NM_API size_t nm_spmm_workspace_bytes(nm_dtype ab_dtype, int64_t R, int64_t K, i
  * (requires alpha == 1 and beta == 0, else NM_ERR_UNSUPPORTED; no overflow
  * while K <= 262144, since |sum| <= K/2 * 2^14); NM_F32 / NM_BF16 store
  * alpha * float(sum) + beta * Y (the conversion of sums beyond 2^24 rounds).
- * With NM_S32 output, T % 4 == 0 and 16-byte aligned Y and ldy, the tiles of
- * a partly filled last wave are split along K: a first small kernel zeroes
- * their part of Y, then each piece adds its exact partial sums into it, so
- * the result is the same bits as without the split.
  * A bounded wait inside the kernel that gives up records NM_ERR_TIMEOUT in a
  * device status word, read and cleared by nm_last_device_status().
  */

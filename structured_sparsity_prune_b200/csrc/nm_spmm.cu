@@ -291,14 +291,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                "r"(smem_u32(src)), "r"(x), "r"(y)
                : "memory");
 }
-// the same box added element by element into global memory (s32 here: exact,
-// so the order of the additions does not matter)
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int x, int y) {
-  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(smem_u32(src)), "r"(x), "r"(y)
-               : "memory");
-}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // the bulk stores committed by this thread have finished reading shared memory
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
@@ -479,12 +471,9 @@ struct Params {
   int y_vec;    // 1: Y and ldy allow 16-byte vector stores
   int y_tma;    // 1: bf16 output with beta == 0 leaves through staged bulk tensor stores (pair kernel)
   // Pair kernel work list: items [0, split_from) are whole tiles; the tiles
-  // from split_from on (the last, partly filled wave) are each done as two
-  // half-width items, or, with ks > 0, as ks items over consecutive ranges of
-  // K whose exact s32 sums are added into Y (zeroed first) by bulk tensor
-  // reductions.
+  // from split_from on are each done as two half-width items (the last,
+  // partly filled wave then takes half as long).
   int split_from, num_work;
-  int ks;
   int n_ymaps;  // output tensor maps the staged stores go through (1, or one per destination GPU)
   float alpha, beta;
   uint64_t wait_ns;  // limit of every bounded wait (kWaitLimitNs unless a test shortens it)
@@ -513,28 +502,13 @@ __device__ __forceinline__ void grouped_tile(const Params& p, int t, int& mt, in
   }
 }
 
-// Work item w of the pair kernel: its tile (mt, nt), first output column,
-// whether it is a half-width item, its K-stage range and whether its sums are
-// added into Y rather than stored.
+// Work item w of the pair kernel: its tile (mt, nt), first output column and
+// whether it is a half-width item.
 struct PairWork {
   int mt, nt, col0, narrow;
-  int kb0, kb1, reduce;
 };
 __device__ __forceinline__ PairWork pair_work(const Params& p, int w, int n_total) {
   PairWork k;
-  k.kb0 = 0;
-  k.kb1 = p.k_blocks;
-  k.reduce = 0;
-  if (p.ks > 0 && w >= p.split_from) {  // every piece holds at least one stage (ks <= k_blocks)
-    const int j = w - p.split_from, piece = j % p.ks;
-    grouped_tile(p, p.split_from + j / p.ks, k.mt, k.nt);
-    k.narrow = 0;
-    k.col0 = k.nt * n_total;
-    k.kb0 = int(int64_t(piece) * p.k_blocks / p.ks);
-    k.kb1 = int(int64_t(piece + 1) * p.k_blocks / p.ks);
-    k.reduce = 1;
-    return k;
-  }
   const bool narrow = w >= p.split_from;
   const int t = narrow ? p.split_from + ((w - p.split_from) >> 1) : w;
   grouped_tile(p, t, k.mt, k.nt);
@@ -917,7 +891,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const int b_boxes = (C::kCanSplit && wk.narrow) ? 64 / K_::kAtomCols : C::kBBoxes;
         const int b_cols = (C::kCanSplit && wk.narrow) ? 64 : C::kNHalf;
         const uint32_t tx = 2u * uint32_t(C::kABytes + b_boxes * C::kBBoxBytes + C::kEBytes);
-        for (int kb = wk.kb0; kb < wk.kb1; ++kb, ++it) {
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           if (int64_t(it) == p.skip_it) continue;  // test hook: neither CTA fills this step's stage
           const int s = int(it % STAGES);
           const uint32_t round = it / STAGES;
@@ -946,14 +920,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       uint32_t it = 0, local = 0;
       bool ok = true;
       for (int w = pair; w < num_work && ok; w += num_pairs, ++local) {
-        const PairWork wk = pair_work(p, w, N_TOTAL);
-        const uint32_t idesc = wk.narrow ? idesc_narrow : idesc_full;
+        const uint32_t idesc = w >= p.split_from ? idesc_narrow : idesc_full;
         const int buf = int(local % C::kAccBufs);
         const uint32_t use = local / C::kAccBufs;
         if (!mbar_wait(&acc_empty[buf], (use & 1u) ^ 1u, abort_flag, p.wait_ns)) { ok = false; break; }
         fence_after_sync();
         const uint32_t d_tmem = tmem_base + uint32_t(buf * N_TOTAL);
-        for (int kb = wk.kb0; kb < wk.kb1; ++kb, ++it) {
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
           const int s = int(it % STAGES);
           const uint32_t round = it / STAGES;
           if (!mbar_wait(&full[s], round & 1u, abort_flag, p.wait_ns)) { ok = false; break; }
@@ -974,7 +947,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                                              K_::kB32Atom ? 512u : 1024u, K_::kB32Atom ? kLayoutSW128_32B : kLayoutSW128);
             uint32_t e_col, sel;
             meta_operand<KD>(e_tmem, k2, e_col, sel);
-            mma_sp_pair<KD>(d_tmem, adesc, bdesc, e_col, idesc | sel, (kb > wk.kb0 || k2 > 0) ? 1u : 0u);
+            mma_sp_pair<KD>(d_tmem, adesc, bdesc, e_col, idesc | sel, (kb > 0 || k2 > 0) ? 1u : 0u);
           }
           mma_commit_pair(&empty[s]);
         }
@@ -1050,12 +1023,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0 && row0 < p.R && c_base + c < p.T) {  // boxes start inside Y
-            if (wk.reduce) {
-              tma_reduce_add_2d(&ymaps.m[0], smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes, c_base + c, row0);
-            } else {
-              for (int j = 0; j < n_ymaps; ++j)
-                tma_store_2d(&ymaps.m[j], smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes, c_base + c, row0);
-            }
+            for (int j = 0; j < n_ymaps; ++j)
+              tma_store_2d(&ymaps.m[j], smem + C::kOutOff + (warp - 2) * C::kOutSlotBytes, c_base + c, row0);
             bulk_commit();
           }
         }
@@ -1257,20 +1226,6 @@ bool make_map_image(CUtensorMap* map, const uint8_t* img, int64_t rows16, int bo
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Zeroes the output tiles [split_from, split_from + gridDim.x) of the pair
-// kernel's order (s32 output, 16-byte rows) before their K pieces are added.
-__global__ void zero_tiles_kernel(Params p, int n_total) {
-  int mt, nt;
-  grouped_tile(p, p.split_from + int(blockIdx.x), mt, nt);
-  const int r0 = mt * 2 * kBlockM, c0 = nt * n_total;
-  const int rows = min(2 * kBlockM, p.R - r0), quads = min(n_total, p.T - c0) / 4;  // T % 4 == 0 here
-  for (int i = int(threadIdx.x); i < rows * quads; i += int(blockDim.x)) {
-    const int r = i / quads, c = i - r * quads;
-    reinterpret_cast<uint4*>(static_cast<uint32_t*>(p.Y) + size_t(r0 + r) * size_t(p.ldy) + c0)[c] =
-        make_uint4(0u, 0u, 0u, 0u);
-  }
-}
-
 template <int N_TOTAL, int STAGES, Kind KD, int NMAP = 1>
 nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& me, const YMaps<NMAP>& my,
                       const Params& p, bool tail_split, cudaStream_t s) {
@@ -1280,33 +1235,17 @@ nm_status launch_pair(const CUtensorMap& ma, const CUtensorMap& mb, const CUtens
   if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes) != NM_OK) return NM_ERR_CUDA;
   const int tiles = p.m_tiles * p.n_tiles;
   const int max_pairs = sm_count() / 2;
-  int pairs = tiles < max_pairs ? tiles : max_pairs;
+  const int pairs = tiles < max_pairs ? tiles : max_pairs;
   Params q = p;
   q.split_from = tiles;
   q.num_work = tiles;
-  q.ks = 0;
   // A last wave that fills at most half of the pairs is done in half-width
   // items (whole B atoms per CTA, so only for 256-column tiles of 16- and
   // 32-bit operands).
   const int rem = tiles % pairs;
-  // int8 operands with the exact s32 output (whose sums may be added in any
-  // order) split the tiles of such a wave along K instead: ks pieces per tile
-  // spread over the pairs, each adding its partial sums into Y, which a
-  // small kernel zeroes first.  Their 128-column B atoms rule out half-width
-  // items.  A single partly filled wave (tiles <= pairs) is split the same way.
-  const int last = tiles > max_pairs ? tiles % max_pairs : tiles;
   if (C::kCanSplit && tiles > pairs && rem > 0 && 2 * rem <= pairs && tail_split) {
     q.split_from = tiles - rem;
     q.num_work = tiles + rem;
-  } else if (KD == Kind::S8 && NMAP == 1 && p.y_s32 && p.y_tma && tail_split && last > 0 && 2 * last <= max_pairs) {
-    const int ks = min(p.k_blocks, max_pairs / last);
-    if (ks >= 2) {
-      q.split_from = tiles - last;
-      q.num_work = q.split_from + last * ks;
-      q.ks = ks;
-      pairs = q.num_work < max_pairs ? q.num_work : max_pairs;
-      zero_tiles_kernel<<<last, 256, 0, s>>>(q, N_TOTAL);
-    }
   }
   kern<<<2 * pairs, kPairThreads, C::kSmemBytes, s>>>(ma, mb, me, my, q);
   return launch_status();
@@ -1365,7 +1304,6 @@ nm_status run(const void* values, const uint8_t* meta_img, const void* X, int64_
   if (n_peers > 0) Y = static_cast<uint8_t*>(peer_y[0]) + size_t(row0) * size_t(ldy) * 2;
   Params p;
   p.n_ymaps = 1;
-  p.ks = 0;
   p.wait_ns = o.wait_ns;
   p.skip_it = o.skip_it;
   p.y_tma = 0;

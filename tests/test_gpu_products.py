@@ -155,32 +155,6 @@ def test_int8_full_size_decode_weight(T):
     assert np.array_equal(Y.numpy()[rows].astype(np.float64), ref)
 
 
-# (R, K, T): a partly filled last wave of 256 x 256 tiles, split along K into
-# pieces whose exact sums are added into the zeroed output
-K_SPLIT_CASES = [(512, 4096, 512),     # one wave of 4 tiles, 16 pieces each
-                 (10240, 1024, 512),   # 80 tiles: a last wave of 6, 4 pieces each (every K stage its own piece)
-                 (1000, 768, 300),     # ragged rows and columns, 3 pieces
-                 (256, 512, 256),      # a single tile in 2 pieces
-                 (2304, 2048, 1024)]   # one wave of 36 tiles, 2 pieces each
-
-
-@pytest.mark.parametrize("R,K,T", K_SPLIT_CASES)
-def test_int8_k_split_last_wave_is_exact(R, K, T):
-    """The int32 output with the last wave split along K equals the whole-tile
-    result bit for bit, and both equal the exact sum."""
-    W, X = _s8_case(R, K, T, 7 * R + K + T)
-    Y, values, meta = _s8_gpu(W, X)
-    img = nm.nm_meta_to_sm100_s8(meta, R, K)
-    Y1 = nm.nm_spmm_test(values, img, _dev_x(X, 16), y_dtype=torch.int32, kernel="pair256", tail_split=False)
-    torch.cuda.synchronize()
-    assert nm.nm_last_device_status() == 0
-    assert torch.equal(Y, Y1.cpu())
-    rows = None if R <= 2304 else _sample_rows(R, 2)
-    ref = _s8_ref(W, X, rows=rows)
-    got = Y.numpy() if rows is None else Y.numpy()[rows]
-    assert np.array_equal(got.astype(np.float64), ref)
-
-
 # ---------------------------------------------------------------- TF32 1:2
 def _tf32_gpu(W, X, y_dtype=torch.float32, kernel=None, alpha=1.0, beta=0.0, Y0=None):
     R, K = W.shape
