@@ -71,6 +71,7 @@ def transposable_int_ops(M: int) -> float:
     return 2.0 * comps + 7.0 * M * M + 2.0 * M * M
 SPARSE_RATIO = 2.0   # 2:4 sparse tensor peak = 2x dense (dense-equivalent flops)
 PEER_WAIT_NS = 2_000_000_000   # limit of the row-split step's wait for every GPU's rows of H
+IPC_MAPPINGS = []              # (address, offset) of every other GPU's buffer this process mapped
 # dense throughput of the int8 and tf32 tensor-core kinds relative to bf16 (nominal B200 figures:
 # 4.5 POPS int8, 1.1 PFLOPS tf32 against 2.25 PFLOPS bf16); applied to the measured bf16 peak
 KIND_RATIO = {"int8": 2.0, "pairs": 0.5}
@@ -453,7 +454,7 @@ class Step:
             torch.cuda.synchronize()              # zeroed before any peer can write
         every = [None] * world_
         dist_.all_gather_object(every, mine)
-        self.peer_H, self.peer_F, self._opened = [[], []], [], []
+        self.peer_H, self.peer_F = [[], []], []
         for j in range(world_):
             if j == rank_:
                 self.peer_H[0].append(self.H_bufs[0])
@@ -463,7 +464,7 @@ class Step:
             addrs = []
             for h, off in every[j]:
                 addrs.append(nm.nm_ipc_open(h, off))
-                self._opened.append((addrs[-1], off))
+                IPC_MAPPINGS.append((addrs[-1], off))
             self.peer_H[0].append(addrs[0])
             self.peer_H[1].append(addrs[1])
             self.peer_F.append(addrs[2])
@@ -1219,7 +1220,10 @@ def main():
                 "clocks": clk, "kernels": kernels}
         print(json.dumps(line), flush=True)
     if pg:
-        pg.barrier()
+        torch.cuda.synchronize()
+        pg.barrier()                # no rank's kernels touch another GPU's buffers any more
+        while IPC_MAPPINGS:
+            nm.nm_ipc_close(*IPC_MAPPINGS.pop())
         pg.destroy_process_group()
 
 

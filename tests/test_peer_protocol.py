@@ -174,6 +174,8 @@ def _run(world, steps, single_buffer=False, slow_rank=1):
     for t in threads:
         t.join(timeout=120)
         assert not t.is_alive()
+    assert len(bench.IPC_MAPPINGS) == 3 * world * (world - 1)   # two H buffers and the flags of every other rank
+    bench.IPC_MAPPINGS.clear()
     return ranks, errors
 
 
