@@ -1,7 +1,9 @@
 /*
  * nm.h -- C ABI of libnm: N:M fine-grained structured sparsity on NVIDIA
  * B200 (sm_100a).  Mask selection, 2:4 compression / decompression, the
- * tensor-core metadata image, and the 2:4-sparse x dense product.
+ * tensor-core metadata image, the 2:4-sparse x dense product, and that
+ * product split by output rows over several GPUs (peer stores, completion
+ * flags, IPC mappings).
  *
  * Conventions shared by every call
  * --------------------------------
