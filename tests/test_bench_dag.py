@@ -291,3 +291,4 @@ def test_row_split_mlp_fused_exchange():
                 reads_j, writes_j = rec.log[j]
                 if (writes_j & reads_i) or (reads_j & writes_i) or (writes_j & writes_i):
                     assert j in before[i], (names[j], names[i])
+    bench.IPC_MAPPINGS.clear()

@@ -144,6 +144,7 @@ def _bf16(*shape):
 
 
 def _run(world, steps, single_buffer=False, slow_rank=1):
+    bench.IPC_MAPPINGS.clear()                # whatever earlier tests in this process mapped
     R, K, T = 256 * world, 64, 8
     wl = {"W": _bf16(R, K), "W2": _bf16(K, R), "X": _bf16(K, T), "R": R, "K": K, "T": T}
     shared = {"objs": [None] * world, "barrier": threading.Barrier(world, timeout=60)}
